@@ -1,0 +1,268 @@
+"""COAT oracle -- TEST INFRASTRUCTURE ONLY.
+
+Python face of the plain C oracle (``coat_oracle.c``) plus an unquantized
+binary64 AdamW.  Only the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package; the CUDA library
+and its binding never do.
+
+Pages cited (by title and section):
+  COAT summary, "COAT: 压缩优化器状态和激活以实现内存高效的 FP8 训练"
+  (blog.daoxuan.cc/posts/57954): sections on the AdamW rule and why v is
+  sensitive, the expansion function f(x) = sign(x)|x|^k with
+  k = log(R_E4M3)/log(R_X), mixed granularity (1xG groups and Group Scaling).
+  LLM Atlas "systems/numerics" (llm-atlas.k1412.top): section 03 "FP8"
+  (format limits) and section 08 "Adam -> AdamW" (the update rule).
+
+Parity status: pinned by tests/test_oracle_*.py; the magnitude of the error
+reduction from the expansion function is "parity unpinned" (direction only).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+E4M3 = 0
+E5M2 = 1
+
+_lib = None
+
+
+class AdamWCfg(ctypes.Structure):
+    _fields_ = [
+        ("beta1", ctypes.c_float),
+        ("beta2", ctypes.c_float),
+        ("lr", ctypes.c_float),
+        ("eps", ctypes.c_float),
+        ("weight_decay", ctypes.c_float),
+        ("step", ctypes.c_int64),
+        ("group_size", ctypes.c_int64),
+        ("m_fmt", ctypes.c_int32),
+        ("v_fmt", ctypes.c_int32),
+        ("k_range", ctypes.c_int32),
+        ("k_max", ctypes.c_float),
+        ("force_k1", ctypes.c_int32),
+    ]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        L.orc_exmy_value.restype = ctypes.c_double
+        L.orc_exmy_value.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_uint32,
+                                     ctypes.c_uint32]
+        L.orc_fp8_decode.restype = ctypes.c_double
+        L.orc_fp8_decode.argtypes = [ctypes.c_uint8, ctypes.c_int]
+        L.orc_fp8_encode.restype = ctypes.c_uint8
+        L.orc_fp8_encode.argtypes = [ctypes.c_float, ctypes.c_int]
+        for name in ("orc_fp8_max", "orc_fp8_min_subnormal", "orc_fp8_range"):
+            getattr(L, name).restype = ctypes.c_double
+            getattr(L, name).argtypes = [ctypes.c_int]
+        L.orc_bf16_to_f32.restype = ctypes.c_float
+        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.orc_f32_to_bf16.restype = ctypes.c_uint16
+        L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.orc_fp8_encode_array.restype = None
+        L.orc_fp8_encode_array.argtypes = [P, i64, ctypes.c_int, P]
+        L.orc_f32_to_bf16_array.restype = None
+        L.orc_f32_to_bf16_array.argtypes = [P, i64, P]
+        L.orc_state_dequant_one.restype = ctypes.c_float
+        L.orc_state_dequant_one.argtypes = [ctypes.c_uint8, ctypes.c_float, ctypes.c_float,
+                                            ctypes.c_int]
+        L.orc_quantize_state.restype = ctypes.c_int
+        L.orc_quantize_state.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                         ctypes.c_int, P, P, P]
+        L.orc_dequant.restype = ctypes.c_int
+        L.orc_dequant.argtypes = [P, P, P, i64, i64, ctypes.c_int, P]
+        L.orc_adamw_fp8_step.restype = ctypes.c_int
+        L.orc_adamw_fp8_step.argtypes = [P, P, P, P, P, P, P, P, i64,
+                                         ctypes.POINTER(AdamWCfg), P, P]
+        L.orc_group_quant_1xG.restype = ctypes.c_int
+        L.orc_group_quant_1xG.argtypes = [P, i64, i64, i64, i64, ctypes.c_int, P, P]
+        L.orc_group_scaling_pertensor.restype = ctypes.c_int
+        L.orc_group_scaling_pertensor.argtypes = [P, i64, i64, ctypes.c_int, P, ctypes.c_int,
+                                                  P, P]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle buffers must be contiguous"
+    return a.ctypes.data
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (rc={rc})")
+
+
+# ---- formats ---------------------------------------------------------------
+
+def exmy_value(ebits: int, mbits: int, bias: int, e: int, m: int) -> float:
+    return lib().orc_exmy_value(ebits, mbits, bias, e, m)
+
+
+def fp8_decode(code: int, fmt: int) -> float:
+    return lib().orc_fp8_decode(code, fmt)
+
+
+def fp8_encode(y: float, fmt: int) -> int:
+    return lib().orc_fp8_encode(y, fmt)
+
+
+def fp8_encode_array(y: np.ndarray, fmt: int) -> np.ndarray:
+    """fp8_encode applied to every element (the loop runs in C)."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    out = np.empty(y.shape, dtype=np.uint8)
+    lib().orc_fp8_encode_array(_ptr(y), y.size, fmt, _ptr(out))
+    return out
+
+
+def fp8_max(fmt: int) -> float:
+    return lib().orc_fp8_max(fmt)
+
+
+def fp8_min_subnormal(fmt: int) -> float:
+    return lib().orc_fp8_min_subnormal(fmt)
+
+
+def fp8_range(fmt: int) -> float:
+    return lib().orc_fp8_range(fmt)
+
+
+def bf16_to_f32(b: int) -> float:
+    return lib().orc_bf16_to_f32(b)
+
+
+def f32_to_bf16(f: float) -> int:
+    return lib().orc_f32_to_bf16(f)
+
+
+# ---- optimizer states ------------------------------------------------------
+
+def n_groups(n: int, G: int) -> int:
+    return (n + G - 1) // G
+
+
+def quantize_state(x: np.ndarray, G: int, fmt: int, k_range: int = 0, k_max: float = 64.0,
+                   force_k1: bool = False):
+    """FP32 state -> (codes u8[n], k f32[ngroups], s f32[ngroups])."""
+    x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1)
+    n = x.size
+    code = np.empty(n, dtype=np.uint8)
+    k = np.empty(n_groups(n, G), dtype=np.float32)
+    s = np.empty(n_groups(n, G), dtype=np.float32)
+    _check(lib().orc_quantize_state(_ptr(x), n, G, fmt, k_range, k_max, int(force_k1),
+                                    _ptr(code), _ptr(k), _ptr(s)), "quantize_state")
+    return code, k, s
+
+
+def dequant(q: np.ndarray, k: np.ndarray | None, s: np.ndarray, G: int, fmt: int) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8).reshape(-1)
+    s = np.ascontiguousarray(s, dtype=np.float32).reshape(-1)
+    kk = None if k is None else np.ascontiguousarray(k, dtype=np.float32).reshape(-1)
+    out = np.empty(q.size, dtype=np.float32)
+    _check(lib().orc_dequant(_ptr(q), _ptr(kk), _ptr(s), q.size, G, fmt, _ptr(out)), "dequant")
+    return out
+
+
+def to_bf16_array(x: np.ndarray) -> np.ndarray:
+    """binary32 -> BF16 bits, nearest-even, for every element (loop in C)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib().orc_f32_to_bf16_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def adamw_fp8_step(theta, grad_bf16, m_code, m_k, m_s, v_code, v_k, v_s, *, beta1, beta2, lr,
+                   eps, weight_decay, step, group_size, m_fmt=E4M3, v_fmt=E4M3, k_range=0,
+                   k_max=64.0, force_k1=False, return_moments=False):
+    """One COAT step; returns new copies (inputs untouched).
+
+    Returns (theta, m_code, m_k, m_s, v_code, v_k, v_s) and, with
+    return_moments, the FP32 m_t and v_t before re-quantization.
+    """
+    th = np.array(theta, dtype=np.float32, copy=True).reshape(-1)
+    g = np.ascontiguousarray(grad_bf16, dtype=np.uint16).reshape(-1)
+    mc = np.array(m_code, dtype=np.uint8, copy=True).reshape(-1)
+    vc = np.array(v_code, dtype=np.uint8, copy=True).reshape(-1)
+    mk = np.array(m_k, dtype=np.float32, copy=True).reshape(-1)
+    ms = np.array(m_s, dtype=np.float32, copy=True).reshape(-1)
+    vk = np.array(v_k, dtype=np.float32, copy=True).reshape(-1)
+    vs = np.array(v_s, dtype=np.float32, copy=True).reshape(-1)
+    n = th.size
+    assert g.size == n and mc.size == n and vc.size == n
+    assert mk.size == n_groups(n, group_size) == vk.size
+    cfg = AdamWCfg(beta1, beta2, lr, eps, weight_decay, step, group_size, m_fmt, v_fmt,
+                   k_range, k_max, int(force_k1))
+    mt = np.empty(n, dtype=np.float32) if return_moments else None
+    vt = np.empty(n, dtype=np.float32) if return_moments else None
+    _check(lib().orc_adamw_fp8_step(_ptr(th), _ptr(g), _ptr(mc), _ptr(mk), _ptr(ms), _ptr(vc),
+                                    _ptr(vk), _ptr(vs), n, ctypes.byref(cfg), _ptr(mt),
+                                    _ptr(vt)), "adamw_fp8_step")
+    out = (th, mc, mk, ms, vc, vk, vs)
+    return out + (mt, vt) if return_moments else out
+
+
+def adamw_fp64(theta, grad, m, v, *, step, beta1, beta2, lr, eps, weight_decay):
+    """Unquantized AdamW in binary64 (LLM Atlas, section 08 "Adam -> AdamW").
+
+    m_t = b1 m + (1-b1) g ; v_t = b2 v + (1-b2) g^2 ;
+    theta_t = (1 - lr*wd) theta - lr * m_hat / (sqrt(v_hat) + eps).
+    Returns (theta_t, m_t, v_t) as float64 arrays.
+    """
+    theta = np.asarray(theta, dtype=np.float64)
+    g = np.asarray(grad, dtype=np.float64)
+    m = np.asarray(m, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    b1, b2 = float(np.float32(beta1)), float(np.float32(beta2))
+    m_t = b1 * m + (1.0 - b1) * g
+    v_t = b2 * v + (1.0 - b2) * g * g
+    m_hat = m_t / (1.0 - b1 ** step)
+    v_hat = v_t / (1.0 - b2 ** step)
+    th = theta * (1.0 - float(np.float32(lr)) * float(np.float32(weight_decay)))
+    th = th - float(np.float32(lr)) * m_hat / (np.sqrt(v_hat) + float(np.float32(eps)))
+    return th, m_t, v_t
+
+
+# ---- activations -----------------------------------------------------------
+
+def group_quant_1xG(x_bf16: np.ndarray, G: int, fmt: int = E4M3):
+    """x_bf16: uint16 [rows, cols] -> (q u8 [rows, cols], scale f32 [rows, cols/G])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    q = np.empty((rows, cols), dtype=np.uint8)
+    sc = np.empty((rows, cols // G), dtype=np.float32)
+    _check(lib().orc_group_quant_1xG(_ptr(x), rows, cols, cols, G, fmt, _ptr(q), _ptr(sc)),
+           "group_quant_1xG")
+    return q, sc
+
+
+def group_scaling_pertensor(x_bf16: np.ndarray, G: int, fmt: int = E4M3,
+                            group_amax: np.ndarray | None = None):
+    """Flat BF16 -> (q u8[n], scale float, group_amax f32[ceil(n/G)])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16).reshape(-1)
+    n = x.size
+    pre = group_amax is not None
+    ga = (np.array(group_amax, dtype=np.float32, copy=True) if pre
+          else np.empty(n_groups(n, G), dtype=np.float32))
+    q = np.empty(n, dtype=np.uint8)
+    sc = np.empty(1, dtype=np.float32)
+    _check(lib().orc_group_scaling_pertensor(_ptr(x), n, G, fmt, _ptr(ga), int(pre), _ptr(q),
+                                             _ptr(sc)), "group_scaling_pertensor")
+    return q, float(sc[0]), ga
+
+
+def threads_used() -> int:
+    return 1
+
+
+__all__ = [n for n in dir() if not n.startswith("_")]

@@ -1,0 +1,245 @@
+"""Pins of the oracle's optimizer-state path (CPU only).
+
+AdamW part: the binary64 reference equals torch.optim.AdamW (a library
+routine), and the oracle's binary32 step equals that reference up to
+binary32 rounding.  Quantization part: invariants that follow from the
+definition of f(x) = sign(x)|x|^k and k = log(R_E4M3) / log(R_X) (COAT
+summary page, section "扩展函数：把窄分布拉宽"): sign preservation, the group
+maximum on the format maximum, the group minimum on the format minimum, a
+closed-form round-trip error bound, k = 1 for all-zero / all-equal groups,
+re-quantization idempotence, and the direction of the error reduction.
+"""
+import numpy as np
+import pytest
+import torch
+
+from quantized_optimizer_states_b200 import inputs
+
+E4M3, E5M2 = 0, 1
+H = inputs.HYPER
+
+
+def _f32(x):
+    return float(np.float32(x))
+
+
+# ---------------------------------------------------------------- AdamW ----
+
+def test_fp64_adamw_equals_torch_adamw(orc):
+    """LLM Atlas section 08 "Adam -> AdamW": the binary64 reference must be
+    torch's AdamW (decoupled decay, eps outside the root, bias-corrected)."""
+    rng = np.random.default_rng(3)
+    n = 4096
+    theta0 = rng.normal(0, 0.02, n)
+    p = torch.nn.Parameter(torch.tensor(theta0, dtype=torch.float64))
+    opt = torch.optim.AdamW([p], lr=_f32(H["lr"]), betas=(_f32(H["beta1"]), _f32(H["beta2"])),
+                            eps=_f32(H["eps"]), weight_decay=_f32(H["weight_decay"]),
+                            foreach=False)
+    th, m, v = theta0.copy(), np.zeros(n), np.zeros(n)
+    for t in range(1, 4):
+        g = rng.normal(0, 1e-3, n)
+        p.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+        th, m, v = orc.adamw_fp64(th, g, m, v, step=t, **H)
+        ref = p.detach().numpy()
+        assert np.max(np.abs(th - ref) / np.maximum(np.abs(ref), 1e-30)) < 1e-12
+        st = opt.state[p]
+        assert np.allclose(m, st["exp_avg"].numpy(), rtol=1e-12, atol=0)
+        assert np.allclose(v, st["exp_avg_sq"].numpy(), rtol=1e-12, atol=0)
+
+
+def _state(orc, n, G, v_fmt=E4M3, seed=5, w=None):
+    w = w or inputs.tiny(seed)
+    x = inputs.host_step_inputs(w, n)
+    mc, mk, ms = orc.quantize_state(x["m0"], G, E4M3)
+    vc, vk, vs = orc.quantize_state(x["v0"], G, v_fmt)
+    return x, (mc, mk, ms, vc, vk, vs)
+
+
+@pytest.mark.parametrize("v_fmt", [E4M3, E5M2])
+def test_fp32_step_matches_fp64_adamw_on_same_states(orc, v_fmt):
+    """The binary32 step (before re-quantization) is AdamW: theta_t, m_t and
+    v_t agree with the binary64 reference fed the same dequantized states.
+    A dropped bias correction, a sign error in the decay, eps inside the
+    root or swapped moments all fail this by orders of magnitude."""
+    n, G, t = 8192, 128, 10
+    x, (mc, mk, ms, vc, vk, vs) = _state(orc, n, G, v_fmt)
+    m_in = orc.dequant(mc, mk, ms, G, E4M3)
+    v_in = orc.dequant(vc, vk, vs, G, v_fmt)
+    out = orc.adamw_fp8_step(x["theta"], x["grad"], mc, mk, ms, vc, vk, vs, step=t, group_size=G,
+                             v_fmt=v_fmt, return_moments=True, **H)
+    th32, mt32, vt32 = out[0], out[7], out[8]
+    g = torch.from_numpy(x["grad"].view(np.int16)).view(torch.bfloat16).double().numpy()
+    th64, mt64, vt64 = orc.adamw_fp64(x["theta"], g, m_in, v_in, step=t, **H)
+    # each moment is a sum of two rounded products: the binary32 error is a
+    # few units of 2^-24 of the summands' magnitude (m_t may cancel to ~0)
+    b1, b2 = _f32(H["beta1"]), _f32(H["beta2"])
+    mag_m = np.abs(b1 * m_in) + np.abs((1 - b1) * g)
+    mag_v = np.abs(b2 * v_in) + np.abs((1 - b2) * g * g)
+    assert np.max(np.abs(mt32 - mt64) / np.maximum(mag_m, 1e-30)) < 4 * 2.0 ** -24
+    assert np.max(np.abs(vt32 - vt64) / np.maximum(mag_v, 1e-30)) < 4 * 2.0 ** -24
+    den = np.maximum(np.abs(th64), H["lr"])
+    assert np.max(np.abs(th32 - th64) / den) < 1e-6
+
+
+# ---------------------------------------------------- state quantization ----
+
+def _groups(a, G):
+    n = a.size
+    return [a[i:i + G] for i in range(0, n, G)]
+
+
+@pytest.mark.parametrize("fmt,k_range", [(E4M3, 0), (E5M2, 0), (E5M2, 1)])
+@pytest.mark.parametrize("dist", ["m", "v"])
+def test_quantize_invariants(orc, fmt, k_range, dist):
+    rng = np.random.default_rng(21)
+    G, n = 128, 128 * 64
+    x = (rng.normal(0, 1e-4, n) if dist == "m" else rng.lognormal(-18, 1, n)).astype(np.float32)
+    x[::97] = 0.0
+    code, k, s = orc.quantize_state(x, G, fmt, k_range=k_range, k_max=0.0)
+    top = 0x7E if fmt == E4M3 else 0x7B
+    fmax = orc.fp8_max(fmt)
+    R = orc.fp8_range(fmt if k_range == 1 else E4M3)
+    for gi, (xg, cg) in enumerate(zip(_groups(x, G), _groups(code, G))):
+        nz = xg != 0
+        # sign preservation, zero -> code 0
+        assert np.all(cg[~nz] == 0)
+        assert np.all((cg[nz] >> 7) == (xg[nz] < 0))
+        a = np.abs(xg)
+        imax = np.argmax(a)
+        assert cg[imax] & 0x7F == top
+        # the smallest nonzero magnitude lands on fmt_max / R (the bottom of the
+        # target range): code 0x01 for E4M3, the code of 0.25 for E5M2/R_E4M3
+        imin = np.argmin(np.where(nz, a, np.inf))
+        want = orc.fp8_encode(fmax / R, fmt)
+        assert cg[imin] & 0x7F == want
+        # k from the definition of the range ratio
+        assert k[gi] > 0
+    # stored scale: x_max = fmt_max^(1/k) * s
+    for gi, xg in enumerate(_groups(x, G)):
+        M = np.max(np.abs(xg))
+        assert abs(fmax ** (1.0 / k[gi]) * s[gi] - M) <= 4e-7 * M
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_roundtrip_error_bound(orc, fmt):
+    """Closed form: where the expanded value y is a normal FP8 number, RNE
+    gives |y'-y|/y <= 2^-(mbits+1), so |x'-x|/x <= (1+2^-(mbits+1))^(1/k) - 1
+    (plus binary32 rounding).  A wrong scale, k or exponent sign breaks it."""
+    rng = np.random.default_rng(8)
+    G, n = 128, 128 * 200
+    x = rng.lognormal(-18, 1.0, n).astype(np.float32) * np.sign(rng.normal(size=n)).astype(
+        np.float32)
+    code, k, s = orc.quantize_state(x, G, fmt, k_max=0.0)
+    xr = orc.dequant(code, k, s, G, fmt)
+    mbits = 3 if fmt == E4M3 else 2
+    min_normal = 2.0 ** -6 if fmt == E4M3 else 2.0 ** -14
+    dec = np.array([abs(orc.fp8_decode(int(c), fmt)) for c in code])
+    kk = np.repeat(k, G)[:n].astype(np.float64)
+    bound = (1.0 + 2.0 ** -(mbits + 1)) ** (1.0 / kk) - 1.0 + 3e-7
+    rel = np.abs(xr.astype(np.float64) - x) / np.abs(x)
+    normal = dec > min_normal          # y itself then lies in the normal range
+    assert normal.mean() > 0.9
+    assert np.all(rel[normal] <= bound[normal])
+
+
+def test_all_zero_and_all_equal_groups(orc):
+    G = 64
+    x = np.zeros(3 * G, dtype=np.float32)
+    x[G:2 * G] = -3.5e-6                       # all equal magnitudes
+    x[2 * G:] = np.where(np.arange(G) % 2, 2e-3, -2e-3)
+    code, k, s = orc.quantize_state(x, G, E4M3)
+    assert k[0] == 1.0 and s[0] == 0.0 and np.all(code[:G] == 0)
+    assert k[1] == 1.0 and np.all(code[G:2 * G] == 0xFE)
+    assert k[2] == 1.0 and np.all(code[2 * G:] & 0x7F == 0x7E)
+    assert s[1] == np.float32(3.5e-6 / 448.0)
+    xr = orc.dequant(code, k, s, G, E4M3)
+    assert np.all(xr[:G] == 0)
+    assert np.allclose(xr[G:], x[G:], rtol=1e-6, atol=0)
+
+
+def test_k_clamp_for_near_equal_group(orc):
+    G = 128
+    x = np.linspace(1.0, 1.01, G).astype(np.float32) * 1e-7
+    _, k, _ = orc.quantize_state(x, G, E4M3, k_max=64.0)
+    assert k[0] == 64.0
+    _, k0, _ = orc.quantize_state(x, G, E4M3, k_max=0.0)
+    assert k0[0] > 64.0
+
+
+def test_requantization_idempotent(orc):
+    """dequant -> quantize gives back the same codes: the dequantized group
+    has R_X' = R_target^(1/k), hence the same k (COAT's expansion is exactly
+    undone by the 1/k power).  Ties may flip at binary32 rounding; allow a
+    tiny fraction, one code apart."""
+    rng = np.random.default_rng(9)
+    G, n = 128, 128 * 512
+    for fmt, x in ((E4M3, rng.normal(0, 1e-4, n)), (E5M2, rng.lognormal(-18, 1, n))):
+        x = x.astype(np.float32)
+        c1, k1, s1 = orc.quantize_state(x, G, fmt)
+        xr = orc.dequant(c1, k1, s1, G, fmt)
+        c2, k2, s2 = orc.quantize_state(xr, G, fmt)
+        diff = c1.astype(np.int32) - c2.astype(np.int32)
+        assert np.mean(diff != 0) < 1e-3
+        assert np.all(np.abs(diff) <= 1)
+        assert np.allclose(k1, k2, rtol=1e-5)
+
+
+def test_typical_k_ranges(orc):
+    """COAT summary, section "扩展函数": k for m is typically 1-3 and for v
+    5-15.  On page-typical states (m ~ N(0, 1e-4); v with a narrow group-local
+    spread, logN(-18, 0.25)) the median k must fall in those ranges."""
+    rng = np.random.default_rng(10)
+    G, n = 128, 128 * 1024
+    _, km, _ = orc.quantize_state(rng.normal(0, 1e-4, n).astype(np.float32), G, E4M3)
+    _, kv, _ = orc.quantize_state(rng.lognormal(-18, 0.25, n).astype(np.float32), G, E4M3)
+    assert 1.0 <= np.median(km) <= 3.0
+    assert 5.0 <= np.median(kv) <= 15.0
+
+
+@pytest.mark.parametrize("dist", ["m", "v"])
+def test_expansion_reduces_error_direction(orc, dist):
+    """COAT summary, section "扩展函数": the expansion lowers the quantization
+    error against plain per-group scaling (k = 1).  Only the direction is
+    pinned; the quoted 1.63x was measured on real OLMo states."""
+    rng = np.random.default_rng(12)
+    G, n = 128, 128 * 1024
+    x = (rng.normal(0, 1e-4, n) if dist == "m" else rng.lognormal(-18, 0.5, n)).astype(np.float32)
+    errs = []
+    for force in (False, True):
+        c, k, s = orc.quantize_state(x, G, E4M3, force_k1=force)
+        xr = orc.dequant(c, k, s, G, E4M3).astype(np.float64)
+        errs.append(np.linalg.norm(xr - x) / np.linalg.norm(x))
+    assert errs[0] < errs[1]
+
+
+@pytest.mark.parametrize("G", [32, 64, 128, 256, 1024])
+@pytest.mark.parametrize("v_fmt", [E4M3, E5M2])
+def test_brute_force_tiny_three_steps(orc, G, v_fmt):
+    """N = 2048, three steps against an unquantized binary64 AdamW run; the
+    quantized run stays close (reported error bounds, not exact)."""
+    n = 2048 + 77                       # ragged tail group
+    w = inputs.tiny(17)
+    x = inputs.host_step_inputs(w, n)
+    mc, mk, ms = orc.quantize_state(x["m0"], G, E4M3)
+    vc, vk, vs = orc.quantize_state(x["v0"], G, v_fmt)
+    th = x["theta"]
+    th64 = th.astype(np.float64)
+    m64 = orc.dequant(mc, mk, ms, G, E4M3).astype(np.float64)
+    v64 = orc.dequant(vc, vk, vs, G, v_fmt).astype(np.float64)
+    rng = np.random.default_rng(99)
+    for t in range(10, 13):
+        g32 = (rng.normal(0, 1e-3, n)).astype(np.float32)
+        gb = orc.to_bf16_array(g32)
+        g = np.array([orc.bf16_to_f32(int(b)) for b in gb], dtype=np.float64)
+        th, mc, mk, ms, vc, vk, vs = orc.adamw_fp8_step(th, gb, mc, mk, ms, vc, vk, vs, step=t,
+                                                         group_size=G, v_fmt=v_fmt, **H)
+        th64, m64, v64 = orc.adamw_fp64(th64, g, m64, v64, step=t, **H)
+    m_q = orc.dequant(mc, mk, ms, G, E4M3)
+    v_q = orc.dequant(vc, vk, vs, G, v_fmt)
+    rel = lambda a, b: float(np.linalg.norm(a - b) / np.linalg.norm(b))
+    assert rel(m_q, m64) < 0.06
+    assert rel(v_q, v64) < 0.12
+    assert rel(th, th64) < 1e-4
+    assert np.all(np.isfinite(th))
+

@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark of the fused COAT FP8-state AdamW step on B200.
+
+One step = one coat_adamw_fp8_step over the whole OLMo-7B-shaped parameter
+set (6,888,095,744 FP32 parameters, BF16 gradients, FP8 m/v with per-group
+k and scale, G = 128) resident in HBM.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--v-fmt e4m3|e5m2]
+  python bench.py --impl reference ...    # the CPU oracle on a bounded sample
+
+Multi-GPU (torchrun): every rank owns its own full parameter set (the step
+has no cross-rank exchange), so per-GPU work is fixed: weak scaling, value =
+parameters stepped by all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "params/s for fused FP8-state AdamW step (OLMo-7B set); % of B200 HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["quantized_optimizer_states_b200/csrc/step_kernels.cuh",
+                  "quantized_optimizer_states_b200/csrc/fp8_device.cuh"]
+
+
+def bytes_per_param(G: int) -> float:
+    """Algorithmic HBM bytes per parameter of one fused step: theta read +
+    write (8), BF16 gradient read (2), m and v codes read + write (4), and
+    per group (k, s) x 2 states x 4 B x (read + write) = 32 B over G."""
+    return 14.0 + 32.0 / G
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def recorded_traffic(n: int, G: int):
+    """DRAM bytes per launch from the committed ncu summary, scaled to n
+    parameters; None if the kernel source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "adamw_fp8_step_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except OSError:
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash() or rec.get("group_size") != G:
+        return None
+    return rec["dram_bytes_per_param"] * n
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.uuid = uuid
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.uuid:
+                cmd[1:1] = ["-i", self.uuid]
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[4:8]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def cpu_baseline(workload, G: int, sample: int, v_fmt: int):
+    """The oracle (single-threaded C) on the first `sample` parameters."""
+    import oracle
+    from quantized_optimizer_states_b200 import inputs
+    x = inputs.host_step_inputs(workload, sample)
+    st = oracle.quantize_state(x["m0"], G, 0) + oracle.quantize_state(x["v0"], G, v_fmt)
+    t0 = time.perf_counter()
+    oracle.adamw_fp8_step(x["theta"], x["grad"], *st, step=10, group_size=G, v_fmt=v_fmt,
+                          **inputs.HYPER)
+    dt = time.perf_counter() - t0
+    return {"value": sample / dt, "unit": "params/s", "cores": oracle.threads_used(),
+            "kind": "oracle",
+            "sample": f"first {sample} parameters of the {workload.name} set, one step"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed on bounded samples."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from quantized_optimizer_states_b200 import inputs
+    import oracle
+    v_fmt = 0 if args.v_fmt == "e4m3" else 1
+    w = inputs.olmo_7b(v_fmt=args.v_fmt)
+    G = w.group_size
+    sample = args.ref_sample
+    x = inputs.host_step_inputs(w, sample)
+    st = oracle.quantize_state(x["m0"], G, 0) + oracle.quantize_state(x["v0"], G, v_fmt)
+    th = x["theta"]
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        out = oracle.adamw_fp8_step(th, x["grad"], *st, step=10 + i, group_size=G, v_fmt=v_fmt,
+                                    **inputs.HYPER)
+        dt = time.perf_counter() - t0
+        th, st = out[0], out[1:7]
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = sample * len(times) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"olmo-7b set (bounded sample of {sample} parameters per step)",
+                   "group_size": G, "m_fmt": "e4m3", "v_fmt": args.v_fmt},
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": oracle.threads_used(),
+                         "kind": "oracle",
+                         "sample": f"first {sample} parameters of the olmo-7b set per step"},
+        "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="coat", choices=["coat", "reference"])
+    ap.add_argument("--v-fmt", default="e4m3", choices=["e4m3", "e5m2"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-sample", type=int, default=1 << 25)
+    ap.add_argument("--ref-sample", type=int, default=1 << 22)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="olmo-7b", choices=["olmo-7b", "olmo-1b", "sweep"])
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "coat":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import quantized_optimizer_states_b200 as coat
+    from quantized_optimizer_states_b200 import inputs
+    from quantized_optimizer_states_b200 import build as coat_build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    coat_build.build()
+    coat.load()
+
+    v_fmt = coat.COAT_E4M3 if args.v_fmt == "e4m3" else coat.COAT_E5M2
+    if args.workload == "olmo-7b":
+        w = inputs.olmo_7b(seed=1237 + rank, v_fmt=args.v_fmt)
+    elif args.workload == "olmo-1b":
+        w = inputs.olmo_1b(seed=1235 + rank)
+        w.v_fmt = args.v_fmt
+    else:
+        w = inputs.sweep(128, args.v_fmt, "late", seed=1238 + rank)
+    n, G = w.n, w.group_size
+    ng = -(-n // G)
+    hyper = dict(w.hyper)
+
+    # ---- inputs resident in HBM --------------------------------------------------
+    theta, grad, chunks = inputs.device_step_inputs(w, dev)
+    m_code = torch.empty(n, dtype=torch.uint8, device=dev)
+    v_code = torch.empty(n, dtype=torch.uint8, device=dev)
+    m_k = torch.empty(ng, dtype=torch.float32, device=dev)
+    m_s = torch.empty_like(m_k)
+    v_k = torch.empty_like(m_k)
+    v_s = torch.empty_like(m_k)
+    for off, m0, v0 in chunks():
+        c = m0.numel()
+        g0, g1 = off // G, -(-(off + c) // G)
+        coat.coat_quantize_state(m0, m_code[off:off + c], m_k[g0:g1], m_s[g0:g1], group_size=G,
+                                 fmt=coat.COAT_E4M3)
+        coat.coat_quantize_state(v0, v_code[off:off + c], v_k[g0:g1], v_s[g0:g1], group_size=G,
+                                 fmt=v_fmt)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream(dev)
+    step_no = [w.step]
+
+    def step():
+        coat.coat_adamw_fp8_step(theta, grad, m_code, m_k, m_s, v_code, v_k, v_s,
+                                 step=step_no[0], group_size=G, v_fmt=v_fmt, **hyper)
+        step_no[0] += 1
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    total_ms = evs[0].elapsed_time(evs[-1])
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * n * args.steps / (total_ms / 1e3)
+    kernel_ms = sum(per) / len(per)
+
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = bytes_per_param(G) * n / (kernel_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(n, G),
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6650 GB/s",
+                "algorithmic_bytes_per_param": bytes_per_param(G),
+                "frac_of_8TBs_spec": achieved / 8000.0}
+
+    # ---- end to end: gradients from pinned host memory each step ----------------
+    e2e = None
+    if args.e2e_steps > 0:
+        host_grad = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
+        host_grad.copy_(grad)
+        result = torch.empty(4, dtype=torch.float32, pin_memory=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+        def e2e_step():
+            grad.copy_(host_grad, non_blocking=True)
+            step()
+            result[0:1].copy_(m_k[-1:], non_blocking=True)
+            result[1:2].copy_(m_s[-1:], non_blocking=True)
+            result[2:3].copy_(v_k[-1:], non_blocking=True)
+            result[3:4].copy_(v_s[-1:], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * n * args.e2e_steps / (e2e_ms / 1e3), "unit": "params/s",
+               "h2d_bytes_per_step": 2 * n, "d2h_bytes_per_step": 16,
+               "what": "BF16 gradients copied from pinned host memory every step, then the "
+                       "step, then a 16-byte read-back of the last group's (k, s) pairs"}
+        del host_grad
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, G, args.cpu_sample, v_fmt)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{w.name} set: {n} FP32 params, BF16 grads, FP8 m (e4m3) / "
+                                   f"v ({args.v_fmt}) + per-group k, scale",
+                       "group_size": G, "m_fmt": "e4m3", "v_fmt": args.v_fmt,
+                       "params_per_gpu": n, "parallelism": f"{world} independent shards",
+                       "l2": f"no flush needed: {bytes_per_param(G) * n / 1e9:.1f} GB moved "
+                             "per step, far above the 126 MB L2"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "kernel_ms": kernel_ms,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

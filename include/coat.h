@@ -1,0 +1,216 @@
+/*
+ * coat.h -- C ABI of the B200 (sm_100a) COAT library, libcoat.so.
+ *
+ * COAT compresses AdamW's optimizer states and the saved activations of a
+ * transformer to FP8.  This library implements the data-parallel hot path:
+ * one fused AdamW step over FP8 first and second moments with COAT's
+ * dynamic-range expansion, plus COAT's two activation quantizers.
+ *
+ * Sources, by page title and section:
+ *   [COAT]  "COAT: 压缩优化器状态和激活以实现内存高效的 FP8 训练"
+ *           (blog.daoxuan.cc/posts/57954).  Sections used:
+ *           "为什么二阶动量对量化比一阶动量更敏感" -- the AdamW rule and its
+ *             hyper-parameters beta1, beta2, eta, eps, lambda;
+ *           "二阶动量的动态范围反而更小" -- E4M3 range 448 / 2^-9;
+ *           "扩展函数：把窄分布拉宽" -- f(x) = sign(x)|x|^k applied before
+ *             quantization, k = log(R_E4M3) / log(R_X) recomputed for every
+ *             group at every step, dequantization by the 1/k power, and the
+ *             E4M3+E4M3 / E4M3+E5M2 format pairs;
+ *           "混合粒度：线性层和非线性层分开处理" -- 1xG group quantization
+ *             along channels for nonlinear-layer inputs, and Group Scaling
+ *             (max per 1xG run, then max of that small intermediate) for the
+ *             per-tensor scale of linear-layer inputs;
+ *           "结果和边界" -- k follows the target format's range.
+ *   [ATLAS] "LLM Atlas / systems / numerics" (llm-atlas.k1412.top),
+ *           section 03 "FP8" (E4M3 max 448, min subnormal 2^-9; E5M2 max
+ *           57344, min subnormal 2^-16) and section 08 "Adam -> AdamW"
+ *           (m_t, v_t, the bias-corrected update with eps outside the root,
+ *           theta <- (1 - eta*lambda) theta + delta).
+ *
+ * Common conventions
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless
+ *     stated otherwise.  The library allocates no memory on any call.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call is asynchronous on that stream; the return value reports only
+ *     the host-side argument checks and the launch itself.
+ *   - Buffers that the kernels access with 16-byte vector instructions
+ *     (parameters, gradients, codes, activations) must start on a 16-byte
+ *     boundary, otherwise COAT_ERR_MISALIGNED is returned and nothing runs.
+ *     Per-group metadata arrays need only natural (4-byte) alignment.
+ *   - Group size G: a power of two, 16 <= G <= 4096
+ *     (COAT_ERR_UNSUPPORTED otherwise).
+ *   - Sizes are element counts.  n == 0 is valid and launches nothing.
+ *   - Errors never leave partial work behind: argument errors are found
+ *     before any launch.  COAT_ERR_CUDA means a launch failed; call
+ *     coat_last_cuda_error() for the CUDA error code.
+ *   - FP8 encoding is round-to-nearest-even with saturation to +-max
+ *     (hardware cvt ... satfinite); NaN encodes as 0x7F.
+ */
+#ifndef COAT_H
+#define COAT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum coat_status {
+    COAT_OK = 0,
+    COAT_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad hyper-parameter */
+    COAT_ERR_MISALIGNED = 2,  /* a vector-accessed buffer is not 16-byte aligned */
+    COAT_ERR_UNSUPPORTED = 3, /* format / group size / flag combination not built */
+    COAT_ERR_CUDA = 4,        /* a CUDA launch or query failed */
+    COAT_ERR_NONFINITE = 5,   /* reserved: non-finite gradient detection */
+    COAT_ERR_TIMEOUT = 6      /* reserved: a bounded device wait ran out */
+} coat_status_t;
+
+typedef enum coat_fp8 {
+    COAT_E4M3 = 0, /* 1 sign, 4 exponent (bias 7), 3 mantissa; max 448, no inf */
+    COAT_E5M2 = 1  /* 1 sign, 5 exponent (bias 15), 2 mantissa; max 57344 */
+} coat_fp8_t;
+
+/* cfg.flags */
+#define COAT_FORCE_K1 0x1 /* ablation: k = 1 for every group (no expansion) */
+
+/* Hyper-parameters and layout of one COAT AdamW step ([COAT] AdamW
+ * section; [ATLAS] section 08). */
+typedef struct coat_adamw_cfg {
+    float beta1;        /* first-moment decay, 0 <= beta1 < 1 */
+    float beta2;        /* second-moment decay, 0 <= beta2 < 1 */
+    float lr;           /* eta */
+    float eps;          /* added to sqrt(v_hat) */
+    float weight_decay; /* lambda; the decay applied is (1 - eta*lambda) */
+    int64_t step;       /* t >= 1, already incremented for this step */
+    int32_t group_size; /* G, power of two in [16, 4096] */
+    int32_t m_fmt;      /* COAT_E4M3 (the only first-moment format COAT uses) */
+    int32_t v_fmt;      /* COAT_E4M3 or COAT_E5M2 */
+    int32_t k_range;    /* 0: k targets the E4M3 range for both states;
+                           1: k targets the storage format's own range */
+    float k_max;        /* upper clamp for k (0 = none); 64 recommended */
+    int32_t flags;      /* COAT_FORCE_K1 or 0 */
+} coat_adamw_cfg_t;
+
+/*
+ * coat_adamw_fp8_step -- one fused COAT AdamW step, in place.
+ * [COAT] sections on AdamW and on the expansion function; [ATLAS] 08.
+ *
+ * Layout: n parameters in one flat buffer; groups are the runs
+ * [i*G, (i+1)*G) of that buffer (the last may be shorter);
+ * ngroups = ceil(n / G).
+ *   param    float32[n]   FP32 master weights theta (read, written)
+ *   grad     uint16[n]    BF16 gradient bit patterns (read)
+ *   m_code   uint8[n]     first moment, FP8 codes in m_fmt (read, written)
+ *   m_k      float32[ngroups]  per-group expansion exponent k of m
+ *   m_scale  float32[ngroups]  per-group scale s of m
+ *   v_code, v_k, v_scale  the same for the second moment in v_fmt
+ * Stored state per group: x = sign(d) * |d|^(1/k) * s for decoded FP8 d
+ * (an all-zero group stores k = 1, s = 0).
+ *
+ * Per element: g = float(grad); m, v = dequantized states;
+ *   m_t = beta1*m + (1-beta1)*g;  v_t = beta2*v + (1-beta2)*g*g;
+ *   theta = (1 - lr*wd)*theta - lr * (m_t/(1-beta1^t)) / (sqrt(v_t/(1-beta2^t)) + eps).
+ * Per group, for each of m_t and v_t: M = max|x|, mn = min nonzero |x|,
+ *   k = log(R)/log(M/mn) with R = 448/2^-9 (k_range 0) or the storage
+ *   format's max/min-subnormal (k_range 1), clamped to k_max, k = 1 when
+ *   M == mn; s = M * fmt_max^(-1/k); code = sign(x) . RNE(fmt_max * (|x|/M)^k).
+ * Alignment: param, grad, m_code, v_code 16-byte aligned.
+ * Errors: INVALID_ARG (null pointer, n < 0, step < 1, betas outside [0,1),
+ * k_max < 0), UNSUPPORTED (G, formats, flags), MISALIGNED, CUDA.
+ * Buffers must not overlap.  Results are bit-reproducible run to run.
+ */
+coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m_code,
+                                  float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
+                                  float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
+                                  void *stream);
+
+/*
+ * coat_quantize_state -- compress an FP32 optimizer state into COAT's FP8
+ * form (the re-quantization half of the step, on its own): used to
+ * initialize or convert states.  [COAT] "扩展函数".
+ *   x      float32[n]        input (16-byte aligned)
+ *   code   uint8[n]          output codes in `fmt` (16-byte aligned)
+ *   k, scale float32[ceil(n/G)]  outputs
+ * k_range, k_max, flags as in coat_adamw_cfg_t.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA.
+ */
+coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size, int32_t fmt,
+                                  int32_t k_range, float k_max, int32_t flags, uint8_t *code,
+                                  float *k, float *scale, void *stream);
+
+/*
+ * coat_dequant -- decode FP8 codes to FP32 or BF16.
+ * [COAT] "扩展函数" (inverse by the 1/k power) and "混合粒度" (activation
+ * scales).
+ *   q      uint8[n] codes in `fmt` (16-byte aligned)
+ *   k      float32[ceil(n/G)] per-group exponents, or NULL for k = 1
+ *          (activations: x = decode(q) * s exactly)
+ *   scale  float32[ceil(n/G)] per-group scales; G = n (or any G >= n)
+ *          with a single scale gives per-tensor dequantization
+ *   out    float32[n] (out_bf16 == 0) or BF16 bits uint16[n] (out_bf16 != 0,
+ *          nearest-even rounding of the FP32 value), 16-byte aligned
+ * Here G may be any positive count (it only maps element -> scale index).
+ * Errors: INVALID_ARG, UNSUPPORTED (fmt), MISALIGNED, CUDA.
+ */
+coat_status_t coat_dequant(const uint8_t *q, const float *k, const float *scale, int64_t n,
+                           int64_t group_size, int32_t fmt, int32_t out_bf16, void *out,
+                           void *stream);
+
+/*
+ * coat_group_quant_1xG -- COAT's 1xG group quantization of a nonlinear-layer
+ * input.  [COAT] "混合粒度": groups of G consecutive channels of one token.
+ *   x      BF16 bits, row-major [rows, cols] with row stride ld >= cols
+ *          (16-byte aligned; ld a multiple of 8)
+ *   q      uint8 [rows, cols], row stride cols (16-byte aligned)
+ *   scale  float32 [rows, cols/G], s = amax/fmt_max per group
+ * Codes: RNE_satfinite(x * (fmt_max/amax)), the product rounded to FP32
+ * first; a group with amax <= 2^-100 (e.g. all zero) uses s = 1.
+ * Requires cols % G == 0.  Bit-exact by construction.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA.
+ */
+coat_status_t coat_group_quant_1xG(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                   int32_t group_size, int32_t fmt, uint8_t *q, float *scale,
+                                   void *stream);
+
+/* Bytes of workspace coat_group_scaling_quant_pertensor needs for n values
+ * in groups of G: (ceil(n/G) + 1) float32 slots.  Host function, no GPU. */
+int64_t coat_group_scaling_workspace_bytes(int64_t n, int32_t group_size);
+
+/*
+ * coat_group_scaling_quant_pertensor -- COAT's "Group Scaling" per-tensor
+ * FP8 quantization of a linear-layer input.  [COAT] "混合粒度": (i) the max
+ * of each 1xG run goes to a small intermediate; (ii) the max of that
+ * intermediate is the tensor's amax; (iii) one cast with s = amax/fmt_max.
+ *   x          BF16 bits [n] (16-byte aligned)
+ *   workspace  float32[ceil(n/G) + 1] (4-byte aligned).  Slots
+ *              [0, ceil(n/G)) hold the per-group maxima: written by step (i)
+ *              when amax_precomputed == 0, or filled beforehand by the
+ *              producing kernel when amax_precomputed != 0 (step (i) is then
+ *              skipped).  The last slot is scratch for step (ii).
+ *   q          uint8[n] codes (16-byte aligned)
+ *   scale      float32[1], the per-tensor scale s (amax <= 2^-100 gives 1)
+ * Bit-exact: amax is an exact max and s, the reciprocal and the product
+ * are single IEEE operations.  Calls on the same workspace must not
+ * overlap on the GPU.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA.
+ */
+coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
+                                                 int32_t group_size, int32_t fmt,
+                                                 float *workspace, int32_t amax_precomputed,
+                                                 uint8_t *q, float *scale, void *stream);
+
+/* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
+ * this thread (0 if none). */
+int32_t coat_last_cuda_error(void);
+
+/* A static, human-readable name for a status code. */
+const char *coat_status_string(coat_status_t status);
+
+/* Library version as (major << 16) | (minor << 8) | patch. */
+int32_t coat_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COAT_H */

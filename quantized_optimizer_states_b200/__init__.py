@@ -1,0 +1,24 @@
+"""COAT FP8 optimizer-state step and activation quantizers for B200 (sm_100a).
+
+The compute lives in libcoat.so (hand-written CUDA, C ABI in include/coat.h);
+this package is its thin ctypes binding plus helpers for sharding and
+synthetic inputs.  The library is loaded on first use and a missing library
+raises -- there is no CPU path.
+"""
+from ._lib import (  # noqa: F401
+    COAT_E4M3,
+    COAT_E5M2,
+    COAT_FORCE_K1,
+    CoatError,
+    coat_adamw_fp8_step,
+    coat_dequant,
+    coat_group_quant_1xG,
+    coat_group_scaling_quant_pertensor,
+    coat_group_scaling_workspace_bytes,
+    coat_quantize_state,
+    coat_status_string,
+    coat_version,
+    load,
+)
+
+__version__ = "0.1.0"

@@ -1,0 +1,203 @@
+"""ctypes binding of libcoat.so (declared in include/coat.h).
+
+Argument marshalling only: torch tensors are passed as device pointers and
+the current CUDA stream as the stream handle; every step of the computation
+runs in the library's kernels.  If the library is missing or cannot be
+loaded the functions raise -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libcoat.so")
+
+COAT_E4M3 = 0
+COAT_E5M2 = 1
+COAT_FORCE_K1 = 0x1
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "misaligned", 3: "unsupported", 4: "CUDA error",
+          5: "non-finite", 6: "timeout"}
+
+
+class CoatError(RuntimeError):
+    def __init__(self, fn: str, status: int, cuda_err: int = 0):
+        msg = f"{fn} failed: {STATUS.get(status, status)} (status {status})"
+        if status == 4:
+            msg += f", cudaError {cuda_err}"
+        super().__init__(msg)
+        self.status = status
+
+
+class CoatAdamwCfg(ctypes.Structure):
+    """Mirror of coat_adamw_cfg_t."""
+    _fields_ = [
+        ("beta1", ctypes.c_float),
+        ("beta2", ctypes.c_float),
+        ("lr", ctypes.c_float),
+        ("eps", ctypes.c_float),
+        ("weight_decay", ctypes.c_float),
+        ("step", ctypes.c_int64),
+        ("group_size", ctypes.c_int32),
+        ("m_fmt", ctypes.c_int32),
+        ("v_fmt", ctypes.c_int32),
+        ("k_range", ctypes.c_int32),
+        ("k_max", ctypes.c_float),
+        ("flags", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+# name -> (restype, argtypes)
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_F = ctypes.c_float
+SIGNATURES = {
+    "coat_adamw_fp8_step": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
+                                   ctypes.POINTER(CoatAdamwCfg), _P]),
+    "coat_quantize_state": (_I32, [_P, _I64, _I32, _I32, _I32, _F, _I32, _P, _P, _P, _P]),
+    "coat_dequant": (_I32, [_P, _P, _P, _I64, _I64, _I32, _I32, _P, _P]),
+    "coat_group_quant_1xG": (_I32, [_P, _I64, _I64, _I64, _I32, _I32, _P, _P, _P]),
+    "coat_group_scaling_workspace_bytes": (_I64, [_I64, _I32]),
+    "coat_group_scaling_quant_pertensor": (_I32, [_P, _I64, _I32, _I32, _P, _I32, _P, _P, _P]),
+    "coat_last_cuda_error": (_I32, []),
+    "coat_status_string": (ctypes.c_char_p, [_I32]),
+    "coat_version": (_I32, []),
+}
+
+
+def load(path: str = LIB_PATH):
+    """Load libcoat.so once; raise if it is not there."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"libcoat.so not found at {path}: build it with "
+                "`python -m quantized_optimizer_states_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(name: str, status: int):
+    if status != 0:
+        raise CoatError(name, status, load().coat_last_cuda_error())
+
+
+def _stream(stream):
+    if stream is not None:
+        return ctypes.c_void_p(int(stream))
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t, dtype=None, what="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _u16(t, what):
+    """BF16 or int16/uint16 tensors are all passed as their bit patterns."""
+    import torch
+    if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise ValueError(f"{what} must hold BF16 bit patterns, got {t.dtype}")
+    return _ptr(t, None, what)
+
+
+def coat_adamw_fp8_step(param, grad, m_code, m_k, m_scale, v_code, v_k, v_scale, *, beta1: float,
+                        beta2: float, lr: float, eps: float, weight_decay: float, step: int,
+                        group_size: int = 128, m_fmt: int = COAT_E4M3, v_fmt: int = COAT_E4M3,
+                        k_range: int = 0, k_max: float = 64.0, flags: int = 0, stream=None):
+    """One fused COAT AdamW step, in place (see include/coat.h)."""
+    import torch
+    cfg = CoatAdamwCfg(beta1, beta2, lr, eps, weight_decay, step, group_size, m_fmt, v_fmt,
+                       k_range, k_max, flags)
+    st = load().coat_adamw_fp8_step(
+        _ptr(param, torch.float32, "param"), _u16(grad, "grad"),
+        _ptr(m_code, torch.uint8, "m_code"), _ptr(m_k, torch.float32, "m_k"),
+        _ptr(m_scale, torch.float32, "m_scale"), _ptr(v_code, torch.uint8, "v_code"),
+        _ptr(v_k, torch.float32, "v_k"), _ptr(v_scale, torch.float32, "v_scale"),
+        param.numel(), ctypes.byref(cfg), _stream(stream))
+    _check("coat_adamw_fp8_step", st)
+
+
+def coat_quantize_state(x, code, k, scale, *, group_size: int = 128, fmt: int = COAT_E4M3,
+                        k_range: int = 0, k_max: float = 64.0, flags: int = 0, stream=None):
+    import torch
+    st = load().coat_quantize_state(
+        _ptr(x, torch.float32, "x"), x.numel(), group_size, fmt, k_range, k_max, flags,
+        _ptr(code, torch.uint8, "code"), _ptr(k, torch.float32, "k"),
+        _ptr(scale, torch.float32, "scale"), _stream(stream))
+    _check("coat_quantize_state", st)
+
+
+def coat_dequant(q, k, scale, out, *, group_size: int, fmt: int = COAT_E4M3, stream=None):
+    """out: float32 tensor (FP32 output) or bfloat16 tensor (BF16 output)."""
+    import torch
+    out_bf16 = out.dtype == torch.bfloat16
+    if not out_bf16 and out.dtype != torch.float32:
+        raise ValueError("out must be float32 or bfloat16")
+    st = load().coat_dequant(
+        _ptr(q, torch.uint8, "q"), _ptr(k, torch.float32, "k") if k is not None else None,
+        _ptr(scale, torch.float32, "scale"), q.numel(), group_size, fmt, int(out_bf16),
+        _ptr(out, None, "out"), _stream(stream))
+    _check("coat_dequant", st)
+
+
+def coat_group_quant_1xG(x, q, scale, *, group_size: int = 128, fmt: int = COAT_E4M3,
+                         stream=None):
+    """x: [rows, cols] BF16 (row stride x.stride(0)), q: uint8 [rows, cols],
+    scale: float32 [rows, cols // group_size]."""
+    import torch
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    rows, cols = x.shape
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise ValueError("x must hold BF16 bit patterns")
+    st = load().coat_group_quant_1xG(
+        ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), group_size, fmt,
+        _ptr(q, torch.uint8, "q"), _ptr(scale, torch.float32, "scale"), _stream(stream))
+    _check("coat_group_quant_1xG", st)
+
+
+def coat_group_scaling_workspace_bytes(n: int, group_size: int) -> int:
+    return int(load().coat_group_scaling_workspace_bytes(n, group_size))
+
+
+def coat_group_scaling_quant_pertensor(x, workspace, q, scale, *, group_size: int = 128,
+                                       fmt: int = COAT_E4M3, amax_precomputed: bool = False,
+                                       stream=None):
+    """x: BF16 [n]; workspace: float32 [ceil(n/G) + 1]; q: uint8 [n]; scale: float32 [1]."""
+    import torch
+    need = coat_group_scaling_workspace_bytes(x.numel(), group_size)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    st = load().coat_group_scaling_quant_pertensor(
+        _u16(x, "x"), x.numel(), group_size, fmt, _ptr(workspace, torch.float32, "workspace"),
+        int(bool(amax_precomputed)), _ptr(q, torch.uint8, "q"),
+        _ptr(scale, torch.float32, "scale"), _stream(stream))
+    _check("coat_group_scaling_quant_pertensor", st)
+
+
+def coat_version() -> int:
+    return int(load().coat_version())
+
+
+def coat_status_string(status: int) -> str:
+    return load().coat_status_string(status).decode()

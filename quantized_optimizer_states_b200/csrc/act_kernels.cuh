@@ -1,0 +1,260 @@
+// COAT activation quantizers and FP8 dequantization.
+//
+// COAT summary page (blog.daoxuan.cc/posts/57954), section
+// "混合粒度：线性层和非线性层分开处理":
+//   - nonlinear-layer inputs: 1xG group quantization along the channel axis
+//     of each token (not BxB tiles);
+//   - linear-layer inputs: one scale per tensor, found by "Group Scaling":
+//     (i) the max of every 1xG run, cached in a small intermediate (which
+//     the producing kernel can emit), (ii) the max of that G-times-smaller
+//     intermediate, (iii) the cast.
+// Scale convention: s = amax / fmt_max; codes = RNE_satfinite(x * (fmt_max /
+// amax)) with the product rounded to binary32 first, so GPU and CPU agree
+// bit for bit.  amax <= 2^-100 (e.g. an all-zero group) uses s = 1.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp8_device.cuh"
+#include "step_kernels.cuh"
+
+namespace coat {
+
+__device__ __forceinline__ void act_scale(float amax, float fmax, float &s, float &inv) {
+  if (amax > 0x1p-100f) {
+    s = __fdiv_rn(amax, fmax);
+    inv = __fdiv_rn(fmax, amax);
+  } else {
+    s = 1.0f;
+    inv = 1.0f;
+  }
+}
+
+// 16 BF16 values (eight words) -> 16 floats.
+__device__ __forceinline__ void unpack16_bf16(const uint32_t *w, float *x) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[2 * i] = bf16lo_to_float(w[i]);
+    x[2 * i + 1] = bf16hi_to_float(w[i]);
+  }
+}
+
+__device__ __forceinline__ float amax16(const float *x) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
+  return a;
+}
+
+// Max over the threads of one group (lanes = G/16).
+__device__ __forceinline__ float group_max(float a, int lanes, float *red) {
+  const int lim = lanes < 32 ? lanes : 32;
+  for (int off = 1; off < lim; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+  if (lanes > 32) {
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[warp] = a;
+    __syncthreads();
+    const int wpg = lanes >> 5;
+    const int w0 = (warp / wpg) * wpg;
+    a = red[w0];
+    for (int i = 1; i < wpg; ++i) a = fmaxf(a, red[w0 + i]);
+  }
+  return a;
+}
+
+template <int F>
+__device__ __forceinline__ void cast16(const float *x, float inv, uint32_t *out) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+    out[w] = float4_to_fp8x4<F>(__fmul_rn(x[4 * w], inv), __fmul_rn(x[4 * w + 1], inv),
+                                __fmul_rn(x[4 * w + 2], inv), __fmul_rn(x[4 * w + 3], inv));
+}
+
+// ---- 1xG group quantization ---------------------------------------------------
+
+struct GroupQuantParams {
+  const uint16_t *x;
+  int64_t rows, cols, ld;
+  int64_t vec_per_row;  // cols / 16
+  int log2G;
+  uint8_t *q;
+  float *scale;
+};
+
+template <int F>
+__global__ void __launch_bounds__(kThreads) group_quant_1xG_kernel(const GroupQuantParams p) {
+  __shared__ float red[kWarps];
+  const int64_t vid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+  const bool active = vid < p.rows * p.vec_per_row;
+  const int64_t row = active ? vid / p.vec_per_row : 0;
+  const int64_t c0 = (vid - row * p.vec_per_row) * kVec;
+  const int lanes = 1 << (p.log2G - 4);
+  uint32_t w[8];
+  float x[16];
+  if (active) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.ld + c0);
+    uint4 a = src[0], b = src[1];
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = 0;
+  }
+  unpack16_bf16(w, x);
+  const float amax = group_max(amax16(x), lanes, red);
+  float s, inv;
+  act_scale(amax, fmt_max<F>(), s, inv);
+  uint32_t o[4];
+  cast16<F>(x, inv, o);
+  if (active) {
+    *reinterpret_cast<uint4 *>(p.q + row * p.cols + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+    if ((threadIdx.x & (lanes - 1)) == 0)
+      p.scale[row * (p.cols >> p.log2G) + (c0 >> p.log2G)] = s;
+  }
+}
+
+// ---- Group Scaling per-tensor quantization -------------------------------------
+
+struct GroupScalingParams {
+  const uint16_t *x;
+  int64_t n;
+  int64_t ngroups;
+  int log2G;
+  float *group_amax;     // [ngroups]
+  uint32_t *tensor_amax; // bits of the running max (non-negative floats order as integers)
+  uint8_t *q;
+  float *scale;
+};
+
+// Step (i) (+ the block's share of step (ii)): per-group maxima of the BF16
+// input into group_amax, and the block maximum folded into tensor_amax.
+__global__ void __launch_bounds__(kThreads) group_amax_kernel(const GroupScalingParams p) {
+  __shared__ float red[kWarps];
+  __shared__ float blockred[kWarps];
+  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+  const bool active = e0 < p.n;
+  const int lanes = 1 << (p.log2G - 4);
+  uint32_t w[8];
+  float x[16];
+  if (active) {
+    load16_bf16(p.x, e0, p.n, w);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = 0;
+  }
+  unpack16_bf16(w, x);
+  const float gmax = group_max(amax16(x), lanes, red);
+  if (active && (threadIdx.x & (lanes - 1)) == 0) p.group_amax[e0 >> p.log2G] = gmax;
+  // block max of the group maxima
+  float b = gmax;
+  for (int off = 16; off > 0; off >>= 1) b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, off));
+  if ((threadIdx.x & 31) == 0) blockred[threadIdx.x >> 5] = b;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = blockred[0];
+    for (int i = 1; i < kWarps; ++i) m = fmaxf(m, blockred[i]);
+    atomicMax(p.tensor_amax, __float_as_uint(m));
+  }
+}
+
+// Step (ii) alone, when the producer already wrote group_amax: a grid-wide
+// max of the intermediate into tensor_amax.
+__global__ void __launch_bounds__(kThreads) amax_of_groups_kernel(const GroupScalingParams p) {
+  __shared__ float blockred[kWarps];
+  float m = 0.0f;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < p.ngroups;
+       i += static_cast<int64_t>(gridDim.x) * kThreads)
+    m = fmaxf(m, p.group_amax[i]);
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) blockred[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = blockred[0];
+    for (int i = 1; i < kWarps; ++i) r = fmaxf(r, blockred[i]);
+    atomicMax(p.tensor_amax, __float_as_uint(r));
+  }
+}
+
+// Step (iii): the per-tensor cast.
+template <int F>
+__global__ void __launch_bounds__(kThreads) pertensor_cast_kernel(const GroupScalingParams p) {
+  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+  const float amax = __uint_as_float(*p.tensor_amax);
+  float s, inv;
+  act_scale(amax, fmt_max<F>(), s, inv);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.scale = s;
+  if (e0 >= p.n) return;
+  uint32_t w[8];
+  float x[16];
+  load16_bf16(p.x, e0, p.n, w);
+  unpack16_bf16(w, x);
+  uint32_t o[4];
+  cast16<F>(x, inv, o);
+  store16_u8(p.q, e0, p.n, o);
+}
+
+// ---- dequantization ----------------------------------------------------------------
+
+struct DequantParams {
+  const uint8_t *q;
+  const float *k;  // nullable
+  const float *scale;
+  int64_t n;
+  int log2G;       // -1: one scale for the whole tensor
+  int out_bf16;
+  void *out;
+  float log2_tab[8];
+};
+
+__device__ __forceinline__ uint32_t float_to_bf16_rn(float f) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+template <int F>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p) {
+  __shared__ float tab8[8];
+  if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
+  __syncthreads();
+  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+  if (e0 >= p.n) return;
+  const int64_t grp = p.log2G < 0 ? 0 : (e0 >> p.log2G);
+  const float s = p.scale[grp];
+  const float kk = p.k ? p.k[grp] : 1.0f;
+  const bool k1 = kk == 1.0f;
+  const float rk = __frcp_rn(kk);
+  uint32_t w[4];
+  load16_u8(p.q, e0, p.n, w);
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float d[4];
+    fp8x4_to_float<F>(w[i], d);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (p.k)
+        x[4 * i + j] = dequant_one(d[j], s, rk, k1, tab8);
+      else
+        x[4 * i + j] = __fmul_rn(d[j], s);
+    }
+  }
+  if (p.out_bf16) {
+    uint16_t *o = static_cast<uint16_t *>(p.out);
+    if (e0 + 16 <= p.n) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        pk[i] = float_to_bf16_rn(x[2 * i]) | (float_to_bf16_rn(x[2 * i + 1]) << 16);
+      uint4 *dst = reinterpret_cast<uint4 *>(o + e0);
+      dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    } else {
+      for (int i = 0; i < 16; ++i)
+        if (e0 + i < p.n) o[e0 + i] = static_cast<uint16_t>(float_to_bf16_rn(x[i]));
+    }
+  } else {
+    store16_f32(static_cast<float *>(p.out), e0, p.n, x);
+  }
+}
+
+}  // namespace coat

@@ -1,0 +1,287 @@
+// C ABI of libcoat.so: argument checks, the per-call scalar set-up, and the
+// kernel launches.  Declarations and the contract of every entry point are
+// in include/coat.h.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "coat.h"
+
+#include "act_kernels.cuh"
+#include "fp8_device.cuh"
+#include "step_kernels.cuh"
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+coat_status_t launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_last_cuda_error = static_cast<int32_t>(e);
+    return COAT_ERR_CUDA;
+  }
+  return COAT_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_fmt(int32_t f) { return f == COAT_E4M3 || f == COAT_E5M2; }
+
+// log2(G) for a supported group size, else -1.
+int group_log2(int64_t G) {
+  if (G < 16 || G > 4096 || (G & (G - 1)) != 0) return -1;
+  int l = 0;
+  while ((int64_t{1} << l) < G) ++l;
+  return l;
+}
+
+double fmt_max_host(int32_t f) { return f == COAT_E4M3 ? 448.0 : 57344.0; }
+
+double fmt_min_subnormal_host(int32_t f) {
+  return f == COAT_E4M3 ? std::ldexp(1.0, -9) : std::ldexp(1.0, -16);
+}
+
+// The range that k fills: E4M3's for both states (k_range 0), or the
+// storage format's own (k_range 1).
+coat::StateFmtParams state_fmt_params(int32_t store_fmt, int32_t k_range) {
+  const int32_t rf = k_range == 1 ? store_fmt : COAT_E4M3;
+  coat::StateFmtParams f;
+  f.ln_range = std::log(fmt_max_host(rf) / fmt_min_subnormal_host(rf));
+  f.fmax = static_cast<float>(fmt_max_host(store_fmt));
+  f.log2_fmax = static_cast<float>(std::log2(fmt_max_host(store_fmt)));
+  return f;
+}
+
+void fill_log2_table(float *tab) {
+  for (int i = 0; i < 8; ++i) tab[i] = static_cast<float>(std::log2(1.0 + i / 8.0));
+}
+
+unsigned int blocks_for(int64_t elems) {
+  return static_cast<unsigned int>((elems + coat::kElemsPerBlock - 1) / coat::kElemsPerBlock);
+}
+
+constexpr int64_t kMaxElems = int64_t{1} << 44;  // grid-size bound (2^31 blocks x 4096)
+
+}  // namespace
+
+extern "C" {
+
+coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m_code,
+                                  float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
+                                  float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
+                                  void *stream) {
+  if (!cfg || n < 0) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && (!param || !grad || !m_code || !m_k || !m_scale || !v_code || !v_k || !v_scale))
+    return COAT_ERR_INVALID_ARG;
+  if (cfg->step < 1 || !(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) ||
+      !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f) || !(cfg->k_max >= 0.0f) ||
+      !std::isfinite(cfg->lr) || !std::isfinite(cfg->eps) || !std::isfinite(cfg->weight_decay))
+    return COAT_ERR_INVALID_ARG;
+  const int lg = group_log2(cfg->group_size);
+  if (lg < 0 || cfg->m_fmt != COAT_E4M3 || !valid_fmt(cfg->v_fmt) ||
+      (cfg->k_range != 0 && cfg->k_range != 1) || (cfg->flags & ~COAT_FORCE_K1) != 0)
+    return COAT_ERR_UNSUPPORTED;
+  if (n > kMaxElems) return COAT_ERR_UNSUPPORTED;
+  if (n == 0) return COAT_OK;
+  if (!aligned16(param) || !aligned16(grad) || !aligned16(m_code) || !aligned16(v_code))
+    return COAT_ERR_MISALIGNED;
+
+  coat::StepParams p;
+  p.theta = param;
+  p.grad = grad;
+  p.m_code = m_code;
+  p.m_k = m_k;
+  p.m_s = m_scale;
+  p.v_code = v_code;
+  p.v_k = v_k;
+  p.v_s = v_scale;
+  p.n = n;
+  p.log2G = lg;
+  p.beta1 = cfg->beta1;
+  p.beta2 = cfg->beta2;
+  // scalar factors of the rule, each rounded to binary32 once
+  p.c1 = 1.0f - cfg->beta1;
+  p.c2 = 1.0f - cfg->beta2;
+  p.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(cfg->beta1),
+                                            static_cast<double>(cfg->step)));
+  p.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(cfg->beta2),
+                                            static_cast<double>(cfg->step)));
+  {
+    volatile float lr_wd = cfg->lr * cfg->weight_decay;  // keep the product rounded alone
+    p.decay = 1.0f - lr_wd;
+  }
+  p.lr = cfg->lr;
+  p.eps = cfg->eps;
+  p.k_max = cfg->k_max;
+  p.force_k1 = (cfg->flags & COAT_FORCE_K1) ? 1 : 0;
+  p.m = state_fmt_params(COAT_E4M3, cfg->k_range);
+  p.v = state_fmt_params(cfg->v_fmt, cfg->k_range);
+  fill_log2_table(p.log2_tab);
+  if (!(p.bc1 > 0.0f) || !(p.bc2 > 0.0f)) return COAT_ERR_INVALID_ARG;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned int grid = blocks_for(n);
+  if (cfg->v_fmt == COAT_E4M3)
+    coat::adamw_fp8_step_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+  else
+    coat::adamw_fp8_step_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  return launch_status();
+}
+
+coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size, int32_t fmt,
+                                  int32_t k_range, float k_max, int32_t flags, uint8_t *code,
+                                  float *k, float *scale, void *stream) {
+  if (n < 0 || !(k_max >= 0.0f)) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && (!x || !code || !k || !scale)) return COAT_ERR_INVALID_ARG;
+  const int lg = group_log2(group_size);
+  if (lg < 0 || !valid_fmt(fmt) || (k_range != 0 && k_range != 1) ||
+      (flags & ~COAT_FORCE_K1) != 0 || n > kMaxElems)
+    return COAT_ERR_UNSUPPORTED;
+  if (n == 0) return COAT_OK;
+  if (!aligned16(x) || !aligned16(code)) return COAT_ERR_MISALIGNED;
+  coat::QuantParams p;
+  p.x = x;
+  p.code = code;
+  p.k = k;
+  p.s = scale;
+  p.n = n;
+  p.log2G = lg;
+  p.k_max = k_max;
+  p.force_k1 = (flags & COAT_FORCE_K1) ? 1 : 0;
+  p.f = state_fmt_params(fmt, k_range);
+  fill_log2_table(p.log2_tab);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned int grid = blocks_for(n);
+  if (fmt == COAT_E4M3)
+    coat::quantize_state_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+  else
+    coat::quantize_state_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  return launch_status();
+}
+
+coat_status_t coat_dequant(const uint8_t *q, const float *k, const float *scale, int64_t n,
+                           int64_t group_size, int32_t fmt, int32_t out_bf16, void *out,
+                           void *stream) {
+  if (n < 0 || group_size < 1) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && (!q || !scale || !out)) return COAT_ERR_INVALID_ARG;
+  if (!valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
+  int lg = -1;
+  if (group_size < n) {
+    lg = group_log2(group_size);
+    if (lg < 0) return COAT_ERR_UNSUPPORTED;
+  }
+  if (n == 0) return COAT_OK;
+  if (!aligned16(q) || !aligned16(out)) return COAT_ERR_MISALIGNED;
+  coat::DequantParams p;
+  p.q = q;
+  p.k = k;
+  p.scale = scale;
+  p.n = n;
+  p.log2G = lg;
+  p.out_bf16 = out_bf16 ? 1 : 0;
+  p.out = out;
+  fill_log2_table(p.log2_tab);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned int grid = blocks_for(n);
+  if (fmt == COAT_E4M3)
+    coat::dequant_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+  else
+    coat::dequant_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  return launch_status();
+}
+
+coat_status_t coat_group_quant_1xG(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                   int32_t group_size, int32_t fmt, uint8_t *q, float *scale,
+                                   void *stream) {
+  if (rows < 0 || cols < 0 || ld < cols) return COAT_ERR_INVALID_ARG;
+  if (rows > 0 && cols > 0 && (!x || !q || !scale)) return COAT_ERR_INVALID_ARG;
+  const int lg = group_log2(group_size);
+  if (lg < 0 || !valid_fmt(fmt)) return COAT_ERR_UNSUPPORTED;
+  if (cols % group_size != 0) return COAT_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return COAT_OK;
+  if (rows * cols > kMaxElems) return COAT_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(q) || (ld % 8) != 0) return COAT_ERR_MISALIGNED;
+  coat::GroupQuantParams p;
+  p.x = x;
+  p.rows = rows;
+  p.cols = cols;
+  p.ld = ld;
+  p.vec_per_row = cols / coat::kVec;
+  p.log2G = lg;
+  p.q = q;
+  p.scale = scale;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned int grid = blocks_for(rows * cols);
+  if (fmt == COAT_E4M3)
+    coat::group_quant_1xG_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+  else
+    coat::group_quant_1xG_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  return launch_status();
+}
+
+int64_t coat_group_scaling_workspace_bytes(int64_t n, int32_t group_size) {
+  if (n < 0 || group_size < 1) return -1;
+  return ((n + group_size - 1) / group_size + 1) * static_cast<int64_t>(sizeof(float));
+}
+
+coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
+                                                 int32_t group_size, int32_t fmt,
+                                                 float *workspace, int32_t amax_precomputed,
+                                                 uint8_t *q, float *scale, void *stream) {
+  if (n < 0) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && (!x || !workspace || !q || !scale)) return COAT_ERR_INVALID_ARG;
+  const int lg = group_log2(group_size);
+  if (lg < 0 || !valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
+  if (n == 0) return COAT_OK;
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+    return COAT_ERR_MISALIGNED;
+  const int64_t ng = (n + group_size - 1) / group_size;
+  coat::GroupScalingParams p;
+  p.x = x;
+  p.n = n;
+  p.ngroups = ng;
+  p.log2G = lg;
+  p.group_amax = workspace;
+  p.tensor_amax = reinterpret_cast<uint32_t *>(workspace + ng);
+  p.q = q;
+  p.scale = scale;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(p.tensor_amax, 0, sizeof(uint32_t), s) != cudaSuccess) return launch_status();
+  if (amax_precomputed) {
+    // one pass over the small intermediate: a few blocks per SM suffice
+    const int64_t want = (ng + coat::kThreads - 1) / coat::kThreads;
+    const unsigned int grid = static_cast<unsigned int>(want < 1184 ? want : 1184);
+    coat::amax_of_groups_kernel<<<grid, coat::kThreads, 0, s>>>(p);
+  } else {
+    coat::group_amax_kernel<<<blocks_for(n), coat::kThreads, 0, s>>>(p);
+  }
+  const unsigned int grid = blocks_for(n);
+  if (fmt == COAT_E4M3)
+    coat::pertensor_cast_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+  else
+    coat::pertensor_cast_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  return launch_status();
+}
+
+int32_t coat_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *coat_status_string(coat_status_t status) {
+  switch (status) {
+    case COAT_OK: return "ok";
+    case COAT_ERR_INVALID_ARG: return "invalid argument";
+    case COAT_ERR_MISALIGNED: return "buffer not 16-byte aligned";
+    case COAT_ERR_UNSUPPORTED: return "unsupported format, group size or flag";
+    case COAT_ERR_CUDA: return "CUDA error";
+    case COAT_ERR_NONFINITE: return "non-finite input";
+    case COAT_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t coat_version(void) { return (0 << 16) | (1 << 8) | 0; }
+
+}  // extern "C"

@@ -1,0 +1,409 @@
+// COAT FP8-state AdamW step (fused) and the stand-alone state quantizer.
+//
+// COAT summary page (blog.daoxuan.cc/posts/57954):
+//   section "为什么二阶动量对量化比一阶动量更敏感" -- AdamW with decoupled
+//   weight decay on the FP32 master weights;
+//   section "扩展函数：把窄分布拉宽" -- before FP8 encoding each 1xG group of
+//   a moment is expanded by f(x) = sign(x)|x|^k with
+//   k = log(R_target) / log(R_X), R_X = max|x| / min nonzero |x|, k
+//   recomputed per group at every step; decoding takes the 1/k power.
+// LLM Atlas "systems/numerics", section 08 "Adam -> AdamW" -- m_t, v_t,
+// bias correction, eps outside the root, theta <- (1 - eta*lambda) theta + delta.
+//
+// Work decomposition: one thread owns 16 consecutive parameters, so every
+// stream moves in 16-byte vectors (4 x 16 B of theta, 2 x 16 B of BF16
+// gradient, 16 B of each code stream).  A 1xG group is G/16 consecutive
+// threads: up to 32 of them reduce with warp shuffles, larger groups (G >=
+// 1024) finish the reduction through shared memory inside the block.  The
+// whole group stays in registers between the range reduction and the
+// encode, so every byte crosses HBM exactly once.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp8_device.cuh"
+
+namespace coat {
+
+constexpr int kThreads = 256;
+constexpr int kVec = 16;                           // parameters per thread
+constexpr int kElemsPerBlock = kThreads * kVec;    // 4096
+constexpr int kWarps = kThreads / 32;
+
+struct StateFmtParams {
+  double ln_range;   // ln of the range k aims to fill
+  float fmax;        // storage format's largest finite value
+  float log2_fmax;   // log2(fmax)
+};
+
+struct StepParams {
+  float *theta;
+  const uint16_t *grad;
+  uint8_t *m_code;
+  float *m_k;
+  float *m_s;
+  uint8_t *v_code;
+  float *v_k;
+  float *v_s;
+  int64_t n;
+  int log2G;
+  float beta1, beta2, c1, c2, bc1, bc2, decay, lr, eps;
+  float k_max;       // <= 0: no clamp
+  int force_k1;
+  StateFmtParams m, v;
+  float log2_tab[8]; // log2(1 + i/8)
+};
+
+struct QuantParams {
+  const float *x;
+  uint8_t *code;
+  float *k;
+  float *s;
+  int64_t n;
+  int log2G;
+  float k_max;
+  int force_k1;
+  StateFmtParams f;
+  float log2_tab[8];
+};
+
+// Per-group quantization parameters, identical in every lane of the group.
+struct GroupQ {
+  float k;       // expansion exponent (binary32, as stored)
+  float s;       // scale, x = |d|^(1/k) * s
+  int eM;        // exponent of M = max|x|
+  float fM;      // log2 of M's significand
+  bool zero;     // all-zero group
+};
+
+// k and s of a group from its range (M, mn).  k is evaluated in binary64 and
+// rounded once; s in binary32 through the exp2 unit (or an IEEE division when
+// k == 1).
+__device__ __forceinline__ GroupQ group_params(float M, float mn, const StateFmtParams &f,
+                                               float k_max, int force_k1) {
+  GroupQ g;
+  g.zero = !(M > 0.0f);
+  if (g.zero) {
+    g.k = 1.0f;
+    g.s = 0.0f;
+    g.eM = 0;
+    g.fM = 0.0f;
+    return g;
+  }
+  float k;
+  if (force_k1 || M == mn) {
+    k = 1.0f;
+  } else {
+    double kd = f.ln_range / log(static_cast<double>(M) / static_cast<double>(mn));
+    if (k_max > 0.0f && kd > static_cast<double>(k_max)) kd = static_cast<double>(k_max);
+    k = static_cast<float>(kd);
+  }
+  g.k = k;
+  if (k == 1.0f) {
+    g.s = __fdiv_rn(M, f.fmax);
+  } else {
+    g.s = __fmul_rn(M, ex2_approx(-f.log2_fmax * __frcp_rn(k)));
+  }
+  Log2Split ls = log2_split(M);
+  g.eM = ls.e;
+  g.fM = ls.f;
+  return g;
+}
+
+// Expanded, rescaled magnitude y = fmax * (|x| / M)^k of one element, via
+// log2(|x|/M) = (e_x - e_M) + (log2 sig_x - log2 sig_M), so the large integer
+// part is exact.  Zero stays zero.
+__device__ __forceinline__ float expand_one(float x, const GroupQ &g, float fmax) {
+  const float ax = fabsf(x);
+  Log2Split ls = log2_split(ax);
+  const float A = static_cast<float>(ls.e - g.eM) + (ls.f - g.fM);
+  const float y = fmax * ex2_approx(g.k * A);
+  return ax > 0.0f ? y : 0.0f;
+}
+
+// Encode 16 values of one group into 16 codes (element 0 in the low byte of
+// out[0]).  Sign from x; zero -> 0x00; NaN -> 0x7F.
+template <int F>
+__device__ __forceinline__ void encode16(const float *x, const GroupQ &g, uint32_t *out) {
+  const float fmax = fmt_max<F>();
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    float y[4];
+    uint32_t sign = 0, nanm = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float xv = x[4 * w + j];
+      y[j] = g.zero ? 0.0f : expand_one(xv, g, fmax);
+      sign |= (xv < 0.0f ? 0x80u : 0u) << (8 * j);
+      nanm |= (xv != xv ? 0xFFu : 0u) << (8 * j);
+    }
+    uint32_t c = float4_to_fp8x4<F>(y[0], y[1], y[2], y[3]) | sign;
+    out[w] = (c & ~nanm) | (0x7F7F7F7Fu & nanm);
+  }
+}
+
+// Inverse expansion of one decoded value d with group (k, s):
+// x = sign(d) |d|^(1/k) s, exact d*s when k == 1.
+__device__ __forceinline__ float dequant_one(float d, float s, float rk, bool k1,
+                                             const float *tab8) {
+  const float ad = fabsf(d);
+  const float p = k1 ? ad : ex2_approx(__fmul_rn(log2_fp8_value(ad, tab8), rk));
+  float x = __fmul_rn(p, s);
+  x = (ad > 0.0f) ? x : 0.0f;
+  x = (d != d) ? d : x;
+  return copysignf(x, d);
+}
+
+// Max of |x| and min of nonzero |x| over 16 values (NaN ignored).
+__device__ __forceinline__ void range16(const float *x, float &mx, float &mn) {
+  mx = 0.0f;
+  mn = __int_as_float(0x7f800000);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = fabsf(x[i]);
+    mx = fmaxf(mx, a);
+    mn = fminf(mn, a > 0.0f ? a : __int_as_float(0x7f800000));
+  }
+}
+
+// Reduce (max, min) pairs for two states over the threads of a group.
+// lanes = G/16 threads.  For lanes <= 32 the group lives inside one warp;
+// otherwise warp results are combined through shared memory.
+__device__ __forceinline__ void group_reduce2(float &mx0, float &mn0, float &mx1, float &mn1,
+                                              int lanes, float (*red)[kWarps]) {
+  const int lim = lanes < 32 ? lanes : 32;
+  for (int off = 1; off < lim; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mn0 = fminf(mn0, __shfl_xor_sync(0xffffffffu, mn0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    mn1 = fminf(mn1, __shfl_xor_sync(0xffffffffu, mn1, off));
+  }
+  if (lanes > 32) {  // uniform across the block
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+      red[0][warp] = mx0;
+      red[1][warp] = mn0;
+      red[2][warp] = mx1;
+      red[3][warp] = mn1;
+    }
+    __syncthreads();
+    const int wpg = lanes >> 5;
+    const int w0 = (warp / wpg) * wpg;
+    mx0 = red[0][w0];
+    mn0 = red[1][w0];
+    mx1 = red[2][w0];
+    mn1 = red[3][w0];
+    for (int i = 1; i < wpg; ++i) {
+      mx0 = fmaxf(mx0, red[0][w0 + i]);
+      mn0 = fminf(mn0, red[1][w0 + i]);
+      mx1 = fmaxf(mx1, red[2][w0 + i]);
+      mn1 = fminf(mn1, red[3][w0 + i]);
+    }
+  }
+}
+
+// ---- vector I/O with a ragged tail -----------------------------------------
+
+__device__ __forceinline__ void load16_f32(const float *p, int64_t e0, int64_t n, float *v) {
+  if (e0 + 16 <= n) {
+    const float4 *q = reinterpret_cast<const float4 *>(p + e0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 t = q[i];
+      v[4 * i + 0] = t.x;
+      v[4 * i + 1] = t.y;
+      v[4 * i + 2] = t.z;
+      v[4 * i + 3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = (e0 + i < n) ? p[e0 + i] : 0.0f;
+  }
+}
+
+__device__ __forceinline__ void store16_f32(float *p, int64_t e0, int64_t n, const float *v) {
+  if (e0 + 16 <= n) {
+    float4 *q = reinterpret_cast<float4 *>(p + e0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+    for (int i = 0; i < 16; ++i)
+      if (e0 + i < n) p[e0 + i] = v[i];
+  }
+}
+
+// 16 bytes (16 codes or 8 BF16) as four words.
+__device__ __forceinline__ void load16_u8(const uint8_t *p, int64_t e0, int64_t n, uint32_t *w) {
+  if (e0 + 16 <= n) {
+    uint4 t = *reinterpret_cast<const uint4 *>(p + e0);
+    w[0] = t.x;
+    w[1] = t.y;
+    w[2] = t.z;
+    w[3] = t.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = 0;
+    for (int i = 0; i < 16; ++i)
+      if (e0 + i < n) w[i >> 2] |= static_cast<uint32_t>(p[e0 + i]) << (8 * (i & 3));
+  }
+}
+
+__device__ __forceinline__ void store16_u8(uint8_t *p, int64_t e0, int64_t n, const uint32_t *w) {
+  if (e0 + 16 <= n) {
+    *reinterpret_cast<uint4 *>(p + e0) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    for (int i = 0; i < 16; ++i)
+      if (e0 + i < n) p[e0 + i] = static_cast<uint8_t>(w[i >> 2] >> (8 * (i & 3)));
+  }
+}
+
+// 16 BF16 values as eight words (element 2i in the low half of word i).
+__device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64_t n,
+                                            uint32_t *w) {
+  if (e0 + 16 <= n) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p + e0);
+    uint4 a = q[0], b = q[1];
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = 0;
+    for (int i = 0; i < 16; ++i)
+      if (e0 + i < n) w[i >> 1] |= static_cast<uint32_t>(p[e0 + i]) << (16 * (i & 1));
+  }
+}
+
+// ---- the fused step ----------------------------------------------------------
+
+template <int VF>
+__global__ void __launch_bounds__(kThreads)
+adamw_fp8_step_kernel(const StepParams p) {
+  __shared__ float tab8[8];
+  __shared__ float red[4][kWarps];
+  if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
+  __syncthreads();
+
+  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+  const bool active = e0 < p.n;
+  const int64_t grp = e0 >> p.log2G;
+  const int lanes = 1 << (p.log2G - 4);
+
+  float th[16], m[16], v[16];
+  uint32_t gw[8], mw[4], vw[4];
+  float mk = 1.0f, ms = 0.0f, vk = 1.0f, vs = 0.0f;
+  if (active) {
+    load16_f32(p.theta, e0, p.n, th);
+    load16_bf16(p.grad, e0, p.n, gw);
+    load16_u8(p.m_code, e0, p.n, mw);
+    load16_u8(p.v_code, e0, p.n, vw);
+    mk = p.m_k[grp];
+    ms = p.m_s[grp];
+    vk = p.v_k[grp];
+    vs = p.v_s[grp];
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) th[i] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) gw[i] = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mw[i] = vw[i] = 0;
+  }
+
+  // dequantize the stored moments
+  {
+    const float mrk = __frcp_rn(mk), vrk = __frcp_rn(vk);
+    const bool mk1 = mk == 1.0f, vk1 = vk == 1.0f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      float dm[4], dv[4];
+      fp8x4_to_float<kE4M3>(mw[w], dm);
+      fp8x4_to_float<VF>(vw[w], dv);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m[4 * w + j] = dequant_one(dm[j], ms, mrk, mk1, tab8);
+        v[4 * w + j] = dequant_one(dv[j], vs, vrk, vk1, tab8);
+      }
+    }
+  }
+
+  // AdamW, binary32, one rounding per operation in the order of the rule
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t gword = gw[i >> 1];
+    const float g = (i & 1) ? bf16hi_to_float(gword) : bf16lo_to_float(gword);
+    const float mt = __fadd_rn(__fmul_rn(p.beta1, m[i]), __fmul_rn(p.c1, g));
+    const float vt = __fadd_rn(__fmul_rn(p.beta2, v[i]), __fmul_rn(p.c2, __fmul_rn(g, g)));
+    const float mh = __fdiv_rn(mt, p.bc1);
+    const float vh = __fdiv_rn(vt, p.bc2);
+    const float u = __fdiv_rn(mh, __fadd_rn(__fsqrt_rn(vh), p.eps));
+    th[i] = __fsub_rn(__fmul_rn(th[i], p.decay), __fmul_rn(p.lr, u));
+    m[i] = mt;
+    v[i] = vt;
+  }
+  if (active) store16_f32(p.theta, e0, p.n, th);
+
+  // tail elements beyond n must not take part in the group range
+  if (e0 + 16 > p.n) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (e0 + i >= p.n) m[i] = v[i] = 0.0f;
+  }
+
+  // per-group range of the new moments, then k and s
+  float mmx, mmn, vmx, vmn;
+  range16(m, mmx, mmn);
+  range16(v, vmx, vmn);
+  group_reduce2(mmx, mmn, vmx, vmn, lanes, red);
+  const GroupQ gm = group_params(mmx, mmn, p.m, p.k_max, p.force_k1);
+  const GroupQ gv = group_params(vmx, vmn, p.v, p.k_max, p.force_k1);
+
+  // re-expand, rescale and encode
+  uint32_t mo[4], vo[4];
+  encode16<kE4M3>(m, gm, mo);
+  encode16<VF>(v, gv, vo);
+  if (active) {
+    store16_u8(p.m_code, e0, p.n, mo);
+    store16_u8(p.v_code, e0, p.n, vo);
+    if ((threadIdx.x & (lanes - 1)) == 0 || lanes > kThreads) {
+      p.m_k[grp] = gm.k;
+      p.m_s[grp] = gm.s;
+      p.v_k[grp] = gv.k;
+      p.v_s[grp] = gv.s;
+    }
+  }
+}
+
+// ---- stand-alone state quantizer --------------------------------------------
+
+template <int F>
+__global__ void __launch_bounds__(kThreads)
+quantize_state_kernel(const QuantParams p) {
+  __shared__ float red[4][kWarps];
+  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+  const bool active = e0 < p.n;
+  const int64_t grp = e0 >> p.log2G;
+  const int lanes = 1 << (p.log2G - 4);
+  float x[16];
+  if (active) {
+    load16_f32(p.x, e0, p.n, x);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = 0.0f;
+  }
+  float mx, mn, dmx = 0.0f, dmn = 0.0f;
+  range16(x, mx, mn);
+  group_reduce2(mx, mn, dmx, dmn, lanes, red);
+  const GroupQ g = group_params(mx, mn, p.f, p.k_max, p.force_k1);
+  uint32_t o[4];
+  encode16<F>(x, g, o);
+  if (active) {
+    store16_u8(p.code, e0, p.n, o);
+    if ((threadIdx.x & (lanes - 1)) == 0) {
+      p.k[grp] = g.k;
+      p.s[grp] = g.s;
+    }
+  }
+}
+
+}  // namespace coat

@@ -1,0 +1,112 @@
+"""The C ABI library builds, loads without a GPU, and exports every entry
+point that include/*.h declares; host-side argument checks reject bad calls
+before any launch (CPU only: no kernel runs here)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_optimizer_states_b200 import build
+    build.build()
+    import quantized_optimizer_states_b200 as q
+    return q.load()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b(coat_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("coat_adamw_fp8_step", "coat_group_quant_1xG",
+                 "coat_group_scaling_quant_pertensor", "coat_dequant", "coat_quantize_state"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    so = os.path.join(ROOT, "quantized_optimizer_states_b200", "libcoat.so")
+    out = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_host_functions_without_gpu(lib):
+    assert lib.coat_version() == 0x000100
+    assert lib.coat_status_string(2) == b"buffer not 16-byte aligned"
+    assert lib.coat_group_scaling_workspace_bytes(1000, 128) == (8 + 1) * 4
+    assert lib.coat_group_scaling_workspace_bytes(-1, 128) == -1
+
+
+def test_argument_checks_return_before_any_launch(lib):
+    """Invalid calls are rejected on the host: status codes only, no CUDA."""
+    from quantized_optimizer_states_b200._lib import CoatAdamwCfg
+    P = ctypes.c_void_p
+    fake = P(0x10000)      # never dereferenced: every call below fails a host check
+    odd = P(0x10004)
+    cfg = CoatAdamwCfg(0.9, 0.999, 1e-4, 1e-8, 0.1, 10, 128, 0, 0, 0, 64.0, 0)
+    args = [fake] * 8
+    step = lib.coat_adamw_fp8_step
+    assert step(*args, -1, ctypes.byref(cfg), None) == 1               # n < 0
+    assert step(*args, 0, ctypes.byref(cfg), None) == 0                # empty: no launch
+    assert step(None, *args[1:], 16, ctypes.byref(cfg), None) == 1     # null pointer
+    assert step(odd, *args[1:], 16, ctypes.byref(cfg), None) == 2      # misaligned
+    for field, val, want in (("group_size", 96, 3), ("group_size", 8, 3), ("group_size", 8192, 3),
+                             ("m_fmt", 1, 3), ("v_fmt", 2, 3), ("k_range", 2, 3),
+                             ("flags", 0x40, 3), ("step", 0, 1), ("beta1", 1.0, 1),
+                             ("beta2", -0.1, 1), ("k_max", -1.0, 1)):
+        bad = CoatAdamwCfg.from_buffer_copy(cfg)
+        setattr(bad, field, val)
+        assert step(*args, 16, ctypes.byref(bad), None) == want, field
+    assert step(*args, 16, None, None) == 1
+    q = lib.coat_quantize_state
+    assert q(fake, 16, 100, 0, 0, 64.0, 0, fake, fake, fake, None) == 3
+    assert q(odd, 16, 128, 0, 0, 64.0, 0, fake, fake, fake, None) == 2
+    d = lib.coat_dequant
+    assert d(fake, None, fake, 100, 48, 0, 0, fake, None) == 3            # G not a power of 2
+    assert d(fake, None, fake, 100, 0, 0, 0, fake, None) == 1
+    assert d(odd, None, fake, 100, 100, 0, 0, fake, None) == 2
+    g = lib.coat_group_quant_1xG
+    assert g(fake, 4, 200, 200, 128, 0, fake, fake, None) == 1           # cols % G != 0
+    assert g(fake, 4, 256, 100, 128, 0, fake, fake, None) == 1           # ld < cols
+    assert g(fake, 4, 256, 260, 128, 0, fake, fake, None) == 2           # ld not 16-byte rows
+    gs = lib.coat_group_scaling_quant_pertensor
+    assert gs(fake, 100, 128, 5, fake, 0, fake, fake, None) == 3
+    assert gs(odd, 100, 128, 0, fake, 0, fake, fake, None) == 2
+    assert gs(fake, 0, 128, 0, fake, 0, fake, fake, None) == 0
+
+
+def test_product_path_fails_loudly_without_library(tmp_path):
+    from quantized_optimizer_states_b200 import _lib
+    saved = _lib._lib
+    try:
+        _lib._lib = None
+        with pytest.raises(RuntimeError, match="libcoat.so not found"):
+            _lib.load(str(tmp_path / "missing" / "libcoat.so"))
+    finally:
+        _lib._lib = saved
+
+
+def test_product_package_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "quantized_optimizer_states_b200")
+    for path in glob.glob(os.path.join(pkg, "**", "*"), recursive=True):
+        if path.endswith((".py", ".cu", ".cuh", ".h")):
+            src = open(path).read()
+            assert "import oracle" not in src and "from oracle" not in src, path
+            assert "coat_oracle" not in src and "liborc" not in src, path

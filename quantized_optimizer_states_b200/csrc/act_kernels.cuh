@@ -204,7 +204,7 @@ struct DequantParams {
   int log2G;       // -1: one scale for the whole tensor
   int out_bf16;
   void *out;
-  float log2_tab[8];
+  double log2_tab[8];
 };
 
 __device__ __forceinline__ uint32_t float_to_bf16_rn(float f) {
@@ -213,7 +213,7 @@ __device__ __forceinline__ uint32_t float_to_bf16_rn(float f) {
 
 template <int F>
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p) {
-  __shared__ float tab8[8];
+  __shared__ double tab8[8];
   if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
   __syncthreads();
   const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p
   const float s = p.scale[grp];
   const float kk = p.k ? p.k[grp] : 1.0f;
   const bool k1 = kk == 1.0f;
-  const float rk = __frcp_rn(kk);
+  const double rk = 1.0 / static_cast<double>(kk);
   uint32_t w[4];
   load16_u8(p.q, e0, p.n, w);
   float x[16];

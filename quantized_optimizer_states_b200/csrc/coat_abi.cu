@@ -56,8 +56,8 @@ coat::StateFmtParams state_fmt_params(int32_t store_fmt, int32_t k_range) {
   return f;
 }
 
-void fill_log2_table(float *tab) {
-  for (int i = 0; i < 8; ++i) tab[i] = static_cast<float>(std::log2(1.0 + i / 8.0));
+void fill_log2_table(double *tab) {
+  for (int i = 0; i < 8; ++i) tab[i] = std::log2(1.0 + i / 8.0);
 }
 
 unsigned int blocks_for(int64_t elems) {
@@ -153,7 +153,6 @@ coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size,
   p.k_max = k_max;
   p.force_k1 = (flags & COAT_FORCE_K1) ? 1 : 0;
   p.f = state_fmt_params(fmt, k_range);
-  fill_log2_table(p.log2_tab);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned int grid = blocks_for(n);
   if (fmt == COAT_E4M3)

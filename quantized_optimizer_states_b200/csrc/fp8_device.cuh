@@ -109,12 +109,4 @@ __device__ __forceinline__ Log2Split log2_split(float a) {
   return r;
 }
 
-// log2 |d| of a decoded FP8 magnitude (a float with at most three
-// significant mantissa bits after normalisation): exponent plus a table of
-// log2(1 + i/8), i = 0..7, held in shared memory.
-__device__ __forceinline__ float log2_fp8_value(float ad, const float *tab8) {
-  const uint32_t b = __float_as_uint(ad);
-  return static_cast<float>(static_cast<int>(b >> 23) - 127) + tab8[(b >> 20) & 7u];
-}
-
 }  // namespace coat

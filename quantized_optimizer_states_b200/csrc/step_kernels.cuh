@@ -52,7 +52,7 @@ struct StepParams {
   float k_max;       // <= 0: no clamp
   int force_k1;
   StateFmtParams m, v;
-  float log2_tab[8]; // log2(1 + i/8)
+  double log2_tab[8]; // log2(1 + i/8)
 };
 
 struct QuantParams {
@@ -65,7 +65,6 @@ struct QuantParams {
   float k_max;
   int force_k1;
   StateFmtParams f;
-  float log2_tab[8];
 };
 
 // Per-group quantization parameters, identical in every lane of the group.
@@ -144,11 +143,17 @@ __device__ __forceinline__ void encode16(const float *x, const GroupQ &g, uint32
 }
 
 // Inverse expansion of one decoded value d with group (k, s):
-// x = sign(d) |d|^(1/k) s, exact d*s when k == 1.
-__device__ __forceinline__ float dequant_one(float d, float s, float rk, bool k1,
-                                             const float *tab8) {
+// x = sign(d) |d|^(1/k) s.  The power is evaluated as 2^(log2|d| * (1/k)) in
+// binary64 -- log2|d| is exact up to binary64 rounding (integer exponent plus
+// a table of log2(1 + i/8)) -- and rounded once to binary32, i.e. the
+// correctly rounded |d|^(1/k) except in vanishingly rare double-rounding
+// cases; then one binary32 product with s.  When k == 1 it is exactly d*s.
+__device__ __forceinline__ float dequant_one(float d, float s, double rk, bool k1,
+                                             const double *tab8) {
   const float ad = fabsf(d);
-  const float p = k1 ? ad : ex2_approx(__fmul_rn(log2_fp8_value(ad, tab8), rk));
+  const uint32_t b = __float_as_uint(ad);
+  const double L = static_cast<double>(static_cast<int>(b >> 23) - 127) + tab8[(b >> 20) & 7u];
+  const float p = k1 ? ad : static_cast<float>(exp2(L * rk));
   float x = __fmul_rn(p, s);
   x = (ad > 0.0f) ? x : 0.0f;
   x = (d != d) ? d : x;
@@ -279,7 +284,7 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
 template <int VF>
 __global__ void __launch_bounds__(kThreads)
 adamw_fp8_step_kernel(const StepParams p) {
-  __shared__ float tab8[8];
+  __shared__ double tab8[8];
   __shared__ float red[4][kWarps];
   if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
   __syncthreads();
@@ -312,7 +317,7 @@ adamw_fp8_step_kernel(const StepParams p) {
 
   // dequantize the stored moments
   {
-    const float mrk = __frcp_rn(mk), vrk = __frcp_rn(vk);
+    const double mrk = 1.0 / static_cast<double>(mk), vrk = 1.0 / static_cast<double>(vk);
     const bool mk1 = mk == 1.0f, vk1 = vk == 1.0f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {

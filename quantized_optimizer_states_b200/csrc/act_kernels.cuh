@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include "fp8_device.cuh"
+#include "state_codec.cuh"
 #include "step_kernels.cuh"
 
 namespace coat {
@@ -221,7 +222,6 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p
   const int64_t grp = p.log2G < 0 ? 0 : (e0 >> p.log2G);
   const float s = p.scale[grp];
   const float kk = p.k ? p.k[grp] : 1.0f;
-  const bool k1 = kk == 1.0f;
   const double rk = 1.0 / static_cast<double>(kk);
   uint32_t w[4];
   load16_u8(p.q, e0, p.n, w);
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       if (p.k)
-        x[4 * i + j] = dequant_one(d[j], s, rk, k1, tab8);
+        x[4 * i + j] = dequant_exact(d[j], s, rk, tab8);
       else
         x[4 * i + j] = __fmul_rn(d[j], s);
     }

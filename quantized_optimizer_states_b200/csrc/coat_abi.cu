@@ -66,6 +66,22 @@ unsigned int blocks_for(int64_t elems) {
 
 constexpr int64_t kMaxElems = int64_t{1} << 44;  // grid-size bound (2^31 blocks x 4096)
 
+// Launch one instantiation of the step kernel, raising its dynamic shared
+// memory limit first when the decode tables need more than the default.
+coat_status_t launch_step(void (*kernel)(coat::StepParams), unsigned int grid, size_t smem,
+                          cudaStream_t s, const coat::StepParams &p) {
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) {
+      g_last_cuda_error = static_cast<int32_t>(e);
+      return COAT_ERR_CUDA;
+    }
+  }
+  kernel<<<grid, coat::kThreads, smem, s>>>(p);
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -100,6 +116,7 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
   p.v_k = v_k;
   p.v_s = v_scale;
   p.n = n;
+  p.ngroups = (n + cfg->group_size - 1) / cfg->group_size;
   p.log2G = lg;
   p.beta1 = cfg->beta1;
   p.beta2 = cfg->beta2;
@@ -113,6 +130,9 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
   {
     volatile float lr_wd = cfg->lr * cfg->weight_decay;  // keep the product rounded alone
     p.decay = 1.0f - lr_wd;
+    volatile float one = 1.0f;
+    p.rbc1 = one / p.bc1;  // correctly rounded reciprocals for the corrected quotients
+    p.rbc2 = one / p.bc2;
   }
   p.lr = cfg->lr;
   p.eps = cfg->eps;
@@ -125,11 +145,16 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned int grid = blocks_for(n);
-  if (cfg->v_fmt == COAT_E4M3)
-    coat::adamw_fp8_step_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
-  else
-    coat::adamw_fp8_step_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
-  return launch_status();
+  const size_t smem = coat::step_smem_bytes(lg);
+  const bool table = smem > 0;
+  if (cfg->v_fmt == COAT_E4M3) {
+    if (table)
+      return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, true>, grid, smem, s, p);
+    return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, false>, grid, 0, s, p);
+  }
+  if (table)
+    return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, true>, grid, smem, s, p);
+  return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, false>, grid, 0, s, p);
 }
 
 coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size, int32_t fmt,

@@ -17,12 +17,20 @@
 // 1024) finish the reduction through shared memory inside the block.  The
 // whole group stays in registers between the range reduction and the
 // encode, so every byte crosses HBM exactly once.
+//
+// Dequantization must reproduce RN32(|d|^(1/k)) exactly (the new group
+// range depends on the smallest |m_t|, which cancellation in
+// beta1*m + (1-beta1)*g makes sensitive to the last bit).  For G >= 64 every
+// block first builds, in shared memory, the 128-entry decode table of each
+// of its (group, moment) pairs from binary64 factors, so an element costs
+// one table lookup; for G < 64 each element is decoded directly in binary64.
 #pragma once
 
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "fp8_device.cuh"
+#include "state_codec.cuh"
 
 namespace coat {
 
@@ -30,12 +38,7 @@ constexpr int kThreads = 256;
 constexpr int kVec = 16;                           // parameters per thread
 constexpr int kElemsPerBlock = kThreads * kVec;    // 4096
 constexpr int kWarps = kThreads / 32;
-
-struct StateFmtParams {
-  double ln_range;   // ln of the range k aims to fill
-  float fmax;        // storage format's largest finite value
-  float log2_fmax;   // log2(fmax)
-};
+constexpr int kMinTableG = 64;                     // table path for G >= 64
 
 struct StepParams {
   float *theta;
@@ -47,9 +50,10 @@ struct StepParams {
   float *v_k;
   float *v_s;
   int64_t n;
+  int64_t ngroups;
   int log2G;
-  float beta1, beta2, c1, c2, bc1, bc2, decay, lr, eps;
-  float k_max;       // <= 0: no clamp
+  float beta1, beta2, c1, c2, bc1, bc2, rbc1, rbc2, decay, lr, eps;
+  float k_max;        // <= 0: no clamp
   int force_k1;
   StateFmtParams m, v;
   double log2_tab[8]; // log2(1 + i/8)
@@ -67,97 +71,28 @@ struct QuantParams {
   StateFmtParams f;
 };
 
-// Per-group quantization parameters, identical in every lane of the group.
-struct GroupQ {
-  float k;       // expansion exponent (binary32, as stored)
-  float s;       // scale, x = |d|^(1/k) * s
-  int eM;        // exponent of M = max|x|
-  float fM;      // log2 of M's significand
-  bool zero;     // all-zero group
-};
-
-// k and s of a group from its range (M, mn).  k is evaluated in binary64 and
-// rounded once; s in binary32 through the exp2 unit (or an IEEE division when
-// k == 1).
-__device__ __forceinline__ GroupQ group_params(float M, float mn, const StateFmtParams &f,
-                                               float k_max, int force_k1) {
-  GroupQ g;
-  g.zero = !(M > 0.0f);
-  if (g.zero) {
-    g.k = 1.0f;
-    g.s = 0.0f;
-    g.eM = 0;
-    g.fM = 0.0f;
-    return g;
-  }
-  float k;
-  if (force_k1 || M == mn) {
-    k = 1.0f;
-  } else {
-    double kd = f.ln_range / log(static_cast<double>(M) / static_cast<double>(mn));
-    if (k_max > 0.0f && kd > static_cast<double>(k_max)) kd = static_cast<double>(k_max);
-    k = static_cast<float>(kd);
-  }
-  g.k = k;
-  if (k == 1.0f) {
-    g.s = __fdiv_rn(M, f.fmax);
-  } else {
-    g.s = __fmul_rn(M, ex2_approx(-f.log2_fmax * __frcp_rn(k)));
-  }
-  Log2Split ls = log2_split(M);
-  g.eM = ls.e;
-  g.fM = ls.f;
-  return g;
+// Dynamic shared memory of the table path for group size 2^log2G.
+inline size_t step_smem_bytes(int log2G) {
+  if ((1 << log2G) < kMinTableG) return 0;
+  const int tables = 2 * (kElemsPerBlock >> log2G);
+  return static_cast<size_t>(tables) * kTableBytes;
 }
 
-// Expanded, rescaled magnitude y = fmax * (|x| / M)^k of one element, via
-// log2(|x|/M) = (e_x - e_M) + (log2 sig_x - log2 sig_M), so the large integer
-// part is exact.  Zero stays zero.
-__device__ __forceinline__ float expand_one(float x, const GroupQ &g, float fmax) {
-  const float ax = fabsf(x);
-  Log2Split ls = log2_split(ax);
-  const float A = static_cast<float>(ls.e - g.eM) + (ls.f - g.fM);
-  const float y = fmax * ex2_approx(g.k * A);
-  return ax > 0.0f ? y : 0.0f;
+// a / b for a per-launch constant b with r = RN(1/b): q = RN(a r) corrected
+// once with the exact residual a - q b (Markstein's FMA division step).
+__device__ __forceinline__ float div_by_const(float a, float b, float r) {
+  const float q = __fmul_rn(a, r);
+  const float res = __fmaf_rn(-q, b, a);
+  return __fmaf_rn(res, r, q);
 }
 
-// Encode 16 values of one group into 16 codes (element 0 in the low byte of
-// out[0]).  Sign from x; zero -> 0x00; NaN -> 0x7F.
-template <int F>
-__device__ __forceinline__ void encode16(const float *x, const GroupQ &g, uint32_t *out) {
-  const float fmax = fmt_max<F>();
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    float y[4];
-    uint32_t sign = 0, nanm = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float xv = x[4 * w + j];
-      y[j] = g.zero ? 0.0f : expand_one(xv, g, fmax);
-      sign |= (xv < 0.0f ? 0x80u : 0u) << (8 * j);
-      nanm |= (xv != xv ? 0xFFu : 0u) << (8 * j);
-    }
-    uint32_t c = float4_to_fp8x4<F>(y[0], y[1], y[2], y[3]) | sign;
-    out[w] = (c & ~nanm) | (0x7F7F7F7Fu & nanm);
-  }
-}
-
-// Inverse expansion of one decoded value d with group (k, s):
-// x = sign(d) |d|^(1/k) s.  The power is evaluated as 2^(log2|d| * (1/k)) in
-// binary64 -- log2|d| is exact up to binary64 rounding (integer exponent plus
-// a table of log2(1 + i/8)) -- and rounded once to binary32, i.e. the
-// correctly rounded |d|^(1/k) except in vanishingly rare double-rounding
-// cases; then one binary32 product with s.  When k == 1 it is exactly d*s.
-__device__ __forceinline__ float dequant_one(float d, float s, double rk, bool k1,
-                                             const double *tab8) {
-  const float ad = fabsf(d);
-  const uint32_t b = __float_as_uint(ad);
-  const double L = static_cast<double>(static_cast<int>(b >> 23) - 127) + tab8[(b >> 20) & 7u];
-  const float p = k1 ? ad : static_cast<float>(exp2(L * rk));
-  float x = __fmul_rn(p, s);
-  x = (ad > 0.0f) ? x : 0.0f;
-  x = (d != d) ? d : x;
-  return copysignf(x, d);
+// a / b from the hardware reciprocal estimate plus one Markstein correction.
+__device__ __forceinline__ float div_markstein(float a, float b) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(b));
+  const float q = __fmul_rn(a, y);
+  const float res = __fmaf_rn(-q, b, a);
+  return __fmaf_rn(res, y, q);
 }
 
 // Max of |x| and min of nonzero |x| over 16 values (NaN ignored).
@@ -281,13 +216,13 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
 
 // ---- the fused step ----------------------------------------------------------
 
-template <int VF>
+template <int VF, bool TABLE>
 __global__ void __launch_bounds__(kThreads)
 adamw_fp8_step_kernel(const StepParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
   __shared__ double tab8[8];
   __shared__ float red[4][kWarps];
   if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
-  __syncthreads();
 
   const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
   const bool active = e0 < p.n;
@@ -296,16 +231,11 @@ adamw_fp8_step_kernel(const StepParams p) {
 
   float th[16], m[16], v[16];
   uint32_t gw[8], mw[4], vw[4];
-  float mk = 1.0f, ms = 0.0f, vk = 1.0f, vs = 0.0f;
   if (active) {
     load16_f32(p.theta, e0, p.n, th);
     load16_bf16(p.grad, e0, p.n, gw);
     load16_u8(p.m_code, e0, p.n, mw);
     load16_u8(p.v_code, e0, p.n, vw);
-    mk = p.m_k[grp];
-    ms = p.m_s[grp];
-    vk = p.v_k[grp];
-    vs = p.v_s[grp];
   } else {
 #pragma unroll
     for (int i = 0; i < 16; ++i) th[i] = 0.0f;
@@ -314,11 +244,38 @@ adamw_fp8_step_kernel(const StepParams p) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) mw[i] = vw[i] = 0;
   }
+  __syncthreads();  // tab8
 
-  // dequantize the stored moments
-  {
+  // ---- dequantize the stored moments (exact binary32 results) ----
+  if constexpr (TABLE) {
+    const int gpb = kElemsPerBlock >> p.log2G;  // groups per block
+    const int T = 2 * gpb;
+    const TableView tv = table_view(smem, T);
+    const int64_t g0 = static_cast<int64_t>(blockIdx.x) * gpb;
+    auto meta = [&](int j, bool want_s) -> float {
+      const bool vst = j >= gpb;
+      const int64_t g = g0 + (vst ? j - gpb : j);
+      if (g >= p.ngroups) return want_s ? 0.0f : 1.0f;
+      return want_s ? (vst ? p.v_s[g] : p.m_s[g]) : (vst ? p.v_k[g] : p.m_k[g]);
+    };
+    table_phase1(tv, T, tab8, [&](int j) { return meta(j, false); });
+    __syncthreads();
+    table_phase2<VF>(tv, T, gpb, [&](int j) { return meta(j, true); });
+    __syncthreads();
+    table_phase3<VF>(tv, T, gpb, [&](int j) { return meta(j, true); });
+    __syncthreads();
+    const int gb = threadIdx.x >> (p.log2G - 4);
+    lookup16(tv.ent + gb * kTabEntries, mw, m);
+    lookup16(tv.ent + (gpb + gb) * kTabEntries, vw, v);
+  } else {
+    float mk = 1.0f, ms = 0.0f, vk = 1.0f, vs = 0.0f;
+    if (active) {
+      mk = p.m_k[grp];
+      ms = p.m_s[grp];
+      vk = p.v_k[grp];
+      vs = p.v_s[grp];
+    }
     const double mrk = 1.0 / static_cast<double>(mk), vrk = 1.0 / static_cast<double>(vk);
-    const bool mk1 = mk == 1.0f, vk1 = vk == 1.0f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       float dm[4], dv[4];
@@ -326,22 +283,24 @@ adamw_fp8_step_kernel(const StepParams p) {
       fp8x4_to_float<VF>(vw[w], dv);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        m[4 * w + j] = dequant_one(dm[j], ms, mrk, mk1, tab8);
-        v[4 * w + j] = dequant_one(dv[j], vs, vrk, vk1, tab8);
+        m[4 * w + j] = dequant_exact(dm[j], ms, mrk, tab8);
+        v[4 * w + j] = dequant_exact(dv[j], vs, vrk, tab8);
       }
     }
   }
 
-  // AdamW, binary32, one rounding per operation in the order of the rule
+  // ---- AdamW, binary32, one rounding per operation in the order of the rule ----
+  // m^ = m_t / (1 - beta1^t) and v^ = v_t / (1 - beta2^t) by a corrected
+  // reciprocal product; the update quotient by a corrected reciprocal estimate.
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const uint32_t gword = gw[i >> 1];
     const float g = (i & 1) ? bf16hi_to_float(gword) : bf16lo_to_float(gword);
     const float mt = __fadd_rn(__fmul_rn(p.beta1, m[i]), __fmul_rn(p.c1, g));
     const float vt = __fadd_rn(__fmul_rn(p.beta2, v[i]), __fmul_rn(p.c2, __fmul_rn(g, g)));
-    const float mh = __fdiv_rn(mt, p.bc1);
-    const float vh = __fdiv_rn(vt, p.bc2);
-    const float u = __fdiv_rn(mh, __fadd_rn(__fsqrt_rn(vh), p.eps));
+    const float mh = div_by_const(mt, p.bc1, p.rbc1);
+    const float vh = div_by_const(vt, p.bc2, p.rbc2);
+    const float u = div_markstein(mh, __fadd_rn(__fsqrt_rn(vh), p.eps));
     th[i] = __fsub_rn(__fmul_rn(th[i], p.decay), __fmul_rn(p.lr, u));
     m[i] = mt;
     v[i] = vt;
@@ -355,22 +314,39 @@ adamw_fp8_step_kernel(const StepParams p) {
       if (e0 + i >= p.n) m[i] = v[i] = 0.0f;
   }
 
-  // per-group range of the new moments, then k and s
+  // ---- per-group range of the new moments, then k and s ----
   float mmx, mmn, vmx, vmn;
   range16(m, mmx, mmn);
   range16(v, vmx, vmn);
   group_reduce2(mmx, mmn, vmx, vmn, lanes, red);
-  const GroupQ gm = group_params(mmx, mmn, p.m, p.k_max, p.force_k1);
-  const GroupQ gv = group_params(vmx, vmn, p.v, p.k_max, p.force_k1);
+  GroupQ gm, gv;
+  if (lanes >= 2) {
+    // even lanes evaluate m's parameters, odd lanes v's; then swap
+    const bool odd = threadIdx.x & 1;
+    const GroupQ mine = group_params(odd ? vmx : mmx, odd ? vmn : mmn,
+                                     odd ? p.v.ln_range : p.m.ln_range,
+                                     odd ? p.v.fmax : p.m.fmax,
+                                     odd ? p.v.log2_fmax : p.m.log2_fmax, p.k_max, p.force_k1);
+    GroupQ other;
+    other.k = __shfl_xor_sync(0xffffffffu, mine.k, 1);
+    other.s = __shfl_xor_sync(0xffffffffu, mine.s, 1);
+    other.rM = __shfl_xor_sync(0xffffffffu, mine.rM, 1);
+    other.zero = __shfl_xor_sync(0xffffffffu, static_cast<int>(mine.zero), 1) != 0;
+    gm = odd ? other : mine;
+    gv = odd ? mine : other;
+  } else {
+    gm = group_params(mmx, mmn, p.m.ln_range, p.m.fmax, p.m.log2_fmax, p.k_max, p.force_k1);
+    gv = group_params(vmx, vmn, p.v.ln_range, p.v.fmax, p.v.log2_fmax, p.k_max, p.force_k1);
+  }
 
-  // re-expand, rescale and encode
+  // ---- re-expand, rescale and encode ----
   uint32_t mo[4], vo[4];
-  encode16<kE4M3>(m, gm, mo);
-  encode16<VF>(v, gv, vo);
+  encode16<kE4M3>(m, gm, p.m.log2_fmax, mo);
+  encode16<VF>(v, gv, p.v.log2_fmax, vo);
   if (active) {
     store16_u8(p.m_code, e0, p.n, mo);
     store16_u8(p.v_code, e0, p.n, vo);
-    if ((threadIdx.x & (lanes - 1)) == 0 || lanes > kThreads) {
+    if ((threadIdx.x & (lanes - 1)) == 0) {
       p.m_k[grp] = gm.k;
       p.m_s[grp] = gm.s;
       p.v_k[grp] = gv.k;
@@ -399,9 +375,10 @@ quantize_state_kernel(const QuantParams p) {
   float mx, mn, dmx = 0.0f, dmn = 0.0f;
   range16(x, mx, mn);
   group_reduce2(mx, mn, dmx, dmn, lanes, red);
-  const GroupQ g = group_params(mx, mn, p.f, p.k_max, p.force_k1);
+  const GroupQ g = group_params(mx, mn, p.f.ln_range, p.f.fmax, p.f.log2_fmax, p.k_max,
+                                p.force_k1);
   uint32_t o[4];
-  encode16<F>(x, g, o);
+  encode16<F>(x, g, p.f.log2_fmax, o);
   if (active) {
     store16_u8(p.code, e0, p.n, o);
     if ((threadIdx.x & (lanes - 1)) == 0) {

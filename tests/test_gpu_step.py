@@ -156,8 +156,10 @@ def test_state_dequant_parity(lib, orc):
                          group_size=G, fmt=fmt)
         torch.cuda.synchronize()
         got = parity.to_host(out)
-        # inverse expansion through exp2/log2 units: within 1e-6 relative
-        parity.compare_rel("dequant", got, ref, 1e-6)
+        # correctly rounded powers: identical except in vanishingly rare
+        # double-rounding cases, which may differ by one unit in the last place
+        parity.compare_rel("dequant", got, ref, 2.0 ** -23)
+        assert np.count_nonzero(got != ref) <= 1e-5 * got.size
 
 
 def test_deterministic_and_guarded(lib, orc):

@@ -146,15 +146,19 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned int grid = blocks_for(n);
   const size_t smem = coat::step_smem_bytes(lg);
-  const bool table = smem > 0;
+  const int ent = coat::step_table_entries(lg);
   if (cfg->v_fmt == COAT_E4M3) {
-    if (table)
-      return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, true>, grid, smem, s, p);
-    return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, false>, grid, 0, s, p);
+    if (ent == 256)
+      return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, 256>, grid, smem, s, p);
+    if (ent == 128)
+      return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, 128>, grid, smem, s, p);
+    return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, 0>, grid, 0, s, p);
   }
-  if (table)
-    return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, true>, grid, smem, s, p);
-  return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, false>, grid, 0, s, p);
+  if (ent == 256)
+    return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, 256>, grid, smem, s, p);
+  if (ent == 128)
+    return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, 128>, grid, smem, s, p);
+  return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, 0>, grid, 0, s, p);
 }
 
 coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size, int32_t fmt,

@@ -55,6 +55,16 @@ __device__ __forceinline__ double exp2_d(double y) {
   return q * __hiloint2double((n + 1023) << 20, 0);
 }
 
+// 1/x in binary64 from the hardware estimate and two Newton steps.
+__device__ __forceinline__ double recip_d(double x) {
+  double y;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(x));
+  double e = fma(-x, y, 1.0);
+  y = fma(e, y, y);
+  e = fma(-x, y, 1.0);
+  return fma(e, y, y);
+}
+
 // ---- per-group parameters from the group range --------------------------------
 
 struct GroupQ {
@@ -73,38 +83,52 @@ __device__ __forceinline__ GroupQ group_params(float M, float mn, double ln_rang
   g.zero = !(M > 0.0f);
   float k = 1.0f;
   if (!g.zero && !force_k1 && M != mn) {
-    double kd = ln_range / log(static_cast<double>(M) / static_cast<double>(mn));
+    const double ratio = static_cast<double>(M) * recip_d(static_cast<double>(mn));
+    double kd = ln_range * recip_d(log(ratio));
     if (k_max > 0.0f && kd > static_cast<double>(k_max)) kd = static_cast<double>(k_max);
     k = static_cast<float>(kd);
   }
   g.k = k;
+  float rk, rM;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rk) : "f"(k));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rM) : "f"(M));
   if (g.zero)
     g.s = 0.0f;
   else if (k == 1.0f)
     g.s = __fdiv_rn(M, fmax);
   else
-    g.s = __fmul_rn(M, ex2_approx(-log2_fmax * __frcp_rn(k)));
-  g.rM = g.zero ? 0.0f : __frcp_rn(M);
+    g.s = __fmul_rn(M, ex2_approx(-log2_fmax * rk));
+  g.rM = g.zero ? 0.0f : rM;
   return g;
 }
 
 // ---- expansion + encode ---------------------------------------------------------
-// y = fmax * (|x| / M)^k = 2^(k log2(|x| / M) + log2 fmax), signed like x
-// (zero stays +0, so x == 0 encodes as 0x00).
+// y = fmax * (|x| / M)^k = 2^(k log2(|x| / M) + log2 fmax), carrying x's sign
+// bit (+0 encodes as 0x00; -0, which the update can produce only from a
+// negative-zero gradient on a zero moment, as the equal-valued 0x80).
 __device__ __forceinline__ float expand_signed(float x, float rM, float k, float log2_fmax) {
   const float r = __fmul_rn(fabsf(x), rM);
   const float y = ex2_approx(__fmaf_rn(k, lg2_approx(r), log2_fmax));
-  return x < 0.0f ? -y : y;
+  return __uint_as_float(__float_as_uint(y) | (__float_as_uint(x) & 0x80000000u));
 }
 
 template <int F>
 __device__ __forceinline__ void encode16(const float *x, const GroupQ &g, float log2_fmax,
                                          uint32_t *out) {
+  const float2 RM = make_float2(g.rM, g.rM), K = make_float2(g.k, g.k);
+  const float2 LF = make_float2(log2_fmax, log2_fmax);
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     float y[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) y[j] = expand_signed(x[4 * w + j], g.rM, g.k, log2_fmax);
+    for (int j = 0; j < 4; j += 2) {
+      const float x0 = x[4 * w + j], x1 = x[4 * w + j + 1];
+      const float2 r = fmul2(make_float2(fabsf(x0), fabsf(x1)), RM);
+      const float2 z = ffma2(K, make_float2(lg2_approx(r.x), lg2_approx(r.y)), LF);
+      y[j] = __uint_as_float(__float_as_uint(ex2_approx(z.x)) | (__float_as_uint(x0) & 0x80000000u));
+      y[j + 1] =
+          __uint_as_float(__float_as_uint(ex2_approx(z.y)) | (__float_as_uint(x1) & 0x80000000u));
+    }
     out[w] = g.zero ? 0u : float4_to_fp8x4<F>(y[0], y[1], y[2], y[3]);
   }
 }
@@ -128,131 +152,160 @@ __device__ __forceinline__ float dequant_exact(float d, float s, double rk, cons
 }
 
 // ---- per-group dequantization tables --------------------------------------------
-// For a group with exponent k and scale s, entry c (c = 0..127, the code's
-// magnitude bits) holds RN32(RN32(|d_c|^(1/k)) * s).  |d_c| = (1 + f/8) 2^e,
-// so |d_c|^(1/k) = A(e) B(f) with A(e) = 2^(e/k) and B(f) = 2^(log2(1+f/8)/k),
-// both in binary64 (A from powers of 2^(+-1/k)); one product per entry, then
-// the two binary32 roundings the definition has.  Subnormal, zero, inf and
-// NaN codes are patched afterwards.
-constexpr int kTabEntries = 128;
-constexpr int kAOff = 16;   // A(e) at index e + 16, e in [-16, 16]
-constexpr int kASize = 33;
-constexpr int kTableBytes = kTabEntries * 4 + kASize * 8 + 8 * 8;  // 840
+// For a group with exponent k and scale s, entry c holds
+// RN32(RN32(|d_c|^(1/k)) * s) with the sign of code c.  |d_c| = (1 + f/8) 2^e,
+// so |d_c|^(1/k) = A(e) B(f) with A(e) = a^e, a = 2^(1/k), and
+// B(f) = 2^(log2(1 + f/8) / k), all in binary64: a, 1/a and B(2..7) come from
+// exp2_d, B(1) = B(4)^2 / a (since 1.5^2 = 2 * 1.125), and a^e from at most
+// four squarings and four products, so every entry is within ~2^-48 of the
+// exact power before the binary32 roundings of the definition.
+//
+// Every warp builds the tables of the groups its threads touch (with only
+// warp-level synchronisation): 2 per group (m, v), 256 signed entries each
+// (ENT == 256) or 128 magnitude entries plus a sign fix-up at lookup time
+// (ENT == 128, used when a warp holds many small groups).
+constexpr int kTabDoubles = 8;   // a, 1/a, B(2..7)
 
-struct TableView {
-  float *ent;    // [T][128]
-  double *A;     // [T][33]
-  double *B;     // [T][8]
+template <int ENT>
+struct WarpTables {
+  float *ent;    // [TW][ENT]
+  double *D;     // [TW][8]: a, 1/a, B(2), ..., B(7)
+  float *S;      // [TW] scale s
 };
 
-__device__ __forceinline__ TableView table_view(unsigned char *smem, int T) {
-  TableView v;
-  v.ent = reinterpret_cast<float *>(smem);
-  v.A = reinterpret_cast<double *>(smem + static_cast<size_t>(T) * kTabEntries * 4);
-  v.B = v.A + static_cast<size_t>(T) * kASize;
+template <int ENT>
+__host__ __device__ constexpr int warp_table_bytes(int TW) {
+  return ((TW * (ENT * 4 + kTabDoubles * 8 + 4)) + 15) / 16 * 16;
+}
+
+template <int ENT>
+__device__ __forceinline__ WarpTables<ENT> warp_tables(unsigned char *base, int TW) {
+  WarpTables<ENT> v;
+  v.ent = reinterpret_cast<float *>(base);
+  v.D = reinterpret_cast<double *>(base + static_cast<size_t>(TW) * ENT * 4);
+  v.S = reinterpret_cast<float *>(v.D + static_cast<size_t>(TW) * kTabDoubles);
   return v;
 }
 
-// Phase 1: A(e) for e in [-16, 16] (jobs [0, T)) and B(f), f = 1..7
-// (jobs [T, 8T)).  k_of(j) returns table j's k.
-template <class KOf>
-__device__ __forceinline__ void table_phase1(const TableView &tv, int T, const double *log2tab,
-                                             KOf k_of) {
-  for (int job = threadIdx.x; job < 8 * T; job += blockDim.x) {
-    if (job < T) {
-      const double rk = 1.0 / static_cast<double>(k_of(job));
-      const double a = exp2_d(rk), ai = exp2_d(-rk);
-      double *Aj = tv.A + job * kASize;
-      Aj[kAOff] = 1.0;
-      double up = 1.0, dn = 1.0;
+// b^|e| with b = a (e >= 0) or 1/a (e < 0), |e| < 2^BITS, by square-and-multiply.
+template <int BITS>
+__device__ __forceinline__ double ipow(double a, double ai, int e) {
+  double base = e >= 0 ? a : ai;
+  int n = e >= 0 ? e : -e;
+  double r = 1.0;
 #pragma unroll
-      for (int e = 1; e <= 16; ++e) {
-        up *= a;
-        dn *= ai;
-        Aj[kAOff + e] = up;
-        Aj[kAOff - e] = dn;
-      }
-    } else {
-      const int q = job - T;
-      const int j = q / 7;
-      const int f = q - 7 * j + 1;
-      const double rk = 1.0 / static_cast<double>(k_of(j));
-      tv.B[j * 8 + f] = exp2_d(log2tab[f] * rk);
-      if (f == 1) tv.B[j * 8] = 1.0;
-    }
+  for (int bit = 0; bit < BITS; ++bit) {
+    const double t = r * base;
+    r = (n & 1) ? t : r;
+    base *= base;
+    n >>= 1;
   }
+  return r;
 }
 
-// Phase 2: the 128 entries of every table, eight codes per job.  Tables
-// [0, T_m) hold E4M3 first moments; [T_m, T) the second moment in VF.
-template <int VF, class SOf>
-__device__ __forceinline__ void table_phase2(const TableView &tv, int T, int T_m, SOf s_of) {
-  for (int job = threadIdx.x; job < 16 * T; job += blockDim.x) {
-    const int j = job >> 4;
-    const int c0 = (job & 15) << 3;
-    const float s = s_of(j);
-    const double *Aj = tv.A + j * kASize;
-    const double *Bj = tv.B + j * 8;
-    float r[8];
-    if (VF == kE4M3 || j < T_m) {
-      const double a = Aj[kAOff + (c0 >> 3) - 7];
-#pragma unroll
-      for (int f = 0; f < 8; ++f) r[f] = __fmul_rn(static_cast<float>(a * Bj[f]), s);
-    } else {
-      const int E = c0 >> 2;
-      const double a0 = Aj[kAOff + E - 15], a1 = Aj[kAOff + E + 1 - 15];
-#pragma unroll
-      for (int f = 0; f < 4; ++f) {
-        r[f] = __fmul_rn(static_cast<float>(a0 * Bj[2 * f]), s);
-        r[4 + f] = __fmul_rn(static_cast<float>(a1 * Bj[2 * f]), s);
-      }
-    }
-    float4 *dst = reinterpret_cast<float4 *>(tv.ent + j * kTabEntries + c0);
-    dst[0] = make_float4(r[0], r[1], r[2], r[3]);
-    dst[1] = make_float4(r[4], r[5], r[6], r[7]);
-  }
+__device__ __forceinline__ float entry_value(double A, double B, float s) {
+  return __fmul_rn(static_cast<float>(A * B), s);
 }
 
-// Phase 3: zero, subnormal, inf and NaN codes.
-template <int VF, class SOf>
-__device__ __forceinline__ void table_phase3(const TableView &tv, int T, int T_m, SOf s_of) {
-  for (int job = threadIdx.x; job < 9 * T; job += blockDim.x) {
-    const int j = job / 9;
-    const int w = job - 9 * j;
-    const float s = s_of(j);
-    float *ent = tv.ent + j * kTabEntries;
-    const double *Aj = tv.A + j * kASize;
-    const double *Bj = tv.B + j * 8;
-    const bool e4 = (VF == kE4M3 || j < T_m);
-    const int nsub = e4 ? 7 : 3;          // subnormal codes 1..nsub
-    const int emin = e4 ? -9 : -16;       // exponent of the smallest subnormal
-    if (w == 0) {
-      ent[0] = 0.0f;
-    } else if (w <= nsub) {
-      // code w is w * 2^emin = (1 + f/8) 2^(lz + emin), lz = floor(log2 w)
-      const int lz = 31 - __clz(w);
-      const int f = (w << (3 - lz)) & 7;
-      ent[w] = __fmul_rn(static_cast<float>(Aj[kAOff + lz + emin] * Bj[f]), s);
-    } else if (e4) {
-      if (w == 8) ent[127] = s != 0.0f ? __int_as_float(0x7fc00000) : 0.0f;
-    } else if (w >= 4 && w <= 7) {
-      // E5M2: 0x7C = inf, 0x7D..0x7F = NaN
-      const float special = w == 4 ? __int_as_float(0x7f800000) : __int_as_float(0x7fc00000);
-      ent[120 + w] = s != 0.0f ? special : 0.0f;
+// Phase 1 for one job of a warp: table j, slot f (0 = a, 1 = 1/a, 2..7 =
+// B(f)).  mult8 = {1, -1, log2(1 + f/8) for f = 2..7}.
+template <int ENT>
+__device__ __forceinline__ void table_slot(const WarpTables<ENT> &tw, int j, int f, float k,
+                                           float s, const double *mult8) {
+  const double rk = recip_d(static_cast<double>(k));
+  tw.D[j * kTabDoubles + f] = exp2_d(mult8[f] * rk);
+  if (f == 0) tw.S[j] = s;
+}
+
+// Phase 2 for one job: the sixteen codes 16q .. 16q+15 of table j, whose
+// format is E4M3 (e4) or E5M2.  Code 0 and the subnormal codes (q == 0) and
+// the inf / NaN codes (q == 7) are set from their own definitions.
+template <int ENT>
+__device__ __forceinline__ void table_codes(const WarpTables<ENT> &tw, int j, int q, bool e4) {
+  const double *D = tw.D + j * kTabDoubles;
+  const float s = tw.S[j];
+  const double a = D[0], ai = D[1];
+  double B[8];
+  B[0] = 1.0;
+#pragma unroll
+  for (int f = 2; f < 8; ++f) B[f] = D[f];
+  B[1] = B[4] * B[4] * ai;
+  float r[16];
+  const float nan = s != 0.0f ? __int_as_float(0x7fc00000) : 0.0f;
+  if (e4) {
+    // binades 2q, 2q+1: exponents 2q-7, 2q-6 (binade 0 holds the subnormals)
+    const double A0 = ipow<3>(a, ai, 2 * q - 7);
+    const double A1 = A0 * a;
+#pragma unroll
+    for (int f = 0; f < 8; ++f) {
+      r[f] = entry_value(A0, B[f], s);
+      r[8 + f] = entry_value(A1, B[f], s);
     }
+    if (q == 0) {
+      // code w = w * 2^-9: 1 -> 2^-9, 2 -> 2^-8, 3 -> 1.5 2^-8, 4 -> 2^-7,
+      // 5 -> 1.25 2^-7, 6 -> 1.5 2^-7, 7 -> 1.75 2^-7; A0 = A(-7)
+      const double Am8 = A0 * ai, Am9 = Am8 * ai;
+      r[0] = 0.0f;
+      r[1] = entry_value(Am9, 1.0, s);
+      r[2] = entry_value(Am8, 1.0, s);
+      r[3] = entry_value(Am8, B[4], s);
+      r[4] = entry_value(A0, 1.0, s);
+      r[5] = entry_value(A0, B[2], s);
+      r[6] = entry_value(A0, B[4], s);
+      r[7] = entry_value(A0, B[6], s);
+    }
+    if (q == 7) r[15] = nan;  // 0x7F
+  } else {
+    // binades 4q .. 4q+3: exponents 4q-15 .. 4q-12 (binade 0: subnormals,
+    // binade 31: inf and NaN)
+    double A = ipow<4>(a, ai, 4 * q - 15);
+    const double A0 = A;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+#pragma unroll
+      for (int f = 0; f < 4; ++f) r[4 * b + f] = entry_value(A, B[2 * f], s);
+      A *= a;
+    }
+    if (q == 0) {
+      // code w = w * 2^-16: 1 -> 2^-16, 2 -> 2^-15, 3 -> 1.5 2^-15; A0 = A(-15)
+      r[0] = 0.0f;
+      r[1] = entry_value(A0 * ai, 1.0, s);
+      r[2] = entry_value(A0, 1.0, s);
+      r[3] = entry_value(A0, B[4], s);
+    }
+    if (q == 7) {
+      r[12] = s != 0.0f ? __int_as_float(0x7f800000) : 0.0f;  // 0x7C
+      r[13] = nan;
+      r[14] = nan;
+      r[15] = nan;
+    }
+  }
+  float4 *pos = reinterpret_cast<float4 *>(tw.ent + j * ENT + 16 * q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) pos[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+  if constexpr (ENT == 256) {
+    float4 *neg = reinterpret_cast<float4 *>(tw.ent + j * ENT + 128 + 16 * q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      neg[i] = make_float4(-r[4 * i], -r[4 * i + 1], -r[4 * i + 2], -r[4 * i + 3]);
   }
 }
 
 // Table lookup for the 16 codes held in four words (element 0 in the low
-// byte of w[0]): x = entry[c & 0x7F] with the code's sign bit.
+// byte of w[0]).
+template <int ENT>
 __device__ __forceinline__ void lookup16(const float *ent, const uint32_t *w, float *x) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const uint32_t word = w[i >> 2];
     const int sh = 8 * (i & 3);
-    const uint32_t c = (word >> sh) & 0x7Fu;
-    const uint32_t sign = (word << (24 - sh)) & 0x80000000u;
-    x[i] = __uint_as_float(__float_as_uint(ent[c]) | sign);
+    if constexpr (ENT == 256) {
+      x[i] = ent[(word >> sh) & 0xFFu];
+    } else {
+      const uint32_t c = (word >> sh) & 0x7Fu;
+      const uint32_t sign = (word << (24 - sh)) & 0x80000000u;
+      x[i] = __uint_as_float(__float_as_uint(ent[c]) | sign);
+    }
   }
 }
 

@@ -71,11 +71,27 @@ struct QuantParams {
   StateFmtParams f;
 };
 
-// Dynamic shared memory of the table path for group size 2^log2G.
+// Decode-table layout of the step kernel for group size 2^log2G:
+// 0 = direct binary64 decode (G < 64), else table entries per table.
+inline int step_table_entries(int log2G) {
+  const int G = 1 << log2G;
+  if (G < kMinTableG) return 0;
+  return G == 64 ? 128 : 256;
+}
+
+// Tables per warp: 2 (m, v) per group touched by the warp.
+__host__ __device__ inline int step_tables_per_warp(int log2G) {
+  const int gpw = (32 * kVec) >> log2G;
+  return 2 * (gpw > 1 ? gpw : 1);
+}
+
+// Dynamic shared memory of the step kernel for group size 2^log2G.
 inline size_t step_smem_bytes(int log2G) {
-  if ((1 << log2G) < kMinTableG) return 0;
-  const int tables = 2 * (kElemsPerBlock >> log2G);
-  return static_cast<size_t>(tables) * kTableBytes;
+  const int ent = step_table_entries(log2G);
+  if (ent == 0) return 0;
+  const int TW = step_tables_per_warp(log2G);
+  const int per_warp = ent == 128 ? warp_table_bytes<128>(TW) : warp_table_bytes<256>(TW);
+  return static_cast<size_t>(kWarps) * per_warp;
 }
 
 // a / b for a per-launch constant b with r = RN(1/b): q = RN(a r) corrected
@@ -86,25 +102,42 @@ __device__ __forceinline__ float div_by_const(float a, float b, float r) {
   return __fmaf_rn(res, r, q);
 }
 
-// a / b from the hardware reciprocal estimate plus one Markstein correction.
-__device__ __forceinline__ float div_markstein(float a, float b) {
+__device__ __forceinline__ float sqrt_approx(float x) {
   float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(b));
-  const float q = __fmul_rn(a, y);
-  const float res = __fmaf_rn(-q, b, a);
-  return __fmaf_rn(res, y, q);
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-// Max of |x| and min of nonzero |x| over 16 values (NaN ignored).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// theta_t for one element with every operation of the rule correctly
+// rounded: m^ = m_t / bc1, v^ = v_t / bc2, u = m^ / (sqrt(v^) + eps).
+template <class P>
+__device__ __forceinline__ float exact_update(float th, float mt, float vt, const P &p) {
+  const float mh = div_by_const(mt, p.bc1, p.rbc1);
+  const float vh = div_by_const(vt, p.bc2, p.rbc2);
+  const float u = __fdiv_rn(mh, __fadd_rn(__fsqrt_rn(vh), p.eps));
+  return __fsub_rn(__fmul_rn(th, p.decay), __fmul_rn(p.lr, u));
+}
+
+// Max of |x| and min of nonzero |x| over 16 values (NaN ignored by the max).
+// The minimum runs on 2*bits(x) - 2 as unsigned integers: the doubling drops
+// the sign bit, and the -2 wraps +-0 to the largest value, so zeros never win;
+// for non-negative floats the integer order is the numeric order.
 __device__ __forceinline__ void range16(const float *x, float &mx, float &mn) {
   mx = 0.0f;
-  mn = __int_as_float(0x7f800000);
+  uint32_t key = 0xFFFFFFFFu;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float a = fabsf(x[i]);
-    mx = fmaxf(mx, a);
-    mn = fminf(mn, a > 0.0f ? a : __int_as_float(0x7f800000));
+    mx = fmaxf(mx, fabsf(x[i]));
+    key = min(key, __float_as_uint(x[i]) * 2u - 2u);
   }
+  // all-zero (or all-NaN) input gives an infinite minimum
+  mn = key >= 0xFF000000u - 2u ? __int_as_float(0x7f800000) : __uint_as_float((key + 2u) >> 1);
 }
 
 // Reduce (max, min) pairs for two states over the threads of a group.
@@ -216,18 +249,49 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
 
 // ---- the fused step ----------------------------------------------------------
 
-template <int VF, bool TABLE>
+template <int VF, int ENT>
 __global__ void __launch_bounds__(kThreads)
 adamw_fp8_step_kernel(const StepParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ double tab8[8];
+  __shared__ double tab8[8];   // log2(1 + i/8)
+  __shared__ double mult8[8];  // 1, -1, log2(1 + i/8) for i = 2..7
   __shared__ float red[4][kWarps];
-  if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
+  if (threadIdx.x < 8) {
+    const double t = p.log2_tab[threadIdx.x];
+    tab8[threadIdx.x] = t;
+    mult8[threadIdx.x] = threadIdx.x == 0 ? 1.0 : (threadIdx.x == 1 ? -1.0 : t);
+  }
 
   const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
   const bool active = e0 < p.n;
   const int64_t grp = e0 >> p.log2G;
   const int lanes = 1 << (p.log2G - 4);
+
+  // Per-group (k, s) of the decode tables this thread helps to build, loaded
+  // first so that they arrive while the bulk streams are requested.
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  int TW = 0, gpw = 1;
+  int64_t warp_g0 = 0;
+  float kk[4], ss[4];
+  if constexpr (ENT != 0) {
+    TW = step_tables_per_warp(p.log2G);
+    gpw = TW >> 1;
+    warp_g0 = (static_cast<int64_t>(blockIdx.x) * kElemsPerBlock + warp * 32 * kVec) >> p.log2G;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int job = lane + 32 * r;
+      const int j = job >> 3;
+      const bool vst = j >= gpw;
+      const int64_t g = warp_g0 + (vst ? j - gpw : j);
+      kk[r] = 1.0f;
+      ss[r] = 0.0f;
+      if (job < 8 * TW && g < p.ngroups) {
+        kk[r] = vst ? p.v_k[g] : p.m_k[g];
+        ss[r] = vst ? p.v_s[g] : p.m_s[g];
+      }
+    }
+  }
 
   float th[16], m[16], v[16];
   uint32_t gw[8], mw[4], vw[4];
@@ -244,29 +308,27 @@ adamw_fp8_step_kernel(const StepParams p) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) mw[i] = vw[i] = 0;
   }
-  __syncthreads();  // tab8
+  __syncthreads();  // tab8, mult8
 
   // ---- dequantize the stored moments (exact binary32 results) ----
-  if constexpr (TABLE) {
-    const int gpb = kElemsPerBlock >> p.log2G;  // groups per block
-    const int T = 2 * gpb;
-    const TableView tv = table_view(smem, T);
-    const int64_t g0 = static_cast<int64_t>(blockIdx.x) * gpb;
-    auto meta = [&](int j, bool want_s) -> float {
-      const bool vst = j >= gpb;
-      const int64_t g = g0 + (vst ? j - gpb : j);
-      if (g >= p.ngroups) return want_s ? 0.0f : 1.0f;
-      return want_s ? (vst ? p.v_s[g] : p.m_s[g]) : (vst ? p.v_k[g] : p.m_k[g]);
-    };
-    table_phase1(tv, T, tab8, [&](int j) { return meta(j, false); });
-    __syncthreads();
-    table_phase2<VF>(tv, T, gpb, [&](int j) { return meta(j, true); });
-    __syncthreads();
-    table_phase3<VF>(tv, T, gpb, [&](int j) { return meta(j, true); });
-    __syncthreads();
-    const int gb = threadIdx.x >> (p.log2G - 4);
-    lookup16(tv.ent + gb * kTabEntries, mw, m);
-    lookup16(tv.ent + (gpb + gb) * kTabEntries, vw, v);
+  if constexpr (ENT != 0) {
+    // warp-local decode tables: [0, gpw) first moment, [gpw, TW) second
+    const WarpTables<ENT> tw =
+        warp_tables<ENT>(smem + static_cast<size_t>(warp) * warp_table_bytes<ENT>(TW), TW);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int job = lane + 32 * r;
+      if (job < 8 * TW) table_slot(tw, job >> 3, job & 7, kk[r], ss[r], mult8);
+    }
+    __syncwarp();
+    for (int job = lane; job < 8 * TW; job += 32) {
+      const int j = job >> 3;
+      table_codes(tw, j, job & 7, VF == kE4M3 || j < gpw);
+    }
+    __syncwarp();
+    const int lg = gpw > 1 ? (lane >> (p.log2G - 4)) : 0;
+    lookup16<ENT>(tw.ent + lg * ENT, mw, m);
+    lookup16<ENT>(tw.ent + (gpw + lg) * ENT, vw, v);
   } else {
     float mk = 1.0f, ms = 0.0f, vk = 1.0f, vs = 0.0f;
     if (active) {
@@ -290,20 +352,51 @@ adamw_fp8_step_kernel(const StepParams p) {
   }
 
   // ---- AdamW, binary32, one rounding per operation in the order of the rule ----
-  // m^ = m_t / (1 - beta1^t) and v^ = v_t / (1 - beta2^t) by a corrected
-  // reciprocal product; the update quotient by a corrected reciprocal estimate.
+  // m_t and v_t are computed exactly as the rule states (they are the new
+  // states).  The update quotient u = m^ / (sqrt(v^) + eps) is first formed
+  // with reciprocal estimates (relative error below 1e-6, so the product
+  // lr*u is off by at most ~1e-6 of itself); wherever |lr*u| is not at least
+  // twice below max(|theta|, lr) that error could matter for theta, and the
+  // pair is recomputed with correctly rounded division and square root.
+  {
+    const float2 RB1 = make_float2(p.rbc1, p.rbc1), RB2 = make_float2(p.rbc2, p.rbc2);
+    const float2 EPS = make_float2(p.eps, p.eps), DEC = make_float2(p.decay, p.decay);
+    const float2 NLR = make_float2(-p.lr, -p.lr), TWO = make_float2(2.0f, 2.0f);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t gword = gw[i >> 1];
-    const float g = (i & 1) ? bf16hi_to_float(gword) : bf16lo_to_float(gword);
-    const float mt = __fadd_rn(__fmul_rn(p.beta1, m[i]), __fmul_rn(p.c1, g));
-    const float vt = __fadd_rn(__fmul_rn(p.beta2, v[i]), __fmul_rn(p.c2, __fmul_rn(g, g)));
-    const float mh = div_by_const(mt, p.bc1, p.rbc1);
-    const float vh = div_by_const(vt, p.bc2, p.rbc2);
-    const float u = div_markstein(mh, __fadd_rn(__fsqrt_rn(vh), p.eps));
-    th[i] = __fsub_rn(__fmul_rn(th[i], p.decay), __fmul_rn(p.lr, u));
-    m[i] = mt;
-    v[i] = vt;
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t gword = gw[i];
+      const float2 g = make_float2(bf16lo_to_float(gword), bf16hi_to_float(gword));
+      // the new states, exactly as the rule rounds them (scalar IEEE
+      // operations: the packed f32x2 forms did not reproduce these roundings)
+      float2 mt, vt;
+      mt.x = __fadd_rn(__fmul_rn(p.beta1, m[2 * i]), __fmul_rn(p.c1, g.x));
+      mt.y = __fadd_rn(__fmul_rn(p.beta1, m[2 * i + 1]), __fmul_rn(p.c1, g.y));
+      vt.x = __fadd_rn(__fmul_rn(p.beta2, v[2 * i]), __fmul_rn(p.c2, __fmul_rn(g.x, g.x)));
+      vt.y = __fadd_rn(__fmul_rn(p.beta2, v[2 * i + 1]),
+                       __fmul_rn(p.c2, __fmul_rn(g.y, g.y)));
+      const float2 vh = fmul2(vt, RB2);
+      const float2 den = fadd2(make_float2(sqrt_approx(vh.x), sqrt_approx(vh.y)), EPS);
+      const float2 u = fmul2(fmul2(mt, RB1),
+                                  make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+      const float2 th0 = make_float2(th[2 * i], th[2 * i + 1]);
+      const float2 t2 = fmul2(NLR, u);
+      float2 tn = fadd2(fmul2(th0, DEC), t2);
+      const float2 w2 = fmul2(TWO, t2);
+      const bool slow = fabsf(w2.x) > fmaxf(fabsf(tn.x), p.lr) ||
+                        fabsf(w2.y) > fmaxf(fabsf(tn.y), p.lr);
+      if (__any_sync(0xffffffffu, slow)) {
+        if (slow) {
+          tn.x = exact_update(th0.x, mt.x, vt.x, p);
+          tn.y = exact_update(th0.y, mt.y, vt.y, p);
+        }
+      }
+      th[2 * i] = tn.x;
+      th[2 * i + 1] = tn.y;
+      m[2 * i] = mt.x;
+      m[2 * i + 1] = mt.y;
+      v[2 * i] = vt.x;
+      v[2 * i + 1] = vt.y;
+    }
   }
   if (active) store16_f32(p.theta, e0, p.n, th);
 

@@ -82,6 +82,24 @@ coat_status_t launch_step(void (*kernel)(coat::StepParams), unsigned int grid, s
   return launch_status();
 }
 
+// The step kernel is instantiated for each supported group size.
+template <int VF>
+coat_status_t launch_step_for(int lg, unsigned int grid, size_t smem, cudaStream_t s,
+                              const coat::StepParams &p) {
+  switch (lg) {
+    case 4: return launch_step(coat::adamw_fp8_step_kernel<VF, 4>, grid, smem, s, p);
+    case 5: return launch_step(coat::adamw_fp8_step_kernel<VF, 5>, grid, smem, s, p);
+    case 6: return launch_step(coat::adamw_fp8_step_kernel<VF, 6>, grid, smem, s, p);
+    case 7: return launch_step(coat::adamw_fp8_step_kernel<VF, 7>, grid, smem, s, p);
+    case 8: return launch_step(coat::adamw_fp8_step_kernel<VF, 8>, grid, smem, s, p);
+    case 9: return launch_step(coat::adamw_fp8_step_kernel<VF, 9>, grid, smem, s, p);
+    case 10: return launch_step(coat::adamw_fp8_step_kernel<VF, 10>, grid, smem, s, p);
+    case 11: return launch_step(coat::adamw_fp8_step_kernel<VF, 11>, grid, smem, s, p);
+    case 12: return launch_step(coat::adamw_fp8_step_kernel<VF, 12>, grid, smem, s, p);
+  }
+  return COAT_ERR_UNSUPPORTED;
+}
+
 }  // namespace
 
 extern "C" {
@@ -117,7 +135,6 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
   p.v_s = v_scale;
   p.n = n;
   p.ngroups = (n + cfg->group_size - 1) / cfg->group_size;
-  p.log2G = lg;
   p.beta1 = cfg->beta1;
   p.beta2 = cfg->beta2;
   // scalar factors of the rule, each rounded to binary32 once
@@ -146,19 +163,8 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned int grid = blocks_for(n);
   const size_t smem = coat::step_smem_bytes(lg);
-  const int ent = coat::step_table_entries(lg);
-  if (cfg->v_fmt == COAT_E4M3) {
-    if (ent == 256)
-      return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, 256>, grid, smem, s, p);
-    if (ent == 128)
-      return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, 128>, grid, smem, s, p);
-    return launch_step(coat::adamw_fp8_step_kernel<coat::kE4M3, 0>, grid, 0, s, p);
-  }
-  if (ent == 256)
-    return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, 256>, grid, smem, s, p);
-  if (ent == 128)
-    return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, 128>, grid, smem, s, p);
-  return launch_step(coat::adamw_fp8_step_kernel<coat::kE5M2, 0>, grid, 0, s, p);
+  return cfg->v_fmt == COAT_E4M3 ? launch_step_for<coat::kE4M3>(lg, grid, smem, s, p)
+                                 : launch_step_for<coat::kE5M2>(lg, grid, smem, s, p);
 }
 
 coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size, int32_t fmt,

@@ -207,6 +207,14 @@ __device__ __forceinline__ float entry_value(double A, double B, float s) {
   return __fmul_rn(static_cast<float>(A * B), s);
 }
 
+// The decode of a pair of codes, optionally scaled by the caller's factor:
+// RN32(RN32(RN32(A B) * s) * beta), two lanes at a time (products only).
+__device__ __forceinline__ float2 entry_pair(double A0, double B0, double A1, double B1, float2 S,
+                                             float2 BETA) {
+  const float2 p = make_float2(static_cast<float>(A0 * B0), static_cast<float>(A1 * B1));
+  return fmul2(fmul2(p, S), BETA);
+}
+
 // Phase 1 for one job of a warp: table j, slot f (0 = a, 1 = 1/a, 2..7 =
 // B(f)).  mult8 = {1, -1, log2(1 + f/8) for f = 2..7}.
 template <int ENT>
@@ -218,12 +226,16 @@ __device__ __forceinline__ void table_slot(const WarpTables<ENT> &tw, int j, int
 }
 
 // Phase 2 for one job: the sixteen codes 16q .. 16q+15 of table j, whose
-// format is E4M3 (e4) or E5M2.  Code 0 and the subnormal codes (q == 0) and
-// the inf / NaN codes (q == 7) are set from their own definitions.
+// format is E4M3 (e4) or E5M2, each entry multiplied by beta (the table
+// then holds beta * x, the first product of the moment update; beta = 1
+// gives the plain decode).  Code 0 and the subnormal codes (q == 0) and the
+// inf / NaN codes (q == 7) are set from their own definitions.
 template <int ENT>
-__device__ __forceinline__ void table_codes(const WarpTables<ENT> &tw, int j, int q, bool e4) {
+__device__ __forceinline__ void table_codes(const WarpTables<ENT> &tw, int j, int q, bool e4,
+                                            float beta) {
   const double *D = tw.D + j * kTabDoubles;
   const float s = tw.S[j];
+  const float2 S = make_float2(s, s), BETA = make_float2(beta, beta);
   const double a = D[0], ai = D[1];
   double B[8];
   B[0] = 1.0;
@@ -237,22 +249,30 @@ __device__ __forceinline__ void table_codes(const WarpTables<ENT> &tw, int j, in
     const double A0 = ipow<3>(a, ai, 2 * q - 7);
     const double A1 = A0 * a;
 #pragma unroll
-    for (int f = 0; f < 8; ++f) {
-      r[f] = entry_value(A0, B[f], s);
-      r[8 + f] = entry_value(A1, B[f], s);
+    for (int f = 0; f < 8; f += 2) {
+      const float2 lo = entry_pair(A0, B[f], A0, B[f + 1], S, BETA);
+      const float2 hi = entry_pair(A1, B[f], A1, B[f + 1], S, BETA);
+      r[f] = lo.x;
+      r[f + 1] = lo.y;
+      r[8 + f] = hi.x;
+      r[9 + f] = hi.y;
     }
     if (q == 0) {
       // code w = w * 2^-9: 1 -> 2^-9, 2 -> 2^-8, 3 -> 1.5 2^-8, 4 -> 2^-7,
       // 5 -> 1.25 2^-7, 6 -> 1.5 2^-7, 7 -> 1.75 2^-7; A0 = A(-7)
       const double Am8 = A0 * ai, Am9 = Am8 * ai;
+      const float2 e12 = entry_pair(Am9, 1.0, Am8, 1.0, S, BETA);
+      const float2 e34 = entry_pair(Am8, B[4], A0, 1.0, S, BETA);
+      const float2 e56 = entry_pair(A0, B[2], A0, B[4], S, BETA);
+      const float2 e70 = entry_pair(A0, B[6], A0, B[6], S, BETA);
       r[0] = 0.0f;
-      r[1] = entry_value(Am9, 1.0, s);
-      r[2] = entry_value(Am8, 1.0, s);
-      r[3] = entry_value(Am8, B[4], s);
-      r[4] = entry_value(A0, 1.0, s);
-      r[5] = entry_value(A0, B[2], s);
-      r[6] = entry_value(A0, B[4], s);
-      r[7] = entry_value(A0, B[6], s);
+      r[1] = e12.x;
+      r[2] = e12.y;
+      r[3] = e34.x;
+      r[4] = e34.y;
+      r[5] = e56.x;
+      r[6] = e56.y;
+      r[7] = e70.x;
     }
     if (q == 7) r[15] = nan;  // 0x7F
   } else {
@@ -262,16 +282,22 @@ __device__ __forceinline__ void table_codes(const WarpTables<ENT> &tw, int j, in
     const double A0 = A;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-#pragma unroll
-      for (int f = 0; f < 4; ++f) r[4 * b + f] = entry_value(A, B[2 * f], s);
+      const float2 lo = entry_pair(A, B[0], A, B[2], S, BETA);
+      const float2 hi = entry_pair(A, B[4], A, B[6], S, BETA);
+      r[4 * b] = lo.x;
+      r[4 * b + 1] = lo.y;
+      r[4 * b + 2] = hi.x;
+      r[4 * b + 3] = hi.y;
       A *= a;
     }
     if (q == 0) {
       // code w = w * 2^-16: 1 -> 2^-16, 2 -> 2^-15, 3 -> 1.5 2^-15; A0 = A(-15)
+      const float2 e12 = entry_pair(A0 * ai, 1.0, A0, 1.0, S, BETA);
+      const float2 e33 = entry_pair(A0, B[4], A0, B[4], S, BETA);
       r[0] = 0.0f;
-      r[1] = entry_value(A0 * ai, 1.0, s);
-      r[2] = entry_value(A0, 1.0, s);
-      r[3] = entry_value(A0, B[4], s);
+      r[1] = e12.x;
+      r[2] = e12.y;
+      r[3] = e33.x;
     }
     if (q == 7) {
       r[12] = s != 0.0f ? __int_as_float(0x7f800000) : 0.0f;  // 0x7C

@@ -21,9 +21,11 @@
 // Dequantization must reproduce RN32(|d|^(1/k)) exactly (the new group
 // range depends on the smallest |m_t|, which cancellation in
 // beta1*m + (1-beta1)*g makes sensitive to the last bit).  For G >= 64 every
-// block first builds, in shared memory, the 128-entry decode table of each
-// of its (group, moment) pairs from binary64 factors, so an element costs
-// one table lookup; for G < 64 each element is decoded directly in binary64.
+// warp first builds, in shared memory, the 128-entry decode table of each of
+// its (group, moment) pairs from binary64 factors -- holding beta1*m or
+// beta2*v directly -- so an element costs one table lookup; for G < 64 each
+// element is decoded directly in binary64.  The kernel is instantiated per
+// group size, so lane counts, table counts and shifts are compile-time.
 #pragma once
 
 #include <cstdint>
@@ -38,7 +40,8 @@ constexpr int kThreads = 256;
 constexpr int kVec = 16;                           // parameters per thread
 constexpr int kElemsPerBlock = kThreads * kVec;    // 4096
 constexpr int kWarps = kThreads / 32;
-constexpr int kMinTableG = 64;                     // table path for G >= 64
+constexpr int kMinTableLog2G = 6;                  // decode tables for G >= 64
+constexpr int kTabEnt = 128;                       // entries per decode table
 
 struct StepParams {
   float *theta;
@@ -51,7 +54,6 @@ struct StepParams {
   float *v_s;
   int64_t n;
   int64_t ngroups;
-  int log2G;
   float beta1, beta2, c1, c2, bc1, bc2, rbc1, rbc2, decay, lr, eps;
   float k_max;        // <= 0: no clamp
   int force_k1;
@@ -71,27 +73,31 @@ struct QuantParams {
   StateFmtParams f;
 };
 
-// Decode-table layout of the step kernel for group size 2^log2G:
-// 0 = direct binary64 decode (G < 64), else table entries per table.
-inline int step_table_entries(int log2G) {
-  const int G = 1 << log2G;
-  if (G < kMinTableG) return 0;
-  return G == 64 ? 128 : 256;
-}
-
-// Tables per warp: 2 (m, v) per group touched by the warp.
-__host__ __device__ inline int step_tables_per_warp(int log2G) {
-  const int gpw = (32 * kVec) >> log2G;
-  return 2 * (gpw > 1 ? gpw : 1);
-}
+// Compile-time layout of the step kernel for group size 2^LG.
+template <int LG>
+struct StepLayout {
+  static constexpr int kLanes = 1 << (LG - 4);               // threads per group
+  static constexpr bool kTable = LG >= kMinTableLog2G;
+  static constexpr int kGroupsPerWarp = LG <= 9 ? (512 >> LG) : 1;
+  static constexpr int kTablesPerWarp = 2 * kGroupsPerWarp;  // m and v per group
+  static constexpr int kJobs = 8 * kTablesPerWarp;           // per phase, per warp
+  static constexpr int kRounds = (kJobs + 31) / 32;
+  static constexpr int kWarpBytes = kTable ? warp_table_bytes<kTabEnt>(kTablesPerWarp) : 0;
+  static constexpr int kSmemBytes = kWarps * kWarpBytes;
+};
 
 // Dynamic shared memory of the step kernel for group size 2^log2G.
 inline size_t step_smem_bytes(int log2G) {
-  const int ent = step_table_entries(log2G);
-  if (ent == 0) return 0;
-  const int TW = step_tables_per_warp(log2G);
-  const int per_warp = ent == 128 ? warp_table_bytes<128>(TW) : warp_table_bytes<256>(TW);
-  return static_cast<size_t>(kWarps) * per_warp;
+  switch (log2G) {
+    case 6: return StepLayout<6>::kSmemBytes;
+    case 7: return StepLayout<7>::kSmemBytes;
+    case 8: return StepLayout<8>::kSmemBytes;
+    case 9: return StepLayout<9>::kSmemBytes;
+    case 10: return StepLayout<10>::kSmemBytes;
+    case 11: return StepLayout<11>::kSmemBytes;
+    case 12: return StepLayout<12>::kSmemBytes;
+    default: return 0;
+  }
 }
 
 // a / b for a per-launch constant b with r = RN(1/b): q = RN(a r) corrected
@@ -140,11 +146,48 @@ __device__ __forceinline__ void range16(const float *x, float &mx, float &mn) {
   mn = key >= 0xFF000000u - 2u ? __int_as_float(0x7f800000) : __uint_as_float((key + 2u) >> 1);
 }
 
-// Reduce (max, min) pairs for two states over the threads of a group.
-// lanes = G/16 threads.  For lanes <= 32 the group lives inside one warp;
-// otherwise warp results are combined through shared memory.
+// Reduce (max, min) pairs for two states over the LANES threads of a group.
+// For LANES <= 32 the group lives inside one warp; otherwise warp results
+// are combined through shared memory.
+template <int LANES>
 __device__ __forceinline__ void group_reduce2(float &mx0, float &mn0, float &mx1, float &mn1,
-                                              int lanes, float (*red)[kWarps]) {
+                                              float (*red)[kWarps]) {
+  constexpr int lim = LANES < 32 ? LANES : 32;
+#pragma unroll
+  for (int off = 1; off < lim; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mn0 = fminf(mn0, __shfl_xor_sync(0xffffffffu, mn0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    mn1 = fminf(mn1, __shfl_xor_sync(0xffffffffu, mn1, off));
+  }
+  if constexpr (LANES > 32) {
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+      red[0][warp] = mx0;
+      red[1][warp] = mn0;
+      red[2][warp] = mx1;
+      red[3][warp] = mn1;
+    }
+    __syncthreads();
+    constexpr int wpg = LANES >> 5;
+    const int w0 = (warp / wpg) * wpg;
+    mx0 = red[0][w0];
+    mn0 = red[1][w0];
+    mx1 = red[2][w0];
+    mn1 = red[3][w0];
+#pragma unroll
+    for (int i = 1; i < wpg; ++i) {
+      mx0 = fmaxf(mx0, red[0][w0 + i]);
+      mn0 = fminf(mn0, red[1][w0 + i]);
+      mx1 = fmaxf(mx1, red[2][w0 + i]);
+      mn1 = fminf(mn1, red[3][w0 + i]);
+    }
+  }
+}
+
+// Runtime-lane form for the stand-alone quantizer.
+__device__ __forceinline__ void group_reduce2_rt(float &mx0, float &mn0, float &mx1, float &mn1,
+                                                 int lanes, float (*red)[kWarps]) {
   const int lim = lanes < 32 ? lanes : 32;
   for (int off = 1; off < lim; off <<= 1) {
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
@@ -152,7 +195,7 @@ __device__ __forceinline__ void group_reduce2(float &mx0, float &mn0, float &mx1
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
     mn1 = fminf(mn1, __shfl_xor_sync(0xffffffffu, mn1, off));
   }
-  if (lanes > 32) {  // uniform across the block
+  if (lanes > 32) {
     const int warp = threadIdx.x >> 5;
     if ((threadIdx.x & 31) == 0) {
       red[0][warp] = mx0;
@@ -249,9 +292,10 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
 
 // ---- the fused step ----------------------------------------------------------
 
-template <int VF, int ENT>
+template <int VF, int LG>
 __global__ void __launch_bounds__(kThreads)
 adamw_fp8_step_kernel(const StepParams p) {
+  using L = StepLayout<LG>;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ double tab8[8];   // log2(1 + i/8)
   __shared__ double mult8[8];  // 1, -1, log2(1 + i/8) for i = 2..7
@@ -262,35 +306,38 @@ adamw_fp8_step_kernel(const StepParams p) {
     mult8[threadIdx.x] = threadIdx.x == 0 ? 1.0 : (threadIdx.x == 1 ? -1.0 : t);
   }
 
-  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
-  const bool active = e0 < p.n;
-  const int64_t grp = e0 >> p.log2G;
-  const int lanes = 1 << (p.log2G - 4);
-
-  // Per-group (k, s) of the decode tables this thread helps to build, loaded
-  // first so that they arrive while the bulk streams are requested.
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  int TW = 0, gpw = 1;
-  int64_t warp_g0 = 0;
-  float kk[4], ss[4];
-  if constexpr (ENT != 0) {
-    TW = step_tables_per_warp(p.log2G);
-    gpw = TW >> 1;
-    warp_g0 = (static_cast<int64_t>(blockIdx.x) * kElemsPerBlock + warp * 32 * kVec) >> p.log2G;
+  const int64_t blk0 = static_cast<int64_t>(blockIdx.x) * kElemsPerBlock;
+  const int64_t e0 = blk0 + threadIdx.x * kVec;
+  const bool active = e0 < p.n;
+  const int64_t grp = e0 >> LG;
+
+  // Per-group (k, s) of the decode tables this thread helps to build (or of
+  // its own group on the direct path), loaded first so that they arrive
+  // while the bulk streams are requested.
+  const int64_t warp_g0 = (blk0 + warp * 32 * kVec) >> LG;
+  float kk[L::kRounds], ss[L::kRounds];
+  float mk = 1.0f, ms = 0.0f, vk = 1.0f, vs = 0.0f;
+  if constexpr (L::kTable) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < L::kRounds; ++r) {
       const int job = lane + 32 * r;
       const int j = job >> 3;
-      const bool vst = j >= gpw;
-      const int64_t g = warp_g0 + (vst ? j - gpw : j);
+      const bool vst = j >= L::kGroupsPerWarp;
+      const int64_t g = warp_g0 + (vst ? j - L::kGroupsPerWarp : j);
       kk[r] = 1.0f;
       ss[r] = 0.0f;
-      if (job < 8 * TW && g < p.ngroups) {
+      if (job < L::kJobs && g < p.ngroups) {
         kk[r] = vst ? p.v_k[g] : p.m_k[g];
         ss[r] = vst ? p.v_s[g] : p.m_s[g];
       }
     }
+  } else if (active) {
+    mk = p.m_k[grp];
+    ms = p.m_s[grp];
+    vk = p.v_k[grp];
+    vs = p.v_s[grp];
   }
 
   float th[16], m[16], v[16];
@@ -310,33 +357,31 @@ adamw_fp8_step_kernel(const StepParams p) {
   }
   __syncthreads();  // tab8, mult8
 
-  // ---- dequantize the stored moments (exact binary32 results) ----
-  if constexpr (ENT != 0) {
-    // warp-local decode tables: [0, gpw) first moment, [gpw, TW) second
-    const WarpTables<ENT> tw =
-        warp_tables<ENT>(smem + static_cast<size_t>(warp) * warp_table_bytes<ENT>(TW), TW);
+  // ---- beta1 * m and beta2 * v from the stored states (exact binary32) ----
+  if constexpr (L::kTable) {
+    // warp-local decode tables: [0, GPW) first moment, [GPW, 2 GPW) second
+    const WarpTables<kTabEnt> tw = warp_tables<kTabEnt>(
+        smem + static_cast<size_t>(warp) * L::kWarpBytes, L::kTablesPerWarp);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < L::kRounds; ++r) {
       const int job = lane + 32 * r;
-      if (job < 8 * TW) table_slot(tw, job >> 3, job & 7, kk[r], ss[r], mult8);
+      if (job < L::kJobs) table_slot(tw, job >> 3, job & 7, kk[r], ss[r], mult8);
     }
     __syncwarp();
-    for (int job = lane; job < 8 * TW; job += 32) {
-      const int j = job >> 3;
-      table_codes(tw, j, job & 7, VF == kE4M3 || j < gpw);
+#pragma unroll
+    for (int r = 0; r < L::kRounds; ++r) {
+      const int job = lane + 32 * r;
+      if (job < L::kJobs) {
+        const int j = job >> 3;
+        const bool first = j < L::kGroupsPerWarp;
+        table_codes(tw, j, job & 7, VF == kE4M3 || first, first ? p.beta1 : p.beta2);
+      }
     }
     __syncwarp();
-    const int lg = gpw > 1 ? (lane >> (p.log2G - 4)) : 0;
-    lookup16<ENT>(tw.ent + lg * ENT, mw, m);
-    lookup16<ENT>(tw.ent + (gpw + lg) * ENT, vw, v);
+    const int lg = L::kGroupsPerWarp > 1 ? (lane >> (LG - 4)) : 0;
+    lookup16<kTabEnt>(tw.ent + lg * kTabEnt, mw, m);
+    lookup16<kTabEnt>(tw.ent + (L::kGroupsPerWarp + lg) * kTabEnt, vw, v);
   } else {
-    float mk = 1.0f, ms = 0.0f, vk = 1.0f, vs = 0.0f;
-    if (active) {
-      mk = p.m_k[grp];
-      ms = p.m_s[grp];
-      vk = p.v_k[grp];
-      vs = p.v_s[grp];
-    }
     const double mrk = 1.0 / static_cast<double>(mk), vrk = 1.0 / static_cast<double>(vk);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -345,20 +390,22 @@ adamw_fp8_step_kernel(const StepParams p) {
       fp8x4_to_float<VF>(vw[w], dv);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        m[4 * w + j] = dequant_exact(dm[j], ms, mrk, tab8);
-        v[4 * w + j] = dequant_exact(dv[j], vs, vrk, tab8);
+        m[4 * w + j] = __fmul_rn(p.beta1, dequant_exact(dm[j], ms, mrk, tab8));
+        v[4 * w + j] = __fmul_rn(p.beta2, dequant_exact(dv[j], vs, vrk, tab8));
       }
     }
   }
 
   // ---- AdamW, binary32, one rounding per operation in the order of the rule ----
-  // m_t and v_t are computed exactly as the rule states (they are the new
-  // states).  The update quotient u = m^ / (sqrt(v^) + eps) is first formed
-  // with reciprocal estimates (relative error below 1e-6, so the product
-  // lr*u is off by at most ~1e-6 of itself); wherever |lr*u| is not at least
-  // twice below max(|theta|, lr) that error could matter for theta, and the
-  // pair is recomputed with correctly rounded division and square root.
+  // m_t and v_t are computed exactly as the rule rounds them (they are the
+  // new states): scalar IEEE sums of separately rounded products.  The
+  // update quotient u = m^ / (sqrt(v^) + eps) is first formed with
+  // reciprocal estimates (relative error below 1e-6, so lr*u is off by at
+  // most ~1e-6 of itself); wherever |lr*u| is not at least twice below
+  // max(|theta|, lr) that error could matter for theta, and the element is
+  // recomputed with correctly rounded division and square root.
   {
+    const float2 C1 = make_float2(p.c1, p.c1), C2 = make_float2(p.c2, p.c2);
     const float2 RB1 = make_float2(p.rbc1, p.rbc1), RB2 = make_float2(p.rbc2, p.rbc2);
     const float2 EPS = make_float2(p.eps, p.eps), DEC = make_float2(p.decay, p.decay);
     const float2 NLR = make_float2(-p.lr, -p.lr), TWO = make_float2(2.0f, 2.0f);
@@ -366,18 +413,16 @@ adamw_fp8_step_kernel(const StepParams p) {
     for (int i = 0; i < 8; ++i) {
       const uint32_t gword = gw[i];
       const float2 g = make_float2(bf16lo_to_float(gword), bf16hi_to_float(gword));
-      // the new states, exactly as the rule rounds them (scalar IEEE
-      // operations: the packed f32x2 forms did not reproduce these roundings)
+      const float2 cg = fmul2(C1, g);
+      const float2 cgg = fmul2(C2, fmul2(g, g));
       float2 mt, vt;
-      mt.x = __fadd_rn(__fmul_rn(p.beta1, m[2 * i]), __fmul_rn(p.c1, g.x));
-      mt.y = __fadd_rn(__fmul_rn(p.beta1, m[2 * i + 1]), __fmul_rn(p.c1, g.y));
-      vt.x = __fadd_rn(__fmul_rn(p.beta2, v[2 * i]), __fmul_rn(p.c2, __fmul_rn(g.x, g.x)));
-      vt.y = __fadd_rn(__fmul_rn(p.beta2, v[2 * i + 1]),
-                       __fmul_rn(p.c2, __fmul_rn(g.y, g.y)));
+      mt.x = __fadd_rn(m[2 * i], cg.x);
+      mt.y = __fadd_rn(m[2 * i + 1], cg.y);
+      vt.x = __fadd_rn(v[2 * i], cgg.x);
+      vt.y = __fadd_rn(v[2 * i + 1], cgg.y);
       const float2 vh = fmul2(vt, RB2);
       const float2 den = fadd2(make_float2(sqrt_approx(vh.x), sqrt_approx(vh.y)), EPS);
-      const float2 u = fmul2(fmul2(mt, RB1),
-                                  make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+      const float2 u = fmul2(fmul2(mt, RB1), make_float2(rcp_approx(den.x), rcp_approx(den.y)));
       const float2 th0 = make_float2(th[2 * i], th[2 * i + 1]);
       const float2 t2 = fmul2(NLR, u);
       float2 tn = fadd2(fmul2(th0, DEC), t2);
@@ -411,9 +456,9 @@ adamw_fp8_step_kernel(const StepParams p) {
   float mmx, mmn, vmx, vmn;
   range16(m, mmx, mmn);
   range16(v, vmx, vmn);
-  group_reduce2(mmx, mmn, vmx, vmn, lanes, red);
+  group_reduce2<L::kLanes>(mmx, mmn, vmx, vmn, red);
   GroupQ gm, gv;
-  if (lanes >= 2) {
+  if constexpr (L::kLanes >= 2) {
     // even lanes evaluate m's parameters, odd lanes v's; then swap
     const bool odd = threadIdx.x & 1;
     const GroupQ mine = group_params(odd ? vmx : mmx, odd ? vmn : mmn,
@@ -439,7 +484,7 @@ adamw_fp8_step_kernel(const StepParams p) {
   if (active) {
     store16_u8(p.m_code, e0, p.n, mo);
     store16_u8(p.v_code, e0, p.n, vo);
-    if ((threadIdx.x & (lanes - 1)) == 0) {
+    if ((threadIdx.x & (L::kLanes - 1)) == 0) {
       p.m_k[grp] = gm.k;
       p.m_s[grp] = gm.s;
       p.v_k[grp] = gv.k;
@@ -467,7 +512,7 @@ quantize_state_kernel(const QuantParams p) {
   }
   float mx, mn, dmx = 0.0f, dmn = 0.0f;
   range16(x, mx, mn);
-  group_reduce2(mx, mn, dmx, dmn, lanes, red);
+  group_reduce2_rt(mx, mn, dmx, dmn, lanes, red);
   const GroupQ g = group_params(mx, mn, p.f.ln_range, p.f.fmax, p.f.log2_fmax, p.k_max,
                                 p.force_k1);
   uint32_t o[4];

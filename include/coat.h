@@ -199,6 +199,41 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
                                                  float *workspace, int32_t amax_precomputed,
                                                  uint8_t *q, float *scale, void *stream);
 
+/* Capacity, in 1xG groups, of the library-owned scratch that
+ * coat_group_scaling_quant_pertensor_noalloc uses (4 MiB of device memory
+ * per GPU, plus one slot). */
+#define COAT_NOALLOC_MAX_GROUPS (1 << 20)
+
+/*
+ * coat_group_scaling_quant_pertensor_noalloc -- the same Group Scaling
+ * quantization as coat_group_scaling_quant_pertensor (amax_precomputed = 0),
+ * for callers that cannot allocate device memory: for example a serving
+ * process that reserves its whole memory budget at start-up and forbids
+ * allocation afterwards, or a plug-in hosted by a framework that owns every
+ * device allocation and hands the plug-in no allocator.  It takes no
+ * workspace and allocates nothing (no cudaMalloc, no allocating library
+ * call).  (The COAT pages have no counterpart: this is an interface
+ * convenience only.)
+ *
+ * Scratch: a fixed array of COAT_NOALLOC_MAX_GROUPS + 1 float32 slots
+ * compiled into the library as a device variable; every GPU that loads the
+ * library holds it until the process exits.  The first call on a device
+ * resolves that array's address for the current device (a one-time,
+ * non-allocating runtime query), so make the first call on each device
+ * before any stream capture.  Every call shares the array: calls that
+ * overlap on the GPU (on different streams, or from different threads
+ * without ordering) race on it and must be serialised by the caller.
+ *   x      BF16 bits [n] (16-byte aligned)
+ *   q      uint8[n] codes (16-byte aligned)
+ *   scale  float32[1], the per-tensor scale s
+ * Errors: INVALID_ARG, MISALIGNED, CUDA, and UNSUPPORTED for an unsupported
+ * format or group size or when ceil(n/G) > COAT_NOALLOC_MAX_GROUPS.
+ */
+coat_status_t coat_group_scaling_quant_pertensor_noalloc(const uint16_t *x, int64_t n,
+                                                         int32_t group_size, int32_t fmt,
+                                                         uint8_t *q, float *scale,
+                                                         void *stream);
+
 /* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
  * this thread (0 if none). */
 int32_t coat_last_cuda_error(void);

@@ -9,11 +9,13 @@ from ._lib import (  # noqa: F401
     COAT_E4M3,
     COAT_E5M2,
     COAT_FORCE_K1,
+    COAT_NOALLOC_MAX_GROUPS,
     CoatError,
     coat_adamw_fp8_step,
     coat_dequant,
     coat_group_quant_1xG,
     coat_group_scaling_quant_pertensor,
+    coat_group_scaling_quant_pertensor_noalloc,
     coat_group_scaling_workspace_bytes,
     coat_quantize_state,
     coat_status_string,

@@ -63,6 +63,7 @@ SIGNATURES = {
     "coat_group_quant_1xG": (_I32, [_P, _I64, _I64, _I64, _I32, _I32, _P, _P, _P]),
     "coat_group_scaling_workspace_bytes": (_I64, [_I64, _I32]),
     "coat_group_scaling_quant_pertensor": (_I32, [_P, _I64, _I32, _I32, _P, _I32, _P, _P, _P]),
+    "coat_group_scaling_quant_pertensor_noalloc": (_I32, [_P, _I64, _I32, _I32, _P, _P, _P]),
     "coat_last_cuda_error": (_I32, []),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
     "coat_version": (_I32, []),
@@ -193,6 +194,20 @@ def coat_group_scaling_quant_pertensor(x, workspace, q, scale, *, group_size: in
         int(bool(amax_precomputed)), _ptr(q, torch.uint8, "q"),
         _ptr(scale, torch.float32, "scale"), _stream(stream))
     _check("coat_group_scaling_quant_pertensor", st)
+
+
+COAT_NOALLOC_MAX_GROUPS = 1 << 20  # mirrors include/coat.h
+
+
+def coat_group_scaling_quant_pertensor_noalloc(x, q, scale, *, group_size: int = 128,
+                                               fmt: int = COAT_E4M3, stream=None):
+    """Group Scaling quantization with the library's own fixed scratch: no
+    workspace argument and no allocation (see include/coat.h)."""
+    import torch
+    st = load().coat_group_scaling_quant_pertensor_noalloc(
+        _u16(x, "x"), x.numel(), group_size, fmt, _ptr(q, torch.uint8, "q"),
+        _ptr(scale, torch.float32, "scale"), _stream(stream))
+    _check("coat_group_scaling_quant_pertensor_noalloc", st)
 
 
 def coat_version() -> int:

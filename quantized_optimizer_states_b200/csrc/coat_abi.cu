@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -319,3 +320,78 @@ const char *coat_status_string(coat_status_t status) {
 int32_t coat_version(void) { return (0 << 16) | (1 << 8) | 0; }
 
 }  // extern "C"
+
+// ---- Group Scaling with library-owned scratch (no allocation) -----------------
+
+namespace {
+
+constexpr int64_t kNoAllocGroups = COAT_NOALLOC_MAX_GROUPS;
+constexpr int kMaxDevices = 64;
+
+// The per-group maxima [0, kNoAllocGroups) and the tensor-max slot
+// [kNoAllocGroups] of the no-allocation variant, shared by all its calls.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocGroups + 1];
+
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, resolved once
+// per device (host code cannot use the symbol's name as an address).
+coat_status_t noalloc_scratch(float **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    g_last_cuda_error = static_cast<int32_t>(e);
+    return COAT_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return COAT_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr) {
+      g_last_cuda_error = static_cast<int32_t>(e);
+      return COAT_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<float *>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return COAT_OK;
+}
+
+}  // namespace
+
+extern "C" coat_status_t coat_group_scaling_quant_pertensor_noalloc(
+    const uint16_t *x, int64_t n, int32_t group_size, int32_t fmt, uint8_t *q, float *scale,
+    void *stream) {
+  if (n < 0) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && (!x || !q || !scale)) return COAT_ERR_INVALID_ARG;
+  const int lg = group_log2(group_size);
+  if (lg < 0 || !valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
+  if (n == 0) return COAT_OK;
+  if (!aligned16(x) || !aligned16(q)) return COAT_ERR_MISALIGNED;
+  const int64_t ng = (n + group_size - 1) / group_size;
+  if (ng > kNoAllocGroups) return COAT_ERR_UNSUPPORTED;
+  float *ws = nullptr;
+  const coat_status_t st = noalloc_scratch(&ws);
+  if (st != COAT_OK) return st;
+  coat::GroupScalingParams p;
+  p.x = x;
+  p.n = n;
+  p.ngroups = ng;
+  p.log2G = lg;
+  p.group_amax = ws;
+  p.tensor_amax = reinterpret_cast<uint32_t *>(ws + kNoAllocGroups);
+  p.q = q;
+  p.scale = scale;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the tensor maximum accumulates with atomicMax and must start at zero
+  if (cudaMemsetAsync(p.tensor_amax, 0, sizeof(uint32_t), s) != cudaSuccess) return launch_status();
+  coat::group_amax_kernel<<<blocks_for(n), coat::kThreads, 0, s>>>(p);
+  const unsigned int grid = blocks_for(n);
+  if (fmt == COAT_E4M3)
+    coat::pertensor_cast_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+  else
+    coat::pertensor_cast_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  return launch_status();
+}

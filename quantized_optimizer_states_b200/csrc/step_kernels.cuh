@@ -114,6 +114,12 @@ __device__ __forceinline__ float sqrt_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float rsqrt_approx(float x) {
+  float y;
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -400,15 +406,17 @@ adamw_fp8_step_kernel(const StepParams p) {
   // m_t and v_t are computed exactly as the rule rounds them (they are the
   // new states): scalar IEEE sums of separately rounded products.  The
   // update quotient u = m^ / (sqrt(v^) + eps) is first formed with
-  // reciprocal estimates (relative error below 1e-6, so lr*u is off by at
-  // most ~1e-6 of itself); wherever |lr*u| is not at least twice below
-  // max(|theta|, lr) that error could matter for theta, and the element is
-  // recomputed with correctly rounded division and square root.
+  // the reciprocal-square-root estimate (relative error below 1e-6, so lr*u
+  // is off by at most ~1e-6 of itself); wherever |lr*u| is not at least twice
+  // below max(|theta|, lr), or eps is not negligible next to sqrt(v^), that
+  // error could matter for theta, and the element is recomputed with
+  // correctly rounded division and square root.
   {
     const float2 C1 = make_float2(p.c1, p.c1), C2 = make_float2(p.c2, p.c2);
     const float2 RB1 = make_float2(p.rbc1, p.rbc1), RB2 = make_float2(p.rbc2, p.rbc2);
     const float2 EPS = make_float2(p.eps, p.eps), DEC = make_float2(p.decay, p.decay);
     const float2 NLR = make_float2(-p.lr, -p.lr), TWO = make_float2(2.0f, 2.0f);
+    const float2 ONE = make_float2(1.0f, 1.0f), MONE = make_float2(-1.0f, -1.0f);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t gword = gw[i];
@@ -420,15 +428,20 @@ adamw_fp8_step_kernel(const StepParams p) {
       mt.y = __fadd_rn(m[2 * i + 1], cg.y);
       vt.x = __fadd_rn(v[2 * i], cgg.x);
       vt.y = __fadd_rn(v[2 * i + 1], cgg.y);
+      // 1 / (sqrt(v^) + eps) = r / (1 + d) with r = 1/sqrt(v^), d = eps r;
+      // for d <= 2^-10, 1 - d + d^2 is within 2^-30 of 1/(1 + d)
       const float2 vh = fmul2(vt, RB2);
-      const float2 den = fadd2(make_float2(sqrt_approx(vh.x), sqrt_approx(vh.y)), EPS);
-      const float2 u = fmul2(fmul2(mt, RB1), make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+      const float2 r = make_float2(rsqrt_approx(vh.x), rsqrt_approx(vh.y));
+      const float2 d = fmul2(EPS, r);
+      const float2 c = ffma2(d, fadd2(d, MONE), ONE);
+      const float2 u = fmul2(fmul2(fmul2(mt, RB1), r), c);
       const float2 th0 = make_float2(th[2 * i], th[2 * i + 1]);
       const float2 t2 = fmul2(NLR, u);
       float2 tn = fadd2(fmul2(th0, DEC), t2);
       const float2 w2 = fmul2(TWO, t2);
       const bool slow = fabsf(w2.x) > fmaxf(fabsf(tn.x), p.lr) ||
-                        fabsf(w2.y) > fmaxf(fabsf(tn.y), p.lr);
+                        fabsf(w2.y) > fmaxf(fabsf(tn.y), p.lr) || !(d.x <= 0x1p-10f) ||
+                        !(d.y <= 0x1p-10f);
       if (__any_sync(0xffffffffu, slow)) {
         if (slow) {
           tn.x = exact_update(th0.x, mt.x, vt.x, p);

@@ -115,6 +115,7 @@ __device__ __forceinline__ float expand_signed(float x, float rM, float k, float
 template <int F>
 __device__ __forceinline__ void encode16(const float *x, const GroupQ &g, float log2_fmax,
                                          uint32_t *out) {
+  // an all-zero group has rM = 0, so every y is 0 and every code 0x00
   const float2 RM = make_float2(g.rM, g.rM), K = make_float2(g.k, g.k);
   const float2 LF = make_float2(log2_fmax, log2_fmax);
 #pragma unroll
@@ -123,13 +124,13 @@ __device__ __forceinline__ void encode16(const float *x, const GroupQ &g, float 
 #pragma unroll
     for (int j = 0; j < 4; j += 2) {
       const float x0 = x[4 * w + j], x1 = x[4 * w + j + 1];
-      const float2 r = fmul2(make_float2(fabsf(x0), fabsf(x1)), RM);
-      const float2 z = ffma2(K, make_float2(lg2_approx(r.x), lg2_approx(r.y)), LF);
+      const float2 r = fmul2(make_float2(x0, x1), RM);
+      const float2 z = ffma2(K, make_float2(lg2_approx(fabsf(r.x)), lg2_approx(fabsf(r.y))), LF);
       y[j] = __uint_as_float(__float_as_uint(ex2_approx(z.x)) | (__float_as_uint(x0) & 0x80000000u));
       y[j + 1] =
           __uint_as_float(__float_as_uint(ex2_approx(z.y)) | (__float_as_uint(x1) & 0x80000000u));
     }
-    out[w] = g.zero ? 0u : float4_to_fp8x4<F>(y[0], y[1], y[2], y[3]);
+    out[w] = float4_to_fp8x4<F>(y[0], y[1], y[2], y[3]);
   }
 }
 
@@ -236,12 +237,12 @@ __device__ __forceinline__ void table_codes(const WarpTables<ENT> &tw, int j, in
   const double *D = tw.D + j * kTabDoubles;
   const float s = tw.S[j];
   const float2 S = make_float2(s, s), BETA = make_float2(beta, beta);
-  const double a = D[0], ai = D[1];
-  double B[8];
-  B[0] = 1.0;
-#pragma unroll
-  for (int f = 2; f < 8; ++f) B[f] = D[f];
-  B[1] = B[4] * B[4] * ai;
+  const double2 aai = reinterpret_cast<const double2 *>(D)[0];
+  const double2 b23 = reinterpret_cast<const double2 *>(D)[1];
+  const double2 b45 = reinterpret_cast<const double2 *>(D)[2];
+  const double2 b67 = reinterpret_cast<const double2 *>(D)[3];
+  const double a = aai.x, ai = aai.y;
+  const double B[8] = {1.0, b45.x * b45.x * ai, b23.x, b23.y, b45.x, b45.y, b67.x, b67.y};
   float r[16];
   const float nan = s != 0.0f ? __int_as_float(0x7fc00000) : 0.0f;
   if (e4) {

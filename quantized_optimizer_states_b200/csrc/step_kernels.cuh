@@ -41,7 +41,6 @@ constexpr int kVec = 16;                           // parameters per thread
 constexpr int kElemsPerBlock = kThreads * kVec;    // 4096
 constexpr int kWarps = kThreads / 32;
 constexpr int kMinTableLog2G = 6;                  // decode tables for G >= 64
-constexpr int kTabEnt = 128;                       // entries per decode table
 
 struct StepParams {
   float *theta;
@@ -82,13 +81,24 @@ struct StepLayout {
   static constexpr int kTablesPerWarp = 2 * kGroupsPerWarp;  // m and v per group
   static constexpr int kJobs = 8 * kTablesPerWarp;           // per phase, per warp
   static constexpr int kRounds = (kJobs + 31) / 32;
-  static constexpr int kWarpBytes = kTable ? warp_table_bytes<kTabEnt>(kTablesPerWarp) : 0;
-  static constexpr int kSmemBytes = kWarps * kWarpBytes;
+  // 128 magnitude entries per table, the code's sign applied at lookup (the
+  // signed 256-entry form measured slower: twice the shared-memory stores)
+  static constexpr int kEnt = 128;
+  static constexpr int kWarpBytes = kTable ? warp_table_bytes<kEnt>(kTablesPerWarp) : 0;
+  // each warp also stages its 512 theta values (2 KB) through shared memory
+  static constexpr int kThetaBytes = 32 * kVec * 4;
+  static constexpr int kWarpTotal = kThetaBytes + kWarpBytes;
+  static constexpr int kSmemBytes = kWarps * kWarpTotal;
+  // resident blocks per SM the register budget is sized for (64 registers
+  // per thread at 4 blocks); G = 64 is held to 2 by its 16 tables per warp
+  static constexpr int kMinBlocks = LG <= 6 ? 2 : (LG == 11 ? 3 : 4);
 };
 
 // Dynamic shared memory of the step kernel for group size 2^log2G.
 inline size_t step_smem_bytes(int log2G) {
   switch (log2G) {
+    case 4: return StepLayout<4>::kSmemBytes;
+    case 5: return StepLayout<5>::kSmemBytes;
     case 6: return StepLayout<6>::kSmemBytes;
     case 7: return StepLayout<7>::kSmemBytes;
     case 8: return StepLayout<8>::kSmemBytes;
@@ -298,8 +308,32 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
 
 // ---- the fused step ----------------------------------------------------------
 
+// theta of one thread (16 values) copied asynchronously into shared memory
+// (cp.async, zero-filled past n), so no registers are held while it loads.
+// The warp's 512 values are stored chunk-major -- chunk c (values 4c..4c+3)
+// of lane l at float4 index 32c + l -- so that every 16-byte access of the
+// warp touches 512 consecutive bytes (no bank conflicts).
+__device__ __forceinline__ void stage_theta(float4 *warp_th, const float *theta, int64_t e0,
+                                            int64_t n, int lane) {
+  const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(warp_th + lane));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int64_t base = e0 + 4 * c;
+    const int bytes = base + 4 <= n ? 16 : (base < n ? static_cast<int>(n - base) * 4 : 0);
+    const float *src = bytes > 0 ? theta + base : theta;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(sa + 512 * c), "l"(src),
+                 "r"(bytes)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void wait_staged() {
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
 template <int VF, int LG>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, StepLayout<LG>::kMinBlocks)
 adamw_fp8_step_kernel(const StepParams p) {
   using L = StepLayout<LG>;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -346,16 +380,15 @@ adamw_fp8_step_kernel(const StepParams p) {
     vs = p.v_s[grp];
   }
 
-  float th[16], m[16], v[16];
+  float4 *th_s = reinterpret_cast<float4 *>(smem + static_cast<size_t>(warp) * L::kWarpTotal);
+  stage_theta(th_s, p.theta, e0, p.n, lane);
+  float m[16], v[16];
   uint32_t gw[8], mw[4], vw[4];
   if (active) {
-    load16_f32(p.theta, e0, p.n, th);
     load16_bf16(p.grad, e0, p.n, gw);
     load16_u8(p.m_code, e0, p.n, mw);
     load16_u8(p.v_code, e0, p.n, vw);
   } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) th[i] = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) gw[i] = 0;
 #pragma unroll
@@ -366,8 +399,8 @@ adamw_fp8_step_kernel(const StepParams p) {
   // ---- beta1 * m and beta2 * v from the stored states (exact binary32) ----
   if constexpr (L::kTable) {
     // warp-local decode tables: [0, GPW) first moment, [GPW, 2 GPW) second
-    const WarpTables<kTabEnt> tw = warp_tables<kTabEnt>(
-        smem + static_cast<size_t>(warp) * L::kWarpBytes, L::kTablesPerWarp);
+    const WarpTables<L::kEnt> tw = warp_tables<L::kEnt>(
+        smem + static_cast<size_t>(warp) * L::kWarpTotal + L::kThetaBytes, L::kTablesPerWarp);
 #pragma unroll
     for (int r = 0; r < L::kRounds; ++r) {
       const int job = lane + 32 * r;
@@ -385,8 +418,8 @@ adamw_fp8_step_kernel(const StepParams p) {
     }
     __syncwarp();
     const int lg = L::kGroupsPerWarp > 1 ? (lane >> (LG - 4)) : 0;
-    lookup16<kTabEnt>(tw.ent + lg * kTabEnt, mw, m);
-    lookup16<kTabEnt>(tw.ent + (L::kGroupsPerWarp + lg) * kTabEnt, vw, v);
+    lookup16<L::kEnt>(tw.ent + lg * L::kEnt, mw, m);
+    lookup16<L::kEnt>(tw.ent + (L::kGroupsPerWarp + lg) * L::kEnt, vw, v);
   } else {
     const double mrk = 1.0 / static_cast<double>(mk), vrk = 1.0 / static_cast<double>(vk);
 #pragma unroll
@@ -417,46 +450,62 @@ adamw_fp8_step_kernel(const StepParams p) {
     const float2 EPS = make_float2(p.eps, p.eps), DEC = make_float2(p.decay, p.decay);
     const float2 NLR = make_float2(-p.lr, -p.lr), TWO = make_float2(2.0f, 2.0f);
     const float2 ONE = make_float2(1.0f, 1.0f), MONE = make_float2(-1.0f, -1.0f);
+    wait_staged();
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t gword = gw[i];
-      const float2 g = make_float2(bf16lo_to_float(gword), bf16hi_to_float(gword));
-      const float2 cg = fmul2(C1, g);
-      const float2 cgg = fmul2(C2, fmul2(g, g));
-      float2 mt, vt;
-      mt.x = __fadd_rn(m[2 * i], cg.x);
-      mt.y = __fadd_rn(m[2 * i + 1], cg.y);
-      vt.x = __fadd_rn(v[2 * i], cgg.x);
-      vt.y = __fadd_rn(v[2 * i + 1], cgg.y);
-      // 1 / (sqrt(v^) + eps) = r / (1 + d) with r = 1/sqrt(v^), d = eps r;
-      // for d <= 2^-10, 1 - d + d^2 is within 2^-30 of 1/(1 + d)
-      const float2 vh = fmul2(vt, RB2);
-      const float2 r = make_float2(rsqrt_approx(vh.x), rsqrt_approx(vh.y));
-      const float2 d = fmul2(EPS, r);
-      const float2 c = ffma2(d, fadd2(d, MONE), ONE);
-      const float2 u = fmul2(fmul2(fmul2(mt, RB1), r), c);
-      const float2 th0 = make_float2(th[2 * i], th[2 * i + 1]);
-      const float2 t2 = fmul2(NLR, u);
-      float2 tn = fadd2(fmul2(th0, DEC), t2);
-      const float2 w2 = fmul2(TWO, t2);
-      const bool slow = fabsf(w2.x) > fmaxf(fabsf(tn.x), p.lr) ||
-                        fabsf(w2.y) > fmaxf(fabsf(tn.y), p.lr) || !(d.x <= 0x1p-10f) ||
-                        !(d.y <= 0x1p-10f);
-      if (__any_sync(0xffffffffu, slow)) {
-        if (slow) {
-          tn.x = exact_update(th0.x, mt.x, vt.x, p);
-          tn.y = exact_update(th0.y, mt.y, vt.y, p);
+    for (int c = 0; c < 4; ++c) {
+      const float4 th4 = th_s[32 * c + lane];
+      float2 out[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = 2 * c + h;
+        const uint32_t gword = gw[i];
+        const float2 g = make_float2(bf16lo_to_float(gword), bf16hi_to_float(gword));
+        const float2 cg = fmul2(C1, g);
+        const float2 cgg = fmul2(C2, fmul2(g, g));
+        float2 mt, vt;
+        mt.x = __fadd_rn(m[2 * i], cg.x);
+        mt.y = __fadd_rn(m[2 * i + 1], cg.y);
+        vt.x = __fadd_rn(v[2 * i], cgg.x);
+        vt.y = __fadd_rn(v[2 * i + 1], cgg.y);
+        // 1 / (sqrt(v^) + eps) = r / (1 + d) with r = 1/sqrt(v^), d = eps r;
+        // for d <= 2^-10, 1 - d + d^2 is within 2^-30 of 1/(1 + d)
+        const float2 vh = fmul2(vt, RB2);
+        const float2 r = make_float2(rsqrt_approx(vh.x), rsqrt_approx(vh.y));
+        const float2 d = fmul2(EPS, r);
+        const float2 cc = ffma2(d, fadd2(d, MONE), ONE);
+        const float2 u = fmul2(fmul2(fmul2(mt, RB1), r), cc);
+        const float2 th0 = h ? make_float2(th4.z, th4.w) : make_float2(th4.x, th4.y);
+        const float2 t2 = fmul2(NLR, u);
+        float2 tn = fadd2(fmul2(th0, DEC), t2);
+        const float2 w2 = fmul2(TWO, t2);
+        const bool slow = fabsf(w2.x) > fmaxf(fabsf(tn.x), p.lr) ||
+                          fabsf(w2.y) > fmaxf(fabsf(tn.y), p.lr) || !(d.x <= 0x1p-10f) ||
+                          !(d.y <= 0x1p-10f);
+        if (__any_sync(0xffffffffu, slow)) {
+          if (slow) {
+            tn.x = exact_update(th0.x, mt.x, vt.x, p);
+            tn.y = exact_update(th0.y, mt.y, vt.y, p);
+          }
+        }
+        out[h] = tn;
+        m[2 * i] = mt.x;
+        m[2 * i + 1] = mt.y;
+        v[2 * i] = vt.x;
+        v[2 * i + 1] = vt.y;
+      }
+      if (active) {
+        const int64_t base = e0 + 4 * c;
+        if (base + 4 <= p.n) {
+          *reinterpret_cast<float4 *>(p.theta + base) =
+              make_float4(out[0].x, out[0].y, out[1].x, out[1].y);
+        } else {
+          const float o[4] = {out[0].x, out[0].y, out[1].x, out[1].y};
+          for (int j = 0; j < 4; ++j)
+            if (base + j < p.n) p.theta[base + j] = o[j];
         }
       }
-      th[2 * i] = tn.x;
-      th[2 * i + 1] = tn.y;
-      m[2 * i] = mt.x;
-      m[2 * i + 1] = mt.y;
-      v[2 * i] = vt.x;
-      v[2 * i + 1] = vt.y;
     }
   }
-  if (active) store16_f32(p.theta, e0, p.n, th);
 
   // tail elements beyond n must not take part in the group range
   if (e0 + 16 > p.n) {

@@ -307,9 +307,19 @@ __device__ __forceinline__ void table_codes(const WarpTables<ENT> &tw, int j, in
       r[15] = nan;
     }
   }
+  // the eight jobs of a table (q = 0..7) store their 64-byte runs in a
+  // rotated chunk order, so that each store instruction of eight lanes
+  // touches eight different 16-byte bank groups (no bank conflicts)
   float4 *pos = reinterpret_cast<float4 *>(tw.ent + j * ENT + 16 * q);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) pos[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+  for (int i = 0; i < 4; ++i) {
+    const int c = (i + (q >> 1)) & 3;
+    const float4 v = c == 0   ? make_float4(r[0], r[1], r[2], r[3])
+                     : c == 1 ? make_float4(r[4], r[5], r[6], r[7])
+                     : c == 2 ? make_float4(r[8], r[9], r[10], r[11])
+                              : make_float4(r[12], r[13], r[14], r[15]);
+    pos[c] = v;
+  }
   if constexpr (ENT == 256) {
     float4 *neg = reinterpret_cast<float4 *>(tw.ent + j * ENT + 128 + 16 * q);
 #pragma unroll

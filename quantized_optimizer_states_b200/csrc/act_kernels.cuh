@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const GroupScaling
   uint32_t w[8];
   float x[16];
   if (active) {
-    load16_bf16(p.x, e0, p.n, w);
+    load16_bf16<false>(p.x, e0, p.n, w);
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) w[i] = 0;
@@ -188,11 +188,11 @@ __global__ void __launch_bounds__(kThreads) pertensor_cast_kernel(const GroupSca
   if (e0 >= p.n) return;
   uint32_t w[8];
   float x[16];
-  load16_bf16(p.x, e0, p.n, w);
+  load16_bf16<false>(p.x, e0, p.n, w);
   unpack16_bf16(w, x);
   uint32_t o[4];
   cast16<F>(x, inv, o);
-  store16_u8(p.q, e0, p.n, o);
+  store16_u8<false>(p.q, e0, p.n, o);
 }
 
 // ---- dequantization ----------------------------------------------------------------
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p
   const float kk = p.k ? p.k[grp] : 1.0f;
   const double rk = 1.0 / static_cast<double>(kk);
   uint32_t w[4];
-  load16_u8(p.q, e0, p.n, w);
+  load16_u8<false>(p.q, e0, p.n, w);
   float x[16];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p
         if (e0 + i < p.n) o[e0 + i] = static_cast<uint16_t>(float_to_bf16_rn(x[i]));
     }
   } else {
-    store16_f32(static_cast<float *>(p.out), e0, p.n, x);
+    store16_f32<false>(static_cast<float *>(p.out), e0, p.n, x);
   }
 }
 

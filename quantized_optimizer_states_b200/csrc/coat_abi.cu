@@ -65,7 +65,7 @@ unsigned int blocks_for(int64_t elems) {
   return static_cast<unsigned int>((elems + coat::kElemsPerBlock - 1) / coat::kElemsPerBlock);
 }
 
-constexpr int64_t kMaxElems = int64_t{1} << 44;  // grid-size bound (2^31 blocks x 4096)
+constexpr int64_t kMaxElems = int64_t{1} << 42;  // within the grid-size bound (2^31 - 1 blocks x 4096)
 
 // Launch one instantiation of the step kernel, raising its dynamic shared
 // memory limit first when the decode tables need more than the default.
@@ -83,22 +83,42 @@ coat_status_t launch_step(void (*kernel)(coat::StepParams), unsigned int grid, s
   return launch_status();
 }
 
-// The step kernel is instantiated for each supported group size.
-template <int VF>
+// The step kernel is instantiated for each supported group size and for
+// full blocks / the ragged tail block.
+template <int VF, bool FULL>
 coat_status_t launch_step_for(int lg, unsigned int grid, size_t smem, cudaStream_t s,
                               const coat::StepParams &p) {
   switch (lg) {
-    case 4: return launch_step(coat::adamw_fp8_step_kernel<VF, 4>, grid, smem, s, p);
-    case 5: return launch_step(coat::adamw_fp8_step_kernel<VF, 5>, grid, smem, s, p);
-    case 6: return launch_step(coat::adamw_fp8_step_kernel<VF, 6>, grid, smem, s, p);
-    case 7: return launch_step(coat::adamw_fp8_step_kernel<VF, 7>, grid, smem, s, p);
-    case 8: return launch_step(coat::adamw_fp8_step_kernel<VF, 8>, grid, smem, s, p);
-    case 9: return launch_step(coat::adamw_fp8_step_kernel<VF, 9>, grid, smem, s, p);
-    case 10: return launch_step(coat::adamw_fp8_step_kernel<VF, 10>, grid, smem, s, p);
-    case 11: return launch_step(coat::adamw_fp8_step_kernel<VF, 11>, grid, smem, s, p);
-    case 12: return launch_step(coat::adamw_fp8_step_kernel<VF, 12>, grid, smem, s, p);
+    case 4: return launch_step(coat::adamw_fp8_step_kernel<VF, 4, FULL>, grid, smem, s, p);
+    case 5: return launch_step(coat::adamw_fp8_step_kernel<VF, 5, FULL>, grid, smem, s, p);
+    case 6: return launch_step(coat::adamw_fp8_step_kernel<VF, 6, FULL>, grid, smem, s, p);
+    case 7: return launch_step(coat::adamw_fp8_step_kernel<VF, 7, FULL>, grid, smem, s, p);
+    case 8: return launch_step(coat::adamw_fp8_step_kernel<VF, 8, FULL>, grid, smem, s, p);
+    case 9: return launch_step(coat::adamw_fp8_step_kernel<VF, 9, FULL>, grid, smem, s, p);
+    case 10: return launch_step(coat::adamw_fp8_step_kernel<VF, 10, FULL>, grid, smem, s, p);
+    case 11: return launch_step(coat::adamw_fp8_step_kernel<VF, 11, FULL>, grid, smem, s, p);
+    case 12: return launch_step(coat::adamw_fp8_step_kernel<VF, 12, FULL>, grid, smem, s, p);
   }
   return COAT_ERR_UNSUPPORTED;
+}
+
+// One launch over the full 4096-parameter blocks (no bounds checks), then,
+// if n is not a multiple of 4096, one block for the ragged tail.
+template <int VF>
+coat_status_t launch_step_all(int lg, int64_t n, size_t smem, cudaStream_t s,
+                              coat::StepParams p) {
+  const int64_t full = n / coat::kElemsPerBlock;
+  if (full > 0) {
+    p.block0 = 0;
+    const coat_status_t st =
+        launch_step_for<VF, true>(lg, static_cast<unsigned int>(full), smem, s, p);
+    if (st != COAT_OK) return st;
+  }
+  if (n % coat::kElemsPerBlock != 0) {
+    p.block0 = full;
+    return launch_step_for<VF, false>(lg, 1u, smem, s, p);
+  }
+  return COAT_OK;
 }
 
 }  // namespace
@@ -161,11 +181,25 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
   fill_log2_table(p.log2_tab);
   if (!(p.bc1 > 0.0f) || !(p.bc2 > 0.0f)) return COAT_ERR_INVALID_ARG;
 
+  // Bounds of the estimate-based quotient (see step_kernels.cuh): v^ = v_t / bc2
+  // within [2^-120, 2^100] keeps the rsqrt / rcp estimates on normal
+  // numbers, and |m_t| <= 2^100 bc1 eps keeps m^ / (sqrt(v^) + eps) below
+  // 2^100.  A non-normal eps disables the fast form.
+  p.block0 = 0;
+  if (p.eps >= 0x1p-100f && p.eps <= 0x1p+20f) {
+    p.fast_vmin = 0x1p-120f;
+    p.fast_vmax = static_cast<float>(std::ldexp(static_cast<double>(p.bc2), 100));
+    p.fast_mmax = static_cast<float>(std::ldexp(static_cast<double>(p.bc1) * p.eps, 100));
+  } else {
+    p.fast_vmin = 0.0f;
+    p.fast_vmax = 0.0f;
+    p.fast_mmax = -1.0f;
+  }
+
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const unsigned int grid = blocks_for(n);
   const size_t smem = coat::step_smem_bytes(lg);
-  return cfg->v_fmt == COAT_E4M3 ? launch_step_for<coat::kE4M3>(lg, grid, smem, s, p)
-                                 : launch_step_for<coat::kE5M2>(lg, grid, smem, s, p);
+  return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3>(lg, n, smem, s, p)
+                                 : launch_step_all<coat::kE5M2>(lg, n, smem, s, p);
 }
 
 coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size, int32_t fmt,

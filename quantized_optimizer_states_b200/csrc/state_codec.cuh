@@ -152,197 +152,132 @@ __device__ __forceinline__ float dequant_exact(float d, float s, double rk, cons
   return d < 0.0f ? -x : x;
 }
 
-// ---- per-group dequantization tables --------------------------------------------
-// For a group with exponent k and scale s, entry c holds
-// RN32(RN32(|d_c|^(1/k)) * s) with the sign of code c.  |d_c| = (1 + f/8) 2^e,
-// so |d_c|^(1/k) = A(e) B(f) with A(e) = a^e, a = 2^(1/k), and
-// B(f) = 2^(log2(1 + f/8) / k), all in binary64: a, 1/a and B(2..7) come from
-// exp2_d, B(1) = B(4)^2 / a (since 1.5^2 = 2 * 1.125), and a^e from at most
-// four squarings and four products, so every entry is within ~2^-48 of the
-// exact power before the binary32 roundings of the definition.
+// ---- per-group decode tables ---------------------------------------------------
+// For a group with exponent k and scale s, entry c (c = 0..127: a code
+// without its sign bit) holds RN32(RN32(RN32(|d_c|^(1/k)) * s) * beta): the
+// decoded moment already multiplied by its beta, the first product of the
+// moment update (beta = 1 gives the plain decode).  A lookup applies the
+// code's sign.
 //
-// Every warp builds the tables of the groups its threads touch (with only
-// warp-level synchronisation): 2 per group (m, v), 256 signed entries each
-// (ENT == 256) or 128 magnitude entries plus a sign fix-up at lookup time
-// (ENT == 128, used when a warp holds many small groups).
-constexpr int kTabDoubles = 8;   // a, 1/a, B(2..7)
+// Layout: a table takes 512 bytes at a 512-byte-aligned offset of the
+// kernel's dynamic shared memory; entry c sits at byte (4c) XOR swz, with
+// swz = 32 (j & 3) for the warp's table j.  The XOR sends the simultaneous
+// stores of the build (below) to distinct banks, while a lookup still forms
+// its address with one bitwise operation: (4c) ^ (table offset | swz).
+//
+// Build: the L lanes of a table (L = 4, 8 or 16) own the normal codes
+// c0 + 2L i and c0 + 2L i + 1, with c0 = first + 2t for lane t (first = 8 for
+// E4M3, whose codes 8..127 are normal; 4 for E5M2, codes 4..123).  A normal
+// code is (1 + f 2^-mb) 2^e, so |d|^(1/k) = 2^((e + log2(1 + f 2^-mb)) / k),
+// and the values of one lane advance by the constant factor M = 2^(H/k), H
+// the binades per step (L/4 for E4M3, L/2 for E5M2).  A lane evaluates its
+// two starting powers and a = 2^(1/k) with the binary64 exp2 and steps them
+// with binary64 products: after at most 15 steps each is within ~2^-47 of
+// the exact power, so its rounding to binary32 is the correctly rounded
+// power except in vanishingly rare cases.  Code 0, the subnormal codes and
+// the inf / NaN codes are set from their own definitions by lanes 0..3.
+constexpr int kTableBytes = 512;
 
-template <int ENT>
-struct WarpTables {
-  float *ent;    // [TW][ENT]
-  double *D;     // [TW][8]: a, 1/a, B(2), ..., B(7)
-  float *S;      // [TW] scale s
-};
+// log2(1 + i/8), i = 0..7, binary64
+__constant__ double c_log2_1p8th[8] = {
+    0.0, 0x1.5c01a39fbd688p-3, 0x1.49a784bcd1b8bp-2, 0x1.d6753e032ea0fp-2,
+    0x1.2b803473f7ad1p-1, 0x1.66a008e4788ccp-1, 0x1.9d5d9fd5010b3p-1, 0x1.d053f6d260896p-1};
 
-template <int ENT>
-__host__ __device__ constexpr int warp_table_bytes(int TW) {
-  return ((TW * (ENT * 4 + kTabDoubles * 8 + 4)) + 15) / 16 * 16;
+// RN32(RN32(RN32(q) * s) * beta)
+__device__ __forceinline__ float table_entry(double q, float s, float beta) {
+  return __fmul_rn(__fmul_rn(static_cast<float>(q), s), beta);
 }
 
-template <int ENT>
-__device__ __forceinline__ WarpTables<ENT> warp_tables(unsigned char *base, int TW) {
-  WarpTables<ENT> v;
-  v.ent = reinterpret_cast<float *>(base);
-  v.D = reinterpret_cast<double *>(base + static_cast<size_t>(TW) * ENT * 4);
-  v.S = reinterpret_cast<float *>(v.D + static_cast<size_t>(TW) * kTabDoubles);
-  return v;
+__device__ __forceinline__ void st_shared_f32(unsigned char *smem, uint32_t off, float v) {
+  *reinterpret_cast<float *>(smem + off) = v;
 }
 
-// b^|e| with b = a (e >= 0) or 1/a (e < 0), |e| < 2^BITS, by square-and-multiply.
-template <int BITS>
-__device__ __forceinline__ double ipow(double a, double ai, int e) {
-  double base = e >= 0 ? a : ai;
-  int n = e >= 0 ? e : -e;
-  double r = 1.0;
-#pragma unroll
-  for (int bit = 0; bit < BITS; ++bit) {
-    const double t = r * base;
-    r = (n & 1) ? t : r;
-    base *= base;
-    n >>= 1;
-  }
-  return r;
+__device__ __forceinline__ void st_shared_f32x2(unsigned char *smem, uint32_t off, float2 v) {
+  *reinterpret_cast<float2 *>(smem + off) = v;
 }
 
-__device__ __forceinline__ float entry_value(double A, double B, float s) {
-  return __fmul_rn(static_cast<float>(A * B), s);
-}
-
-// The decode of a pair of codes, optionally scaled by the caller's factor:
-// RN32(RN32(RN32(A B) * s) * beta), two lanes at a time (products only).
-__device__ __forceinline__ float2 entry_pair(double A0, double B0, double A1, double B1, float2 S,
-                                             float2 BETA) {
-  const float2 p = make_float2(static_cast<float>(A0 * B0), static_cast<float>(A1 * B1));
-  return fmul2(fmul2(p, S), BETA);
-}
-
-// Phase 1 for one job of a warp: table j, slot f (0 = a, 1 = 1/a, 2..7 =
-// B(f)).  mult8 = {1, -1, log2(1 + f/8) for f = 2..7}.
-template <int ENT>
-__device__ __forceinline__ void table_slot(const WarpTables<ENT> &tw, int j, int f, float k,
-                                           float s, const double *mult8) {
+// Lane t (0 <= t < L) of the L lanes that build one table.  key = the
+// table's offset in `smem` (a multiple of 512) | swz.  The caller
+// synchronises the warp before the first lookup.
+template <int L>
+__device__ __forceinline__ void build_table(unsigned char *smem, uint32_t key, int t, bool e4,
+                                            float k, float s, float beta) {
+  static_assert(L == 4 || L == 8 || L == 16, "lanes per table");
   const double rk = recip_d(static_cast<double>(k));
-  tw.D[j * kTabDoubles + f] = exp2_d(mult8[f] * rk);
-  if (f == 0) tw.S[j] = s;
-}
+  const int c0 = (e4 ? 8 : 4) + 2 * t;
+  const int ex = e4 ? (c0 >> 3) - 7 : (c0 >> 2) - 15;  // exponent of the lane's first binade
+  const int i0 = e4 ? (c0 & 7) : 2 * (c0 & 3);         // log2 index of its two codes
+  const int i1 = e4 ? i0 + 1 : i0 + 2;
+  const double ed = static_cast<double>(ex);
+  double P0 = exp2_d((ed + c_log2_1p8th[i0]) * rk);
+  double P1 = exp2_d((ed + c_log2_1p8th[i1]) * rk);
+  const double a = exp2_d(rk);
+  double M = a;
+#pragma unroll
+  for (int h = 4; h < L; h <<= 1) M *= M;  // a^(L/4)
+  if (!e4) M *= M;                         // E5M2 steps twice as many binades
+  const float nanv = s != 0.0f ? __int_as_float(0x7fc00000) : 0.0f;
+  const float infv = s != 0.0f ? __int_as_float(0x7f800000) : 0.0f;
 
-// Phase 2 for one job: the sixteen codes 16q .. 16q+15 of table j, whose
-// format is E4M3 (e4) or E5M2, each entry multiplied by beta (the table
-// then holds beta * x, the first product of the moment update; beta = 1
-// gives the plain decode).  Code 0 and the subnormal codes (q == 0) and the
-// inf / NaN codes (q == 7) are set from their own definitions.
-template <int ENT>
-__device__ __forceinline__ void table_codes(const WarpTables<ENT> &tw, int j, int q, bool e4,
-                                            float beta) {
-  const double *D = tw.D + j * kTabDoubles;
-  const float s = tw.S[j];
-  const float2 S = make_float2(s, s), BETA = make_float2(beta, beta);
-  const double2 aai = reinterpret_cast<const double2 *>(D)[0];
-  const double2 b23 = reinterpret_cast<const double2 *>(D)[1];
-  const double2 b45 = reinterpret_cast<const double2 *>(D)[2];
-  const double2 b67 = reinterpret_cast<const double2 *>(D)[3];
-  const double a = aai.x, ai = aai.y;
-  const double B[8] = {1.0, b45.x * b45.x * ai, b23.x, b23.y, b45.x, b45.y, b67.x, b67.y};
-  float r[16];
-  const float nan = s != 0.0f ? __int_as_float(0x7fc00000) : 0.0f;
-  if (e4) {
-    // binades 2q, 2q+1: exponents 2q-7, 2q-6 (binade 0 holds the subnormals)
-    const double A0 = ipow<3>(a, ai, 2 * q - 7);
-    const double A1 = A0 * a;
-#pragma unroll
-    for (int f = 0; f < 8; f += 2) {
-      const float2 lo = entry_pair(A0, B[f], A0, B[f + 1], S, BETA);
-      const float2 hi = entry_pair(A1, B[f], A1, B[f + 1], S, BETA);
-      r[f] = lo.x;
-      r[f + 1] = lo.y;
-      r[8 + f] = hi.x;
-      r[9 + f] = hi.y;
+  // Code 0 and the subnormal codes, from the lane's starting power P0
+  // (binade 1): E4M3 code w is w 2^-9, E5M2 code w is w 2^-16.  The inf
+  // (E5M2 0x7C) and NaN codes hold inf / NaN (0 in an all-zero group).
+  if (t < 4) {
+    const double ai = recip_d(a);
+    const double q1 = P0 * ai, q2 = q1 * ai, q3 = q2 * ai;
+    const float v1 = table_entry(q1, s, beta), v2 = table_entry(q2, s, beta);
+    const float v3 = table_entry(q3, s, beta);
+    // E4M3: lane 0 (P0 = 2^(-6/k)): 0, 2^-9, 2^-8, 2^-7 at codes 0, 1, 2, 4;
+    // lane 1 (1.25 2^-6): code 5; lane 2 (1.5 2^-6): codes 3, 6; lane 3 (1.75 2^-6): code 7.
+    // E5M2: lane 0 (2^(-14/k)): 0, 2^-16, 2^-15 at codes 0, 1, 2; lane 1
+    // (1.5 2^-14): code 3; lanes 2, 3: codes 124..127 (inf, NaN x 3).
+    if (t == 0 || (!e4 && t >= 2)) {
+      const int pc = t == 0 ? 0 : (t == 2 ? 124 : 126);
+      const float2 pv = t == 0 ? make_float2(0.0f, e4 ? v3 : v2)
+                               : make_float2(t == 2 ? infv : nanv, nanv);
+      st_shared_f32x2(smem, (4u * pc) ^ key, pv);
     }
-    if (q == 0) {
-      // code w = w * 2^-9: 1 -> 2^-9, 2 -> 2^-8, 3 -> 1.5 2^-8, 4 -> 2^-7,
-      // 5 -> 1.25 2^-7, 6 -> 1.5 2^-7, 7 -> 1.75 2^-7; A0 = A(-7)
-      const double Am8 = A0 * ai, Am9 = Am8 * ai;
-      const float2 e12 = entry_pair(Am9, 1.0, Am8, 1.0, S, BETA);
-      const float2 e34 = entry_pair(Am8, B[4], A0, 1.0, S, BETA);
-      const float2 e56 = entry_pair(A0, B[2], A0, B[4], S, BETA);
-      const float2 e70 = entry_pair(A0, B[6], A0, B[6], S, BETA);
-      r[0] = 0.0f;
-      r[1] = e12.x;
-      r[2] = e12.y;
-      r[3] = e34.x;
-      r[4] = e34.y;
-      r[5] = e56.x;
-      r[6] = e56.y;
-      r[7] = e70.x;
+    if (e4 || t < 2) {
+      const int sc = e4 ? (t == 0 ? 2 : (t == 1 ? 5 : (t == 2 ? 3 : 7))) : (t == 0 ? 2 : 3);
+      const float sv = (e4 && !(t & 1)) ? v2 : v1;
+      st_shared_f32(smem, (4u * sc) ^ key, sv);
     }
-    if (q == 7) r[15] = nan;  // 0x7F
-  } else {
-    // binades 4q .. 4q+3: exponents 4q-15 .. 4q-12 (binade 0: subnormals,
-    // binade 31: inf and NaN)
-    double A = ipow<4>(a, ai, 4 * q - 15);
-    const double A0 = A;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const float2 lo = entry_pair(A, B[0], A, B[2], S, BETA);
-      const float2 hi = entry_pair(A, B[4], A, B[6], S, BETA);
-      r[4 * b] = lo.x;
-      r[4 * b + 1] = lo.y;
-      r[4 * b + 2] = hi.x;
-      r[4 * b + 3] = hi.y;
-      A *= a;
-    }
-    if (q == 0) {
-      // code w = w * 2^-16: 1 -> 2^-16, 2 -> 2^-15, 3 -> 1.5 2^-15; A0 = A(-15)
-      const float2 e12 = entry_pair(A0 * ai, 1.0, A0, 1.0, S, BETA);
-      const float2 e33 = entry_pair(A0, B[4], A0, B[4], S, BETA);
-      r[0] = 0.0f;
-      r[1] = e12.x;
-      r[2] = e12.y;
-      r[3] = e33.x;
-    }
-    if (q == 7) {
-      r[12] = s != 0.0f ? __int_as_float(0x7f800000) : 0.0f;  // 0x7C
-      r[13] = nan;
-      r[14] = nan;
-      r[15] = nan;
-    }
+    if (e4 && !(t & 1)) st_shared_f32(smem, (4u * (t == 0 ? 4 : 6)) ^ key, v1);
   }
-  // the eight jobs of a table (q = 0..7) store their 64-byte runs in a
-  // rotated chunk order, so that each store instruction of eight lanes
-  // touches eight different 16-byte bank groups (no bank conflicts)
-  float4 *pos = reinterpret_cast<float4 *>(tw.ent + j * ENT + 16 * q);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = (i + (q >> 1)) & 3;
-    const float4 v = c == 0   ? make_float4(r[0], r[1], r[2], r[3])
-                     : c == 1 ? make_float4(r[4], r[5], r[6], r[7])
-                     : c == 2 ? make_float4(r[8], r[9], r[10], r[11])
-                              : make_float4(r[12], r[13], r[14], r[15]);
-    pos[c] = v;
-  }
-  if constexpr (ENT == 256) {
-    float4 *neg = reinterpret_cast<float4 *>(tw.ent + j * ENT + 128 + 16 * q);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      neg[i] = make_float4(-r[4 * i], -r[4 * i + 1], -r[4 * i + 2], -r[4 * i + 3]);
-  }
-}
 
-// Table lookup for the 16 codes held in four words (element 0 in the low
-// byte of w[0]).
-template <int ENT>
-__device__ __forceinline__ void lookup16(const float *ent, const uint32_t *w, float *x) {
+  // the normal codes
+  constexpr int NI = (120 + 2 * L - 1) / (2 * L);
+  const float2 S = make_float2(s, s), B = make_float2(beta, beta);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t word = w[i >> 2];
-    const int sh = 8 * (i & 3);
-    if constexpr (ENT == 256) {
-      x[i] = ent[(word >> sh) & 0xFFu];
+  for (int i = 0; i < NI; ++i) {
+    const int c = c0 + 2 * L * i;
+    float2 v = fmul2(fmul2(make_float2(static_cast<float>(P0), static_cast<float>(P1)), S), B);
+    if (i == NI - 1) {
+      if (e4 && c == 126) v.y = nanv;  // E4M3 0x7F is NaN
+      if (c < (e4 ? 128 : 124)) st_shared_f32x2(smem, (4u * c) ^ key, v);
     } else {
-      const uint32_t c = (word >> sh) & 0x7Fu;
-      const uint32_t sign = (word << (24 - sh)) & 0x80000000u;
-      x[i] = __uint_as_float(__float_as_uint(ent[c]) | sign);
+      st_shared_f32x2(smem, (4u * c) ^ key, v);
     }
+    P0 *= M;
+    P1 *= M;
+  }
+}
+
+// x[i] = sign(code i) * entry(|code i|) for the 16 codes in w[0..3] (element
+// 0 in the low byte of w[0]); key = table offset | swz.
+__device__ __forceinline__ void lookup16(const unsigned char *smem, uint32_t key,
+                                         const uint32_t *w, float *x) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t wd = w[q];
+    const float e0 = *reinterpret_cast<const float *>(smem + (((wd << 2) & 0x1FCu) ^ key));
+    const float e1 = *reinterpret_cast<const float *>(smem + (((wd >> 6) & 0x1FCu) ^ key));
+    const float e2 = *reinterpret_cast<const float *>(smem + (((wd >> 14) & 0x1FCu) ^ key));
+    const float e3 = *reinterpret_cast<const float *>(smem + (((wd >> 22) & 0x1FCu) ^ key));
+    x[4 * q + 0] = __uint_as_float(__float_as_uint(e0) | ((wd << 24) & 0x80000000u));
+    x[4 * q + 1] = __uint_as_float(__float_as_uint(e1) | ((wd << 16) & 0x80000000u));
+    x[4 * q + 2] = __uint_as_float(__float_as_uint(e2) | ((wd << 8) & 0x80000000u));
+    x[4 * q + 3] = __uint_as_float(__float_as_uint(e3) | (wd & 0x80000000u));
   }
 }
 

@@ -22,10 +22,21 @@
 // range depends on the smallest |m_t|, which cancellation in
 // beta1*m + (1-beta1)*g makes sensitive to the last bit).  For G >= 64 every
 // warp first builds, in shared memory, the 128-entry decode table of each of
-// its (group, moment) pairs from binary64 factors -- holding beta1*m or
-// beta2*v directly -- so an element costs one table lookup; for G < 64 each
-// element is decoded directly in binary64.  The kernel is instantiated per
-// group size, so lane counts, table counts and shifts are compile-time.
+// its (group, moment) pairs (binary64 power chains, state_codec.cuh) --
+// holding beta1*m or beta2*v directly -- so an element costs one table
+// lookup; for G < 64 each element is decoded directly in binary64.
+//
+// The update quotient u = m^ / (sqrt(v^) + eps) is evaluated branch-free with
+// one correction step per operation (division by the bias corrections with
+// their correctly rounded reciprocals, the square root from the rsqrt
+// estimate, the quotient from the rcp estimate), each of which yields the
+// correctly rounded result except in vanishingly rare near-midpoint cases;
+// a warp whose moments fall outside the range where those estimates are
+// valid (zero-free tiny, huge or infinite values) takes the fully IEEE path.
+//
+// The kernel is instantiated per group size, so lane counts, table counts
+// and shifts are compile-time, and per launch shape: full blocks (no bounds
+// checks) and the one ragged tail block of a launch.
 #pragma once
 
 #include <cstdint>
@@ -35,6 +46,7 @@
 #include "state_codec.cuh"
 
 namespace coat {
+
 
 constexpr int kThreads = 256;
 constexpr int kVec = 16;                           // parameters per thread
@@ -53,7 +65,13 @@ struct StepParams {
   float *v_s;
   int64_t n;
   int64_t ngroups;
+  int64_t block0;     // index of this launch's first block of kElemsPerBlock parameters
   float beta1, beta2, c1, c2, bc1, bc2, rbc1, rbc2, decay, lr, eps;
+  // The estimate-based quotient is used for a thread's 16 elements when
+  // max|m_t| <= fast_mmax, max v_t <= fast_vmax and every nonzero v_t >=
+  // fast_vmin (bounds from the bias corrections and eps); otherwise, or when
+  // fast_mmax < 0, the warp takes the fully IEEE path.
+  float fast_mmax, fast_vmin, fast_vmax;
   float k_max;        // <= 0: no clamp
   int force_k1;
   StateFmtParams m, v;
@@ -77,17 +95,14 @@ template <int LG>
 struct StepLayout {
   static constexpr int kLanes = 1 << (LG - 4);               // threads per group
   static constexpr bool kTable = LG >= kMinTableLog2G;
-  static constexpr int kGroupsPerWarp = LG <= 9 ? (512 >> LG) : 1;
-  static constexpr int kTablesPerWarp = 2 * kGroupsPerWarp;  // m and v per group
-  static constexpr int kJobs = 8 * kTablesPerWarp;           // per phase, per warp
-  static constexpr int kRounds = (kJobs + 31) / 32;
-  // 128 magnitude entries per table, the code's sign applied at lookup (the
-  // signed 256-entry form measured slower: twice the shared-memory stores)
-  static constexpr int kEnt = 128;
-  static constexpr int kWarpBytes = kTable ? warp_table_bytes<kEnt>(kTablesPerWarp) : 0;
+  static constexpr int kGPW = LG <= 9 ? (512 >> LG) : 1;     // groups a warp touches
+  static constexpr int kTW = 2 * kGPW;                       // tables per warp (m and v)
+  static constexpr int kL = kTW >= 8 ? 4 : 32 / kTW;         // lanes building one table
+  static constexpr int kRounds = kTW >= 8 ? kTW / 8 : 1;     // tables per lane
+  static constexpr int kTableBytesPerWarp = kTable ? kTW * kTableBytes : 0;
   // each warp also stages its 512 theta values (2 KB) through shared memory
   static constexpr int kThetaBytes = 32 * kVec * 4;
-  static constexpr int kWarpTotal = kThetaBytes + kWarpBytes;
+  static constexpr int kWarpTotal = kTableBytesPerWarp + kThetaBytes;  // multiple of 512
   static constexpr int kSmemBytes = kWarps * kWarpTotal;
   // resident blocks per SM the register budget is sized for (64 registers
   // per thread at 4 blocks); G = 64 is held to 2 by its 16 tables per warp
@@ -118,12 +133,6 @@ __device__ __forceinline__ float div_by_const(float a, float b, float r) {
   return __fmaf_rn(res, r, q);
 }
 
-__device__ __forceinline__ float sqrt_approx(float x) {
-  float y;
-  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 __device__ __forceinline__ float rsqrt_approx(float x) {
   float y;
   asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -136,6 +145,39 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
+// Packed binary32 pairs through PTX.  The code generator may still fuse a
+// packed product that feeds a packed sum into one packed fma, even with the
+// explicit rounding mode, so a product whose rounding the rule fixes is
+// never summed with add2_rn: those sums are scalar __fadd_rn, which is never
+// contracted.  The packed fma below is used only where a fused operation is
+// intended (the correction steps).
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+
 // theta_t for one element with every operation of the rule correctly
 // rounded: m^ = m_t / bc1, v^ = v_t / bc2, u = m^ / (sqrt(v^) + eps).
 template <class P>
@@ -144,6 +186,33 @@ __device__ __forceinline__ float exact_update(float th, float mt, float vt, cons
   const float vh = div_by_const(vt, p.bc2, p.rbc2);
   const float u = __fdiv_rn(mh, __fadd_rn(__fsqrt_rn(vh), p.eps));
   return __fsub_rn(__fmul_rn(th, p.decay), __fmul_rn(p.lr, u));
+}
+
+// The same for two elements from the estimates (see the file comment):
+// m^, v^ by Markstein division; sqrt(v^) = s + (v^ - s^2) y/2 with s = v^ y,
+// y = rsqrt(v^); u = q0 + (m^ - q0 d) r with d = sqrt(v^) + eps, r = rcp(d),
+// q0 = m^ r.  v^ = 0 is covered by evaluating y at max(v^, 2^-126).
+template <class P>
+__device__ __forceinline__ float2 fast_update2(float2 th, float2 mt, float2 vt, const P &p) {
+  const float2 RB1 = make_float2(p.rbc1, p.rbc1), NB1 = make_float2(-p.bc1, -p.bc1);
+  const float2 RB2 = make_float2(p.rbc2, p.rbc2), NB2 = make_float2(-p.bc2, -p.bc2);
+  const float2 EPS = make_float2(p.eps, p.eps), DEC = make_float2(p.decay, p.decay);
+  const float2 NLR = make_float2(-p.lr, -p.lr), HALF = make_float2(0.5f, 0.5f);
+  float2 q = mul2_rn(mt, RB1);
+  const float2 mh = fma2_rn(fma2_rn(q, NB1, mt), RB1, q);
+  q = mul2_rn(vt, RB2);
+  const float2 vh = fma2_rn(fma2_rn(q, NB2, vt), RB2, q);
+  const float2 y = make_float2(rsqrt_approx(fmaxf(vh.x, 0x1p-126f)),
+                               rsqrt_approx(fmaxf(vh.y, 0x1p-126f)));
+  const float2 sv = mul2_rn(vh, y);
+  const float2 e = fma2_rn(neg2(sv), sv, vh);
+  const float2 sq = fma2_rn(e, mul2_rn(y, HALF), sv);
+  const float2 den = add2_rn(sq, EPS);
+  const float2 r = make_float2(rcp_approx(den.x), rcp_approx(den.y));
+  const float2 q0 = mul2_rn(mh, r);
+  const float2 u = fma2_rn(fma2_rn(neg2(q0), den, mh), r, q0);
+  const float2 a = mul2_rn(th, DEC), t2 = mul2_rn(NLR, u);
+  return make_float2(__fadd_rn(a.x, t2.x), __fadd_rn(a.y, t2.y));
 }
 
 // Max of |x| and min of nonzero |x| over 16 values (NaN ignored by the max).
@@ -160,6 +229,46 @@ __device__ __forceinline__ void range16(const float *x, float &mx, float &mn) {
   }
   // all-zero (or all-NaN) input gives an infinite minimum
   mn = key >= 0xFF000000u - 2u ? __int_as_float(0x7f800000) : __uint_as_float((key + 2u) >> 1);
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// The same for 16 values that are +0, positive or NaN (the second moment):
+// the maximum needs no |.|, and bits(x) - 1 read as a float is, for x > 0,
+// the float just below x (order preserved) and NaN for +0, which the
+// minimum ignores.
+__device__ __forceinline__ void range16_nonneg(const float *x, float &mx, float &mn) {
+  float a = fmax3(x[0], x[1], x[2]);
+  a = fmax3(a, x[3], x[4]);
+  a = fmax3(a, x[5], x[6]);
+  a = fmax3(a, x[7], x[8]);
+  a = fmax3(a, x[9], x[10]);
+  a = fmax3(a, x[11], x[12]);
+  a = fmax3(a, x[13], x[14]);
+  mx = fmaxf(fmaxf(a, x[15]), 0.0f);
+  float k[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) k[i] = __uint_as_float(__float_as_uint(x[i]) - 1u);
+  float b = fmin3(k[0], k[1], k[2]);
+  b = fmin3(b, k[3], k[4]);
+  b = fmin3(b, k[5], k[6]);
+  b = fmin3(b, k[7], k[8]);
+  b = fmin3(b, k[9], k[10]);
+  b = fmin3(b, k[11], k[12]);
+  b = fmin3(b, k[13], k[14]);
+  b = fminf(b, k[15]);
+  // all-zero input leaves NaN: infinite minimum
+  mn = b != b ? __int_as_float(0x7f800000) : __uint_as_float(__float_as_uint(b) + 1u);
 }
 
 // Reduce (max, min) pairs for two states over the LANES threads of a group.
@@ -235,10 +344,11 @@ __device__ __forceinline__ void group_reduce2_rt(float &mx0, float &mn0, float &
   }
 }
 
-// ---- vector I/O with a ragged tail -----------------------------------------
+// ---- vector I/O; FULL = the 16 values are all inside [0, n) --------------------
 
+template <bool FULL>
 __device__ __forceinline__ void load16_f32(const float *p, int64_t e0, int64_t n, float *v) {
-  if (e0 + 16 <= n) {
+  if (FULL || e0 + 16 <= n) {
     const float4 *q = reinterpret_cast<const float4 *>(p + e0);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -254,8 +364,9 @@ __device__ __forceinline__ void load16_f32(const float *p, int64_t e0, int64_t n
   }
 }
 
+template <bool FULL>
 __device__ __forceinline__ void store16_f32(float *p, int64_t e0, int64_t n, const float *v) {
-  if (e0 + 16 <= n) {
+  if (FULL || e0 + 16 <= n) {
     float4 *q = reinterpret_cast<float4 *>(p + e0);
 #pragma unroll
     for (int i = 0; i < 4; ++i) q[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -265,9 +376,10 @@ __device__ __forceinline__ void store16_f32(float *p, int64_t e0, int64_t n, con
   }
 }
 
-// 16 bytes (16 codes or 8 BF16) as four words.
+// 16 bytes (16 codes) as four words.
+template <bool FULL>
 __device__ __forceinline__ void load16_u8(const uint8_t *p, int64_t e0, int64_t n, uint32_t *w) {
-  if (e0 + 16 <= n) {
+  if (FULL || e0 + 16 <= n) {
     uint4 t = *reinterpret_cast<const uint4 *>(p + e0);
     w[0] = t.x;
     w[1] = t.y;
@@ -281,8 +393,9 @@ __device__ __forceinline__ void load16_u8(const uint8_t *p, int64_t e0, int64_t 
   }
 }
 
+template <bool FULL>
 __device__ __forceinline__ void store16_u8(uint8_t *p, int64_t e0, int64_t n, const uint32_t *w) {
-  if (e0 + 16 <= n) {
+  if (FULL || e0 + 16 <= n) {
     *reinterpret_cast<uint4 *>(p + e0) = make_uint4(w[0], w[1], w[2], w[3]);
   } else {
     for (int i = 0; i < 16; ++i)
@@ -291,9 +404,10 @@ __device__ __forceinline__ void store16_u8(uint8_t *p, int64_t e0, int64_t n, co
 }
 
 // 16 BF16 values as eight words (element 2i in the low half of word i).
+template <bool FULL>
 __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64_t n,
                                             uint32_t *w) {
-  if (e0 + 16 <= n) {
+  if (FULL || e0 + 16 <= n) {
     const uint4 *q = reinterpret_cast<const uint4 *>(p + e0);
     uint4 a = q[0], b = q[1];
     w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
@@ -306,24 +420,29 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
   }
 }
 
-// ---- the fused step ----------------------------------------------------------
-
 // theta of one thread (16 values) copied asynchronously into shared memory
 // (cp.async, zero-filled past n), so no registers are held while it loads.
 // The warp's 512 values are stored chunk-major -- chunk c (values 4c..4c+3)
 // of lane l at float4 index 32c + l -- so that every 16-byte access of the
 // warp touches 512 consecutive bytes (no bank conflicts).
+template <bool FULL>
 __device__ __forceinline__ void stage_theta(float4 *warp_th, const float *theta, int64_t e0,
                                             int64_t n, int lane) {
   const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(warp_th + lane));
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     const int64_t base = e0 + 4 * c;
-    const int bytes = base + 4 <= n ? 16 : (base < n ? static_cast<int>(n - base) * 4 : 0);
-    const float *src = bytes > 0 ? theta + base : theta;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(sa + 512 * c), "l"(src),
-                 "r"(bytes)
-                 : "memory");
+    if constexpr (FULL) {
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa + 512 * c),
+                   "l"(theta + base)
+                   : "memory");
+    } else {
+      const int bytes = base + 4 <= n ? 16 : (base < n ? static_cast<int>(n - base) * 4 : 0);
+      const float *src = bytes > 0 ? theta + base : theta;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(sa + 512 * c),
+                   "l"(src), "r"(bytes)
+                   : "memory");
+    }
   }
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
@@ -332,43 +451,42 @@ __device__ __forceinline__ void wait_staged() {
   asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
 
-template <int VF, int LG>
+// ---- the fused step ----------------------------------------------------------
+
+template <int VF, int LG, bool FULL>
 __global__ void __launch_bounds__(kThreads, StepLayout<LG>::kMinBlocks)
 adamw_fp8_step_kernel(const StepParams p) {
   using L = StepLayout<LG>;
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ double tab8[8];   // log2(1 + i/8)
-  __shared__ double mult8[8];  // 1, -1, log2(1 + i/8) for i = 2..7
+  __shared__ double tab8[8];   // log2(1 + i/8), direct decode (G < 64)
   __shared__ float red[4][kWarps];
-  if (threadIdx.x < 8) {
-    const double t = p.log2_tab[threadIdx.x];
-    tab8[threadIdx.x] = t;
-    mult8[threadIdx.x] = threadIdx.x == 0 ? 1.0 : (threadIdx.x == 1 ? -1.0 : t);
+  if constexpr (!L::kTable) {
+    if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
   }
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int64_t blk0 = static_cast<int64_t>(blockIdx.x) * kElemsPerBlock;
+  const int64_t blk0 = (p.block0 + static_cast<int64_t>(blockIdx.x)) * kElemsPerBlock;
   const int64_t e0 = blk0 + threadIdx.x * kVec;
-  const bool active = e0 < p.n;
+  const bool active = FULL || e0 < p.n;
   const int64_t grp = e0 >> LG;
+  const uint32_t warp_off = static_cast<uint32_t>(warp * L::kWarpTotal);
 
-  // Per-group (k, s) of the decode tables this thread helps to build (or of
-  // its own group on the direct path), loaded first so that they arrive
-  // while the bulk streams are requested.
+  // Per-group (k, s) of the decode tables this lane builds (or of its own
+  // group on the direct path), loaded first so that they arrive while the
+  // bulk streams are requested.
   const int64_t warp_g0 = (blk0 + warp * 32 * kVec) >> LG;
   float kk[L::kRounds], ss[L::kRounds];
   float mk = 1.0f, ms = 0.0f, vk = 1.0f, vs = 0.0f;
   if constexpr (L::kTable) {
 #pragma unroll
     for (int r = 0; r < L::kRounds; ++r) {
-      const int job = lane + 32 * r;
-      const int j = job >> 3;
-      const bool vst = j >= L::kGroupsPerWarp;
-      const int64_t g = warp_g0 + (vst ? j - L::kGroupsPerWarp : j);
+      const int j = r * (32 / L::kL) + lane / L::kL;
+      const bool vst = j >= L::kGPW;
+      const int64_t g = warp_g0 + (vst ? j - L::kGPW : j);
       kk[r] = 1.0f;
       ss[r] = 0.0f;
-      if (job < L::kJobs && g < p.ngroups) {
+      if (FULL || g < p.ngroups) {
         kk[r] = vst ? p.v_k[g] : p.m_k[g];
         ss[r] = vst ? p.v_s[g] : p.m_s[g];
       }
@@ -380,47 +498,39 @@ adamw_fp8_step_kernel(const StepParams p) {
     vs = p.v_s[grp];
   }
 
-  float4 *th_s = reinterpret_cast<float4 *>(smem + static_cast<size_t>(warp) * L::kWarpTotal);
-  stage_theta(th_s, p.theta, e0, p.n, lane);
+  float4 *th_s = reinterpret_cast<float4 *>(smem + warp_off + L::kTableBytesPerWarp);
+  stage_theta<FULL>(th_s, p.theta, e0, p.n, lane);
   float m[16], v[16];
   uint32_t gw[8], mw[4], vw[4];
   if (active) {
-    load16_bf16(p.grad, e0, p.n, gw);
-    load16_u8(p.m_code, e0, p.n, mw);
-    load16_u8(p.v_code, e0, p.n, vw);
+    load16_bf16<FULL>(p.grad, e0, p.n, gw);
+    load16_u8<FULL>(p.m_code, e0, p.n, mw);
+    load16_u8<FULL>(p.v_code, e0, p.n, vw);
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) gw[i] = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) mw[i] = vw[i] = 0;
   }
-  __syncthreads();  // tab8, mult8
 
   // ---- beta1 * m and beta2 * v from the stored states (exact binary32) ----
   if constexpr (L::kTable) {
     // warp-local decode tables: [0, GPW) first moment, [GPW, 2 GPW) second
-    const WarpTables<L::kEnt> tw = warp_tables<L::kEnt>(
-        smem + static_cast<size_t>(warp) * L::kWarpTotal + L::kThetaBytes, L::kTablesPerWarp);
 #pragma unroll
     for (int r = 0; r < L::kRounds; ++r) {
-      const int job = lane + 32 * r;
-      if (job < L::kJobs) table_slot(tw, job >> 3, job & 7, kk[r], ss[r], mult8);
+      const int j = r * (32 / L::kL) + lane / L::kL;
+      const bool vst = j >= L::kGPW;
+      const uint32_t key = (warp_off + j * kTableBytes) | (32u * (j & 3));
+      build_table<L::kL>(smem, key, lane % L::kL, VF == kE4M3 || !vst, kk[r], ss[r],
+                         vst ? p.beta2 : p.beta1);
     }
     __syncwarp();
-#pragma unroll
-    for (int r = 0; r < L::kRounds; ++r) {
-      const int job = lane + 32 * r;
-      if (job < L::kJobs) {
-        const int j = job >> 3;
-        const bool first = j < L::kGroupsPerWarp;
-        table_codes(tw, j, job & 7, VF == kE4M3 || first, first ? p.beta1 : p.beta2);
-      }
-    }
-    __syncwarp();
-    const int lg = L::kGroupsPerWarp > 1 ? (lane >> (LG - 4)) : 0;
-    lookup16<L::kEnt>(tw.ent + lg * L::kEnt, mw, m);
-    lookup16<L::kEnt>(tw.ent + (L::kGroupsPerWarp + lg) * L::kEnt, vw, v);
+    const int lg = L::kGPW > 1 ? (lane >> (LG - 4)) : 0;
+    const int jm = lg, jv = L::kGPW + lg;
+    lookup16(smem, (warp_off + jm * kTableBytes) | (32u * (jm & 3)), mw, m);
+    lookup16(smem, (warp_off + jv * kTableBytes) | (32u * (jv & 3)), vw, v);
   } else {
+    __syncthreads();  // tab8
     const double mrk = 1.0 / static_cast<double>(mk), vrk = 1.0 / static_cast<double>(vk);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -435,89 +545,68 @@ adamw_fp8_step_kernel(const StepParams p) {
     }
   }
 
-  // ---- AdamW, binary32, one rounding per operation in the order of the rule ----
-  // m_t and v_t are computed exactly as the rule rounds them (they are the
-  // new states): scalar IEEE sums of separately rounded products.  The
-  // update quotient u = m^ / (sqrt(v^) + eps) is first formed with
-  // the reciprocal-square-root estimate (relative error below 1e-6, so lr*u
-  // is off by at most ~1e-6 of itself); wherever |lr*u| is not at least twice
-  // below max(|theta|, lr), or eps is not negligible next to sqrt(v^), that
-  // error could matter for theta, and the element is recomputed with
-  // correctly rounded division and square root.
+  // ---- the new moments, binary32, one rounding per operation (scalar sums) ----
   {
     const float2 C1 = make_float2(p.c1, p.c1), C2 = make_float2(p.c2, p.c2);
-    const float2 RB1 = make_float2(p.rbc1, p.rbc1), RB2 = make_float2(p.rbc2, p.rbc2);
-    const float2 EPS = make_float2(p.eps, p.eps), DEC = make_float2(p.decay, p.decay);
-    const float2 NLR = make_float2(-p.lr, -p.lr), TWO = make_float2(2.0f, 2.0f);
-    const float2 ONE = make_float2(1.0f, 1.0f), MONE = make_float2(-1.0f, -1.0f);
-    wait_staged();
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float4 th4 = th_s[32 * c + lane];
-      float2 out[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int i = 2 * c + h;
-        const uint32_t gword = gw[i];
-        const float2 g = make_float2(bf16lo_to_float(gword), bf16hi_to_float(gword));
-        const float2 cg = fmul2(C1, g);
-        const float2 cgg = fmul2(C2, fmul2(g, g));
-        float2 mt, vt;
-        mt.x = __fadd_rn(m[2 * i], cg.x);
-        mt.y = __fadd_rn(m[2 * i + 1], cg.y);
-        vt.x = __fadd_rn(v[2 * i], cgg.x);
-        vt.y = __fadd_rn(v[2 * i + 1], cgg.y);
-        // 1 / (sqrt(v^) + eps) = r / (1 + d) with r = 1/sqrt(v^), d = eps r;
-        // for d <= 2^-10, 1 - d + d^2 is within 2^-30 of 1/(1 + d)
-        const float2 vh = fmul2(vt, RB2);
-        const float2 r = make_float2(rsqrt_approx(vh.x), rsqrt_approx(vh.y));
-        const float2 d = fmul2(EPS, r);
-        const float2 cc = ffma2(d, fadd2(d, MONE), ONE);
-        const float2 u = fmul2(fmul2(fmul2(mt, RB1), r), cc);
-        const float2 th0 = h ? make_float2(th4.z, th4.w) : make_float2(th4.x, th4.y);
-        const float2 t2 = fmul2(NLR, u);
-        float2 tn = fadd2(fmul2(th0, DEC), t2);
-        const float2 w2 = fmul2(TWO, t2);
-        const bool slow = fabsf(w2.x) > fmaxf(fabsf(tn.x), p.lr) ||
-                          fabsf(w2.y) > fmaxf(fabsf(tn.y), p.lr) || !(d.x <= 0x1p-10f) ||
-                          !(d.y <= 0x1p-10f);
-        if (__any_sync(0xffffffffu, slow)) {
-          if (slow) {
-            tn.x = exact_update(th0.x, mt.x, vt.x, p);
-            tn.y = exact_update(th0.y, mt.y, vt.y, p);
-          }
-        }
-        out[h] = tn;
-        m[2 * i] = mt.x;
-        m[2 * i + 1] = mt.y;
-        v[2 * i] = vt.x;
-        v[2 * i + 1] = vt.y;
-      }
-      if (active) {
-        const int64_t base = e0 + 4 * c;
-        if (base + 4 <= p.n) {
-          *reinterpret_cast<float4 *>(p.theta + base) =
-              make_float4(out[0].x, out[0].y, out[1].x, out[1].y);
-        } else {
-          const float o[4] = {out[0].x, out[0].y, out[1].x, out[1].y};
-          for (int j = 0; j < 4; ++j)
-            if (base + j < p.n) p.theta[base + j] = o[j];
-        }
-      }
+    for (int i = 0; i < 8; ++i) {
+      const float2 g = make_float2(bf16lo_to_float(gw[i]), bf16hi_to_float(gw[i]));
+      const float2 cg = mul2_rn(C1, g), cgg = mul2_rn(C2, mul2_rn(g, g));
+      m[2 * i] = __fadd_rn(m[2 * i], cg.x);
+      m[2 * i + 1] = __fadd_rn(m[2 * i + 1], cg.y);
+      v[2 * i] = __fadd_rn(v[2 * i], cgg.x);
+      v[2 * i + 1] = __fadd_rn(v[2 * i + 1], cgg.y);
     }
   }
-
   // tail elements beyond n must not take part in the group range
-  if (e0 + 16 > p.n) {
+  if (!FULL && e0 + 16 > p.n) {
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       if (e0 + i >= p.n) m[i] = v[i] = 0.0f;
   }
 
-  // ---- per-group range of the new moments, then k and s ----
+  // ---- this thread's range of the new moments ----
   float mmx, mmn, vmx, vmn;
   range16(m, mmx, mmn);
-  range16(v, vmx, vmn);
+  range16_nonneg(v, vmx, vmn);
+
+  // ---- theta_t = (1 - lr wd) theta - lr m^ / (sqrt(v^) + eps) ----
+  {
+    const bool fast = mmx <= p.fast_mmax && vmx <= p.fast_vmax && vmn >= p.fast_vmin;
+    const bool slow = __any_sync(0xffffffffu, !fast);
+    wait_staged();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float4 th4 = th_s[32 * c + lane];
+      float o[4];
+      if (!slow) {
+        const float2 a = fast_update2(make_float2(th4.x, th4.y),
+                                      make_float2(m[4 * c], m[4 * c + 1]),
+                                      make_float2(v[4 * c], v[4 * c + 1]), p);
+        const float2 b = fast_update2(make_float2(th4.z, th4.w),
+                                      make_float2(m[4 * c + 2], m[4 * c + 3]),
+                                      make_float2(v[4 * c + 2], v[4 * c + 3]), p);
+        o[0] = a.x;
+        o[1] = a.y;
+        o[2] = b.x;
+        o[3] = b.y;
+      } else {
+        o[0] = exact_update(th4.x, m[4 * c], v[4 * c], p);
+        o[1] = exact_update(th4.y, m[4 * c + 1], v[4 * c + 1], p);
+        o[2] = exact_update(th4.z, m[4 * c + 2], v[4 * c + 2], p);
+        o[3] = exact_update(th4.w, m[4 * c + 3], v[4 * c + 3], p);
+      }
+      const int64_t base = e0 + 4 * c;
+      if (FULL || base + 4 <= p.n) {
+        *reinterpret_cast<float4 *>(p.theta + base) = make_float4(o[0], o[1], o[2], o[3]);
+      } else {
+        for (int j = 0; j < 4; ++j)
+          if (base + j < p.n) p.theta[base + j] = o[j];
+      }
+    }
+  }
+
+  // ---- per-group range of the new moments, then k and s ----
   group_reduce2<L::kLanes>(mmx, mmn, vmx, vmn, red);
   GroupQ gm, gv;
   if constexpr (L::kLanes >= 2) {
@@ -544,8 +633,8 @@ adamw_fp8_step_kernel(const StepParams p) {
   encode16<kE4M3>(m, gm, p.m.log2_fmax, mo);
   encode16<VF>(v, gv, p.v.log2_fmax, vo);
   if (active) {
-    store16_u8(p.m_code, e0, p.n, mo);
-    store16_u8(p.v_code, e0, p.n, vo);
+    store16_u8<FULL>(p.m_code, e0, p.n, mo);
+    store16_u8<FULL>(p.v_code, e0, p.n, vo);
     if ((threadIdx.x & (L::kLanes - 1)) == 0) {
       p.m_k[grp] = gm.k;
       p.m_s[grp] = gm.s;
@@ -567,7 +656,7 @@ quantize_state_kernel(const QuantParams p) {
   const int lanes = 1 << (p.log2G - 4);
   float x[16];
   if (active) {
-    load16_f32(p.x, e0, p.n, x);
+    load16_f32<false>(p.x, e0, p.n, x);
   } else {
 #pragma unroll
     for (int i = 0; i < 16; ++i) x[i] = 0.0f;
@@ -580,7 +669,7 @@ quantize_state_kernel(const QuantParams p) {
   uint32_t o[4];
   encode16<F>(x, g, p.f.log2_fmax, o);
   if (active) {
-    store16_u8(p.code, e0, p.n, o);
+    store16_u8<false>(p.code, e0, p.n, o);
     if ((threadIdx.x & (lanes - 1)) == 0) {
       p.k[grp] = g.k;
       p.s[grp] = g.s;

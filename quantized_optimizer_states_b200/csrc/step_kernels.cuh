@@ -12,7 +12,8 @@
 //
 // Work decomposition: one thread owns 16 consecutive parameters, so every
 // stream moves in 16-byte vectors (4 x 16 B of theta, 2 x 16 B of BF16
-// gradient, 16 B of each code stream).  A 1xG group is G/16 consecutive
+// gradient, 16 B of each code stream).  Dynamic shared memory holds only the
+// warps' decode tables.  A 1xG group is G/16 consecutive
 // threads: up to 32 of them reduce with warp shuffles, larger groups (G >=
 // 1024) finish the reduction through shared memory inside the block.  The
 // whole group stays in registers between the range reduction and the
@@ -100,9 +101,7 @@ struct StepLayout {
   static constexpr int kL = kTW >= 8 ? 4 : 32 / kTW;         // lanes building one table
   static constexpr int kRounds = kTW >= 8 ? kTW / 8 : 1;     // tables per lane
   static constexpr int kTableBytesPerWarp = kTable ? kTW * kTableBytes : 0;
-  // each warp also stages its 512 theta values (2 KB) through shared memory
-  static constexpr int kThetaBytes = 32 * kVec * 4;
-  static constexpr int kWarpTotal = kTableBytesPerWarp + kThetaBytes;  // multiple of 512
+  static constexpr int kWarpTotal = kTableBytesPerWarp;  // multiple of 512
   static constexpr int kSmemBytes = kWarps * kWarpTotal;
   // resident blocks per SM the register budget is sized for (64 registers
   // per thread at 4 blocks); G = 64 is held to 2 by its 16 tables per warp
@@ -420,37 +419,6 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
   }
 }
 
-// theta of one thread (16 values) copied asynchronously into shared memory
-// (cp.async, zero-filled past n), so no registers are held while it loads.
-// The warp's 512 values are stored chunk-major -- chunk c (values 4c..4c+3)
-// of lane l at float4 index 32c + l -- so that every 16-byte access of the
-// warp touches 512 consecutive bytes (no bank conflicts).
-template <bool FULL>
-__device__ __forceinline__ void stage_theta(float4 *warp_th, const float *theta, int64_t e0,
-                                            int64_t n, int lane) {
-  const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(warp_th + lane));
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const int64_t base = e0 + 4 * c;
-    if constexpr (FULL) {
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa + 512 * c),
-                   "l"(theta + base)
-                   : "memory");
-    } else {
-      const int bytes = base + 4 <= n ? 16 : (base < n ? static_cast<int>(n - base) * 4 : 0);
-      const float *src = bytes > 0 ? theta + base : theta;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(sa + 512 * c),
-                   "l"(src), "r"(bytes)
-                   : "memory");
-    }
-  }
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void wait_staged() {
-  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-}
-
 // ---- the fused step ----------------------------------------------------------
 
 template <int VF, int LG, bool FULL>
@@ -498,8 +466,6 @@ adamw_fp8_step_kernel(const StepParams p) {
     vs = p.v_s[grp];
   }
 
-  float4 *th_s = reinterpret_cast<float4 *>(smem + warp_off + L::kTableBytesPerWarp);
-  stage_theta<FULL>(th_s, p.theta, e0, p.n, lane);
   float m[16], v[16];
   uint32_t gw[8], mw[4], vw[4];
   if (active) {
@@ -558,6 +524,20 @@ adamw_fp8_step_kernel(const StepParams p) {
       v[2 * i + 1] = __fadd_rn(v[2 * i + 1], cgg.y);
     }
   }
+  // theta is loaded only now, when the codes and gradients are consumed, so
+  // that its 16 registers are not held through the table build; the range
+  // below runs while it is in flight
+  float4 th[4];
+  if (FULL || e0 + 16 <= p.n) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) th[c] = *reinterpret_cast<const float4 *>(p.theta + e0 + 4 * c);
+  } else {
+    float t16[16];
+    load16_f32<false>(p.theta, e0, p.n, t16);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      th[c] = make_float4(t16[4 * c], t16[4 * c + 1], t16[4 * c + 2], t16[4 * c + 3]);
+  }
   // tail elements beyond n must not take part in the group range
   if (!FULL && e0 + 16 > p.n) {
 #pragma unroll
@@ -574,10 +554,9 @@ adamw_fp8_step_kernel(const StepParams p) {
   {
     const bool fast = mmx <= p.fast_mmax && vmx <= p.fast_vmax && vmn >= p.fast_vmin;
     const bool slow = __any_sync(0xffffffffu, !fast);
-    wait_staged();
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const float4 th4 = th_s[32 * c + lane];
+      const float4 th4 = th[c];
       float o[4];
       if (!slow) {
         const float2 a = fast_update2(make_float2(th4.x, th4.y),

@@ -234,6 +234,28 @@ coat_status_t coat_group_scaling_quant_pertensor_noalloc(const uint16_t *x, int6
                                                          uint8_t *q, float *scale,
                                                          void *stream);
 
+/*
+ * coat_swiglu_group_amax -- a producing kernel with Group Scaling's step (i)
+ * fused in.  [COAT] "混合粒度": the per-1xG maxima of a linear layer's
+ * input are emitted by the kernel that produces it, so the per-tensor
+ * quantizer only reads the G-times-smaller intermediate before its cast.
+ * This producer is the SwiGLU of a GLU MLP ([COAT] "激活为什么难压"), whose
+ * output feeds the down projection:
+ *   out[i] = RN_bf16(silu(gate[i]) * up[i]),  silu(g) = g / (1 + e^-g),
+ * evaluated in binary32 (the library expf, then IEEE division and product,
+ * then round to nearest even BF16).
+ *   gate, up    BF16 bits [n] (16-byte aligned)
+ *   out         BF16 bits [n] (16-byte aligned)
+ *   group_amax  float32[ceil(n/G)] (4-byte aligned): max |out| over each
+ *               1xG run of the flat output (the last run may be shorter) --
+ *               exactly the slots coat_group_scaling_quant_pertensor reads
+ *               when called on `out` with amax_precomputed != 0
+ * Errors: INVALID_ARG, UNSUPPORTED (group size), MISALIGNED, CUDA.
+ */
+coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, int64_t n,
+                                     int32_t group_size, uint16_t *out, float *group_amax,
+                                     void *stream);
+
 /* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
  * this thread (0 if none). */
 int32_t coat_last_cuda_error(void);

@@ -261,6 +261,50 @@ def group_scaling_pertensor(x_bf16: np.ndarray, G: int, fmt: int = E4M3,
     return q, float(sc[0]), ga
 
 
+BF16_MAX = float.fromhex("0x1.fep+127")
+
+
+def round_to_bf16(x) -> np.ndarray:
+    """binary64 values -> BF16 bit patterns, round to nearest even, with BF16
+    subnormals and overflow to infinity (QA page on BF16: 8 exponent bits, 7
+    explicit mantissa bits).  x = m 2^e with 0.5 <= |m| < 1 keeps 8
+    significant bits: rint(x 2^(8-e)) 2^(e-8); below 2^-126 the quantum is
+    the subnormal spacing 2^-133."""
+    x = np.asarray(x, dtype=np.float64)
+    with np.errstate(invalid="ignore", over="ignore"):
+        _, e = np.frexp(x)
+        e = np.maximum(e, -125)
+        q = np.ldexp(np.rint(np.ldexp(x, 8 - e)), e - 8)
+        q = np.where(np.abs(q) > BF16_MAX, np.copysign(np.inf, x), q)
+    return (q.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f64(b) -> np.ndarray:
+    b = np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def swiglu_bf16(gate_bf16: np.ndarray, up_bf16: np.ndarray) -> np.ndarray:
+    """SwiGLU of BF16 inputs, the producer of a GLU MLP's down-projection
+    input (COAT summary page, sections "激活为什么难压" and "混合粒度"):
+    RN_bf16(silu(g) u) with silu(g) = g / (1 + e^-g), evaluated in binary64
+    and rounded once to BF16."""
+    g = bf16_bits_to_f64(gate_bf16)
+    u = bf16_bits_to_f64(up_bf16)
+    with np.errstate(over="ignore"):
+        h = g / (1.0 + np.exp(-g)) * u
+    return round_to_bf16(h)
+
+
+def group_amax_of(x_bf16: np.ndarray, G: int) -> np.ndarray:
+    """Per-1xG max |x| of a flat BF16 tensor (a shorter last group allowed)."""
+    x = np.abs(bf16_bits_to_f64(np.ascontiguousarray(x_bf16).reshape(-1)))
+    ng = n_groups(x.size, G)
+    pad = np.zeros(ng * G)
+    pad[:x.size] = x
+    return pad.reshape(ng, G).max(axis=1).astype(np.float32)
+
+
 def threads_used() -> int:
     return 1
 

@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     coat_group_scaling_workspace_bytes,
     coat_quantize_state,
     coat_status_string,
+    coat_swiglu_group_amax,
     coat_version,
     load,
 )

@@ -64,6 +64,7 @@ SIGNATURES = {
     "coat_group_scaling_workspace_bytes": (_I64, [_I64, _I32]),
     "coat_group_scaling_quant_pertensor": (_I32, [_P, _I64, _I32, _I32, _P, _I32, _P, _P, _P]),
     "coat_group_scaling_quant_pertensor_noalloc": (_I32, [_P, _I64, _I32, _I32, _P, _P, _P]),
+    "coat_swiglu_group_amax": (_I32, [_P, _P, _I64, _I32, _P, _P, _P]),
     "coat_last_cuda_error": (_I32, []),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
     "coat_version": (_I32, []),
@@ -208,6 +209,21 @@ def coat_group_scaling_quant_pertensor_noalloc(x, q, scale, *, group_size: int =
         _u16(x, "x"), x.numel(), group_size, fmt, _ptr(q, torch.uint8, "q"),
         _ptr(scale, torch.float32, "scale"), _stream(stream))
     _check("coat_group_scaling_quant_pertensor_noalloc", st)
+
+
+def coat_swiglu_group_amax(gate, up, out, group_amax, *, group_size: int = 128, stream=None):
+    """out = RN_bf16(silu(gate) * up) and the per-1xG maxima of out, ready
+    for coat_group_scaling_quant_pertensor(..., amax_precomputed=True)."""
+    import torch
+    if gate.numel() != up.numel() or out.numel() != gate.numel():
+        raise ValueError("gate, up and out must have the same number of elements")
+    ng = -(-gate.numel() // group_size)
+    if group_amax.numel() < ng:
+        raise ValueError(f"group_amax needs {ng} float32 slots")
+    st = load().coat_swiglu_group_amax(
+        _u16(gate, "gate"), _u16(up, "up"), gate.numel(), group_size, _u16(out, "out"),
+        _ptr(group_amax, torch.float32, "group_amax"), _stream(stream))
+    _check("coat_swiglu_group_amax", st)
 
 
 def coat_version() -> int:

@@ -195,6 +195,67 @@ __global__ void __launch_bounds__(kThreads) pertensor_cast_kernel(const GroupSca
   store16_u8<false>(p.q, e0, p.n, o);
 }
 
+// ---- a producer with Group Scaling's step (i) fused in: SwiGLU -------------------
+// COAT summary page, section "混合粒度": the per-1xG maxima of a linear
+// layer's input are emitted by the kernel that produces that input, so the
+// per-tensor quantizer only reads the G-times-smaller intermediate (step
+// (ii)) before its cast.  SwiGLU produces the input of an MLP's down
+// projection (the GLU layers of section "激活为什么难压"):
+//   out = RN_bf16(silu(gate) * up), silu(g) = g / (1 + e^-g),
+// evaluated in binary32 (expf, then IEEE division and product); the maxima
+// are taken over the BF16 outputs, i.e. exactly the values the quantizer
+// will read.
+
+struct SwigluParams {
+  const uint16_t *gate;
+  const uint16_t *up;
+  int64_t n;
+  int log2G;
+  uint16_t *out;
+  float *group_amax;  // [ceil(n / G)]
+};
+
+__global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const SwigluParams p) {
+  __shared__ float red[kWarps];
+  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+  const bool active = e0 < p.n;
+  const int lanes = 1 << (p.log2G - 4);
+  uint32_t gw[8], uw[8];
+  if (active) {
+    load16_bf16<false>(p.gate, e0, p.n, gw);
+    load16_bf16<false>(p.up, e0, p.n, uw);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) gw[i] = uw[i] = 0;
+  }
+  float g[16], u[16], h[16];
+  unpack16_bf16(gw, g);
+  unpack16_bf16(uw, u);
+  uint32_t ow[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float a = __fmul_rn(__fdiv_rn(g[2 * i], __fadd_rn(1.0f, expf(-g[2 * i]))), u[2 * i]);
+    const float b =
+        __fmul_rn(__fdiv_rn(g[2 * i + 1], __fadd_rn(1.0f, expf(-g[2 * i + 1]))), u[2 * i + 1]);
+    const uint32_t ba = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a)));
+    const uint32_t bb = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(b)));
+    ow[i] = ba | (bb << 16);
+    h[2 * i] = bf16lo_to_float(ow[i]);
+    h[2 * i + 1] = bf16hi_to_float(ow[i]);
+  }
+  const float gmax = group_max(amax16(h), lanes, red);
+  if (!active) return;
+  if (e0 + 16 <= p.n) {
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + e0);
+    dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    dst[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+  } else {
+    for (int i = 0; i < 16; ++i)
+      if (e0 + i < p.n) p.out[e0 + i] = static_cast<uint16_t>(ow[i >> 1] >> (16 * (i & 1)));
+  }
+  if ((threadIdx.x & (lanes - 1)) == 0) p.group_amax[e0 >> p.log2G] = gmax;
+}
+
 // ---- dequantization ----------------------------------------------------------------
 
 struct DequantParams {

@@ -336,6 +336,29 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
   return launch_status();
 }
 
+coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, int64_t n,
+                                     int32_t group_size, uint16_t *out, float *group_amax,
+                                     void *stream) {
+  if (n < 0) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && (!gate || !up || !out || !group_amax)) return COAT_ERR_INVALID_ARG;
+  const int lg = group_log2(group_size);
+  if (lg < 0 || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
+  if (n == 0) return COAT_OK;
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(group_amax) & 3u) != 0)
+    return COAT_ERR_MISALIGNED;
+  coat::SwigluParams p;
+  p.gate = gate;
+  p.up = up;
+  p.n = n;
+  p.log2G = lg;
+  p.out = out;
+  p.group_amax = group_amax;
+  coat::swiglu_group_amax_kernel<<<blocks_for(n), coat::kThreads, 0,
+                                   static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
+}
+
 int32_t coat_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char *coat_status_string(coat_status_t status) {

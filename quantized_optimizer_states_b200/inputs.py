@@ -241,3 +241,28 @@ def device_activations(w: ActWorkload, device):
                                                                    generator=gen)
     x[:, ch] *= mult
     return x.to(torch.bfloat16)
+
+
+def host_swiglu_inputs(w: ActWorkload, rows: int | None = None):
+    """(gate, up) uint16 BF16 bits [rows, cols] for the SwiGLU producer:
+    gate ~ N(0, 1.5^2), up ~ N(0, 1) with the workload's GLU-style spike
+    channels scaled by U[spike_lo, spike_hi] per token."""
+    rows = w.rows if rows is None else rows
+    rng = np.random.default_rng(w.seed + 17)
+    gate = (rng.standard_normal((rows, w.cols)) * 1.5).astype(np.float32)
+    up = rng.standard_normal((rows, w.cols)).astype(np.float32)
+    ch = _spike_channels(w, rng)
+    up[:, ch] *= rng.uniform(w.spike_lo, w.spike_hi, (rows, ch.size)).astype(np.float32)
+    return _bf16_bits(gate).reshape(rows, w.cols), _bf16_bits(up).reshape(rows, w.cols)
+
+
+def device_swiglu_inputs(w: ActWorkload, device):
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed + 17)
+    gate = torch.randn(w.rows, w.cols, device=device, generator=gen) * 1.5
+    up = torch.randn(w.rows, w.cols, device=device, generator=gen)
+    ch = torch.from_numpy(_spike_channels(w, np.random.default_rng(w.seed + 17))).to(device)
+    up[:, ch] *= torch.empty(w.rows, ch.numel(), device=device).uniform_(
+        w.spike_lo, w.spike_hi, generator=gen)
+    return gate.to(torch.bfloat16), up.to(torch.bfloat16)

@@ -1,0 +1,118 @@
+"""The SwiGLU producer with Group Scaling's step (i) fused in
+(coat_swiglu_group_amax), against the oracle, and the per-tensor quantizer
+fed with its maxima."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_optimizer_states_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from quantized_optimizer_states_b200 import build
+    build.build()
+    import quantized_optimizer_states_b200 as q
+    q.load()
+    return q
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def _run(lib, gate, up, G):
+    n = gate.size
+    out = torch.empty(n, dtype=torch.int16, device="cuda")
+    ga = torch.full((-(-n // G),), -1.0, dtype=torch.float32, device="cuda")
+    lib.coat_swiglu_group_amax(_dev(gate.reshape(-1)), _dev(up.reshape(-1)), out, ga,
+                               group_size=G)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().view(np.uint16), ga.cpu().numpy()
+
+
+def _near_midpoint(gate, up, idx):
+    """Is the exact binary64 product within 2^-18 (relative) of a BF16
+    rounding midpoint?  Only there may binary32 evaluation round the other way."""
+    g = oracle.bf16_bits_to_f64(gate.reshape(-1)[idx])
+    u = oracle.bf16_bits_to_f64(up.reshape(-1)[idx])
+    h = g / (1.0 + np.exp(-g)) * u
+    m, e = np.frexp(h)
+    frac = np.abs(np.ldexp(h, 8 - np.maximum(e, -125)))
+    dist = np.abs(frac - np.floor(frac) - 0.5)
+    return dist <= 2.0**-18 * 256
+
+
+def _check_out(got, ref, gate, up):
+    """Equal, except at most 1e-3 of the elements that are one BF16 step
+    apart next to a rounding midpoint."""
+    diff = np.nonzero(got != ref)[0]
+    assert diff.size <= max(1, 1e-3 * got.size), diff.size
+    if diff.size:
+        step = np.abs(got[diff].astype(np.int32) - ref[diff].astype(np.int32))
+        assert np.all(step == 1)
+        assert np.all(_near_midpoint(gate, up, diff))
+
+
+@pytest.mark.parametrize("G", [32, 128, 1024])
+def test_swiglu_matches_oracle_and_maxima_are_exact(lib, G):
+    w = inputs.activations()
+    gate, up = inputs.host_swiglu_inputs(w, rows=64)
+    got, ga = _run(lib, gate, up, G)
+    ref = oracle.swiglu_bf16(gate.reshape(-1), up.reshape(-1))
+    _check_out(got, ref, gate, up)
+    # the fused maxima are exactly the maxima of the BF16 output
+    assert np.array_equal(ga, oracle.group_amax_of(got, G))
+
+
+def test_ragged_length_and_special_values(lib):
+    G = 128
+    vals = np.array([0.0, -0.0, 1.0, -1.0, 100.0, -100.0, 3e38, -3e38, 1e-40], dtype=np.float32)
+    rng = np.random.default_rng(3)
+    n = 3 * G + 37
+    gate = oracle.round_to_bf16(rng.choice(vals, n).astype(np.float64))
+    up = oracle.round_to_bf16(rng.normal(0, 2, n))
+    got, ga = _run(lib, gate, up, G)
+    ref = oracle.swiglu_bf16(gate, up)
+    fin = np.isfinite(oracle.bf16_bits_to_f64(ref))
+    assert np.array_equal(np.isfinite(oracle.bf16_bits_to_f64(got)), fin)
+    _check_out(got[fin], ref[fin], gate[fin], up[fin])
+    assert np.array_equal(ga, oracle.group_amax_of(got, G))
+
+
+def test_fused_maxima_feed_group_scaling(lib):
+    """Producer maxima + the per-tensor quantizer (step (i) skipped) give the
+    same codes and scale as the oracle's Group Scaling on the same BF16
+    tensor -- bit-exact."""
+    G = 128
+    w = inputs.activations()
+    gate, up = inputs.host_swiglu_inputs(w, rows=32)
+    n = gate.size
+    out = torch.empty(n, dtype=torch.int16, device="cuda")
+    ws = torch.empty(lib.coat_group_scaling_workspace_bytes(n, G) // 4, dtype=torch.float32,
+                     device="cuda")
+    lib.coat_swiglu_group_amax(_dev(gate.reshape(-1)), _dev(up.reshape(-1)), out, ws,
+                               group_size=G)
+    q = torch.empty(n, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(1, dtype=torch.float32, device="cuda")
+    lib.coat_group_scaling_quant_pertensor(out, ws, q, sc, group_size=G, amax_precomputed=True)
+    torch.cuda.synchronize()
+    h = out.cpu().numpy().view(np.uint16)
+    q_ref, s_ref, _ = oracle.group_scaling_pertensor(h, G, 0)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert float(sc.item()) == s_ref
+
+
+def test_argument_errors(lib):
+    from quantized_optimizer_states_b200._lib import CoatError
+    x = torch.zeros(256, dtype=torch.int16, device="cuda")
+    ga = torch.zeros(4, dtype=torch.float32, device="cuda")
+    with pytest.raises(CoatError):
+        lib.coat_swiglu_group_amax(x, x, x, ga, group_size=100)
+    with pytest.raises(ValueError):
+        lib.coat_swiglu_group_amax(x, x[:128], x, ga, group_size=128)

@@ -1,0 +1,105 @@
+"""ZeRO-1 style data-parallel COAT step over torch.distributed.
+
+In data-parallel training every rank computes a full BF16 gradient of the
+same parameters.  The optimizer state -- FP32 master weights and the FP8
+moments with their per-group k and s (COAT summary page, section
+"扩展函数：把窄分布拉宽") -- is partitioned across the ranks at 1xG group
+boundaries, so each rank keeps 1/world of it.  One step:
+
+  1. reduce-scatter of the gradients: each rank receives, over its shard,
+     the mean of all ranks' gradients (summed in binary32 by the collective,
+     divided by the rank count, rounded to BF16 nearest-even);
+  2. the COAT step on the shard (one `coat_adamw_fp8_step` call);
+  3. all-gather of the updated master weights.
+
+No 1xG group straddles two shards, so the sharded step computes exactly
+what a single-rank step over the whole buffer computes on the reduced
+gradient.  The collectives go through the default (or given) process group:
+NCCL over NVLink/NVSwitch on B200 nodes, gloo on CPU for the tests.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import _lib
+
+
+def shard_length(n: int, group_size: int, world: int) -> int:
+    """Per-rank length: ceil(n / world) rounded up to a multiple of
+    max(G, 16), so every shard is whole groups and 16-byte aligned for all
+    element sizes."""
+    if n < 0 or group_size < 1 or world < 1:
+        raise ValueError("bad shard arguments")
+    unit = max(group_size, 16)
+    per = -(-n // world)
+    return -(-per // unit) * unit
+
+
+def _coat_step(shard: "Zero1Shard", grad_shard: torch.Tensor, t: int, hyper: dict):
+    _lib.coat_adamw_fp8_step(
+        shard.master, grad_shard, shard.m_code, shard.m_k, shard.m_s, shard.v_code, shard.v_k,
+        shard.v_s, step=t, group_size=shard.group_size, v_fmt=shard.v_fmt,
+        k_range=shard.k_range, k_max=shard.k_max, **hyper)
+
+
+class Zero1Shard:
+    """This rank's share of the COAT optimizer state for one flat parameter
+    buffer of n elements.
+
+    `theta` is the full FP32 parameter buffer (the same on every rank); the
+    rank keeps a copy of its shard as master weights.  Fresh moments are
+    all-zero groups (codes 0, k = 1, s = 0).
+    """
+
+    def __init__(self, theta: torch.Tensor, *, group_size: int = 128, v_fmt: int = 0,
+                 k_range: int = 0, k_max: float = 64.0, group=None):
+        self.pg = group
+        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+        self.n = theta.numel()
+        self.group_size, self.v_fmt, self.k_range, self.k_max = group_size, v_fmt, k_range, k_max
+        self.L = shard_length(self.n, group_size, self.world)
+        dev = theta.device
+        lo = self.rank * self.L
+        self.master = torch.zeros(self.L, dtype=torch.float32, device=dev)
+        hi = min(self.n, lo + self.L)
+        if hi > lo:
+            self.master[:hi - lo].copy_(theta.reshape(-1)[lo:hi])
+        ng = self.L // group_size
+        self.m_code = torch.zeros(self.L, dtype=torch.uint8, device=dev)
+        self.v_code = torch.zeros(self.L, dtype=torch.uint8, device=dev)
+        self.m_k = torch.ones(ng, dtype=torch.float32, device=dev)
+        self.v_k = torch.ones(ng, dtype=torch.float32, device=dev)
+        self.m_s = torch.zeros(ng, dtype=torch.float32, device=dev)
+        self.v_s = torch.zeros(ng, dtype=torch.float32, device=dev)
+
+    def reduce_gradient(self, grad: torch.Tensor) -> torch.Tensor:
+        """Mean over ranks of the full BF16 gradients, this rank's shard, as
+        BF16 (binary32 sum, division by the rank count, nearest-even BF16)."""
+        full = torch.zeros(self.world * self.L, dtype=torch.float32, device=grad.device)
+        full[:self.n].copy_(grad.reshape(-1))
+        part = torch.empty(self.L, dtype=torch.float32, device=grad.device)
+        if self.world > 1:
+            dist.reduce_scatter_tensor(part, full, op=dist.ReduceOp.SUM, group=self.pg)
+            part.div_(float(self.world))
+        else:
+            part.copy_(full)
+        return part.to(torch.bfloat16)
+
+    def gather_params(self) -> torch.Tensor:
+        """The full updated FP32 parameter buffer (first n elements)."""
+        full = torch.empty(self.world * self.L, dtype=torch.float32, device=self.master.device)
+        if self.world > 1:
+            dist.all_gather_into_tensor(full, self.master, group=self.pg)
+        else:
+            full.copy_(self.master)
+        return full[:self.n]
+
+    def step(self, grad: torch.Tensor, t: int, hyper: dict, step_fn=None) -> torch.Tensor:
+        """One data-parallel step with this rank's full BF16 gradient `grad`;
+        returns the full updated parameters.  `step_fn(shard, grad_shard, t,
+        hyper)` replaces the CUDA step (the CPU tests pass the oracle)."""
+        g = self.reduce_gradient(grad)
+        (step_fn or _coat_step)(self, g, t, hyper)
+        return self.gather_params()

@@ -143,3 +143,30 @@ def test_dequantized_moments_shape(optim):
     assert m.shape == v.shape == opt.flat_master().shape
     assert torch.all(v >= 0)
     assert torch.isfinite(m).all() and torch.isfinite(v).all()
+
+
+def test_zero1_shard_single_rank_is_the_plain_step(optim):
+    """Without a process group the ZeRO-1 shard is the whole (padded) buffer:
+    its step equals a direct coat_adamw_fp8_step."""
+    import quantized_optimizer_states_b200 as q
+    from quantized_optimizer_states_b200 import zero
+    n = 3 * 128 + 50
+    g = torch.Generator().manual_seed(4)
+    theta = (torch.randn(n, generator=g) * 0.02).cuda()
+    sh = zero.Zero1Shard(theta, group_size=128)
+    L = sh.L
+    th = torch.zeros(L, device="cuda")
+    th[:n] = theta
+    mc = torch.zeros(L, dtype=torch.uint8, device="cuda")
+    vc = torch.zeros_like(mc)
+    ng = L // 128
+    mk, vk = torch.ones(ng, device="cuda"), torch.ones(ng, device="cuda")
+    ms, vs = torch.zeros(ng, device="cuda"), torch.zeros(ng, device="cuda")
+    for t in (1, 2):
+        grad = (torch.randn(n, generator=g) * 1e-3).to(torch.bfloat16).cuda()
+        full = sh.step(grad, t, H)
+        gp = torch.zeros(L, dtype=torch.bfloat16, device="cuda")
+        gp[:n] = grad
+        q.coat_adamw_fp8_step(th, gp, mc, mk, ms, vc, vk, vs, step=t, group_size=128, **H)
+        assert torch.equal(full, th[:n])
+        assert torch.equal(sh.m_code, mc) and torch.equal(sh.v_code, vc)

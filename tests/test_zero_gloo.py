@@ -1,0 +1,111 @@
+"""ZeRO-1 sharded COAT step (quantized_optimizer_states_b200.zero) with two
+gloo ranks on CPU.  The CUDA step is replaced by the oracle on each shard;
+the sharded result must equal one oracle step over the whole buffer on the
+rank-mean gradient, bit for bit (groups never straddle shards)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+from quantized_optimizer_states_b200 import inputs, zero
+
+H = inputs.HYPER
+G = 128
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_shard_length():
+    assert zero.shard_length(1000, 128, 2) == 512
+    assert zero.shard_length(1024, 128, 2) == 512
+    assert zero.shard_length(1025, 128, 2) == 640
+    assert zero.shard_length(7, 16, 3) == 16
+    assert zero.shard_length(0, 128, 4) == 0
+    with pytest.raises(ValueError):
+        zero.shard_length(10, 0, 2)
+
+
+def _inputs(n, world, steps):
+    rng = np.random.default_rng(42)
+    theta = rng.normal(0, 0.02, n).astype(np.float32)
+    grads = rng.normal(0, 1e-3, (steps, world, n)).astype(np.float32)
+    return theta, grads
+
+
+def _oracle_step_fn():
+    import oracle
+    import torch
+
+    def step_fn(shard, g_shard, t, hyper):
+        gb = g_shard.view(torch.int16).numpy().view(np.uint16)
+        st = tuple(x.numpy() for x in (shard.m_code, shard.m_k, shard.m_s, shard.v_code,
+                                       shard.v_k, shard.v_s))
+        out = oracle.adamw_fp8_step(shard.master.numpy(), gb, *st, step=t, group_size=G,
+                                    **hyper)
+        for dst, src in zip((shard.master, shard.m_code, shard.m_k, shard.m_s, shard.v_code,
+                             shard.v_k, shard.v_s), out[:7]):
+            dst.copy_(torch.from_numpy(np.ascontiguousarray(src)))
+    return step_fn
+
+
+def _worker(rank, world, port, n, steps, q):
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        theta, grads = _inputs(n, world, steps)
+        sh = zero.Zero1Shard(torch.from_numpy(theta), group_size=G)
+        step_fn = _oracle_step_fn()
+        full = None
+        for t in range(steps):
+            g = torch.from_numpy(grads[t, rank]).to(torch.bfloat16)
+            full = sh.step(g, 10 + t, H, step_fn=step_fn)
+        q.put((rank, full.numpy().copy(), sh.L))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_match_the_single_rank_step():
+    import oracle
+    import torch
+    world, n, steps = 2, 5 * 128 + 77, 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, n, steps, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+
+    # reference: one rank, whole buffer, gradient = BF16(mean over ranks)
+    theta, grads = _inputs(n, world, steps)
+    L = zero.shard_length(n, G, world)
+    npad = world * L
+    th = np.zeros(npad, np.float32)
+    th[:n] = theta
+    z = np.zeros(npad, np.uint8)
+    ng = npad // G
+    st = (z, np.ones(ng, np.float32), np.zeros(ng, np.float32), z.copy(),
+          np.ones(ng, np.float32), np.zeros(ng, np.float32))
+    for t in range(steps):
+        gsum = torch.zeros(npad, dtype=torch.float32)
+        for r in range(world):
+            gsum[:n] += torch.from_numpy(grads[t, r]).to(torch.bfloat16).float()
+        gmean = (gsum / world).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        out = oracle.adamw_fp8_step(th, gmean, *st, step=10 + t, group_size=G, **H)
+        th, st = out[0], out[1:7]
+    for rank, full, Lr in res:
+        assert Lr == L
+        assert np.array_equal(full, th[:n]), f"rank {rank}"

@@ -54,6 +54,8 @@ coat::StateFmtParams state_fmt_params(int32_t store_fmt, int32_t k_range) {
   f.ln_range = std::log(fmt_max_host(rf) / fmt_min_subnormal_host(rf));
   f.fmax = static_cast<float>(fmt_max_host(store_fmt));
   f.log2_fmax = static_cast<float>(std::log2(fmt_max_host(store_fmt)));
+  volatile float one = 1.0f;
+  f.rfmax = one / f.fmax;  // correctly rounded reciprocal
   return f;
 }
 

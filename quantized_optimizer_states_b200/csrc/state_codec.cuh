@@ -22,6 +22,7 @@ struct StateFmtParams {
   double ln_range;   // ln of the range k aims to fill
   float fmax;        // storage format's largest finite value
   float log2_fmax;   // log2(fmax), binary32
+  float rfmax;       // RN(1 / fmax)
 };
 
 // ---- binary64 exp2 -----------------------------------------------------------
@@ -74,30 +75,61 @@ struct GroupQ {
   bool zero;   // all-zero group
 };
 
+// ln(x) for a positive normal binary64 x, without branches: x = 2^e m with
+// m in [~sqrt(1/2), ~sqrt(2)), ln m = 2 atanh(s) = 2 (s + s^3/3 + s^5/5 + ...)
+// with s = (m - 1)/(m + 1), |s| <= 0.1716, summed to s^21 (remainder below
+// 2^-56 of the result); e ln 2 with ln 2 split in two parts.  Error a few
+// units of 2^-53.
+__device__ __forceinline__ double log_d(double x) {
+  const int hi = __double2hiint(x), lo = __double2loint(x);
+  const int frac = hi & 0x000FFFFF;
+  const int big = frac > 0x6A09E ? 1 : 0;  // m >= ~sqrt(2): use m/2, e + 1
+  const int e = (hi >> 20) - 1023 + big;
+  const double m = __hiloint2double((frac | 0x3FF00000) - (big << 20), lo);
+  const double s = (m - 1.0) * recip_d(m + 1.0);
+  const double s2 = s * s;
+  double p = 1.0 / 21.0;
+  p = fma(p, s2, 1.0 / 19.0);
+  p = fma(p, s2, 1.0 / 17.0);
+  p = fma(p, s2, 1.0 / 15.0);
+  p = fma(p, s2, 1.0 / 13.0);
+  p = fma(p, s2, 1.0 / 11.0);
+  p = fma(p, s2, 1.0 / 9.0);
+  p = fma(p, s2, 1.0 / 7.0);
+  p = fma(p, s2, 1.0 / 5.0);
+  p = fma(p, s2, 1.0 / 3.0);
+  const double lnm = fma(2.0 * s * s2, p, 2.0 * s);
+  constexpr double kLn2Hi = 0x1.62e42fefa3800p-1;  // ln 2, leading 43 bits
+  constexpr double kLn2Lo = 0x1.ef35793c76730p-45; // ln 2 - kLn2Hi
+  const double ed = static_cast<double>(e);
+  return fma(ed, kLn2Hi, fma(ed, kLn2Lo, lnm));
+}
+
 // k = ln(R_target) / ln(M / mn) in binary64, rounded once, clamped to k_max;
-// k = 1 when M == mn.  s = M * fmax^(-1/k) (binary32 through the exp2 unit;
-// an IEEE quotient when k == 1).
+// k = 1 when M == mn (or for an all-zero group, or when forced).
+// s = M * fmax^(-1/k) (binary32 through the exp2 unit), or the correctly
+// rounded quotient M / fmax when k == 1 (Markstein division by the constant
+// fmax with its rounded reciprocal).  Every branch is a select, so the
+// binary64 chain can be scheduled together with independent work.
 __device__ __forceinline__ GroupQ group_params(float M, float mn, double ln_range, float fmax,
-                                               float log2_fmax, float k_max, int force_k1) {
+                                               float log2_fmax, float rfmax, float k_max,
+                                               int force_k1) {
   GroupQ g;
   g.zero = !(M > 0.0f);
-  float k = 1.0f;
-  if (!g.zero && !force_k1 && M != mn) {
-    const double ratio = static_cast<double>(M) * recip_d(static_cast<double>(mn));
-    double kd = ln_range * recip_d(log(ratio));
-    if (k_max > 0.0f && kd > static_cast<double>(k_max)) kd = static_cast<double>(k_max);
-    k = static_cast<float>(kd);
-  }
+  const bool expand = !g.zero && !force_k1 && M != mn;
+  const double Md = static_cast<double>(expand ? M : 2.0f);
+  const double mnd = static_cast<double>(expand ? mn : 1.0f);
+  double kd = ln_range * recip_d(log_d(Md * recip_d(mnd)));
+  kd = (k_max > 0.0f && kd > static_cast<double>(k_max)) ? static_cast<double>(k_max) : kd;
+  const float k = expand ? static_cast<float>(kd) : 1.0f;
   g.k = k;
   float rk, rM;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rk) : "f"(k));
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rM) : "f"(M));
-  if (g.zero)
-    g.s = 0.0f;
-  else if (k == 1.0f)
-    g.s = __fdiv_rn(M, fmax);
-  else
-    g.s = __fmul_rn(M, ex2_approx(-log2_fmax * rk));
+  const float q = __fmul_rn(M, rfmax);
+  const float s1 = __fmaf_rn(__fmaf_rn(-q, fmax, M), rfmax, q);  // M / fmax
+  const float sk = __fmul_rn(M, ex2_approx(-log2_fmax * rk));
+  g.s = g.zero ? 0.0f : (k == 1.0f ? s1 : sk);
   g.rM = g.zero ? 0.0f : rM;
   return g;
 }

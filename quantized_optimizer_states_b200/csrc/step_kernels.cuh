@@ -550,37 +550,43 @@ adamw_fp8_step_kernel(const StepParams p) {
   range16(m, mmx, mmn);
   range16_nonneg(v, vmx, vmn);
 
+  const bool slow = __any_sync(0xffffffffu, !(mmx <= p.fast_mmax && vmx <= p.fast_vmax &&
+                                                 vmn >= p.fast_vmin));
+
   // ---- theta_t = (1 - lr wd) theta - lr m^ / (sqrt(v^) + eps) ----
+  // The estimate-based form runs unconditionally; a warp with a thread
+  // outside its range then recomputes and rewrites its parameters with the
+  // fully IEEE operations.
   {
-    const bool fast = mmx <= p.fast_mmax && vmx <= p.fast_vmax && vmn >= p.fast_vmin;
-    const bool slow = __any_sync(0xffffffffu, !fast);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const float4 th4 = th[c];
-      float o[4];
-      if (!slow) {
-        const float2 a = fast_update2(make_float2(th4.x, th4.y),
-                                      make_float2(m[4 * c], m[4 * c + 1]),
-                                      make_float2(v[4 * c], v[4 * c + 1]), p);
-        const float2 b = fast_update2(make_float2(th4.z, th4.w),
-                                      make_float2(m[4 * c + 2], m[4 * c + 3]),
-                                      make_float2(v[4 * c + 2], v[4 * c + 3]), p);
-        o[0] = a.x;
-        o[1] = a.y;
-        o[2] = b.x;
-        o[3] = b.y;
-      } else {
-        o[0] = exact_update(th4.x, m[4 * c], v[4 * c], p);
-        o[1] = exact_update(th4.y, m[4 * c + 1], v[4 * c + 1], p);
-        o[2] = exact_update(th4.z, m[4 * c + 2], v[4 * c + 2], p);
-        o[3] = exact_update(th4.w, m[4 * c + 3], v[4 * c + 3], p);
-      }
+      const float2 a = fast_update2(make_float2(th4.x, th4.y),
+                                    make_float2(m[4 * c], m[4 * c + 1]),
+                                    make_float2(v[4 * c], v[4 * c + 1]), p);
+      const float2 b = fast_update2(make_float2(th4.z, th4.w),
+                                    make_float2(m[4 * c + 2], m[4 * c + 3]),
+                                    make_float2(v[4 * c + 2], v[4 * c + 3]), p);
       const int64_t base = e0 + 4 * c;
       if (FULL || base + 4 <= p.n) {
-        *reinterpret_cast<float4 *>(p.theta + base) = make_float4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<float4 *>(p.theta + base) = make_float4(a.x, a.y, b.x, b.y);
       } else {
+        const float o[4] = {a.x, a.y, b.x, b.y};
         for (int j = 0; j < 4; ++j)
           if (base + j < p.n) p.theta[base + j] = o[j];
+      }
+    }
+    if (slow) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float4 th4 = th[c];
+        const float o[4] = {exact_update(th4.x, m[4 * c], v[4 * c], p),
+                            exact_update(th4.y, m[4 * c + 1], v[4 * c + 1], p),
+                            exact_update(th4.z, m[4 * c + 2], v[4 * c + 2], p),
+                            exact_update(th4.w, m[4 * c + 3], v[4 * c + 3], p)};
+        const int64_t base = e0 + 4 * c;
+        for (int j = 0; j < 4; ++j)
+          if (FULL || base + j < p.n) p.theta[base + j] = o[j];
       }
     }
   }
@@ -594,7 +600,8 @@ adamw_fp8_step_kernel(const StepParams p) {
     const GroupQ mine = group_params(odd ? vmx : mmx, odd ? vmn : mmn,
                                      odd ? p.v.ln_range : p.m.ln_range,
                                      odd ? p.v.fmax : p.m.fmax,
-                                     odd ? p.v.log2_fmax : p.m.log2_fmax, p.k_max, p.force_k1);
+                                     odd ? p.v.log2_fmax : p.m.log2_fmax,
+                                     odd ? p.v.rfmax : p.m.rfmax, p.k_max, p.force_k1);
     GroupQ other;
     other.k = __shfl_xor_sync(0xffffffffu, mine.k, 1);
     other.s = __shfl_xor_sync(0xffffffffu, mine.s, 1);
@@ -603,8 +610,10 @@ adamw_fp8_step_kernel(const StepParams p) {
     gm = odd ? other : mine;
     gv = odd ? mine : other;
   } else {
-    gm = group_params(mmx, mmn, p.m.ln_range, p.m.fmax, p.m.log2_fmax, p.k_max, p.force_k1);
-    gv = group_params(vmx, vmn, p.v.ln_range, p.v.fmax, p.v.log2_fmax, p.k_max, p.force_k1);
+    gm = group_params(mmx, mmn, p.m.ln_range, p.m.fmax, p.m.log2_fmax, p.m.rfmax, p.k_max,
+                      p.force_k1);
+    gv = group_params(vmx, vmn, p.v.ln_range, p.v.fmax, p.v.log2_fmax, p.v.rfmax, p.k_max,
+                      p.force_k1);
   }
 
   // ---- re-expand, rescale and encode ----
@@ -643,8 +652,8 @@ quantize_state_kernel(const QuantParams p) {
   float mx, mn, dmx = 0.0f, dmn = 0.0f;
   range16(x, mx, mn);
   group_reduce2_rt(mx, mn, dmx, dmn, lanes, red);
-  const GroupQ g = group_params(mx, mn, p.f.ln_range, p.f.fmax, p.f.log2_fmax, p.k_max,
-                                p.force_k1);
+  const GroupQ g = group_params(mx, mn, p.f.ln_range, p.f.fmax, p.f.log2_fmax, p.f.rfmax,
+                                p.k_max, p.force_k1);
   uint32_t o[4];
   encode16<F>(x, g, p.f.log2_fmax, o);
   if (active) {

@@ -181,6 +181,99 @@ def run_reference(args):
     return 0
 
 
+def run_activations(args):
+    """The activation-side kernels on the activation workload (BF16 [16384,
+    2048], G = 128, E4M3): 1xG quantization, Group Scaling (standalone: steps
+    (i)-(iii)), the SwiGLU producer with fused maxima followed by Group
+    Scaling's steps (ii)-(iii), and dequantization.  The tensor (64 MiB of
+    BF16) fits in L2, so a 256 MiB buffer is written before every timed
+    launch to flush it; each launch is timed alone with CUDA events.  One
+    JSON line: elements/s of the 1xG quantizer as the headline, every
+    kernel's time, achieved GB/s and fraction of the measured HBM copy
+    bandwidth in `kernels`."""
+    import torch
+    import quantized_optimizer_states_b200 as coat
+    from quantized_optimizer_states_b200 import build as coat_build
+    from quantized_optimizer_states_b200 import inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    coat_build.build()
+    coat.load()
+    w = inputs.activations()
+    G = w.group_size
+    x = inputs.device_activations(w, dev)
+    gate, up = inputs.device_swiglu_inputs(w, dev)
+    n = x.numel()
+    ng = n // G
+    q = torch.empty(n, dtype=torch.uint8, device=dev)
+    sc = torch.empty(ng, dtype=torch.float32, device=dev)
+    ws = torch.empty(coat.coat_group_scaling_workspace_bytes(n, G) // 4, dtype=torch.float32,
+                     device=dev)
+    s1 = torch.empty(1, dtype=torch.float32, device=dev)
+    h = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(n, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    xf = x.reshape(-1)
+    cases = {
+        # name: (callable, algorithmic bytes per element)
+        "group_quant_1xG": (lambda: coat.coat_group_quant_1xG(x, q, sc, group_size=G),
+                            2 + 1 + 4.0 / G),
+        "group_scaling_standalone": (
+            lambda: coat.coat_group_scaling_quant_pertensor(xf, ws, q, s1, group_size=G),
+            2 + 2 + 1 + 8.0 / G),
+        "swiglu_fused_amax": (
+            lambda: coat.coat_swiglu_group_amax(gate.reshape(-1), up.reshape(-1), h, ws,
+                                                group_size=G),
+            2 + 2 + 2 + 4.0 / G),
+        "group_scaling_after_producer": (
+            lambda: coat.coat_group_scaling_quant_pertensor(h, ws, q, s1, group_size=G,
+                                                            amax_precomputed=True),
+            2 + 1 + 4.0 / G),
+        "dequant_pertensor": (
+            lambda: coat.coat_dequant(q, None, s1, out, group_size=n), 1 + 4),
+    }
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    res = {}
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(None)
+    sampler.start()
+    time.sleep(0.3)
+    for name, (fn, bpe) in cases.items():
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        gbs = bpe * n / (ms / 1e3) / 1e9
+        res[name] = {"ms": ms, "elements_per_s": n / (ms / 1e3), "GB/s": gbs,
+                     "frac_of_hbm": gbs / peak, "algorithmic_bytes_per_element": bpe}
+    clocks = sampler.stop()
+    head = res["group_quant_1xG"]
+    line = {"metric": "elements/s for 1xG FP8 activation quantization (BF16 [16384, 2048], G=128)",
+            "value": head["elements_per_s"], "unit": "elements/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "activations [16384, 2048] BF16 with GLU spike channels",
+                       "group_size": G, "fmt": "e4m3",
+                       "l2": "256 MiB buffer written before every timed launch"},
+            "roofline": {"bound": "hbm", "achieved": head["GB/s"], "peak": peak, "unit": "GB/s",
+                         "frac": head["frac_of_hbm"], "traffic": None,
+                         "peak_source": f"{peak_kind} copy bandwidth"},
+            "kernels": res, "clocks": clocks,
+            "gpu_launches": args.steps * (1 + 2 + 1 + 2 + 1)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -192,12 +285,18 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=1 << 25)
     ap.add_argument("--ref-sample", type=int, default=1 << 22)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="olmo-7b", choices=["olmo-7b", "olmo-1b", "sweep"])
+    ap.add_argument("--workload", default="olmo-7b",
+                    choices=["olmo-7b", "olmo-1b", "sweep", "activations"])
+    ap.add_argument("--group-size", type=int, default=128, help="sweep workload only")
+    ap.add_argument("--regime", default="late", choices=["early", "late", "typical"],
+                    help="sweep workload only")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "coat":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "activations":
+        return run_activations(args)
 
     import torch
     import torch.distributed as dist
@@ -225,7 +324,7 @@ def main():
         w = inputs.olmo_1b(seed=1235 + rank)
         w.v_fmt = args.v_fmt
     else:
-        w = inputs.sweep(128, args.v_fmt, "late", seed=1238 + rank)
+        w = inputs.sweep(args.group_size, args.v_fmt, args.regime, seed=1238 + rank)
     n, G = w.n, w.group_size
     ng = -(-n // G)
     hyper = dict(w.hyper)

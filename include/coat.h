@@ -242,8 +242,9 @@ coat_status_t coat_group_scaling_quant_pertensor_noalloc(const uint16_t *x, int6
  * This producer is the SwiGLU of a GLU MLP ([COAT] "激活为什么难压"), whose
  * output feeds the down projection:
  *   out[i] = RN_bf16(silu(gate[i]) * up[i]),  silu(g) = g / (1 + e^-g),
- * evaluated in binary32 (the library expf, then IEEE division and product,
- * then round to nearest even BF16).
+ * evaluated in binary32 with the hardware exp2 and reciprocal estimates
+ * (relative error ~2^-20), then rounded to nearest even BF16: the correctly
+ * rounded BF16 value except next to a rounding midpoint.
  *   gate, up    BF16 bits [n] (16-byte aligned)
  *   out         BF16 bits [n] (16-byte aligned)
  *   group_amax  float32[ceil(n/G)] (4-byte aligned): max |out| over each

@@ -72,6 +72,17 @@ __device__ __forceinline__ void cast16(const float *x, float inv, uint32_t *out)
                                 __fmul_rn(x[4 * w + 2], inv), __fmul_rn(x[4 * w + 3], inv));
 }
 
+// These kernels stream 2-6 bytes per element and nothing else, so each thread
+// handles kActV vectors of 16 elements (kActV consecutive 256-thread tiles
+// per block) and issues all of their loads before any arithmetic: twice the
+// bytes in flight per thread.
+constexpr int kActV = 2;
+
+inline unsigned int act_blocks(int64_t elems) {
+  const int64_t per = static_cast<int64_t>(kElemsPerBlock) * kActV;
+  return static_cast<unsigned int>((elems + per - 1) / per);
+}
+
 // ---- 1xG group quantization ---------------------------------------------------
 
 struct GroupQuantParams {
@@ -85,33 +96,42 @@ struct GroupQuantParams {
 
 template <int F>
 __global__ void __launch_bounds__(kThreads) group_quant_1xG_kernel(const GroupQuantParams p) {
-  __shared__ float red[kWarps];
-  const int64_t vid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-  const bool active = vid < p.rows * p.vec_per_row;
-  const int64_t row = active ? vid / p.vec_per_row : 0;
-  const int64_t c0 = (vid - row * p.vec_per_row) * kVec;
+  __shared__ float red[kActV][kWarps];
   const int lanes = 1 << (p.log2G - 4);
-  uint32_t w[8];
-  float x[16];
-  if (active) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.ld + c0);
-    uint4 a = src[0], b = src[1];
-    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-  } else {
+  const int64_t nvec = p.rows * p.vec_per_row;
+  uint32_t w[kActV][8];
+  int64_t row[kActV], c0[kActV];
+  bool active[kActV];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = 0;
+  for (int v = 0; v < kActV; ++v) {
+    const int64_t vid = (static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x;
+    active[v] = vid < nvec;
+    row[v] = active[v] ? vid / p.vec_per_row : 0;
+    c0[v] = (vid - row[v] * p.vec_per_row) * kVec;
+    if (active[v]) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row[v] * p.ld + c0[v]);
+      const uint4 a = src[0], b = src[1];
+      w[v][0] = a.x; w[v][1] = a.y; w[v][2] = a.z; w[v][3] = a.w;
+      w[v][4] = b.x; w[v][5] = b.y; w[v][6] = b.z; w[v][7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[v][i] = 0;
+    }
   }
-  unpack16_bf16(w, x);
-  const float amax = group_max(amax16(x), lanes, red);
-  float s, inv;
-  act_scale(amax, fmt_max<F>(), s, inv);
-  uint32_t o[4];
-  cast16<F>(x, inv, o);
-  if (active) {
-    *reinterpret_cast<uint4 *>(p.q + row * p.cols + c0) = make_uint4(o[0], o[1], o[2], o[3]);
-    if ((threadIdx.x & (lanes - 1)) == 0)
-      p.scale[row * (p.cols >> p.log2G) + (c0 >> p.log2G)] = s;
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    float x[16];
+    unpack16_bf16(w[v], x);
+    const float amax = group_max(amax16(x), lanes, red[v]);
+    float s, inv;
+    act_scale(amax, fmt_max<F>(), s, inv);
+    uint32_t o[4];
+    cast16<F>(x, inv, o);
+    if (active[v]) {
+      *reinterpret_cast<uint4 *>(p.q + row[v] * p.cols + c0[v]) = make_uint4(o[0], o[1], o[2], o[3]);
+      if ((threadIdx.x & (lanes - 1)) == 0)
+        p.scale[row[v] * (p.cols >> p.log2G) + (c0[v] >> p.log2G)] = s;
+    }
   }
 }
 
@@ -131,24 +151,31 @@ struct GroupScalingParams {
 // Step (i) (+ the block's share of step (ii)): per-group maxima of the BF16
 // input into group_amax, and the block maximum folded into tensor_amax.
 __global__ void __launch_bounds__(kThreads) group_amax_kernel(const GroupScalingParams p) {
-  __shared__ float red[kWarps];
+  __shared__ float red[kActV][kWarps];
   __shared__ float blockred[kWarps];
-  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
-  const bool active = e0 < p.n;
   const int lanes = 1 << (p.log2G - 4);
-  uint32_t w[8];
-  float x[16];
-  if (active) {
-    load16_bf16<false>(p.x, e0, p.n, w);
-  } else {
+  uint32_t w[kActV][8];
+  int64_t e0[kActV];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = 0;
+  for (int v = 0; v < kActV; ++v) {
+    e0[v] = ((static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x) * kVec;
+    if (e0[v] < p.n) {
+      load16_bf16<false>(p.x, e0[v], p.n, w[v]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[v][i] = 0;
+    }
   }
-  unpack16_bf16(w, x);
-  const float gmax = group_max(amax16(x), lanes, red);
-  if (active && (threadIdx.x & (lanes - 1)) == 0) p.group_amax[e0 >> p.log2G] = gmax;
+  float b = 0.0f;
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    float x[16];
+    unpack16_bf16(w[v], x);
+    const float gmax = group_max(amax16(x), lanes, red[v]);
+    if (e0[v] < p.n && (threadIdx.x & (lanes - 1)) == 0) p.group_amax[e0[v] >> p.log2G] = gmax;
+    b = fmaxf(b, gmax);
+  }
   // block max of the group maxima
-  float b = gmax;
   for (int off = 16; off > 0; off >>= 1) b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, off));
   if ((threadIdx.x & 31) == 0) blockred[threadIdx.x >> 5] = b;
   __syncthreads();
@@ -180,19 +207,26 @@ __global__ void __launch_bounds__(kThreads) amax_of_groups_kernel(const GroupSca
 // Step (iii): the per-tensor cast.
 template <int F>
 __global__ void __launch_bounds__(kThreads) pertensor_cast_kernel(const GroupScalingParams p) {
-  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+  uint32_t w[kActV][8];
+  int64_t e0[kActV];
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    e0[v] = ((static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x) * kVec;
+    if (e0[v] < p.n) load16_bf16<false>(p.x, e0[v], p.n, w[v]);
+  }
   const float amax = __uint_as_float(*p.tensor_amax);
   float s, inv;
   act_scale(amax, fmt_max<F>(), s, inv);
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.scale = s;
-  if (e0 >= p.n) return;
-  uint32_t w[8];
-  float x[16];
-  load16_bf16<false>(p.x, e0, p.n, w);
-  unpack16_bf16(w, x);
-  uint32_t o[4];
-  cast16<F>(x, inv, o);
-  store16_u8<false>(p.q, e0, p.n, o);
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    if (e0[v] >= p.n) continue;
+    float x[16];
+    unpack16_bf16(w[v], x);
+    uint32_t o[4];
+    cast16<F>(x, inv, o);
+    store16_u8<false>(p.q, e0[v], p.n, o);
+  }
 }
 
 // ---- a producer with Group Scaling's step (i) fused in: SwiGLU -------------------
@@ -202,9 +236,11 @@ __global__ void __launch_bounds__(kThreads) pertensor_cast_kernel(const GroupSca
 // (ii)) before its cast.  SwiGLU produces the input of an MLP's down
 // projection (the GLU layers of section "激活为什么难压"):
 //   out = RN_bf16(silu(gate) * up), silu(g) = g / (1 + e^-g),
-// evaluated in binary32 (expf, then IEEE division and product); the maxima
-// are taken over the BF16 outputs, i.e. exactly the values the quantizer
-// will read.
+// evaluated in binary32 with the special-function exp2 and reciprocal
+// (relative error ~2^-20 for |g| < 64, far below BF16's 2^-9 spacing: the
+// BF16 result is the correctly rounded one except next to a rounding
+// midpoint); the maxima are taken over the BF16 outputs, i.e. exactly the
+// values the quantizer will read.
 
 struct SwigluParams {
   const uint16_t *gate;
@@ -216,44 +252,50 @@ struct SwigluParams {
 };
 
 __global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const SwigluParams p) {
-  __shared__ float red[kWarps];
-  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
-  const bool active = e0 < p.n;
+  __shared__ float red[kActV][kWarps];
   const int lanes = 1 << (p.log2G - 4);
-  uint32_t gw[8], uw[8];
-  if (active) {
-    load16_bf16<false>(p.gate, e0, p.n, gw);
-    load16_bf16<false>(p.up, e0, p.n, uw);
-  } else {
+  uint32_t gw[kActV][8], uw[kActV][8];
+  int64_t e0[kActV];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) gw[i] = uw[i] = 0;
-  }
-  float g[16], u[16], h[16];
-  unpack16_bf16(gw, g);
-  unpack16_bf16(uw, u);
-  uint32_t ow[8];
+  for (int v = 0; v < kActV; ++v) {
+    e0[v] = ((static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x) * kVec;
+    if (e0[v] < p.n) {
+      load16_bf16<false>(p.gate, e0[v], p.n, gw[v]);
+      load16_bf16<false>(p.up, e0[v], p.n, uw[v]);
+    } else {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float a = __fmul_rn(__fdiv_rn(g[2 * i], __fadd_rn(1.0f, expf(-g[2 * i]))), u[2 * i]);
-    const float b =
-        __fmul_rn(__fdiv_rn(g[2 * i + 1], __fadd_rn(1.0f, expf(-g[2 * i + 1]))), u[2 * i + 1]);
-    const uint32_t ba = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a)));
-    const uint32_t bb = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(b)));
-    ow[i] = ba | (bb << 16);
-    h[2 * i] = bf16lo_to_float(ow[i]);
-    h[2 * i + 1] = bf16hi_to_float(ow[i]);
+      for (int i = 0; i < 8; ++i) gw[v][i] = uw[v][i] = 0;
+    }
   }
-  const float gmax = group_max(amax16(h), lanes, red);
-  if (!active) return;
-  if (e0 + 16 <= p.n) {
-    uint4 *dst = reinterpret_cast<uint4 *>(p.out + e0);
-    dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-    dst[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
-  } else {
-    for (int i = 0; i < 16; ++i)
-      if (e0 + i < p.n) p.out[e0 + i] = static_cast<uint16_t>(ow[i >> 1] >> (16 * (i & 1)));
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    float g[16], u[16], h[16];
+    unpack16_bf16(gw[v], g);
+    unpack16_bf16(uw[v], u);
+    uint32_t ow[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float a = __fmul_rn(__fdividef(g[2 * i], 1.0f + __expf(-g[2 * i])), u[2 * i]);
+      const float b =
+          __fmul_rn(__fdividef(g[2 * i + 1], 1.0f + __expf(-g[2 * i + 1])), u[2 * i + 1]);
+      const uint32_t ba = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a)));
+      const uint32_t bb = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(b)));
+      ow[i] = ba | (bb << 16);
+      h[2 * i] = bf16lo_to_float(ow[i]);
+      h[2 * i + 1] = bf16hi_to_float(ow[i]);
+    }
+    const float gmax = group_max(amax16(h), lanes, red[v]);
+    if (e0[v] >= p.n) continue;
+    if (e0[v] + 16 <= p.n) {
+      uint4 *dst = reinterpret_cast<uint4 *>(p.out + e0[v]);
+      dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      dst[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+    } else {
+      for (int i = 0; i < 16; ++i)
+        if (e0[v] + i < p.n) p.out[e0[v] + i] = static_cast<uint16_t>(ow[i >> 1] >> (16 * (i & 1)));
+    }
+    if ((threadIdx.x & (lanes - 1)) == 0) p.group_amax[e0[v] >> p.log2G] = gmax;
   }
-  if ((threadIdx.x & (lanes - 1)) == 0) p.group_amax[e0 >> p.log2G] = gmax;
 }
 
 // ---- dequantization ----------------------------------------------------------------
@@ -273,32 +315,7 @@ __device__ __forceinline__ uint32_t float_to_bf16_rn(float f) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
-template <int F>
-__global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p) {
-  __shared__ double tab8[8];
-  if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
-  __syncthreads();
-  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
-  if (e0 >= p.n) return;
-  const int64_t grp = p.log2G < 0 ? 0 : (e0 >> p.log2G);
-  const float s = p.scale[grp];
-  const float kk = p.k ? p.k[grp] : 1.0f;
-  const double rk = 1.0 / static_cast<double>(kk);
-  uint32_t w[4];
-  load16_u8<false>(p.q, e0, p.n, w);
-  float x[16];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float d[4];
-    fp8x4_to_float<F>(w[i], d);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (p.k)
-        x[4 * i + j] = dequant_exact(d[j], s, rk, tab8);
-      else
-        x[4 * i + j] = __fmul_rn(d[j], s);
-    }
-  }
+__device__ __forceinline__ void store16_out(const DequantParams &p, int64_t e0, const float *x) {
   if (p.out_bf16) {
     uint16_t *o = static_cast<uint16_t *>(p.out);
     if (e0 + 16 <= p.n) {
@@ -315,6 +332,59 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p
     }
   } else {
     store16_f32<false>(static_cast<float *>(p.out), e0, p.n, x);
+  }
+}
+
+// States (k given): x = sign(d) RN32(|d|^(1/k)) s per element, binary64.
+template <int F>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p) {
+  __shared__ double tab8[8];
+  if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
+  __syncthreads();
+  const int64_t e0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+  if (e0 >= p.n) return;
+  const int64_t grp = p.log2G < 0 ? 0 : (e0 >> p.log2G);
+  const float s = p.scale[grp];
+  const double rk = 1.0 / static_cast<double>(p.k[grp]);
+  uint32_t w[4];
+  load16_u8<false>(p.q, e0, p.n, w);
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float d[4];
+    fp8x4_to_float<F>(w[i], d);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) x[4 * i + j] = dequant_exact(d[j], s, rk, tab8);
+  }
+  store16_out(p, e0, x);
+}
+
+// Activations (no k): x = d * s, one binary32 product; kActV vectors per thread.
+template <int F>
+__global__ void __launch_bounds__(kThreads) dequant_linear_kernel(const DequantParams p) {
+  uint32_t w[kActV][4];
+  int64_t e0[kActV];
+  float s[kActV];
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    e0[v] = ((static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x) * kVec;
+    if (e0[v] < p.n) {
+      load16_u8<false>(p.q, e0[v], p.n, w[v]);
+      s[v] = p.scale[p.log2G < 0 ? 0 : (e0[v] >> p.log2G)];
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    if (e0[v] >= p.n) continue;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float d[4];
+      fp8x4_to_float<F>(w[v][i], d);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[4 * i + j] = __fmul_rn(d[j], s[v]);
+    }
+    store16_out(p, e0[v], x);
   }
 }
 

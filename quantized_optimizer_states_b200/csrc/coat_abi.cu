@@ -257,11 +257,19 @@ coat_status_t coat_dequant(const uint8_t *q, const float *k, const float *scale,
   p.out = out;
   fill_log2_table(p.log2_tab);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const unsigned int grid = blocks_for(n);
-  if (fmt == COAT_E4M3)
-    coat::dequant_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
-  else
-    coat::dequant_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  if (k) {
+    const unsigned int grid = blocks_for(n);
+    if (fmt == COAT_E4M3)
+      coat::dequant_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+    else
+      coat::dequant_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  } else {
+    const unsigned int grid = coat::act_blocks(n);
+    if (fmt == COAT_E4M3)
+      coat::dequant_linear_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+    else
+      coat::dequant_linear_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  }
   return launch_status();
 }
 
@@ -286,7 +294,7 @@ coat_status_t coat_group_quant_1xG(const uint16_t *x, int64_t rows, int64_t cols
   p.q = q;
   p.scale = scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const unsigned int grid = blocks_for(rows * cols);
+  const unsigned int grid = coat::act_blocks(rows * cols);
   if (fmt == COAT_E4M3)
     coat::group_quant_1xG_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
   else
@@ -328,9 +336,9 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
     const unsigned int grid = static_cast<unsigned int>(want < 1184 ? want : 1184);
     coat::amax_of_groups_kernel<<<grid, coat::kThreads, 0, s>>>(p);
   } else {
-    coat::group_amax_kernel<<<blocks_for(n), coat::kThreads, 0, s>>>(p);
+    coat::group_amax_kernel<<<coat::act_blocks(n), coat::kThreads, 0, s>>>(p);
   }
-  const unsigned int grid = blocks_for(n);
+  const unsigned int grid = coat::act_blocks(n);
   if (fmt == COAT_E4M3)
     coat::pertensor_cast_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
   else
@@ -356,7 +364,7 @@ coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, i
   p.log2G = lg;
   p.out = out;
   p.group_amax = group_amax;
-  coat::swiglu_group_amax_kernel<<<blocks_for(n), coat::kThreads, 0,
+  coat::swiglu_group_amax_kernel<<<coat::act_blocks(n), coat::kThreads, 0,
                                    static_cast<cudaStream_t>(stream)>>>(p);
   return launch_status();
 }
@@ -446,8 +454,8 @@ extern "C" coat_status_t coat_group_scaling_quant_pertensor_noalloc(
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the tensor maximum accumulates with atomicMax and must start at zero
   if (cudaMemsetAsync(p.tensor_amax, 0, sizeof(uint32_t), s) != cudaSuccess) return launch_status();
-  coat::group_amax_kernel<<<blocks_for(n), coat::kThreads, 0, s>>>(p);
-  const unsigned int grid = blocks_for(n);
+  coat::group_amax_kernel<<<coat::act_blocks(n), coat::kThreads, 0, s>>>(p);
+  const unsigned int grid = coat::act_blocks(n);
   if (fmt == COAT_E4M3)
     coat::pertensor_cast_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
   else

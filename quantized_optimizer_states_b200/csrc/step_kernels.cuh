@@ -104,10 +104,11 @@ struct StepLayout {
   static constexpr int kWarpTotal = kTableBytesPerWarp;  // multiple of 512
   static constexpr int kSmemBytes = kWarps * kWarpTotal;
   // resident blocks per SM the register budget is sized for (64 registers
-  // per thread at 4 blocks); G = 64 is held to 2 by its 16 tables per warp;
-  // groups spanning several warps (G >= 1024) run faster at 3 blocks with
-  // 80 registers (measured: 311 vs 196 G params/s at G = 1024)
-  static constexpr int kMinBlocks = LG <= 6 ? 2 : (LG >= 10 ? 3 : 4);
+  // per thread at 4 blocks).  G = 64 (16 tables, 64 KB of shared memory per
+  // block) fits 3 blocks; groups spanning several warps (G >= 1024) also run
+  // faster at 3 blocks with 80 registers (measured: 311 vs 196 G params/s at
+  // G = 1024, 260 vs 233 at G = 64); the direct-decode G < 64 kernels use 2
+  static constexpr int kMinBlocks = LG <= 5 ? 2 : ((LG == 6 || LG >= 10) ? 3 : 4);
 };
 
 // Dynamic shared memory of the step kernel for group size 2^log2G.

@@ -235,6 +235,18 @@ coat_status_t coat_group_scaling_quant_pertensor_noalloc(const uint16_t *x, int6
                                                          void *stream);
 
 /*
+ * coat_fp8_encode -- the FP8 cast alone: code = RNE_satfinite(y), the last
+ * operation of every quantizer here.  [ATLAS] 03 "FP8": E4M3 (bias 7, max
+ * 448, no infinity) and E5M2 (bias 15, max 57344); round to nearest even;
+ * finite values beyond the largest magnitude and infinities saturate to
+ * +-max; NaN gives a NaN code (either sign).
+ *   y  float32[n] (16-byte aligned)
+ *   q  uint8[n] codes (16-byte aligned)
+ * Errors: INVALID_ARG, UNSUPPORTED (format), MISALIGNED, CUDA.
+ */
+coat_status_t coat_fp8_encode(const float *y, int64_t n, int32_t fmt, uint8_t *q, void *stream);
+
+/*
  * coat_swiglu_group_amax -- a producing kernel with Group Scaling's step (i)
  * fused in.  [COAT] "混合粒度": the per-1xG maxima of a linear layer's
  * input are emitted by the kernel that produces it, so the per-tensor

@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     CoatError,
     coat_adamw_fp8_step,
     coat_dequant,
+    coat_fp8_encode,
     coat_group_quant_1xG,
     coat_group_scaling_quant_pertensor,
     coat_group_scaling_quant_pertensor_noalloc,

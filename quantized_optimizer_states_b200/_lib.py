@@ -65,6 +65,7 @@ SIGNATURES = {
     "coat_group_scaling_quant_pertensor": (_I32, [_P, _I64, _I32, _I32, _P, _I32, _P, _P, _P]),
     "coat_group_scaling_quant_pertensor_noalloc": (_I32, [_P, _I64, _I32, _I32, _P, _P, _P]),
     "coat_swiglu_group_amax": (_I32, [_P, _P, _I64, _I32, _P, _P, _P]),
+    "coat_fp8_encode": (_I32, [_P, _I64, _I32, _P, _P]),
     "coat_last_cuda_error": (_I32, []),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
     "coat_version": (_I32, []),
@@ -224,6 +225,16 @@ def coat_swiglu_group_amax(gate, up, out, group_amax, *, group_size: int = 128, 
         _u16(gate, "gate"), _u16(up, "up"), gate.numel(), group_size, _u16(out, "out"),
         _ptr(group_amax, torch.float32, "group_amax"), _stream(stream))
     _check("coat_swiglu_group_amax", st)
+
+
+def coat_fp8_encode(y, q, *, fmt: int = COAT_E4M3, stream=None):
+    """q = RNE_satfinite FP8 codes of the float32 tensor y."""
+    import torch
+    if q.numel() != y.numel():
+        raise ValueError("y and q must have the same number of elements")
+    st = load().coat_fp8_encode(_ptr(y, torch.float32, "y"), y.numel(), fmt,
+                                _ptr(q, torch.uint8, "q"), _stream(stream))
+    _check("coat_fp8_encode", st)
 
 
 def coat_version() -> int:

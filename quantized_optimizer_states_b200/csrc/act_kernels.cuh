@@ -298,6 +298,37 @@ __global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const Swigl
   }
 }
 
+// ---- the FP8 cast alone -------------------------------------------------------------
+// code = RNE_satfinite(y): round to nearest even, finite values beyond the
+// format's largest magnitude (and infinities) saturate to +-max, NaN gives a
+// NaN code (LLM Atlas "systems/numerics", section 03 "FP8": E4M3 max 448,
+// E5M2 max 57344).  The hardware cvt that every quantizer here ends with.
+struct EncodeParams {
+  const float *y;
+  int64_t n;
+  uint8_t *q;
+};
+
+template <int F>
+__global__ void __launch_bounds__(kThreads) fp8_encode_kernel(const EncodeParams p) {
+  float x[kActV][16];
+  int64_t e0[kActV];
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    e0[v] = ((static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x) * kVec;
+    if (e0[v] < p.n) load16_f32<false>(p.y, e0[v], p.n, x[v]);
+  }
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    if (e0[v] >= p.n) continue;
+    uint32_t o[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      o[w] = float4_to_fp8x4<F>(x[v][4 * w], x[v][4 * w + 1], x[v][4 * w + 2], x[v][4 * w + 3]);
+    store16_u8<false>(p.q, e0[v], p.n, o);
+  }
+}
+
 // ---- dequantization ----------------------------------------------------------------
 
 struct DequantParams {

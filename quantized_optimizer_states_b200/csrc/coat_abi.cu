@@ -369,6 +369,25 @@ coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, i
   return launch_status();
 }
 
+coat_status_t coat_fp8_encode(const float *y, int64_t n, int32_t fmt, uint8_t *q,
+                              void *stream) {
+  if (n < 0) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && (!y || !q)) return COAT_ERR_INVALID_ARG;
+  if (!valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
+  if (n == 0) return COAT_OK;
+  if (!aligned16(y) || !aligned16(q)) return COAT_ERR_MISALIGNED;
+  coat::EncodeParams p;
+  p.y = y;
+  p.n = n;
+  p.q = q;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fmt == COAT_E4M3)
+    coat::fp8_encode_kernel<coat::kE4M3><<<coat::act_blocks(n), coat::kThreads, 0, s>>>(p);
+  else
+    coat::fp8_encode_kernel<coat::kE5M2><<<coat::act_blocks(n), coat::kThreads, 0, s>>>(p);
+  return launch_status();
+}
+
 int32_t coat_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char *coat_status_string(coat_status_t status) {

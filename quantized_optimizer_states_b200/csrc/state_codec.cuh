@@ -75,7 +75,8 @@ struct GroupQ {
   bool zero;   // all-zero group
 };
 
-// ln(x) for a positive normal binary64 x, without branches: x = 2^e m with
+// ln(x) for a positive normal binary64 x (+inf and NaN are returned as they
+// are), without branches: x = 2^e m with
 // m in [~sqrt(1/2), ~sqrt(2)), ln m = 2 atanh(s) = 2 (s + s^3/3 + s^5/5 + ...)
 // with s = (m - 1)/(m + 1), |s| <= 0.1716, summed to s^21 (remainder below
 // 2^-56 of the result); e ln 2 with ln 2 split in two parts.  Error a few
@@ -102,7 +103,8 @@ __device__ __forceinline__ double log_d(double x) {
   constexpr double kLn2Hi = 0x1.62e42fefa3800p-1;  // ln 2, leading 43 bits
   constexpr double kLn2Lo = 0x1.ef35793c76730p-45; // ln 2 - kLn2Hi
   const double ed = static_cast<double>(e);
-  return fma(ed, kLn2Hi, fma(ed, kLn2Lo, lnm));
+  const double r = fma(ed, kLn2Hi, fma(ed, kLn2Lo, lnm));
+  return x < __longlong_as_double(0x7FF0000000000000LL) ? r : x;  // inf, NaN pass through
 }
 
 // k = ln(R_target) / ln(M / mn) in binary64, rounded once, clamped to k_max;

@@ -218,3 +218,53 @@ def test_argument_errors(lib):
     e0 = torch.empty(0, dtype=torch.float32, device="cuda")
     lib.coat_adamw_fp8_step(e0, g[:0], mc[:0], meta[0], meta[1], vc[:0], meta[2], meta[3],
                             group_size=128, **base)
+
+
+def _step_cfg(orc, lib, x, st, *, G, t, v_fmt, hyper):
+    cfg = dict(step=t, group_size=G, v_fmt=v_fmt, k_range=0, k_max=64.0, **hyper)
+    ref = orc.adamw_fp8_step(x["theta"], x["grad"], *st, return_moments=True, **cfg)
+    got = parity.gpu_step(lib, x["theta"], x["grad"], *st, flags=0, **cfg)
+    return parity.assert_step_parity(got, ref, hyper["lr"], G, v_fmt,
+                                     moments=(ref[7], ref[8]))
+
+
+def test_exact_path_when_the_estimates_are_disabled(lib, orc):
+    """eps = 0 leaves the estimate-based quotient's range: every warp takes
+    the fully IEEE path."""
+    x = inputs.host_step_inputs(inputs.tiny(61), 3 * 4096 + 100)
+    st = _init_states(orc, x, 128, E4M3)
+    _step_cfg(orc, lib, x, st, G=128, t=10, v_fmt=E4M3, hyper=dict(H, eps=0.0))
+
+
+def test_exact_path_for_out_of_range_moments(lib, orc):
+    """A group whose second moment is tiny (v_t < 2^-120 with a zero
+    gradient) and one whose gradients are huge (v_t far above the estimates'
+    range) make their warps rewrite theta with the IEEE operations; the
+    other warps keep the estimate-based result.  All against the oracle."""
+    G = 128
+    n = 8 * 4096
+    x = inputs.host_step_inputs(inputs.tiny(62), n)
+    x["v0"][3 * G:4 * G] = 1e-38
+    x["grad"][3 * G:4 * G] = 0
+    big = orc.to_bf16_array(np.full(G, 1e19, dtype=np.float32))
+    x["grad"][9 * G:10 * G] = big
+    x["grad"][9 * G + 1:10 * G:2] ^= 0x8000          # alternate signs
+    st = _init_states(orc, x, G, E4M3)
+    _step_cfg(orc, lib, x, st, G=G, t=10, v_fmt=E4M3, hyper=H)
+
+
+@pytest.mark.parametrize("G", [128, 1024])
+def test_group_parameters_special_cases(lib, orc, G):
+    """Branch-free k and s on all-equal groups (k = 1, s = M / fmax), a
+    group whose range would exceed k_max (clamped) and ordinary groups,
+    with v in E5M2."""
+    n = 6 * G
+    x = inputs.host_step_inputs(inputs.tiny(63), n)
+    x["m0"][:G] = 3e-4
+    x["v0"][:G] = 5e-8
+    x["grad"][:G] = 0
+    x["m0"][G:2 * G] = np.where(np.arange(G) % 2, 1e-4, 1.0001e-4).astype(np.float32)
+    x["v0"][G:2 * G] = np.where(np.arange(G) % 2, 2e-8, 2.00001e-8).astype(np.float32)
+    x["grad"][G:2 * G] = 0
+    st = _init_states(orc, x, G, E5M2)
+    _step_cfg(orc, lib, x, st, G=G, t=10, v_fmt=E5M2, hyper=H)

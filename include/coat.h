@@ -61,7 +61,7 @@ typedef enum coat_status {
     COAT_ERR_MISALIGNED = 2,  /* a vector-accessed buffer is not 16-byte aligned */
     COAT_ERR_UNSUPPORTED = 3, /* format / group size / flag combination not built */
     COAT_ERR_CUDA = 4,        /* a CUDA launch or query failed */
-    COAT_ERR_NONFINITE = 5,   /* reserved: non-finite gradient detection */
+    COAT_ERR_NONFINITE = 5,   /* reserved */
     COAT_ERR_TIMEOUT = 6      /* reserved: a bounded device wait ran out */
 } coat_status_t;
 
@@ -123,6 +123,37 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
                                   float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
                                   float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
                                   void *stream);
+
+/*
+ * coat_count_nonfinite_bf16 -- *count += the number of BF16 values in x that
+ * are +-inf or NaN (all-ones exponent).  The caller zeroes *count first.
+ * With coat_adamw_fp8_step_guarded this skips a step on overflowed
+ * gradients without a host round trip (the pages define no behaviour for
+ * non-finite gradients; skipping the step is the usual mixed-precision
+ * convention).
+ *   x      BF16 bits [n] (16-byte aligned)
+ *   count  uint32[1] (4-byte aligned), accumulated atomically
+ * Errors: INVALID_ARG, UNSUPPORTED (n too large), MISALIGNED, CUDA.
+ */
+coat_status_t coat_count_nonfinite_bf16(const uint16_t *x, int64_t n, uint32_t *count,
+                                        void *stream);
+
+/*
+ * coat_adamw_fp8_step_guarded -- coat_adamw_fp8_step, except that the
+ * kernel first reads the device word *skip_if_nonzero and, if it is not
+ * zero, returns without reading or writing anything else: parameters,
+ * codes, k and s keep their values (for example, skip_if_nonzero = the
+ * count of coat_count_nonfinite_bf16 on grad).  The decision is made on the
+ * device, so the call stays asynchronous; cfg->step is still the caller's
+ * step count (a skipped step leaves it to the caller whether to advance it).
+ * Arguments and errors as coat_adamw_fp8_step; skip_if_nonzero must be a
+ * 4-byte-aligned device pointer (INVALID_ARG if NULL, MISALIGNED).
+ */
+coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, uint8_t *m_code,
+                                          float *m_k, float *m_scale, uint8_t *v_code,
+                                          float *v_k, float *v_scale, int64_t n,
+                                          const coat_adamw_cfg_t *cfg,
+                                          const uint32_t *skip_if_nonzero, void *stream);
 
 /*
  * coat_quantize_state -- compress an FP32 optimizer state into COAT's FP8

@@ -66,6 +66,9 @@ SIGNATURES = {
     "coat_group_scaling_quant_pertensor_noalloc": (_I32, [_P, _I64, _I32, _I32, _P, _P, _P]),
     "coat_swiglu_group_amax": (_I32, [_P, _P, _I64, _I32, _P, _P, _P]),
     "coat_fp8_encode": (_I32, [_P, _I64, _I32, _P, _P]),
+    "coat_count_nonfinite_bf16": (_I32, [_P, _I64, _P, _P]),
+    "coat_adamw_fp8_step_guarded": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
+                                           ctypes.POINTER(CoatAdamwCfg), _P, _P]),
     "coat_last_cuda_error": (_I32, []),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
     "coat_version": (_I32, []),
@@ -124,18 +127,38 @@ def _u16(t, what):
 def coat_adamw_fp8_step(param, grad, m_code, m_k, m_scale, v_code, v_k, v_scale, *, beta1: float,
                         beta2: float, lr: float, eps: float, weight_decay: float, step: int,
                         group_size: int = 128, m_fmt: int = COAT_E4M3, v_fmt: int = COAT_E4M3,
-                        k_range: int = 0, k_max: float = 64.0, flags: int = 0, stream=None):
-    """One fused COAT AdamW step, in place (see include/coat.h)."""
+                        k_range: int = 0, k_max: float = 64.0, flags: int = 0,
+                        skip_if_nonzero=None, stream=None):
+    """One fused COAT AdamW step, in place (see include/coat.h).  With
+    skip_if_nonzero (a CUDA int32/uint32 tensor of one element) the guarded
+    form runs: the step is a no-op when that word is nonzero."""
     import torch
     cfg = CoatAdamwCfg(beta1, beta2, lr, eps, weight_decay, step, group_size, m_fmt, v_fmt,
                        k_range, k_max, flags)
-    st = load().coat_adamw_fp8_step(
-        _ptr(param, torch.float32, "param"), _u16(grad, "grad"),
-        _ptr(m_code, torch.uint8, "m_code"), _ptr(m_k, torch.float32, "m_k"),
-        _ptr(m_scale, torch.float32, "m_scale"), _ptr(v_code, torch.uint8, "v_code"),
-        _ptr(v_k, torch.float32, "v_k"), _ptr(v_scale, torch.float32, "v_scale"),
-        param.numel(), ctypes.byref(cfg), _stream(stream))
-    _check("coat_adamw_fp8_step", st)
+    args = [_ptr(param, torch.float32, "param"), _u16(grad, "grad"),
+            _ptr(m_code, torch.uint8, "m_code"), _ptr(m_k, torch.float32, "m_k"),
+            _ptr(m_scale, torch.float32, "m_scale"), _ptr(v_code, torch.uint8, "v_code"),
+            _ptr(v_k, torch.float32, "v_k"), _ptr(v_scale, torch.float32, "v_scale"),
+            param.numel(), ctypes.byref(cfg)]
+    if skip_if_nonzero is None:
+        st = load().coat_adamw_fp8_step(*args, _stream(stream))
+        _check("coat_adamw_fp8_step", st)
+    else:
+        if skip_if_nonzero.dtype not in (torch.int32, torch.uint32):
+            raise ValueError("skip_if_nonzero must be an int32/uint32 tensor")
+        st = load().coat_adamw_fp8_step_guarded(*args, _ptr(skip_if_nonzero, None, "skip"),
+                                                _stream(stream))
+        _check("coat_adamw_fp8_step_guarded", st)
+
+
+def coat_count_nonfinite_bf16(x, count, *, stream=None):
+    """count[0] += number of inf/NaN values in the BF16 tensor x."""
+    import torch
+    if count.dtype not in (torch.int32, torch.uint32):
+        raise ValueError("count must be an int32/uint32 tensor")
+    st = load().coat_count_nonfinite_bf16(_u16(x, "x"), x.numel(), _ptr(count, None, "count"),
+                                          _stream(stream))
+    _check("coat_count_nonfinite_bf16", st)
 
 
 def coat_quantize_state(x, code, k, scale, *, group_size: int = 128, fmt: int = COAT_E4M3,

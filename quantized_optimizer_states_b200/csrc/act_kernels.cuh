@@ -329,6 +329,41 @@ __global__ void __launch_bounds__(kThreads) fp8_encode_kernel(const EncodeParams
   }
 }
 
+// ---- non-finite gradient count ----------------------------------------------------
+// *count += number of BF16 values with an all-ones exponent (inf or NaN).
+struct CountParams {
+  const uint16_t *x;
+  int64_t n;
+  uint32_t *count;
+};
+
+__global__ void __launch_bounds__(kThreads) count_nonfinite_bf16_kernel(const CountParams p) {
+  __shared__ uint32_t part[kWarps];
+  uint32_t c = 0;
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    const int64_t e0 =
+        ((static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x) * kVec;
+    if (e0 < p.n) {
+      uint32_t w[8];
+      load16_bf16<false>(p.x, e0, p.n, w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c += ((w[i] & 0x7F80u) == 0x7F80u) ? 1u : 0u;
+        c += ((w[i] & 0x7F800000u) == 0x7F800000u) ? 1u : 0u;
+      }
+    }
+  }
+  for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+    for (int i = 0; i < kWarps; ++i) t += part[i];
+    if (t) atomicAdd(p.count, t);
+  }
+}
+
 // ---- dequantization ----------------------------------------------------------------
 
 struct DequantParams {

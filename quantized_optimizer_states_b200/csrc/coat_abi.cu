@@ -123,14 +123,10 @@ coat_status_t launch_step_all(int lg, int64_t n, size_t smem, cudaStream_t s,
   return COAT_OK;
 }
 
-}  // namespace
 
-extern "C" {
-
-coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m_code,
-                                  float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
-                                  float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
-                                  void *stream) {
+coat_status_t step_impl(float *param, const uint16_t *grad, uint8_t *m_code, float *m_k,
+                        float *m_scale, uint8_t *v_code, float *v_k, float *v_scale, int64_t n,
+                        const coat_adamw_cfg_t *cfg, const uint32_t *skip, void *stream) {
   if (!cfg || n < 0) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!param || !grad || !m_code || !m_k || !m_scale || !v_code || !v_k || !v_scale))
     return COAT_ERR_INVALID_ARG;
@@ -188,6 +184,7 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
   // numbers, and |m_t| <= 2^100 bc1 eps keeps m^ / (sqrt(v^) + eps) below
   // 2^100.  A non-normal eps disables the fast form.
   p.block0 = 0;
+  p.skip = skip;
   if (p.eps >= 0x1p-100f && p.eps <= 0x1p+20f) {
     p.fast_vmin = 0x1p-120f;
     p.fast_vmax = static_cast<float>(std::ldexp(static_cast<double>(p.bc2), 100));
@@ -202,6 +199,45 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
   const size_t smem = coat::step_smem_bytes(lg);
   return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3>(lg, n, smem, s, p)
                                  : launch_step_all<coat::kE5M2>(lg, n, smem, s, p);
+}
+
+}  // namespace
+
+extern "C" {
+
+coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m_code,
+                                  float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
+                                  float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
+                                  void *stream) {
+  return step_impl(param, grad, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg, nullptr,
+                   stream);
+}
+
+coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, uint8_t *m_code,
+                                          float *m_k, float *m_scale, uint8_t *v_code,
+                                          float *v_k, float *v_scale, int64_t n,
+                                          const coat_adamw_cfg_t *cfg,
+                                          const uint32_t *skip_if_nonzero, void *stream) {
+  if (!skip_if_nonzero || (reinterpret_cast<uintptr_t>(skip_if_nonzero) & 3u) != 0)
+    return skip_if_nonzero ? COAT_ERR_MISALIGNED : COAT_ERR_INVALID_ARG;
+  return step_impl(param, grad, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
+                   skip_if_nonzero, stream);
+}
+
+coat_status_t coat_count_nonfinite_bf16(const uint16_t *x, int64_t n, uint32_t *count,
+                                        void *stream) {
+  if (n < 0 || !count) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && !x) return COAT_ERR_INVALID_ARG;
+  if (n > kMaxElems) return COAT_ERR_UNSUPPORTED;
+  if (n == 0) return COAT_OK;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(count) & 3u) != 0) return COAT_ERR_MISALIGNED;
+  coat::CountParams p;
+  p.x = x;
+  p.n = n;
+  p.count = count;
+  coat::count_nonfinite_bf16_kernel<<<coat::act_blocks(n), coat::kThreads, 0,
+                                      static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
 }
 
 coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size, int32_t fmt,

@@ -67,6 +67,7 @@ struct StepParams {
   int64_t n;
   int64_t ngroups;
   int64_t block0;     // index of this launch's first block of kElemsPerBlock parameters
+  const uint32_t *skip;  // nullable: a nonzero word here makes the step a no-op
   float beta1, beta2, c1, c2, bc1, bc2, rbc1, rbc2, decay, lr, eps;
   // The estimate-based quotient is used for a thread's 16 elements when
   // max|m_t| <= fast_mmax, max v_t <= fast_vmax and every nonzero v_t >=
@@ -441,6 +442,10 @@ adamw_fp8_step_kernel(const StepParams p) {
   if constexpr (!L::kTable) {
     if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
   }
+
+  // guarded form: the whole grid leaves before touching anything (the word
+  // is the same for every thread, so no barrier below is split)
+  if (p.skip != nullptr && *p.skip != 0u) return;
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;

@@ -82,11 +82,14 @@ class CoatAdamW(torch.optim.Optimizer):
       k_range: 0 = k fills E4M3's range for both moments, 1 = the storage
         format's own range.
       k_max: clamp of the expansion exponent (0 = none).
+      skip_nonfinite: count inf/NaN gradients first (on the device) and skip
+        the whole step of a parameter group that has any; the group's step
+        counter then does not advance (one host read of the count per step).
     """
 
     def __init__(self, params, lr: float = 1e-3, betas=(0.9, 0.999), eps: float = 1e-8,
                  weight_decay: float = 1e-2, *, group_size: int = 128, v_fmt="e4m3",
-                 k_range: int = 0, k_max: float = 64.0):
+                 k_range: int = 0, k_max: float = 64.0, skip_nonfinite: bool = False):
         if not 0.0 <= betas[0] < 1.0 or not 0.0 <= betas[1] < 1.0:
             raise ValueError("betas must be in [0, 1)")
         if lr < 0.0 or eps < 0.0 or weight_decay < 0.0:
@@ -97,6 +100,8 @@ class CoatAdamW(torch.optim.Optimizer):
                         group_size=group_size, v_fmt=_FMT[v_fmt], k_range=k_range,
                         k_max=k_max)
         super().__init__(params, defaults)
+        self.skip_nonfinite = skip_nonfinite
+        self.skipped_steps = 0
         self._flat: list[_FlatGroup] = [self._build(g) for g in self.param_groups]
 
     # ---- flat buffers --------------------------------------------------------
@@ -152,6 +157,12 @@ class CoatAdamW(torch.optim.Optimizer):
                 loss = closure()
         for group, fg in zip(self.param_groups, self._flat):
             self._gather_grads(fg)
+            if self.skip_nonfinite:
+                count = torch.zeros(1, dtype=torch.int32, device=fg.grad.device)
+                _lib.coat_count_nonfinite_bf16(fg.grad, count)
+                if int(count.item()) != 0:
+                    self.skipped_steps += 1
+                    continue
             fg.step += 1
             b1, b2 = group["betas"]
             _lib.coat_adamw_fp8_step(

@@ -67,12 +67,12 @@ unsigned int blocks_for(int64_t elems) {
   return static_cast<unsigned int>((elems + coat::kElemsPerBlock - 1) / coat::kElemsPerBlock);
 }
 
-constexpr int64_t kMaxElems = int64_t{1} << 42;  // within the grid-size bound (2^31 - 1 blocks x 4096)
+constexpr int64_t kMaxElems = int64_t{1} << 42;  // within the grid-size bound (2^31 - 1 blocks x 2048)
 
 // Launch one instantiation of the step kernel, raising its dynamic shared
 // memory limit first when the decode tables need more than the default.
-coat_status_t launch_step(void (*kernel)(coat::StepParams), unsigned int grid, size_t smem,
-                          cudaStream_t s, const coat::StepParams &p) {
+coat_status_t launch_step(void (*kernel)(coat::StepParams), unsigned int grid, int block,
+                          size_t smem, cudaStream_t s, const coat::StepParams &p) {
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(
         kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -81,48 +81,48 @@ coat_status_t launch_step(void (*kernel)(coat::StepParams), unsigned int grid, s
       return COAT_ERR_CUDA;
     }
   }
-  kernel<<<grid, coat::kThreads, smem, s>>>(p);
+  kernel<<<grid, block, smem, s>>>(p);
   return launch_status();
 }
 
 // The step kernel is instantiated for each supported group size and for
 // full blocks / the ragged tail block.
 template <int VF, bool FULL>
-coat_status_t launch_step_for(int lg, unsigned int grid, size_t smem, cudaStream_t s,
+coat_status_t launch_step_for(int lg, unsigned int grid, int block, size_t smem, cudaStream_t s,
                               const coat::StepParams &p) {
   switch (lg) {
-    case 4: return launch_step(coat::adamw_fp8_step_kernel<VF, 4, FULL>, grid, smem, s, p);
-    case 5: return launch_step(coat::adamw_fp8_step_kernel<VF, 5, FULL>, grid, smem, s, p);
-    case 6: return launch_step(coat::adamw_fp8_step_kernel<VF, 6, FULL>, grid, smem, s, p);
-    case 7: return launch_step(coat::adamw_fp8_step_kernel<VF, 7, FULL>, grid, smem, s, p);
-    case 8: return launch_step(coat::adamw_fp8_step_kernel<VF, 8, FULL>, grid, smem, s, p);
-    case 9: return launch_step(coat::adamw_fp8_step_kernel<VF, 9, FULL>, grid, smem, s, p);
-    case 10: return launch_step(coat::adamw_fp8_step_kernel<VF, 10, FULL>, grid, smem, s, p);
-    case 11: return launch_step(coat::adamw_fp8_step_kernel<VF, 11, FULL>, grid, smem, s, p);
-    case 12: return launch_step(coat::adamw_fp8_step_kernel<VF, 12, FULL>, grid, smem, s, p);
+#define COAT_LAUNCH(LGV) \
+  case LGV:              \
+    return launch_step(coat::adamw_fp8_step_kernel<VF, LGV, FULL>, grid, block, smem, s, p);
+    COAT_LAUNCH(4) COAT_LAUNCH(5) COAT_LAUNCH(6) COAT_LAUNCH(7) COAT_LAUNCH(8)
+    COAT_LAUNCH(9) COAT_LAUNCH(10) COAT_LAUNCH(11) COAT_LAUNCH(12)
+#undef COAT_LAUNCH
   }
   return COAT_ERR_UNSUPPORTED;
 }
 
-// One launch over the full 4096-parameter blocks (no bounds checks), then,
-// if n is not a multiple of 4096, one block for the ragged tail.
+// One launch over the full blocks (no bounds checks), then, if n is not a
+// multiple of the block's parameter count, one block for the ragged tail.
 template <int VF>
-coat_status_t launch_step_all(int lg, int64_t n, size_t smem, cudaStream_t s,
-                              coat::StepParams p) {
-  const int64_t full = n / coat::kElemsPerBlock;
+coat_status_t launch_step_all(int lg, int64_t n, cudaStream_t s, coat::StepParams p) {
+  size_t smem = 0;
+  int block = 0;
+  coat::step_launch_shape(lg, smem, block);
+  if (block == 0) return COAT_ERR_UNSUPPORTED;
+  const int64_t per = static_cast<int64_t>(block) * coat::kVec;
+  const int64_t full = n / per;
   if (full > 0) {
     p.block0 = 0;
     const coat_status_t st =
-        launch_step_for<VF, true>(lg, static_cast<unsigned int>(full), smem, s, p);
+        launch_step_for<VF, true>(lg, static_cast<unsigned int>(full), block, smem, s, p);
     if (st != COAT_OK) return st;
   }
-  if (n % coat::kElemsPerBlock != 0) {
+  if (n % per != 0) {
     p.block0 = full;
-    return launch_step_for<VF, false>(lg, 1u, smem, s, p);
+    return launch_step_for<VF, false>(lg, 1u, block, smem, s, p);
   }
   return COAT_OK;
 }
-
 
 coat_status_t step_impl(float *param, const uint16_t *grad, uint8_t *m_code, float *m_k,
                         float *m_scale, uint8_t *v_code, float *v_k, float *v_scale, int64_t n,
@@ -196,9 +196,8 @@ coat_status_t step_impl(float *param, const uint16_t *grad, uint8_t *m_code, flo
   }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t smem = coat::step_smem_bytes(lg);
-  return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3>(lg, n, smem, s, p)
-                                 : launch_step_all<coat::kE5M2>(lg, n, smem, s, p);
+  return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3>(lg, n, s, p)
+                                 : launch_step_all<coat::kE5M2>(lg, n, s, p);
 }
 
 }  // namespace

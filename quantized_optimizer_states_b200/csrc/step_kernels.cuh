@@ -66,7 +66,7 @@ struct StepParams {
   float *v_s;
   int64_t n;
   int64_t ngroups;
-  int64_t block0;     // index of this launch's first block of kElemsPerBlock parameters
+  int64_t block0;     // index of this launch's first block (of StepLayout::kBlockElems)
   const uint32_t *skip;  // nullable: a nonzero word here makes the step a no-op
   float beta1, beta2, c1, c2, bc1, bc2, rbc1, rbc2, decay, lr, eps;
   // The estimate-based quotient is used for a thread's 16 elements when
@@ -95,6 +95,15 @@ struct QuantParams {
 // Compile-time layout of the step kernel for group size 2^LG.
 template <int LG>
 struct StepLayout {
+  // Threads per block: 64 (2 warps), or the threads of one group where that
+  // is more (128 for G = 2048, 256 for G = 4096).  Small blocks finish at
+  // different times, so the warps of an SM spread over the kernel's phases
+  // (table build, update, encode) and use the special-function, FP64 and
+  // shared-memory pipes more evenly (measured against 256-thread blocks:
+  // +7% at G = 128, +10% at G = 256, +15% at G = 1024).
+  static constexpr int kBlock = LG >= 12 ? 256 : (LG == 11 ? 128 : 64);
+  static constexpr int kBlockWarps = kBlock / 32;
+  static constexpr int kBlockElems = kBlock * kVec;
   static constexpr int kLanes = 1 << (LG - 4);               // threads per group
   static constexpr bool kTable = LG >= kMinTableLog2G;
   static constexpr int kGPW = LG <= 9 ? (512 >> LG) : 1;     // groups a warp touches
@@ -103,28 +112,33 @@ struct StepLayout {
   static constexpr int kRounds = kTW >= 8 ? kTW / 8 : 1;     // tables per lane
   static constexpr int kTableBytesPerWarp = kTable ? kTW * kTableBytes : 0;
   static constexpr int kWarpTotal = kTableBytesPerWarp;  // multiple of 512
-  static constexpr int kSmemBytes = kWarps * kWarpTotal;
-  // resident blocks per SM the register budget is sized for (64 registers
-  // per thread at 4 blocks).  G = 64 (16 tables, 64 KB of shared memory per
-  // block) fits 3 blocks; groups spanning several warps (G >= 1024) also run
-  // faster at 3 blocks with 80 registers (measured: 311 vs 196 G params/s at
-  // G = 1024, 260 vs 233 at G = 64); the direct-decode G < 64 kernels use 2
-  static constexpr int kMinBlocks = LG <= 5 ? 2 : ((LG == 6 || LG >= 10) ? 3 : 4);
+  static constexpr int kSmemBytes = kBlockWarps * kWarpTotal;
+  // resident warps per SM the register budget is sized for: 32 (64
+  // registers per thread); 24 for G = 64 (16 tables, 32 KB of shared memory
+  // per 4 warps) and for groups spanning several warps (G >= 1024), which run
+  // faster with 80 registers (measured: 311 vs 196 G params/s at G = 1024,
+  // 260 vs 233 at G = 64); 16 for the direct-decode G < 64 kernels
+  static constexpr int kMinWarps = LG <= 5 ? 16 : ((LG == 6 || LG >= 10) ? 24 : 32);
+  static constexpr int kMinBlocks = kMinWarps / kBlockWarps;
 };
 
-// Dynamic shared memory of the step kernel for group size 2^log2G.
-inline size_t step_smem_bytes(int log2G) {
+// Dynamic shared memory, threads per block and parameters per block of the
+// step kernel for group size 2^log2G (host side).
+template <int LG>
+struct StepLaunch {
+  static constexpr size_t kSmem = StepLayout<LG>::kSmemBytes;
+  static constexpr int kBlock = StepLayout<LG>::kBlock;
+};
+
+inline void step_launch_shape(int log2G, size_t &smem, int &block) {
   switch (log2G) {
-    case 4: return StepLayout<4>::kSmemBytes;
-    case 5: return StepLayout<5>::kSmemBytes;
-    case 6: return StepLayout<6>::kSmemBytes;
-    case 7: return StepLayout<7>::kSmemBytes;
-    case 8: return StepLayout<8>::kSmemBytes;
-    case 9: return StepLayout<9>::kSmemBytes;
-    case 10: return StepLayout<10>::kSmemBytes;
-    case 11: return StepLayout<11>::kSmemBytes;
-    case 12: return StepLayout<12>::kSmemBytes;
-    default: return 0;
+#define COAT_STEP_SHAPE(LGV) \
+  case LGV: smem = StepLaunch<LGV>::kSmem; block = StepLaunch<LGV>::kBlock; return;
+    COAT_STEP_SHAPE(4) COAT_STEP_SHAPE(5) COAT_STEP_SHAPE(6) COAT_STEP_SHAPE(7)
+    COAT_STEP_SHAPE(8) COAT_STEP_SHAPE(9) COAT_STEP_SHAPE(10) COAT_STEP_SHAPE(11)
+    COAT_STEP_SHAPE(12)
+#undef COAT_STEP_SHAPE
+    default: smem = 0; block = 0; return;
   }
 }
 
@@ -277,9 +291,9 @@ __device__ __forceinline__ void range16_nonneg(const float *x, float &mx, float 
 // Reduce (max, min) pairs for two states over the LANES threads of a group.
 // For LANES <= 32 the group lives inside one warp; otherwise warp results
 // are combined through shared memory.
-template <int LANES>
+template <int LANES, int BLOCK_WARPS>
 __device__ __forceinline__ void group_reduce2(float &mx0, float &mn0, float &mx1, float &mn1,
-                                              float (*red)[kWarps]) {
+                                              float (*red)[BLOCK_WARPS]) {
   constexpr int lim = LANES < 32 ? LANES : 32;
 #pragma unroll
   for (int off = 1; off < lim; off <<= 1) {
@@ -297,7 +311,7 @@ __device__ __forceinline__ void group_reduce2(float &mx0, float &mn0, float &mx1
       red[3][warp] = mn1;
     }
     constexpr int wpg = LANES >> 5;
-    if constexpr (wpg * 32 == kThreads) {
+    if constexpr (wpg == BLOCK_WARPS) {
       __syncthreads();
     } else {
       // only the warps of this group wait for one another (named barrier
@@ -433,12 +447,12 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
 // ---- the fused step ----------------------------------------------------------
 
 template <int VF, int LG, bool FULL>
-__global__ void __launch_bounds__(kThreads, StepLayout<LG>::kMinBlocks)
+__global__ void __launch_bounds__(StepLayout<LG>::kBlock, StepLayout<LG>::kMinBlocks)
 adamw_fp8_step_kernel(const StepParams p) {
   using L = StepLayout<LG>;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ double tab8[8];   // log2(1 + i/8), direct decode (G < 64)
-  __shared__ float red[4][kWarps];
+  __shared__ float red[4][L::kBlockWarps];
   if constexpr (!L::kTable) {
     if (threadIdx.x < 8) tab8[threadIdx.x] = p.log2_tab[threadIdx.x];
   }
@@ -449,7 +463,7 @@ adamw_fp8_step_kernel(const StepParams p) {
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int64_t blk0 = (p.block0 + static_cast<int64_t>(blockIdx.x)) * kElemsPerBlock;
+  const int64_t blk0 = (p.block0 + static_cast<int64_t>(blockIdx.x)) * L::kBlockElems;
   const int64_t e0 = blk0 + threadIdx.x * kVec;
   const bool active = FULL || e0 < p.n;
   const int64_t grp = e0 >> LG;
@@ -607,7 +621,7 @@ adamw_fp8_step_kernel(const StepParams p) {
   }
 
   // ---- per-group range of the new moments, then k and s ----
-  group_reduce2<L::kLanes>(mmx, mmn, vmx, vmn, red);
+  group_reduce2<L::kLanes, L::kBlockWarps>(mmx, mmn, vmx, vmn, red);
   GroupQ gm, gv;
   if constexpr (L::kLanes >= 2) {
     // even lanes evaluate m's parameters, odd lanes v's; then swap

@@ -76,11 +76,9 @@ __device__ __forceinline__ float bf16hi_to_float(uint32_t w) {
 
 // ---- packed binary32 pairs (sm_100 f32x2 instructions) -------------------------
 // Each lane is an IEEE binary32 operation rounded to nearest even.  A packed
-// product feeding a packed sum may be contracted into a packed fma by the
-// compiler, so these are used only where that is harmless: the moment
-// updates, which must round every product, use scalar operations.
+// product feeding a packed sum may be fused into a packed fma by the code
+// generator, so these are used only where no product is then summed.
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 // ---- special-function-unit approximations ----------------------------------
@@ -94,28 +92,6 @@ __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// log2 of a positive finite float split as (integer exponent, log2 of the
-// significand in [1, 2)).  Subnormal inputs are renormalised first, so the
-// integer part is exact and the fraction carries only the significand's
-// approximation error.
-struct Log2Split {
-  int e;
-  float f;
-};
-
-__device__ __forceinline__ Log2Split log2_split(float a) {
-  uint32_t b = __float_as_uint(a);
-  int adj = 0;
-  if (b < 0x00800000u) {  // subnormal: scale by 2^24 (exact)
-    b = __float_as_uint(a * 16777216.0f);
-    adj = 24;
-  }
-  Log2Split r;
-  r.e = static_cast<int>(b >> 23) - 127 - adj;
-  r.f = lg2_approx(__uint_as_float((b & 0x007FFFFFu) | 0x3F800000u));
-  return r;
 }
 
 }  // namespace coat

@@ -140,12 +140,6 @@ __device__ __forceinline__ GroupQ group_params(float M, float mn, double ln_rang
 // y = fmax * (|x| / M)^k = 2^(k log2(|x| / M) + log2 fmax), carrying x's sign
 // bit (+0 encodes as 0x00; -0, which the update can produce only from a
 // negative-zero gradient on a zero moment, as the equal-valued 0x80).
-__device__ __forceinline__ float expand_signed(float x, float rM, float k, float log2_fmax) {
-  const float r = __fmul_rn(fabsf(x), rM);
-  const float y = ex2_approx(__fmaf_rn(k, lg2_approx(r), log2_fmax));
-  return __uint_as_float(__float_as_uint(y) | (__float_as_uint(x) & 0x80000000u));
-}
-
 template <int F>
 __device__ __forceinline__ void encode16(const float *x, const GroupQ &g, float log2_fmax,
                                          uint32_t *out) {

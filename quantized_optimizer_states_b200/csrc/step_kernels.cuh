@@ -12,10 +12,11 @@
 //
 // Work decomposition: one thread owns 16 consecutive parameters, so every
 // stream moves in 16-byte vectors (4 x 16 B of theta, 2 x 16 B of BF16
-// gradient, 16 B of each code stream).  Dynamic shared memory holds only the
-// warps' decode tables.  A 1xG group is G/16 consecutive
+// gradient, 16 B of each code stream); blocks are small (64 threads, more
+// only where one group needs it, see StepLayout).  Dynamic shared memory
+// holds only the warps' decode tables.  A 1xG group is G/16 consecutive
 // threads: up to 32 of them reduce with warp shuffles, larger groups (G >=
-// 1024) finish the reduction through shared memory inside the block.  The
+// 1024) finish the reduction through shared memory among their warps.  The
 // whole group stays in registers between the range reduction and the
 // encode, so every byte crosses HBM exactly once.
 //
@@ -38,6 +39,10 @@
 // The kernel is instantiated per group size, so lane counts, table counts
 // and shifts are compile-time, and per launch shape: full blocks (no bounds
 // checks) and the one ragged tail block of a launch.
+//
+// kThreads / kElemsPerBlock below are the 256-thread block shape of the
+// other kernels of the library (the stand-alone quantizer and the
+// activation kernels).
 #pragma once
 
 #include <cstdint>

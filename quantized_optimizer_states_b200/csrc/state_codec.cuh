@@ -225,17 +225,21 @@ __device__ __forceinline__ void st_shared_f32x2(unsigned char *smem, uint32_t of
 }
 
 // Lane t (0 <= t < L) of the L lanes that build one table.  key = the
-// table's offset in `smem` (a multiple of 512) | swz.  The caller
-// synchronises the warp before the first lookup.
-template <int L>
+// table's offset in `smem` (a multiple of 512) | swz.  kMixed: the lanes of
+// the warp build tables of both formats (E4M3 first moments beside E5M2
+// second moments), so e4 differs between them.  The caller synchronises the
+// warp before the first lookup.
+template <int L, bool kMixed>
 __device__ __forceinline__ void build_table(unsigned char *smem, uint32_t key, int t, bool e4,
                                             float k, float s, float beta) {
   static_assert(L == 4 || L == 8 || L == 16, "lanes per table");
   const double rk = recip_d(static_cast<double>(k));
-  const int c0 = (e4 ? 8 : 4) + 2 * t;
-  const int ex = e4 ? (c0 >> 3) - 7 : (c0 >> 2) - 15;  // exponent of the lane's first binade
-  const int i0 = e4 ? (c0 & 7) : 2 * (c0 & 3);         // log2 index of its two codes
-  const int i1 = e4 ? i0 + 1 : i0 + 2;
+  // f = 0 (E4M3: 3 mantissa bits, bias 7) or 1 (E5M2: 2 bits, bias 15)
+  const int f = e4 ? 0 : 1;
+  const int c0 = 8 - 4 * f + 2 * t;
+  const int ex = (c0 >> (3 - f)) - 7 - 8 * f;  // exponent of the lane's first binade
+  const int i0 = (c0 & (7 >> f)) << f;         // log2(1 + i/8) index of its two codes
+  const int i1 = i0 + 1 + f;
   const double ed = static_cast<double>(ex);
   double P0 = exp2_d((ed + c_log2_1p8th[i0]) * rk);
   double P1 = exp2_d((ed + c_log2_1p8th[i1]) * rk);
@@ -243,7 +247,7 @@ __device__ __forceinline__ void build_table(unsigned char *smem, uint32_t key, i
   double M = a;
 #pragma unroll
   for (int h = 4; h < L; h <<= 1) M *= M;  // a^(L/4)
-  if (!e4) M *= M;                         // E5M2 steps twice as many binades
+  M = e4 ? M : M * M;                      // E5M2 steps twice as many binades
   const float nanv = s != 0.0f ? __int_as_float(0x7fc00000) : 0.0f;
   const float infv = s != 0.0f ? __int_as_float(0x7f800000) : 0.0f;
 
@@ -259,18 +263,31 @@ __device__ __forceinline__ void build_table(unsigned char *smem, uint32_t key, i
     // lane 1 (1.25 2^-6): code 5; lane 2 (1.5 2^-6): codes 3, 6; lane 3 (1.75 2^-6): code 7.
     // E5M2: lane 0 (2^(-14/k)): 0, 2^-16, 2^-15 at codes 0, 1, 2; lane 1
     // (1.5 2^-14): code 3; lanes 2, 3: codes 124..127 (inf, NaN x 3).
-    if (t == 0 || (!e4 && t >= 2)) {
-      const int pc = t == 0 ? 0 : (t == 2 ? 124 : 126);
-      const float2 pv = t == 0 ? make_float2(0.0f, e4 ? v3 : v2)
-                               : make_float2(t == 2 ? infv : nanv, nanv);
-      st_shared_f32x2(smem, (4u * pc) ^ key, pv);
-    }
-    if (e4 || t < 2) {
-      const int sc = e4 ? (t == 0 ? 2 : (t == 1 ? 5 : (t == 2 ? 3 : 7))) : (t == 0 ? 2 : 3);
-      const float sv = (e4 && !(t & 1)) ? v2 : v1;
+    const int pc = t == 0 ? 0 : (t == 2 ? 124 : 126);
+    const float2 pv = t == 0 ? make_float2(0.0f, e4 ? v3 : v2)
+                             : make_float2(t == 2 ? infv : nanv, nanv);
+    if constexpr (kMixed) {
+      // the same three stores in every lane, without divergent branches: a
+      // lane with less to store repeats one of its stores (same address,
+      // same bits)
+      const int sc = e4 ? (t == 0 ? 2 : (t == 1 ? 5 : (t == 2 ? 3 : 7)))
+                        : (t == 0 ? 2 : (t == 1 ? 3 : pc));
+      const float sv = e4 ? ((t & 1) ? v1 : v2) : (t < 2 ? v1 : pv.x);
+      const bool two = e4 && !(t & 1);
+      const int sb = two ? (t == 0 ? 4 : 6) : sc;
+      const float svb = two ? v1 : sv;
+      if (t == 0 || !e4) st_shared_f32x2(smem, (4u * pc) ^ key, pv);
       st_shared_f32(smem, (4u * sc) ^ key, sv);
+      st_shared_f32(smem, (4u * sb) ^ key, svb);
+    } else {
+      if (t == 0 || (!e4 && t >= 2)) st_shared_f32x2(smem, (4u * pc) ^ key, pv);
+      if (e4 || t < 2) {
+        const int sc = e4 ? (t == 0 ? 2 : (t == 1 ? 5 : (t == 2 ? 3 : 7))) : (t == 0 ? 2 : 3);
+        const float sv = (e4 && !(t & 1)) ? v2 : v1;
+        st_shared_f32(smem, (4u * sc) ^ key, sv);
+      }
+      if (e4 && !(t & 1)) st_shared_f32(smem, (4u * (t == 0 ? 4 : 6)) ^ key, v1);
     }
-    if (e4 && !(t & 1)) st_shared_f32(smem, (4u * (t == 0 ? 4 : 6)) ^ key, v1);
   }
 
   // the normal codes
@@ -282,7 +299,8 @@ __device__ __forceinline__ void build_table(unsigned char *smem, uint32_t key, i
     float2 v = fmul2(fmul2(make_float2(static_cast<float>(P0), static_cast<float>(P1)), S), B);
     if (i == NI - 1) {
       if (e4 && c == 126) v.y = nanv;  // E4M3 0x7F is NaN
-      if (c < (e4 ? 128 : 124)) st_shared_f32x2(smem, (4u * c) ^ key, v);
+      // with L = 4 the last pair of every lane lies within its format's 128 codes
+      if (L == 4 || c < (e4 ? 128 : 124)) st_shared_f32x2(smem, (4u * c) ^ key, v);
     } else {
       st_shared_f32x2(smem, (4u * c) ^ key, v);
     }

@@ -521,8 +521,8 @@ adamw_fp8_step_kernel(const StepParams p) {
       const int j = r * (32 / L::kL) + lane / L::kL;
       const bool vst = j >= L::kGPW;
       const uint32_t key = (warp_off + j * kTableBytes) | (32u * (j & 3));
-      build_table<L::kL>(smem, key, lane % L::kL, VF == kE4M3 || !vst, kk[r], ss[r],
-                         vst ? p.beta2 : p.beta1);
+      build_table<L::kL, VF != kE4M3>(smem, key, lane % L::kL, VF == kE4M3 || !vst, kk[r],
+                                      ss[r], vst ? p.beta2 : p.beta1);
     }
     __syncwarp();
     const int lg = L::kGPW > 1 ? (lane >> (LG - 4)) : 0;

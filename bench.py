@@ -181,17 +181,23 @@ def run_reference(args):
     return 0
 
 
+ACT_RING = 8  # distinct activation tensors cycled by the activation bench
+
+
 def run_activations(args):
     """The activation-side kernels on the activation workload (BF16 [16384,
     2048], G = 128, E4M3): 1xG quantization, Group Scaling (standalone: steps
     (i)-(iii)), the SwiGLU producer with fused maxima followed by Group
-    Scaling's steps (ii)-(iii), and dequantization.  The tensor (64 MiB of
-    BF16) fits in L2, so a 256 MiB buffer is read before every timed
-    launch to flush it; each launch is timed alone with CUDA events.  One
-    JSON line: elements/s of the 1xG quantizer as the headline, every
-    kernel's time, achieved GB/s and fraction of the measured HBM copy
-    bandwidth in `kernels`.  The flush reads the buffer (leaving clean
-    lines), so no write-back of flush data lands in the timed launch."""
+    Scaling's steps (ii)-(iii), and dequantization.
+
+    Steady state: each kernel is launched back to back over a ring of
+    ACT_RING distinct input (and output) sets -- 8 x 64 MiB of BF16 input
+    alone, four times the 126 MB L2 -- so every launch reads its input from
+    HBM, and one pair of CUDA events brackets the K timed launches (the
+    event timer ticks in ~2 us steps on this part, too coarse for a single
+    20 us launch).  One JSON line: elements/s of the 1xG quantizer as the
+    headline; every kernel's time per launch, achieved GB/s and fraction of
+    the measured HBM copy bandwidth in `kernels`."""
     import torch
     import quantized_optimizer_states_b200 as coat
     from quantized_optimizer_states_b200 import build as coat_build
@@ -200,41 +206,46 @@ def run_activations(args):
     torch.cuda.set_device(dev)
     coat_build.build()
     coat.load()
-    w = inputs.activations()
-    G = w.group_size
-    x = inputs.device_activations(w, dev)
-    gate, up = inputs.device_swiglu_inputs(w, dev)
-    n = x.numel()
+    w0 = inputs.activations()
+    G = w0.group_size
+    n = w0.rows * w0.cols
     ng = n // G
-    q = torch.empty(n, dtype=torch.uint8, device=dev)
-    sc = torch.empty(ng, dtype=torch.float32, device=dev)
-    ws = torch.empty(coat.coat_group_scaling_workspace_bytes(n, G) // 4, dtype=torch.float32,
-                     device=dev)
-    s1 = torch.empty(1, dtype=torch.float32, device=dev)
-    h = torch.empty(n, dtype=torch.bfloat16, device=dev)
-    out = torch.empty(n, dtype=torch.float32, device=dev)
-    # L2 flush by reading 256 MiB: the cache is left holding clean lines, so
-    # the timed kernel does not also pay for writing back a flush's dirty data
-    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
-    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
-    xf = x.reshape(-1)
+    wsn = coat.coat_group_scaling_workspace_bytes(n, G) // 4
+    ring = []
+    for r in range(ACT_RING):
+        w = inputs.activations(seed=w0.seed + 101 * r)
+        gate, up = inputs.device_swiglu_inputs(w, dev)
+        ring.append({
+            "x": inputs.device_activations(w, dev), "gate": gate.reshape(-1), "up": up.reshape(-1),
+            "q": torch.empty(n, dtype=torch.uint8, device=dev),
+            "sc": torch.empty(ng, dtype=torch.float32, device=dev),
+            "ws": torch.empty(wsn, dtype=torch.float32, device=dev),
+            "ws_h": torch.empty(wsn, dtype=torch.float32, device=dev),
+            "s1": torch.empty(1, dtype=torch.float32, device=dev),
+            "h": torch.empty(n, dtype=torch.bfloat16, device=dev),
+            "out": torch.empty(n, dtype=torch.float32, device=dev)})
+    for b in ring:  # the producer's outputs that the after-producer case reads
+        coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"], group_size=G)
     cases = {
-        # name: (callable, algorithmic bytes per element)
-        "group_quant_1xG": (lambda: coat.coat_group_quant_1xG(x, q, sc, group_size=G),
+        # name: (callable on one ring slot, algorithmic bytes per element)
+        "group_quant_1xG": (lambda b: coat.coat_group_quant_1xG(b["x"], b["q"], b["sc"],
+                                                                group_size=G),
                             2 + 1 + 4.0 / G),
         "group_scaling_standalone": (
-            lambda: coat.coat_group_scaling_quant_pertensor(xf, ws, q, s1, group_size=G),
+            lambda b: coat.coat_group_scaling_quant_pertensor(b["x"].reshape(-1), b["ws"], b["q"],
+                                                              b["s1"], group_size=G),
             2 + 2 + 1 + 8.0 / G),
         "swiglu_fused_amax": (
-            lambda: coat.coat_swiglu_group_amax(gate.reshape(-1), up.reshape(-1), h, ws,
-                                                group_size=G),
+            lambda b: coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"],
+                                                  group_size=G),
             2 + 2 + 2 + 4.0 / G),
         "group_scaling_after_producer": (
-            lambda: coat.coat_group_scaling_quant_pertensor(h, ws, q, s1, group_size=G,
-                                                            amax_precomputed=True),
+            lambda b: coat.coat_group_scaling_quant_pertensor(b["h"], b["ws_h"], b["q"], b["s1"],
+                                                              group_size=G,
+                                                              amax_precomputed=True),
             2 + 1 + 4.0 / G),
         "dequant_pertensor": (
-            lambda: coat.coat_dequant(q, None, s1, out, group_size=n), 1 + 4),
+            lambda b: coat.coat_dequant(b["q"], None, b["s1"], b["out"], group_size=n), 1 + 4),
     }
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
@@ -244,18 +255,16 @@ def run_activations(args):
     sampler.start()
     time.sleep(0.3)
     for name, (fn, bpe) in cases.items():
-        for _ in range(args.warmup):
-            fn()
-        ts = []
-        for _ in range(args.steps):
-            torch.sum(flush, dim=(0,), out=flush_sink)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            fn()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        ms = statistics.median(ts)
+        for i in range(max(args.warmup, ACT_RING)):
+            fn(ring[i % ACT_RING])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            fn(ring[i % ACT_RING])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
         gbs = bpe * n / (ms / 1e3) / 1e9
         res[name] = {"ms": ms, "elements_per_s": n / (ms / 1e3), "GB/s": gbs,
                      "frac_of_hbm": gbs / peak, "algorithmic_bytes_per_element": bpe}
@@ -268,7 +277,8 @@ def run_activations(args):
             "data": "synthetic",
             "config": {"workload": "activations [16384, 2048] BF16 with GLU spike channels",
                        "group_size": G, "fmt": "e4m3",
-                       "l2": "256 MiB buffer read before every timed launch"},
+                       "l2": f"inputs larger than L2: a ring of {ACT_RING} distinct input sets "
+                             "(512 MiB of BF16 activations) launched back to back"},
             "roofline": {"bound": "hbm", "achieved": head["GB/s"], "peak": peak, "unit": "GB/s",
                          "frac": head["frac_of_hbm"], "traffic": None,
                          "peak_source": f"{peak_kind} copy bandwidth"},

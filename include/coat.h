@@ -304,6 +304,19 @@ coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, i
  * this thread (0 if none). */
 int32_t coat_last_cuda_error(void);
 
+/* Streamed activation kernels (coat_group_quant_1xG on contiguous rows,
+ * the cast of coat_group_scaling_quant_pertensor[_noalloc]) move
+ * 4096-element tiles into shared memory with bulk asynchronous copies and
+ * wait for each on an mbarrier.  Every such wait is
+ * bounded: one that runs out abandons the rest of its block's tiles (their
+ * outputs are then not written) and adds 1 to a device counter.
+ * coat_bulk_wait_timeouts synchronises the current device, stores the
+ * counter in *count (host pointer) and, if reset != 0, sets it to zero.
+ * A non-zero count means outputs of the calls since the last reset are
+ * incomplete.
+ * Errors: INVALID_ARG (count NULL), CUDA. */
+coat_status_t coat_bulk_wait_timeouts(uint32_t *count, int32_t reset);
+
 /* A static, human-readable name for a status code. */
 const char *coat_status_string(coat_status_t status);
 

@@ -12,6 +12,7 @@ from ._lib import (  # noqa: F401
     COAT_NOALLOC_MAX_GROUPS,
     CoatError,
     coat_adamw_fp8_step,
+    coat_bulk_wait_timeouts,
     coat_count_nonfinite_bf16,
     coat_dequant,
     coat_fp8_encode,

@@ -70,6 +70,7 @@ SIGNATURES = {
     "coat_adamw_fp8_step_guarded": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
                                            ctypes.POINTER(CoatAdamwCfg), _P, _P]),
     "coat_last_cuda_error": (_I32, []),
+    "coat_bulk_wait_timeouts": (_I32, [ctypes.POINTER(ctypes.c_uint32), _I32]),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
     "coat_version": (_I32, []),
 }
@@ -258,6 +259,15 @@ def coat_fp8_encode(y, q, *, fmt: int = COAT_E4M3, stream=None):
     st = load().coat_fp8_encode(_ptr(y, torch.float32, "y"), y.numel(), fmt,
                                 _ptr(q, torch.uint8, "q"), _stream(stream))
     _check("coat_fp8_encode", st)
+
+
+def coat_bulk_wait_timeouts(*, reset: bool = False) -> int:
+    """Bounded shared-memory copy waits of the streamed kernels that ran out
+    since the last reset (synchronises the device); 0 when every output is
+    complete."""
+    c = ctypes.c_uint32(0)
+    _check("coat_bulk_wait_timeouts", load().coat_bulk_wait_timeouts(ctypes.byref(c), int(reset)))
+    return int(c.value)
 
 
 def coat_version() -> int:

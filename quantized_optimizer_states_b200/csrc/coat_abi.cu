@@ -67,6 +67,58 @@ unsigned int blocks_for(int64_t elems) {
   return static_cast<unsigned int>((elems + coat::kElemsPerBlock - 1) / coat::kElemsPerBlock);
 }
 
+// Launch of an activation-side kernel with programmatic stream serialization:
+// the kernel may be scheduled while the kernel before it on `s` drains, and
+// it waits for that kernel (pdl_enter) before its first global access.
+template <class... KArgs, class... Args>
+void launch_act(void (*kernel)(KArgs...), unsigned int grid, size_t smem, cudaStream_t s,
+                Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(coat::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, args...);  // a failure is reported by launch_status()
+}
+
+// Streamed launch (tiles through shared memory by bulk copies) over the whole
+// 4096-element tiles of n elements.  Returns the elements it covers; the
+// caller hands the remainder to the plain kernel.
+template <auto K, class P>
+int64_t launch_stream(const P &p, int64_t n, size_t stage_bytes, cudaStream_t s) {
+  const int64_t tiles = n / coat::kElemsPerBlock;
+  if (tiles == 0) return 0;
+  const size_t smem = coat::kBulkStages * stage_bytes;
+  const unsigned int grid = coat::bulk_grid<K>(coat::kThreads, smem, tiles);
+  launch_act(K, grid, smem, s, p, tiles);
+  return tiles * coat::kElemsPerBlock;
+}
+
+// Group Scaling step (iii): the cast, streamed over whole tiles, plain on the rest.
+void launch_pertensor_cast(const coat::GroupScalingParams &p, int32_t fmt, cudaStream_t s) {
+  const int64_t done =
+      fmt == COAT_E4M3
+          ? launch_stream<coat::pertensor_cast_stream_kernel<coat::kE4M3>>(p, p.n,
+                                                                          coat::kTileBf16Bytes, s)
+          : launch_stream<coat::pertensor_cast_stream_kernel<coat::kE5M2>>(p, p.n,
+                                                                          coat::kTileBf16Bytes, s);
+  if (done == p.n) return;
+  coat::GroupScalingParams r = p;
+  r.x += done;
+  r.q += done;
+  r.n -= done;
+  const unsigned int grid = coat::act_blocks(r.n);
+  if (fmt == COAT_E4M3)
+    launch_act(coat::pertensor_cast_kernel<coat::kE4M3>, grid, 0, s, r);
+  else
+    launch_act(coat::pertensor_cast_kernel<coat::kE5M2>, grid, 0, s, r);
+}
+
 constexpr int64_t kMaxElems = int64_t{1} << 42;  // within the grid-size bound (2^31 - 1 blocks x 2048)
 
 // Launch one instantiation of the step kernel, raising its dynamic shared
@@ -299,11 +351,13 @@ coat_status_t coat_dequant(const uint8_t *q, const float *k, const float *scale,
     else
       coat::dequant_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
   } else {
+    // plain loads: a streamed form (bulk copies of the codes) measured
+    // slower here, the kernel being bound by its 4-byte-per-element writes
     const unsigned int grid = coat::act_blocks(n);
     if (fmt == COAT_E4M3)
-      coat::dequant_linear_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+      launch_act(coat::dequant_linear_kernel<coat::kE4M3>, grid, 0, s, p);
     else
-      coat::dequant_linear_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+      launch_act(coat::dequant_linear_kernel<coat::kE5M2>, grid, 0, s, p);
   }
   return launch_status();
 }
@@ -329,11 +383,29 @@ coat_status_t coat_group_quant_1xG(const uint16_t *x, int64_t rows, int64_t cols
   p.q = q;
   p.scale = scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const unsigned int grid = coat::act_blocks(rows * cols);
+  if (ld == cols) {
+    // contiguous rows: stream the flat tensor's whole tiles, then the rest
+    const int64_t n = rows * cols;
+    const int64_t done =
+        fmt == COAT_E4M3
+            ? launch_stream<coat::group_quant_1xG_stream_kernel<coat::kE4M3>>(
+                  p, n, coat::kTileBf16Bytes, s)
+            : launch_stream<coat::group_quant_1xG_stream_kernel<coat::kE5M2>>(
+                  p, n, coat::kTileBf16Bytes, s);
+    if (done == n) return launch_status();
+    // the remainder is whole groups (G divides both cols and the tile)
+    p.x += done;
+    p.q += done;
+    p.scale += done >> lg;
+    p.rows = 1;
+    p.cols = p.ld = n - done;
+    p.vec_per_row = p.cols / coat::kVec;
+  }
+  const unsigned int grid = coat::act_blocks(p.rows * p.cols);
   if (fmt == COAT_E4M3)
-    coat::group_quant_1xG_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
+    launch_act(coat::group_quant_1xG_kernel<coat::kE4M3>, grid, 0, s, p);
   else
-    coat::group_quant_1xG_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+    launch_act(coat::group_quant_1xG_kernel<coat::kE5M2>, grid, 0, s, p);
   return launch_status();
 }
 
@@ -369,15 +441,11 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
     // one pass over the small intermediate: a few blocks per SM suffice
     const int64_t want = (ng + coat::kThreads - 1) / coat::kThreads;
     const unsigned int grid = static_cast<unsigned int>(want < 1184 ? want : 1184);
-    coat::amax_of_groups_kernel<<<grid, coat::kThreads, 0, s>>>(p);
+    launch_act(coat::amax_of_groups_kernel, grid, 0, s, p);
   } else {
-    coat::group_amax_kernel<<<coat::act_blocks(n), coat::kThreads, 0, s>>>(p);
+    launch_act(coat::group_amax_kernel, coat::act_blocks(n), 0, s, p);
   }
-  const unsigned int grid = coat::act_blocks(n);
-  if (fmt == COAT_E4M3)
-    coat::pertensor_cast_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
-  else
-    coat::pertensor_cast_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  launch_pertensor_cast(p, fmt, s);
   return launch_status();
 }
 
@@ -399,8 +467,8 @@ coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, i
   p.log2G = lg;
   p.out = out;
   p.group_amax = group_amax;
-  coat::swiglu_group_amax_kernel<<<coat::act_blocks(n), coat::kThreads, 0,
-                                   static_cast<cudaStream_t>(stream)>>>(p);
+  launch_act(coat::swiglu_group_amax_kernel, coat::act_blocks(n), 0,
+             static_cast<cudaStream_t>(stream), p);
   return launch_status();
 }
 
@@ -417,13 +485,28 @@ coat_status_t coat_fp8_encode(const float *y, int64_t n, int32_t fmt, uint8_t *q
   p.q = q;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (fmt == COAT_E4M3)
-    coat::fp8_encode_kernel<coat::kE4M3><<<coat::act_blocks(n), coat::kThreads, 0, s>>>(p);
+    launch_act(coat::fp8_encode_kernel<coat::kE4M3>, coat::act_blocks(n), 0, s, p);
   else
-    coat::fp8_encode_kernel<coat::kE5M2><<<coat::act_blocks(n), coat::kThreads, 0, s>>>(p);
+    launch_act(coat::fp8_encode_kernel<coat::kE5M2>, coat::act_blocks(n), 0, s, p);
   return launch_status();
 }
 
 int32_t coat_last_cuda_error(void) { return g_last_cuda_error; }
+
+coat_status_t coat_bulk_wait_timeouts(uint32_t *count, int32_t reset) {
+  if (!count) return COAT_ERR_INVALID_ARG;
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpyFromSymbol(&v, coat::g_bulk_wait_timeouts, sizeof(v)) != cudaSuccess)
+    return launch_status();
+  *count = v;
+  if (reset) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(coat::g_bulk_wait_timeouts, &zero, sizeof(zero)) != cudaSuccess)
+      return launch_status();
+  }
+  return COAT_OK;
+}
 
 const char *coat_status_string(coat_status_t status) {
   switch (status) {
@@ -508,11 +591,7 @@ extern "C" coat_status_t coat_group_scaling_quant_pertensor_noalloc(
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the tensor maximum accumulates with atomicMax and must start at zero
   if (cudaMemsetAsync(p.tensor_amax, 0, sizeof(uint32_t), s) != cudaSuccess) return launch_status();
-  coat::group_amax_kernel<<<coat::act_blocks(n), coat::kThreads, 0, s>>>(p);
-  const unsigned int grid = coat::act_blocks(n);
-  if (fmt == COAT_E4M3)
-    coat::pertensor_cast_kernel<coat::kE4M3><<<grid, coat::kThreads, 0, s>>>(p);
-  else
-    coat::pertensor_cast_kernel<coat::kE5M2><<<grid, coat::kThreads, 0, s>>>(p);
+  launch_act(coat::group_amax_kernel, coat::act_blocks(n), 0, s, p);
+  launch_pertensor_cast(p, fmt, s);
   return launch_status();
 }

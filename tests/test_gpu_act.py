@@ -73,6 +73,20 @@ def test_group_quant_strided_rows_and_special_values(lib, orc):
     assert np.array_equal(q, q_ref)
 
 
+def test_group_quant_streamed_group_4096_and_remainders(lib, orc):
+    """Contiguous rows go through the streamed kernel (4096-element tiles by
+    bulk copies) plus the plain kernel for a ragged remainder: G = 4096
+    (a group filling a whole tile), and sizes whose remainder is 0, one group
+    or several groups."""
+    for rows, cols, G in ((5, 8192, 4096), (3, 4096 + 2048, 2048), (7, 1152, 128)):
+        x = inputs.host_activations(inputs.activations(seed=rows), rows=rows)
+        x = np.tile(x, (1, -(-cols // x.shape[1])))[:, :cols].copy()
+        q, sc = _gpu_1xG(lib, x, G, E4M3)
+        q_ref, sc_ref = orc.group_quant_1xG(x, G, E4M3)
+        assert np.array_equal(sc, sc_ref) and np.array_equal(q, q_ref), (rows, cols, G)
+    assert lib.coat_bulk_wait_timeouts(reset=True) == 0
+
+
 def _gpu_group_scaling(lib, x, G, fmt, group_amax=None):
     import torch
     n = x.size
@@ -138,6 +152,36 @@ def test_activation_dequant_bit_exact(lib, orc, fmt):
                      group_size=m, fmt=fmt)
     torch.cuda.synchronize()
     assert np.array_equal(parity.to_host(out1), ref1)
+
+
+@pytest.mark.parametrize("out_bf16", [False, True])
+def test_activation_dequant_full_set(lib, orc, out_bf16):
+    """The activation workload's codes (8192 tiles: every block of the
+    persistent streamed grid cycles its shared-memory stages several times)
+    dequantized per 1xG group, and a per-tensor length that is not a whole
+    number of tiles."""
+    import torch
+    x = inputs.host_activations(inputs.activations())
+    q, sc = orc.group_quant_1xG(x, 128, E4M3)
+    ref = orc.dequant(q.reshape(-1), None, sc.reshape(-1), 128, E4M3)
+    dt = torch.bfloat16 if out_bf16 else torch.float32
+    out = torch.empty(q.size, dtype=dt, device="cuda")
+    lib.coat_dequant(parity.to_dev(q.reshape(-1)), None, parity.to_dev(sc.reshape(-1)), out,
+                     group_size=128, fmt=E4M3)
+    m = q.size - 4096 * 3 - 48
+    s1 = np.array([1.5e-3], dtype=np.float32)
+    out1 = torch.empty(m, dtype=dt, device="cuda")
+    lib.coat_dequant(parity.to_dev(q.reshape(-1)[:m]), None, parity.to_dev(s1), out1,
+                     group_size=m, fmt=E4M3)
+    torch.cuda.synchronize()
+    ref1 = orc.dequant(q.reshape(-1)[:m], None, s1, m, E4M3)
+    if out_bf16:
+        assert np.array_equal(parity.to_host(out).view(np.uint16), orc.to_bf16_array(ref))
+        assert np.array_equal(parity.to_host(out1).view(np.uint16), orc.to_bf16_array(ref1))
+    else:
+        assert np.array_equal(parity.to_host(out), ref)
+        assert np.array_equal(parity.to_host(out1), ref1)
+    assert lib.coat_bulk_wait_timeouts(reset=True) == 0
 
 
 def test_hardware_cvt_matches_oracle_encoder(lib, orc):

@@ -40,9 +40,16 @@ def bytes_per_param(G: int) -> float:
     return 14.0 + 32.0 / G
 
 
-def kernel_source_hash() -> str:
+# sources of the activation quantizers (the traffic record of the 1xG
+# kernel is valid while these are unchanged)
+ACT_KERNEL_SOURCES = ["quantized_optimizer_states_b200/csrc/act_kernels.cuh",
+                      "quantized_optimizer_states_b200/csrc/bulk_pipe.cuh",
+                      "quantized_optimizer_states_b200/csrc/fp8_device.cuh"]
+
+
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in (KERNEL_SOURCES if sources is None else sources):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -69,6 +76,22 @@ def recorded_traffic(n: int, G: int):
     if rec.get("kernel_source_hash") != kernel_source_hash() or rec.get("group_size") != G:
         return None
     return rec["dram_bytes_per_param"] * n
+
+
+def recorded_act_traffic(n: int):
+    """DRAM bytes of one 1xG quantizer launch on the activation workload, from
+    the committed ncu summary; None if its sources changed since the capture
+    or the size differs."""
+    path = os.path.join(ROOT, "profiles", "group_quant_1xG_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except OSError:
+        return None
+    if (rec.get("kernel_source_hash") != kernel_source_hash(ACT_KERNEL_SOURCES)
+            or rec.get("elements") != n):
+        return None
+    return rec["dram_bytes_read"] + rec["dram_bytes_write"]
 
 
 class ClockSampler:
@@ -280,7 +303,7 @@ def run_activations(args):
                        "l2": f"inputs larger than L2: a ring of {ACT_RING} distinct input sets "
                              "(512 MiB of BF16 activations) launched back to back"},
             "roofline": {"bound": "hbm", "achieved": head["GB/s"], "peak": peak, "unit": "GB/s",
-                         "frac": head["frac_of_hbm"], "traffic": None,
+                         "frac": head["frac_of_hbm"], "traffic": recorded_act_traffic(n),
                          "peak_source": f"{peak_kind} copy bandwidth"},
             "kernels": res, "clocks": clocks,
             "gpu_launches": args.steps * (1 + 2 + 1 + 2 + 1)}

@@ -125,6 +125,14 @@ struct StepLayout {
   // 260 vs 233 at G = 64); 16 for the direct-decode G < 64 kernels
   static constexpr int kMinWarps = LG <= 5 ? 16 : ((LG == 6 || LG >= 10) ? 24 : 32);
   static constexpr int kMinBlocks = kMinWarps / kBlockWarps;
+  // groups per block, and whether warp 0 evaluates every (k, s) of the
+  // block (each pair once, read back through shared memory) instead of each
+  // lane of a group evaluating its own copy: for G = 64 and 128, where a
+  // group has 4 or 8 lanes (measured: +3.5% at G = 64, +1-2% at G = 128;
+  // at G = 256 and 512 the two block barriers cost more than they save)
+  static constexpr int kBlockGroups = kBlockElems >> LG;
+  static constexpr bool kShareParams = kTable && LG <= 7 && kBlockWarps >= 2 &&
+                                       2 * kBlockGroups <= 32;
 };
 
 // Dynamic shared memory, threads per block and parameters per block of the
@@ -628,7 +636,43 @@ adamw_fp8_step_kernel(const StepParams p) {
   // ---- per-group range of the new moments, then k and s ----
   group_reduce2<L::kLanes, L::kBlockWarps>(mmx, mmn, vmx, vmn, red);
   GroupQ gm, gv;
-  if constexpr (L::kLanes >= 2) {
+  if constexpr (L::kShareParams) {
+    // The block's (group, state) pairs fit one warp: warp 0 evaluates each
+    // pair once (lane 2 g for group g's first moment, 2 g + 1 for its second)
+    // and the block reads them back, instead of every lane of a group
+    // evaluating its own copy.
+    __shared__ float rng[L::kBlockGroups][4];
+    __shared__ float gq[L::kBlockGroups][2][4];
+    const int gib = threadIdx.x >> (LG - 4);
+    if ((threadIdx.x & (L::kLanes - 1)) == 0) {
+      rng[gib][0] = mmx;
+      rng[gib][1] = mmn;
+      rng[gib][2] = vmx;
+      rng[gib][3] = vmn;
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * L::kBlockGroups) {
+      const int gi = threadIdx.x >> 1;
+      const int odd = threadIdx.x & 1;
+      const GroupQ q = group_params(rng[gi][2 * odd], rng[gi][2 * odd + 1],
+                                    odd ? p.v.ln_range : p.m.ln_range,
+                                    odd ? p.v.fmax : p.m.fmax,
+                                    odd ? p.v.log2_fmax : p.m.log2_fmax,
+                                    odd ? p.v.rfmax : p.m.rfmax, p.k_max, p.force_k1);
+      gq[gi][odd][0] = q.k;
+      gq[gi][odd][1] = q.s;
+      gq[gi][odd][2] = q.rM;
+    }
+    __syncthreads();
+    gm.k = gq[gib][0][0];
+    gm.s = gq[gib][0][1];
+    gm.rM = gq[gib][0][2];
+    gv.k = gq[gib][1][0];
+    gv.s = gq[gib][1][1];
+    gv.rM = gq[gib][1][2];
+    gm.zero = gm.s == 0.0f;
+    gv.zero = gv.s == 0.0f;
+  } else if constexpr (L::kLanes >= 2) {
     // even lanes evaluate m's parameters, odd lanes v's; then swap
     const bool odd = threadIdx.x & 1;
     const GroupQ mine = group_params(odd ? vmx : mmx, odd ? vmn : mmn,

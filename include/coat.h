@@ -26,6 +26,10 @@
  *           57344, min subnormal 2^-16) and section 08 "Adam -> AdamW"
  *           (m_t, v_t, the bias-corrected update with eps outside the root,
  *           theta <- (1 - eta*lambda) theta + delta).
+ *   [QA]    "AI 低精度格式（bfloat16/FP8/TF32）" (codechuan.com): BF16 keeps
+ *           FP32's 8 exponent bits with 7 mantissa bits (conversion is a
+ *           rounding of the low 16 bits); FP32 master weights with
+ *           low-precision gradients.
  *
  * Common conventions
  *   - Every pointer argument is a DEVICE pointer owned by the caller unless
@@ -299,6 +303,45 @@ coat_status_t coat_fp8_encode(const float *y, int64_t n, int32_t fmt, uint8_t *q
 coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, int64_t n,
                                      int32_t group_size, uint16_t *out, float *group_amax,
                                      void *stream);
+
+/*
+ * coat_pack_bf16 -- gather `count` tensors into one flat BF16 buffer with
+ * one launch per 128 tensors: element j of tensor i goes to
+ * dst[offset[i] + j], converted from float32 (round to nearest even, as a
+ * BF16 cast does; NaN stays a NaN) when src_f32 != 0, else copied as BF16
+ * bits; a NULL src[i] fills its slice with zeros.  This lays the
+ * per-parameter BF16 gradients of a parameter group out for one
+ * coat_adamw_fp8_step ([QA]: FP32 -> BF16 by rounding away the low 16 bits;
+ * the flat 1xG layout is this library's, see coat_adamw_fp8_step).
+ *   src     HOST array [count] of device pointers (float32 or BF16 bits)
+ *   numel   HOST array [count]: elements of each tensor (>= 0)
+ *   offset  HOST array [count]: destination offset of each tensor, a
+ *           multiple of 8 (MISALIGNED otherwise), offset + numel <= n
+ *   dst     BF16 bits [n] device buffer (16-byte aligned)
+ * The tables are copied into the kernels' parameter blocks, so nothing is
+ * allocated.  Slices must not overlap (not checked); elements of dst
+ * outside every slice are left as they are.
+ * Errors: INVALID_ARG (NULL tables with count > 0, negative sizes, a slice
+ * outside [0, n), dst NULL), MISALIGNED, UNSUPPORTED (over 2^31 2048-element
+ * chunks in one launch), CUDA.
+ */
+coat_status_t coat_pack_bf16(const void *const *src, const int64_t *numel, const int64_t *offset,
+                             int32_t count, int32_t src_f32, uint16_t *dst, int64_t n,
+                             void *stream);
+
+/*
+ * coat_unpack_bf16 -- the reverse for BF16 parameters: dst[i][j] =
+ * BF16(src[offset[i] + j]) (nearest even) for the `count` tensors, e.g. the
+ * updated float32 master weights of a parameter group written back into its
+ * BF16 parameters.
+ *   src     float32 [n] device buffer (16-byte aligned)
+ *   numel, offset  HOST arrays as in coat_pack_bf16
+ *   dst     HOST array [count] of device pointers to BF16 tensors (not NULL
+ *           where numel > 0)
+ * Errors as coat_pack_bf16.
+ */
+coat_status_t coat_unpack_bf16(const float *src, const int64_t *numel, const int64_t *offset,
+                               int32_t count, void *const *dst, int64_t n, void *stream);
 
 /* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
  * this thread (0 if none). */

@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     COAT_FORCE_K1,
     COAT_NOALLOC_MAX_GROUPS,
     CoatError,
+    PackTable,
     coat_adamw_fp8_step,
     coat_bulk_wait_timeouts,
     coat_count_nonfinite_bf16,
@@ -20,9 +21,11 @@ from ._lib import (  # noqa: F401
     coat_group_scaling_quant_pertensor,
     coat_group_scaling_quant_pertensor_noalloc,
     coat_group_scaling_workspace_bytes,
+    coat_pack_bf16,
     coat_quantize_state,
     coat_status_string,
     coat_swiglu_group_amax,
+    coat_unpack_bf16,
     coat_version,
     load,
 )

@@ -69,6 +69,10 @@ SIGNATURES = {
     "coat_count_nonfinite_bf16": (_I32, [_P, _I64, _P, _P]),
     "coat_adamw_fp8_step_guarded": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
                                            ctypes.POINTER(CoatAdamwCfg), _P, _P]),
+    "coat_pack_bf16": (_I32, [ctypes.POINTER(_P), ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                              _I32, _I32, _P, _I64, _P]),
+    "coat_unpack_bf16": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), _I32,
+                                ctypes.POINTER(_P), _I64, _P]),
     "coat_last_cuda_error": (_I32, []),
     "coat_bulk_wait_timeouts": (_I32, [ctypes.POINTER(ctypes.c_uint32), _I32]),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
@@ -259,6 +263,54 @@ def coat_fp8_encode(y, q, *, fmt: int = COAT_E4M3, stream=None):
     st = load().coat_fp8_encode(_ptr(y, torch.float32, "y"), y.numel(), fmt,
                                 _ptr(q, torch.uint8, "q"), _stream(stream))
     _check("coat_fp8_encode", st)
+
+
+class PackTable:
+    """Host tables (sizes, flat offsets) of a fixed list of tensors, built
+    once, for coat_pack_bf16 / coat_unpack_bf16."""
+
+    def __init__(self, numels, offsets):
+        if len(numels) != len(offsets):
+            raise ValueError("numels and offsets differ in length")
+        self.count = len(numels)
+        self.numel = (_I64 * self.count)(*[int(x) for x in numels])
+        self.offset = (_I64 * self.count)(*[int(x) for x in offsets])
+
+    def pointers(self, tensors):
+        if len(tensors) != self.count:
+            raise ValueError("wrong number of tensors")
+        return (_P * self.count)(*[None if t is None else t.data_ptr() for t in tensors])
+
+
+def coat_pack_bf16(srcs, table: PackTable, dst, *, stream=None):
+    """dst[offset[i] + j] = bf16(srcs[i][j]) for CUDA tensors srcs (all FP32, or
+    all BF16 / int16 / uint16 bit patterns; None = zeros) into the flat BF16
+    tensor dst."""
+    import torch
+    dtypes = {t.dtype for t in srcs if t is not None}
+    bits16 = {torch.bfloat16, torch.int16, torch.uint16}
+    if not dtypes <= {torch.float32} and not dtypes <= bits16:
+        raise ValueError("sources must be all float32 or all BF16 (bit patterns)")
+    for t in srcs:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("sources must be contiguous CUDA tensors")
+    src_f32 = int(dtypes == {torch.float32})
+    _check("coat_pack_bf16", load().coat_pack_bf16(
+        table.pointers(srcs), table.numel, table.offset, table.count, src_f32,
+        _u16(dst, "dst"), dst.numel(), _stream(stream)))
+
+
+def coat_unpack_bf16(src, table: PackTable, dsts, *, stream=None):
+    """dsts[i][j] = bf16(src[offset[i] + j]) from the flat FP32 tensor src into
+    contiguous BF16 CUDA tensors dsts."""
+    for t in dsts:
+        if t is None or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("destinations must be contiguous CUDA tensors")
+        _u16(t, "destination")
+    import torch
+    _check("coat_unpack_bf16", load().coat_unpack_bf16(
+        _ptr(src, torch.float32, "src"), table.numel, table.offset, table.count,
+        table.pointers(dsts), src.numel(), _stream(stream)))
 
 
 def coat_bulk_wait_timeouts(*, reset: bool = False) -> int:

@@ -13,6 +13,7 @@
 
 #include "act_kernels.cuh"
 #include "fp8_device.cuh"
+#include "pack_kernels.cuh"
 #include "step_kernels.cuh"
 
 namespace {
@@ -563,7 +564,65 @@ coat_status_t noalloc_scratch(float **out) {
   return COAT_OK;
 }
 
+// Multi-tensor pack / unpack: argument checks, then one launch per
+// kPackTensors tensors.
+coat_status_t pack_launch(bool unpack, const void *const *ptrs, const int64_t *numel,
+                          const int64_t *offset, int32_t count, int32_t src_f32, void *flat,
+                          int64_t n, void *stream) {
+  if (count < 0 || n < 0) return COAT_ERR_INVALID_ARG;
+  if (count == 0) return COAT_OK;
+  if (!ptrs || !numel || !offset) return COAT_ERR_INVALID_ARG;
+  bool any = false;
+  for (int32_t i = 0; i < count; ++i) {
+    if (numel[i] < 0 || offset[i] < 0 || offset[i] > n - numel[i]) return COAT_ERR_INVALID_ARG;
+    if (numel[i] > 0 && unpack && !ptrs[i]) return COAT_ERR_INVALID_ARG;
+    if (numel[i] > 0 && (offset[i] % 8) != 0) return COAT_ERR_MISALIGNED;
+    any = any || numel[i] > 0;
+  }
+  if (!any) return COAT_OK;
+  if (!flat) return COAT_ERR_INVALID_ARG;
+  if (!aligned16(flat)) return COAT_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int32_t base = 0; base < count; base += coat::kPackTensors) {
+    const int32_t c = count - base < coat::kPackTensors ? count - base : coat::kPackTensors;
+    coat::PackParams p;
+    int64_t chunks = 0;
+    for (int32_t i = 0; i < c; ++i) {
+      p.ptr[i] = ptrs[base + i];
+      p.numel[i] = numel[base + i];
+      p.offset[i] = offset[base + i];
+      p.chunk0[i] = static_cast<int32_t>(chunks);
+      chunks += (numel[base + i] + coat::kPackChunk - 1) / coat::kPackChunk;
+      if (chunks > 0x7fffffff) return COAT_ERR_UNSUPPORTED;
+    }
+    p.chunk0[c] = static_cast<int32_t>(chunks);
+    p.count = c;
+    p.src_f32 = src_f32 ? 1 : 0;
+    p.flat = flat;
+    if (chunks == 0) continue;
+    const unsigned int grid = static_cast<unsigned int>(chunks);
+    if (unpack)
+      coat::unpack_bf16_kernel<<<grid, coat::kPackThreads, 0, s>>>(p);
+    else
+      coat::pack_bf16_kernel<<<grid, coat::kPackThreads, 0, s>>>(p);
+  }
+  return launch_status();
+}
+
 }  // namespace
+
+extern "C" coat_status_t coat_pack_bf16(const void *const *src, const int64_t *numel,
+                                        const int64_t *offset, int32_t count, int32_t src_f32,
+                                        uint16_t *dst, int64_t n, void *stream) {
+  return pack_launch(false, src, numel, offset, count, src_f32, dst, n, stream);
+}
+
+extern "C" coat_status_t coat_unpack_bf16(const float *src, const int64_t *numel,
+                                          const int64_t *offset, int32_t count, void *const *dst,
+                                          int64_t n, void *stream) {
+  return pack_launch(true, const_cast<const void *const *>(dst), numel, offset, count, 1,
+                     const_cast<float *>(src), n, stream);
+}
 
 extern "C" coat_status_t coat_group_scaling_quant_pertensor_noalloc(
     const uint16_t *x, int64_t n, int32_t group_size, int32_t fmt, uint8_t *q, float *scale,

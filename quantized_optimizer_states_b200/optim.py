@@ -20,6 +20,8 @@ the rule).
 * BF16 parameters keep a separate FP32 master copy; their BF16 gradients are
   copied into the flat buffer, and after the step the master values are
   rounded back into the parameters.
+Both moves are one multi-tensor launch per 128 parameters
+(coat_pack_bf16 / coat_unpack_bf16), not one copy per parameter.
 
 Fresh states are all-zero groups (codes 0, k = 1, s = 0).  `state_dict()`
 holds the flat buffers themselves, so saving and loading reproduces the run
@@ -63,6 +65,7 @@ class _FlatGroup:
     v_k: torch.Tensor
     v_s: torch.Tensor
     bf16_params: bool
+    table: _lib.PackTable
     step: int = 0
 
 
@@ -136,16 +139,30 @@ class CoatAdamW(torch.optim.Optimizer):
             m_s=torch.zeros(ng, dtype=torch.float32, device=dev),
             v_k=torch.ones(ng, dtype=torch.float32, device=dev),
             v_s=torch.zeros(ng, dtype=torch.float32, device=dev),
-            bf16_params=bf16)
+            bf16_params=bf16, table=_lib.PackTable([p.numel() for p in ps], offsets))
 
     @torch.no_grad()
     def _gather_grads(self, fg: _FlatGroup):
-        for p, off in zip(fg.params, fg.offsets):
-            dst = fg.grad[off:off + p.numel()]
-            if p.grad is None:
-                dst.zero_()
-            else:
-                dst.copy_(p.grad.reshape(-1))  # FP32 -> BF16 rounds to nearest even
+        want = torch.bfloat16 if fg.bf16_params else torch.float32
+        grads = []
+        for p in fg.params:
+            g = p.grad
+            if g is not None:
+                g = g.detach()
+                if g.dtype != want:
+                    g = g.to(want)
+                if not g.is_contiguous():
+                    g = g.contiguous()
+            grads.append(g)  # None: the slice is zero-filled
+        _lib.coat_pack_bf16(grads, fg.table, fg.grad)
+
+    @torch.no_grad()
+    def _write_back_bf16(self, fg: _FlatGroup):
+        if all(p.is_contiguous() for p in fg.params):
+            _lib.coat_unpack_bf16(fg.master, fg.table, [p.data for p in fg.params])
+        else:
+            for p, off in zip(fg.params, fg.offsets):
+                p.copy_(fg.master[off:off + p.numel()].view_as(p))
 
     # ---- the step --------------------------------------------------------------
 
@@ -172,8 +189,7 @@ class CoatAdamW(torch.optim.Optimizer):
                 group_size=group["group_size"], v_fmt=group["v_fmt"],
                 k_range=group["k_range"], k_max=group["k_max"])
             if fg.bf16_params:
-                for p, off in zip(fg.params, fg.offsets):
-                    p.copy_(fg.master[off:off + p.numel()].view_as(p))
+                self._write_back_bf16(fg)
         return loss
 
     # ---- inspection ------------------------------------------------------------
@@ -219,5 +235,4 @@ class CoatAdamW(torch.optim.Optimizer):
                     getattr(fg, k).copy_(saved[k].to(getattr(fg, k).device))
                 fg.step = int(saved["step"])
                 if fg.bf16_params:
-                    for p, off in zip(fg.params, fg.offsets):
-                        p.copy_(fg.master[off:off + p.numel()].view_as(p))
+                    self._write_back_bf16(fg)

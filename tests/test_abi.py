@@ -92,6 +92,31 @@ def test_argument_checks_return_before_any_launch(lib):
     assert gs(fake, 0, 128, 0, fake, 0, fake, fake, None) == 0
 
 
+def test_pack_argument_checks(lib):
+    """coat_pack_bf16 / coat_unpack_bf16 validate their host tables before any
+    launch (these calls never reach the device)."""
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    fake = P(1 << 20)
+    ptrs = (P * 2)(1 << 20, 1 << 21)
+
+    def tab(*v):
+        return (I64 * len(v))(*v)
+
+    pk, up = lib.coat_pack_bf16, lib.coat_unpack_bf16
+    assert pk(ptrs, tab(8, 8), tab(0, 16), -1, 1, fake, 64, None) == 1    # count < 0
+    assert pk(None, tab(8, 8), tab(0, 16), 2, 1, fake, 64, None) == 1     # no pointer table
+    assert pk(ptrs, tab(8, -1), tab(0, 16), 2, 1, fake, 64, None) == 1    # negative size
+    assert pk(ptrs, tab(8, 8), tab(0, 60), 2, 1, fake, 64, None) == 1     # slice beyond n
+    assert pk(ptrs, tab(8, 8), tab(0, 12), 2, 1, fake, 64, None) == 2     # offset not a multiple of 8
+    assert pk(ptrs, tab(8, 8), tab(0, 16), 2, 1, None, 64, None) == 1     # no destination
+    assert pk(ptrs, tab(8, 8), tab(0, 16), 2, 1, P((1 << 20) + 4), 64, None) == 2
+    assert pk(ptrs, tab(0, 0), tab(0, 16), 2, 1, None, 64, None) == 0     # nothing to move
+    assert pk(None, None, None, 0, 1, None, 0, None) == 0
+    nulls = (P * 2)(None, 1 << 21)
+    assert up(fake, tab(8, 8), tab(0, 16), 2, nulls, 64, None) == 1       # unpack into NULL
+    assert pk(nulls, tab(0, 8), tab(0, 16), 2, 1, P((1 << 20) + 8), 64, None) == 2
+
+
 def test_product_path_fails_loudly_without_library(tmp_path):
     from quantized_optimizer_states_b200 import _lib
     saved = _lib._lib

@@ -313,10 +313,12 @@ def run_activations(args):
 
 def run_optimizer(args):
     """`CoatAdamW.step()` -- the call a training loop makes -- on the OLMo-7B
-    set as 226 FP32 parameters with FP32 gradients: one multi-tensor pack of
-    the gradients into the flat BF16 buffer (coat_pack_bf16) and one fused
-    step.  Reported beside the fused step alone: the pack's share, and the
-    algorithmic bytes of both (pack 4 + 2 B/param, step 14 + 32/G)."""
+    set as 226 FP32 parameters.  Headline: flat_grads=True, the gradients
+    living in one flat FP32 buffer that the parameters' .grad view, read by
+    the step directly (coat_adamw_fp8_step_fp32grad; algorithmic 16 + 32/G
+    B/param).  Beside it: the same optimizer with per-parameter gradient
+    tensors, packed to BF16 first (coat_pack_bf16; 6 + 14 + 32/G B/param),
+    and the pack alone."""
     import torch
     import quantized_optimizer_states_b200 as coat
     from quantized_optimizer_states_b200 import build as coat_build
@@ -331,56 +333,63 @@ def run_optimizer(args):
     gen = torch.Generator(device=dev)
     gen.manual_seed(w.seed)
     stds = inputs._tensor_grad_stds(w, len(w.sizes))
-    params = []
-    for (name, shape), sd in zip(inputs.OLMO_7B, stds):
-        p = torch.nn.Parameter(torch.empty(shape, device=dev).normal_(0.0, w.theta_std,
-                                                                        generator=gen))
-        p.grad = torch.empty(shape, device=dev).normal_(0.0, float(sd), generator=gen)
-        params.append(p)
+    params = [torch.nn.Parameter(torch.empty(shape, device=dev).normal_(0.0, w.theta_std,
+                                                                          generator=gen))
+              for _, shape in inputs.OLMO_7B]
     n = sum(p.numel() for p in params)
     h = w.hyper
     opt = CoatAdamW(params, lr=h["lr"], betas=(h["beta1"], h["beta2"]), eps=h["eps"],
-                    weight_decay=h["weight_decay"], group_size=G)
-    for _ in range(args.warmup):
-        opt.step()
-    torch.cuda.synchronize()
+                    weight_decay=h["weight_decay"], group_size=G, flat_grads=True)
+    with torch.no_grad():
+        for p, sd in zip(params, stds):
+            p.grad.normal_(0.0, float(sd), generator=gen)   # into the flat buffer
     stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
     sampler = ClockSampler(None)
     sampler.start()
     time.sleep(0.3)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        opt.step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    fg = opt._flat[0]
-    e0.record(stream)
-    for _ in range(args.steps):
-        opt._gather_grads(fg)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    pack_ms = e0.elapsed_time(e1) / args.steps
+    assert opt._grads_are_views(opt._flat[0])
+    ms = timed(opt.step)
     clocks = sampler.stop()
+    # per-parameter gradient tensors instead: the optimizer packs them first
+    with torch.no_grad():
+        for p in params:
+            p.grad = p.grad.clone()
+    assert not opt._grads_are_views(opt._flat[0])
+    packed_ms = timed(opt.step)
+    pack_ms = timed(lambda: opt._gather_grads(opt._flat[0]))
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
-    bpp = 6.0 + bytes_per_param(G)
+    bpp = 2.0 + bytes_per_param(G)
     achieved = bpp * n / (ms / 1e3) / 1e9
     line = {"metric": "params/s for CoatAdamW.step() (OLMo-7B set, FP32 parameters and gradients)",
             "value": n / (ms / 1e3), "unit": "params/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"olmo-7b set as {len(params)} FP32 parameters with FP32 "
-                                   "gradients, CoatAdamW(group_size=128)",
+            "config": {"workload": f"olmo-7b set as {len(params)} FP32 parameters, "
+                                   "CoatAdamW(group_size=128, flat_grads=True)",
                        "group_size": G, "params": n,
-                       "l2": "no flush needed: 140 GB moved per step"},
+                       "l2": "no flush needed: 112 GB moved per step"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None,
                          "peak_source": f"{peak_kind} copy bandwidth",
                          "algorithmic_bytes_per_param": bpp},
-            "kernels": {"pack_bf16_ms": pack_ms, "fused_step_ms": ms - pack_ms},
-            "clocks": clocks, "gpu_launches": args.steps * 3}
+            "kernels": {"flat_grads_step_ms": ms, "packed_step_ms": packed_ms,
+                        "pack_bf16_ms": pack_ms,
+                        "packed_params_per_s": n / (packed_ms / 1e3)},
+            "clocks": clocks, "gpu_launches": args.steps}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -143,6 +143,23 @@ coat_status_t coat_count_nonfinite_bf16(const uint16_t *x, int64_t n, uint32_t *
                                         void *stream);
 
 /*
+ * coat_adamw_fp8_step_fp32grad -- coat_adamw_fp8_step with float32 gradients
+ * (e.g. a flat float32 gradient buffer that a framework accumulates into):
+ * each gradient is rounded to BF16 (nearest even) as it is loaded and the
+ * step then proceeds exactly as with that BF16 gradient ([QA]: BF16
+ * gradients, FP32 master weights), so the results are those of
+ * coat_adamw_fp8_step on the rounded gradients.  It saves the separate
+ * float32 -> BF16 pass (6 B per parameter of HBM traffic) at the cost of
+ * reading 4 instead of 2 gradient bytes in the step.
+ *   grad   float32[n] (16-byte aligned)
+ * Other arguments and errors as coat_adamw_fp8_step.
+ */
+coat_status_t coat_adamw_fp8_step_fp32grad(float *param, const float *grad, uint8_t *m_code,
+                                           float *m_k, float *m_scale, uint8_t *v_code,
+                                           float *v_k, float *v_scale, int64_t n,
+                                           const coat_adamw_cfg_t *cfg, void *stream);
+
+/*
  * coat_adamw_fp8_step_guarded -- coat_adamw_fp8_step, except that the
  * kernel first reads the device word *skip_if_nonzero and, if it is not
  * zero, returns without reading or writing anything else: parameters,

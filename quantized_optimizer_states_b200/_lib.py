@@ -69,6 +69,8 @@ SIGNATURES = {
     "coat_count_nonfinite_bf16": (_I32, [_P, _I64, _P, _P]),
     "coat_adamw_fp8_step_guarded": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
                                            ctypes.POINTER(CoatAdamwCfg), _P, _P]),
+    "coat_adamw_fp8_step_fp32grad": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
+                                            ctypes.POINTER(CoatAdamwCfg), _P]),
     "coat_pack_bf16": (_I32, [ctypes.POINTER(_P), ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                               _I32, _I32, _P, _I64, _P]),
     "coat_unpack_bf16": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), _I32,
@@ -134,18 +136,36 @@ def coat_adamw_fp8_step(param, grad, m_code, m_k, m_scale, v_code, v_k, v_scale,
                         group_size: int = 128, m_fmt: int = COAT_E4M3, v_fmt: int = COAT_E4M3,
                         k_range: int = 0, k_max: float = 64.0, flags: int = 0,
                         skip_if_nonzero=None, stream=None):
-    """One fused COAT AdamW step, in place (see include/coat.h).  With
-    skip_if_nonzero (a CUDA int32/uint32 tensor of one element) the guarded
-    form runs: the step is a no-op when that word is nonzero."""
+    """One fused COAT AdamW step, in place (see include/coat.h).  grad holds
+    BF16 gradients (bfloat16 / int16 / uint16 bit patterns) or float32
+    gradients, which the kernel rounds to BF16 as it loads them
+    (coat_adamw_fp8_step_fp32grad).  With skip_if_nonzero (a CUDA
+    int32/uint32 tensor of one element) the guarded form runs: the step is a
+    no-op when that word is nonzero (BF16 gradients only)."""
     import torch
     cfg = CoatAdamwCfg(beta1, beta2, lr, eps, weight_decay, step, group_size, m_fmt, v_fmt,
                        k_range, k_max, flags)
-    args = [_ptr(param, torch.float32, "param"), _u16(grad, "grad"),
+    f32 = grad.dtype == torch.float32
+    if f32 and skip_if_nonzero is not None:
+        raise ValueError("the guarded step takes BF16 gradients")
+    n = param.numel()
+    if grad.numel() != n or m_code.numel() != n or v_code.numel() != n:
+        raise ValueError("grad, m_code and v_code must have as many elements as param")
+    if 16 <= group_size <= 4096 and group_size & (group_size - 1) == 0:
+        # (an unsupported G is reported by the library itself)
+        ng = -(-n // group_size)
+        if min(m_k.numel(), m_scale.numel(), v_k.numel(), v_scale.numel()) < ng:
+            raise ValueError(f"k and scale arrays need ceil(n / G) = {ng} elements")
+    args = [_ptr(param, torch.float32, "param"),
+            _ptr(grad, None, "grad") if f32 else _u16(grad, "grad"),
             _ptr(m_code, torch.uint8, "m_code"), _ptr(m_k, torch.float32, "m_k"),
             _ptr(m_scale, torch.float32, "m_scale"), _ptr(v_code, torch.uint8, "v_code"),
             _ptr(v_k, torch.float32, "v_k"), _ptr(v_scale, torch.float32, "v_scale"),
             param.numel(), ctypes.byref(cfg)]
-    if skip_if_nonzero is None:
+    if f32:
+        st = load().coat_adamw_fp8_step_fp32grad(*args, _stream(stream))
+        _check("coat_adamw_fp8_step_fp32grad", st)
+    elif skip_if_nonzero is None:
         st = load().coat_adamw_fp8_step(*args, _stream(stream))
         _check("coat_adamw_fp8_step", st)
     else:

@@ -139,14 +139,14 @@ coat_status_t launch_step(void (*kernel)(coat::StepParams), unsigned int grid, i
 }
 
 // The step kernel is instantiated for each supported group size and for
-// full blocks / the ragged tail block.
-template <int VF, bool FULL>
+// full blocks / the ragged tail block, and for BF16 / float32 gradients.
+template <int VF, bool FULL, bool GF32>
 coat_status_t launch_step_for(int lg, unsigned int grid, int block, size_t smem, cudaStream_t s,
                               const coat::StepParams &p) {
   switch (lg) {
 #define COAT_LAUNCH(LGV) \
   case LGV:              \
-    return launch_step(coat::adamw_fp8_step_kernel<VF, LGV, FULL>, grid, block, smem, s, p);
+    return launch_step(coat::adamw_fp8_step_kernel<VF, LGV, FULL, GF32>, grid, block, smem, s, p);
     COAT_LAUNCH(4) COAT_LAUNCH(5) COAT_LAUNCH(6) COAT_LAUNCH(7) COAT_LAUNCH(8)
     COAT_LAUNCH(9) COAT_LAUNCH(10) COAT_LAUNCH(11) COAT_LAUNCH(12)
 #undef COAT_LAUNCH
@@ -156,7 +156,7 @@ coat_status_t launch_step_for(int lg, unsigned int grid, int block, size_t smem,
 
 // One launch over the full blocks (no bounds checks), then, if n is not a
 // multiple of the block's parameter count, one block for the ragged tail.
-template <int VF>
+template <int VF, bool GF32>
 coat_status_t launch_step_all(int lg, int64_t n, cudaStream_t s, coat::StepParams p) {
   size_t smem = 0;
   int block = 0;
@@ -167,19 +167,20 @@ coat_status_t launch_step_all(int lg, int64_t n, cudaStream_t s, coat::StepParam
   if (full > 0) {
     p.block0 = 0;
     const coat_status_t st =
-        launch_step_for<VF, true>(lg, static_cast<unsigned int>(full), block, smem, s, p);
+        launch_step_for<VF, true, GF32>(lg, static_cast<unsigned int>(full), block, smem, s, p);
     if (st != COAT_OK) return st;
   }
   if (n % per != 0) {
     p.block0 = full;
-    return launch_step_for<VF, false>(lg, 1u, block, smem, s, p);
+    return launch_step_for<VF, false, GF32>(lg, 1u, block, smem, s, p);
   }
   return COAT_OK;
 }
 
-coat_status_t step_impl(float *param, const uint16_t *grad, uint8_t *m_code, float *m_k,
-                        float *m_scale, uint8_t *v_code, float *v_k, float *v_scale, int64_t n,
-                        const coat_adamw_cfg_t *cfg, const uint32_t *skip, void *stream) {
+coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *m_code,
+                        float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
+                        float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
+                        const uint32_t *skip, void *stream) {
   if (!cfg || n < 0) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!param || !grad || !m_code || !m_k || !m_scale || !v_code || !v_k || !v_scale))
     return COAT_ERR_INVALID_ARG;
@@ -198,7 +199,8 @@ coat_status_t step_impl(float *param, const uint16_t *grad, uint8_t *m_code, flo
 
   coat::StepParams p;
   p.theta = param;
-  p.grad = grad;
+  p.grad = grad_f32 ? nullptr : static_cast<const uint16_t *>(grad);
+  p.grad_f32 = grad_f32 ? static_cast<const float *>(grad) : nullptr;
   p.m_code = m_code;
   p.m_k = m_k;
   p.m_s = m_scale;
@@ -249,8 +251,11 @@ coat_status_t step_impl(float *param, const uint16_t *grad, uint8_t *m_code, flo
   }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3>(lg, n, s, p)
-                                 : launch_step_all<coat::kE5M2>(lg, n, s, p);
+  if (grad_f32)
+    return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3, true>(lg, n, s, p)
+                                   : launch_step_all<coat::kE5M2, true>(lg, n, s, p);
+  return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3, false>(lg, n, s, p)
+                                 : launch_step_all<coat::kE5M2, false>(lg, n, s, p);
 }
 
 }  // namespace
@@ -261,8 +266,16 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
                                   float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
                                   float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
                                   void *stream) {
-  return step_impl(param, grad, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg, nullptr,
-                   stream);
+  return step_impl(param, grad, false, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
+                   nullptr, stream);
+}
+
+coat_status_t coat_adamw_fp8_step_fp32grad(float *param, const float *grad, uint8_t *m_code,
+                                           float *m_k, float *m_scale, uint8_t *v_code,
+                                           float *v_k, float *v_scale, int64_t n,
+                                           const coat_adamw_cfg_t *cfg, void *stream) {
+  return step_impl(param, grad, true, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
+                   nullptr, stream);
 }
 
 coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, uint8_t *m_code,
@@ -272,7 +285,7 @@ coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, ui
                                           const uint32_t *skip_if_nonzero, void *stream) {
   if (!skip_if_nonzero || (reinterpret_cast<uintptr_t>(skip_if_nonzero) & 3u) != 0)
     return skip_if_nonzero ? COAT_ERR_MISALIGNED : COAT_ERR_INVALID_ARG;
-  return step_impl(param, grad, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
+  return step_impl(param, grad, false, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
                    skip_if_nonzero, stream);
 }
 

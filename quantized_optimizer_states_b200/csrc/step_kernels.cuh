@@ -62,7 +62,8 @@ constexpr int kMinTableLog2G = 6;                  // decode tables for G >= 64
 
 struct StepParams {
   float *theta;
-  const uint16_t *grad;
+  const uint16_t *grad;       // BF16 gradients (the kernel's GF32 = false form)
+  const float *grad_f32;      // float32 gradients, rounded to BF16 on load (GF32 = true)
   uint8_t *m_code;
   float *m_k;
   float *m_s;
@@ -459,7 +460,15 @@ __device__ __forceinline__ void load16_bf16(const uint16_t *p, int64_t e0, int64
 
 // ---- the fused step ----------------------------------------------------------
 
-template <int VF, int LG, bool FULL>
+// BF16 pair from two binary32 values, each rounded to nearest even
+// (element lo in the low half, as BF16 words are stored)
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+template <int VF, int LG, bool FULL, bool GF32>
 __global__ void __launch_bounds__(StepLayout<LG>::kBlock, StepLayout<LG>::kMinBlocks)
 adamw_fp8_step_kernel(const StepParams p) {
   using L = StepLayout<LG>;
@@ -511,7 +520,15 @@ adamw_fp8_step_kernel(const StepParams p) {
   float m[16], v[16];
   uint32_t gw[8], mw[4], vw[4];
   if (active) {
-    load16_bf16<FULL>(p.grad, e0, p.n, gw);
+    if constexpr (GF32) {
+      // float32 gradients become the BF16 gradients of the rule right here
+      float g16[16];
+      load16_f32<FULL>(p.grad_f32, e0, p.n, g16);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) gw[i] = bf16x2_rn(g16[2 * i], g16[2 * i + 1]);
+    } else {
+      load16_bf16<FULL>(p.grad, e0, p.n, gw);
+    }
     load16_u8<FULL>(p.m_code, e0, p.n, mw);
     load16_u8<FULL>(p.v_code, e0, p.n, vw);
   } else {

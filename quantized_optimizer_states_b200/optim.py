@@ -23,6 +23,13 @@ the rule).
 Both moves are one multi-tensor launch per 128 parameters
 (coat_pack_bf16 / coat_unpack_bf16), not one copy per parameter.
 
+With flat_grads=True, FP32 parameter groups also get a flat FP32 gradient
+buffer and every parameter's .grad becomes a view into it; backward then
+accumulates in place into the buffer, and the step reads it directly
+(coat_adamw_fp8_step_fp32grad rounds each gradient to BF16 as it loads it),
+so no separate pack pass runs.  zero_grad() zeroes the buffer and keeps the
+views (a .grad replaced by another tensor is noticed and packed instead).
+
 Fresh states are all-zero groups (codes 0, k = 1, s = 0).  `state_dict()`
 holds the flat buffers themselves, so saving and loading reproduces the run
 bit for bit.
@@ -57,7 +64,7 @@ class _FlatGroup:
     offsets: list[int]
     n: int
     master: torch.Tensor
-    grad: torch.Tensor
+    grad: torch.Tensor | None   # flat BF16 gradients (allocated on first use)
     m_code: torch.Tensor
     v_code: torch.Tensor
     m_k: torch.Tensor
@@ -66,6 +73,7 @@ class _FlatGroup:
     v_s: torch.Tensor
     bf16_params: bool
     table: _lib.PackTable
+    grad32: torch.Tensor | None = None   # flat FP32 gradients (flat_grads)
     step: int = 0
 
 
@@ -88,11 +96,14 @@ class CoatAdamW(torch.optim.Optimizer):
       skip_nonfinite: count inf/NaN gradients first (on the device) and skip
         the whole step of a parameter group that has any; the group's step
         counter then does not advance (one host read of the count per step).
+      flat_grads: give FP32 parameter groups a flat FP32 gradient buffer that
+        the parameters' .grad view (see the module docstring).
     """
 
     def __init__(self, params, lr: float = 1e-3, betas=(0.9, 0.999), eps: float = 1e-8,
                  weight_decay: float = 1e-2, *, group_size: int = 128, v_fmt="e4m3",
-                 k_range: int = 0, k_max: float = 64.0, skip_nonfinite: bool = False):
+                 k_range: int = 0, k_max: float = 64.0, skip_nonfinite: bool = False,
+                 flat_grads: bool = False):
         if not 0.0 <= betas[0] < 1.0 or not 0.0 <= betas[1] < 1.0:
             raise ValueError("betas must be in [0, 1)")
         if lr < 0.0 or eps < 0.0 or weight_decay < 0.0:
@@ -106,6 +117,11 @@ class CoatAdamW(torch.optim.Optimizer):
         self.skip_nonfinite = skip_nonfinite
         self.skipped_steps = 0
         self._flat: list[_FlatGroup] = [self._build(g) for g in self.param_groups]
+        if flat_grads:
+            for fg in self._flat:
+                if not fg.bf16_params:
+                    fg.grad32 = torch.zeros(fg.n, dtype=torch.float32, device=fg.master.device)
+                    self._attach_grad_views(fg)
 
     # ---- flat buffers --------------------------------------------------------
 
@@ -133,7 +149,7 @@ class CoatAdamW(torch.optim.Optimizer):
         z8 = lambda: torch.zeros(n, dtype=torch.uint8, device=dev)  # noqa: E731
         return _FlatGroup(
             params=ps, offsets=offsets, n=n, master=master,
-            grad=torch.zeros(n, dtype=torch.bfloat16, device=dev),
+            grad=None,
             m_code=z8(), v_code=z8(),
             m_k=torch.ones(ng, dtype=torch.float32, device=dev),
             m_s=torch.zeros(ng, dtype=torch.float32, device=dev),
@@ -141,8 +157,26 @@ class CoatAdamW(torch.optim.Optimizer):
             v_s=torch.zeros(ng, dtype=torch.float32, device=dev),
             bf16_params=bf16, table=_lib.PackTable([p.numel() for p in ps], offsets))
 
+    def _attach_grad_views(self, fg: _FlatGroup):
+        for p, off in zip(fg.params, fg.offsets):
+            p.grad = fg.grad32[off:off + p.numel()].view_as(p)
+
+    def _grads_are_views(self, fg: _FlatGroup) -> bool:
+        base, size = fg.grad32.data_ptr(), fg.grad32.element_size()
+        return all(p.grad is not None and p.grad.data_ptr() == base + off * size
+                   and p.grad.is_contiguous() for p, off in zip(fg.params, fg.offsets))
+
+    def zero_grad(self, set_to_none: bool = True):
+        super().zero_grad(set_to_none=set_to_none)
+        for fg in self._flat:
+            if fg.grad32 is not None:
+                fg.grad32.zero_()
+                self._attach_grad_views(fg)
+
     @torch.no_grad()
     def _gather_grads(self, fg: _FlatGroup):
+        if fg.grad is None:
+            fg.grad = torch.zeros(fg.n, dtype=torch.bfloat16, device=fg.master.device)
         want = torch.bfloat16 if fg.bf16_params else torch.float32
         grads = []
         for p in fg.params:
@@ -173,7 +207,10 @@ class CoatAdamW(torch.optim.Optimizer):
             with torch.enable_grad():
                 loss = closure()
         for group, fg in zip(self.param_groups, self._flat):
-            self._gather_grads(fg)
+            direct = (fg.grad32 is not None and not self.skip_nonfinite
+                      and self._grads_are_views(fg))
+            if not direct:
+                self._gather_grads(fg)
             if self.skip_nonfinite:
                 count = torch.zeros(1, dtype=torch.int32, device=fg.grad.device)
                 _lib.coat_count_nonfinite_bf16(fg.grad, count)
@@ -183,7 +220,8 @@ class CoatAdamW(torch.optim.Optimizer):
             fg.step += 1
             b1, b2 = group["betas"]
             _lib.coat_adamw_fp8_step(
-                fg.master, fg.grad, fg.m_code, fg.m_k, fg.m_s, fg.v_code, fg.v_k, fg.v_s,
+                fg.master, fg.grad32 if direct else fg.grad, fg.m_code, fg.m_k, fg.m_s,
+                fg.v_code, fg.v_k, fg.v_s,
                 beta1=b1, beta2=b2, lr=group["lr"], eps=group["eps"],
                 weight_decay=group["weight_decay"], step=fg.step,
                 group_size=group["group_size"], v_fmt=group["v_fmt"],

@@ -170,3 +170,51 @@ def test_zero1_shard_single_rank_is_the_plain_step(optim):
         q.coat_adamw_fp8_step(th, gp, mc, mk, ms, vc, vk, vs, step=t, group_size=128, **H)
         assert torch.equal(full, th[:n])
         assert torch.equal(sh.m_code, mc) and torch.equal(sh.v_code, vc)
+
+
+def test_flat_fp32_gradients_match_the_packed_path(optim):
+    """flat_grads=True: .grad are views of one FP32 buffer, the step reads it
+    directly (rounding to BF16 on load); the parameters and states must be
+    bit-identical to the packed path on the same gradients, also when a
+    .grad is replaced by a tensor of its own (that group is packed)."""
+    pa, pb = _model(3), _model(3)
+    oa = _opt(optim, pa, flat_grads=True)
+    ob = _opt(optim, pb)
+    fa, fb = oa._flat[0], ob._flat[0]
+    for t in (1, 2, 3, 4):
+        g = torch.Generator().manual_seed(77 + t)
+        grads = [(torch.randn(p.shape, generator=g) * 1e-3).cuda() for p in pa]
+        for p, q, x in zip(pa, pb, grads):
+            if t == 3 and p is pa[1]:
+                p.grad = x.clone()          # replaced: this step takes the packed path
+            else:
+                p.grad.copy_(x)             # in place into the flat buffer
+            q.grad = x.clone()
+        assert oa._grads_are_views(fa) == (t != 3)
+        oa.step()
+        ob.step()
+        oa.zero_grad()
+        assert oa._grads_are_views(fa)
+        for k in ("master", "m_code", "m_k", "m_s", "v_code", "v_k", "v_s"):
+            assert torch.equal(getattr(fa, k), getattr(fb, k)), (t, k)
+
+
+def test_flat_fp32_gradients_through_backward(optim):
+    """backward accumulates into the flat buffer in place (the .grad stay
+    views), and the result equals the packed path."""
+    torch.manual_seed(5)
+    lin_a = torch.nn.Linear(96, 80).cuda()
+    lin_b = torch.nn.Linear(96, 80).cuda()
+    lin_b.load_state_dict(lin_a.state_dict())
+    oa = _opt(optim, list(lin_a.parameters()), flat_grads=True)
+    ob = _opt(optim, list(lin_b.parameters()))
+    x = torch.randn(32, 96, device="cuda")
+    for _ in range(3):
+        for lin, opt in ((lin_a, oa), (lin_b, ob)):
+            opt.zero_grad()
+            lin(x).square().mean().backward()
+        assert oa._grads_are_views(oa._flat[0])
+        oa.step()
+        ob.step()
+    for pa, pb in zip(lin_a.parameters(), lin_b.parameters()):
+        assert torch.equal(pa, pb)

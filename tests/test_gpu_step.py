@@ -93,6 +93,31 @@ def test_variants(lib, orc, variant):
     _one_step(lib, orc, x, st, **kw)
 
 
+@pytest.mark.parametrize("v_fmt", [E4M3, E5M2])
+def test_fp32_gradients_round_to_bf16(lib, orc, v_fmt):
+    """coat_adamw_fp8_step_fp32grad: float32 gradients rounded to BF16 on
+    load give the oracle's step on the rounded gradients (and the BF16
+    entry point's bits), ragged size included."""
+    import torch
+    G, n = 128, 3 * 4096 + 1000 + 37
+    x = inputs.host_step_inputs(inputs.olmo_1b(), n)
+    rng = np.random.default_rng(11)
+    g32 = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    g32[:3] = [0.0, -0.0, 3.0e-39]                      # zeros and a subnormal
+    gb = orc.to_bf16_array(g32)
+    st = _init_states(orc, x, G, v_fmt)
+    cfg = dict(step=10, group_size=G, v_fmt=v_fmt, **H)
+    ref = orc.adamw_fp8_step(x["theta"], gb, *st, return_moments=True, **cfg)
+    d = [parity.to_dev(x["theta"]), parity.to_dev(g32)] + [parity.to_dev(a) for a in st]
+    lib.coat_adamw_fp8_step(*d, **cfg)
+    torch.cuda.synchronize()
+    got = tuple(parity.to_host(t) for t in (d[0], d[2], d[3], d[4], d[5], d[6], d[7]))
+    parity.assert_step_parity(got, ref, H["lr"], G, v_fmt, moments=(ref[7], ref[8]))
+    same = parity.gpu_step(lib, x["theta"], gb, *st, **cfg)
+    for a, b in zip(got, same):
+        assert np.array_equal(a, b)
+
+
 def test_degenerate_groups(lib, orc):
     """All-zero, all-equal, single-nonzero, zero-gradient groups and a tail
     group of one element."""

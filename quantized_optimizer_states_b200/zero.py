@@ -9,7 +9,9 @@ boundaries, so each rank keeps 1/world of it.  One step:
   1. reduce-scatter of the gradients: each rank receives, over its shard,
      the mean of all ranks' gradients (summed in binary32 by the collective,
      divided by the rank count, rounded to BF16 nearest-even);
-  2. the COAT step on the shard (one `coat_adamw_fp8_step` call);
+  2. the COAT step on the shard (one `coat_adamw_fp8_step` call, which takes
+     the binary32 mean and rounds it to BF16 as it loads it, so no separate
+     conversion pass runs);
   3. all-gather of the updated master weights.
 
 No 1xG group straddles two shards, so the sharded step computes exactly
@@ -74,9 +76,9 @@ class Zero1Shard:
         self.m_s = torch.zeros(ng, dtype=torch.float32, device=dev)
         self.v_s = torch.zeros(ng, dtype=torch.float32, device=dev)
 
-    def reduce_gradient(self, grad: torch.Tensor) -> torch.Tensor:
-        """Mean over ranks of the full BF16 gradients, this rank's shard, as
-        BF16 (binary32 sum, division by the rank count, nearest-even BF16)."""
+    def reduce_gradient_f32(self, grad: torch.Tensor) -> torch.Tensor:
+        """Mean over ranks of the full BF16 gradients, this rank's shard, in
+        binary32 (sum by the collective, division by the rank count)."""
         full = torch.zeros(self.world * self.L, dtype=torch.float32, device=grad.device)
         full[:self.n].copy_(grad.reshape(-1))
         part = torch.empty(self.L, dtype=torch.float32, device=grad.device)
@@ -85,7 +87,12 @@ class Zero1Shard:
             part.div_(float(self.world))
         else:
             part.copy_(full)
-        return part.to(torch.bfloat16)
+        return part
+
+    def reduce_gradient(self, grad: torch.Tensor) -> torch.Tensor:
+        """The same mean rounded to BF16 (nearest even): the gradient the
+        step uses."""
+        return self.reduce_gradient_f32(grad).to(torch.bfloat16)
 
     def gather_params(self) -> torch.Tensor:
         """The full updated FP32 parameter buffer (first n elements)."""
@@ -100,6 +107,8 @@ class Zero1Shard:
         """One data-parallel step with this rank's full BF16 gradient `grad`;
         returns the full updated parameters.  `step_fn(shard, grad_shard, t,
         hyper)` replaces the CUDA step (the CPU tests pass the oracle)."""
-        g = self.reduce_gradient(grad)
-        (step_fn or _coat_step)(self, g, t, hyper)
+        if step_fn is None:
+            _coat_step(self, self.reduce_gradient_f32(grad), t, hyper)  # rounded on load
+        else:
+            step_fn(self, self.reduce_gradient(grad), t, hyper)
         return self.gather_params()

@@ -522,23 +522,30 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantParams p
   store16_out(p, e0, x);
 }
 
-// Activations (no k): x = d * s, one binary32 product; kActV vectors per thread.
+// Activations (no k): x = d * s, one binary32 product; kDeqV vectors per thread.
+constexpr int kDeqV = kActV;
+
+inline unsigned int deq_blocks(int64_t elems) {
+  const int64_t per = static_cast<int64_t>(kElemsPerBlock) * kDeqV;
+  return static_cast<unsigned int>((elems + per - 1) / per);
+}
+
 template <int F>
 __global__ void __launch_bounds__(kThreads) dequant_linear_kernel(const DequantParams p) {
   pdl_enter();
-  uint32_t w[kActV][4];
-  int64_t e0[kActV];
-  float s[kActV];
+  uint32_t w[kDeqV][4];
+  int64_t e0[kDeqV];
+  float s[kDeqV];
 #pragma unroll
-  for (int v = 0; v < kActV; ++v) {
-    e0[v] = ((static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x) * kVec;
+  for (int v = 0; v < kDeqV; ++v) {
+    e0[v] = ((static_cast<int64_t>(blockIdx.x) * kDeqV + v) * kThreads + threadIdx.x) * kVec;
     if (e0[v] < p.n) {
       load16_u8<false>(p.q, e0[v], p.n, w[v]);
       s[v] = p.scale[p.log2G < 0 ? 0 : (e0[v] >> p.log2G)];
     }
   }
 #pragma unroll
-  for (int v = 0; v < kActV; ++v) {
+  for (int v = 0; v < kDeqV; ++v) {
     if (e0[v] >= p.n) continue;
     float x[16];
 #pragma unroll

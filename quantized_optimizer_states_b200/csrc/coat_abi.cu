@@ -367,7 +367,7 @@ coat_status_t coat_dequant(const uint8_t *q, const float *k, const float *scale,
   } else {
     // plain loads: a streamed form (bulk copies of the codes) measured
     // slower here, the kernel being bound by its 4-byte-per-element writes
-    const unsigned int grid = coat::act_blocks(n);
+    const unsigned int grid = coat::deq_blocks(n);
     if (fmt == COAT_E4M3)
       launch_act(coat::dequant_linear_kernel<coat::kE4M3>, grid, 0, s, p);
     else

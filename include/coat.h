@@ -360,6 +360,42 @@ coat_status_t coat_pack_bf16(const void *const *src, const int64_t *numel, const
 coat_status_t coat_unpack_bf16(const float *src, const int64_t *numel, const int64_t *offset,
                                int32_t count, void *const *dst, int64_t n, void *stream);
 
+/*
+ * coat_state_stats -- monitoring of one compressed optimizer state (codes in
+ * `fmt` with per-group k and s, as coat_adamw_fp8_step leaves them).  The
+ * pages define no such report; it counts what COAT's expansion is meant to
+ * produce ([COAT] "扩展函数": every group's maximum on the format's largest
+ * value, k per group and step, typically 1-3 for m and 5-15 for v).  Two
+ * launches: one initialising *stats, one accumulating into it; read it after
+ * the stream reaches them.
+ *   code   uint8[n] (16-byte aligned);  k, scale  float32[ceil(n/G)]
+ *   stats  DEVICE pointer to a coat_state_stats_t (8-byte aligned):
+ *     groups          ceil(n/G)
+ *     zero_groups     groups with scale 0 (all-zero groups)
+ *     k1_groups       other groups stored with k == 1 (no expansion)
+ *     max_codes       codes whose magnitude is the format's largest finite
+ *                     value (0x7E E4M3, 0x7B E5M2): at least one per
+ *                     nonzero group
+ *     zero_codes      codes +-0
+ *     nonfinite_codes inf / NaN codes (0 for states the library wrote)
+ *     k_sum, k_min, k_max  over the nonzero groups (+inf / -inf / 0 when
+ *                     there are none); mean k = k_sum / (groups - zero_groups);
+ *                     k_sum is summed with floating-point atomics, so its
+ *                     last bits can differ between runs (the counts and
+ *                     k_min / k_max are exact)
+ * Errors: INVALID_ARG, UNSUPPORTED (G, fmt), MISALIGNED, CUDA.
+ */
+typedef struct {
+  uint64_t groups, zero_groups, k1_groups;
+  uint64_t max_codes, zero_codes, nonfinite_codes;
+  double k_sum;
+  float k_min, k_max;
+} coat_state_stats_t;
+
+coat_status_t coat_state_stats(const uint8_t *code, const float *k, const float *scale,
+                               int64_t n, int32_t group_size, int32_t fmt,
+                               coat_state_stats_t *stats, void *stream);
+
 /* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
  * this thread (0 if none). */
 int32_t coat_last_cuda_error(void);

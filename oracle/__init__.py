@@ -305,6 +305,31 @@ def group_amax_of(x_bf16: np.ndarray, G: int) -> np.ndarray:
     return pad.reshape(ng, G).max(axis=1).astype(np.float32)
 
 
+def state_stats(code: np.ndarray, k: np.ndarray, s: np.ndarray, G: int, fmt: int) -> dict:
+    """Monitoring counts of one compressed state, written from their
+    definitions (nothing here is on the pages beyond the format maxima of the
+    LLM Atlas "systems/numerics" page, section 03 "FP8"): groups, all-zero
+    groups (scale 0), other groups stored with k == 1, codes at the largest
+    finite magnitude / at +-0 / on inf-NaN patterns, and the sum, min and max
+    of k over the nonzero groups."""
+    code = np.ascontiguousarray(code, dtype=np.uint8).reshape(-1)
+    k = np.asarray(k, dtype=np.float32).reshape(-1)
+    s = np.asarray(s, dtype=np.float32).reshape(-1)
+    ng = n_groups(code.size, G)
+    k, s = k[:ng], s[:ng]
+    top = 0x7E if fmt == E4M3 else 0x7B      # 448 = 0x7E (E4M3), 57344 = 0x7B (E5M2)
+    mag = code & 0x7F
+    nz = s != 0
+    kn = k[nz].astype(np.float64)
+    return {"groups": ng, "zero_groups": int((~nz).sum()),
+            "k1_groups": int((k[nz] == 1.0).sum()),
+            "max_codes": int((mag == top).sum()), "zero_codes": int((mag == 0).sum()),
+            "nonfinite_codes": int((mag > top).sum()),
+            "k_sum": float(kn.sum()) if kn.size else 0.0,
+            "k_min": float(kn.min()) if kn.size else float("inf"),
+            "k_max": float(kn.max()) if kn.size else float("-inf")}
+
+
 def threads_used() -> int:
     return 1
 

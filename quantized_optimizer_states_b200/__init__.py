@@ -23,6 +23,7 @@ from ._lib import (  # noqa: F401
     coat_group_scaling_workspace_bytes,
     coat_pack_bf16,
     coat_quantize_state,
+    coat_state_stats,
     coat_status_string,
     coat_swiglu_group_amax,
     coat_unpack_bf16,

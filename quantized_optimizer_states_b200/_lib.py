@@ -75,6 +75,7 @@ SIGNATURES = {
                               _I32, _I32, _P, _I64, _P]),
     "coat_unpack_bf16": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), _I32,
                                 ctypes.POINTER(_P), _I64, _P]),
+    "coat_state_stats": (_I32, [_P, _P, _P, _I64, _I32, _I32, _P, _P]),
     "coat_last_cuda_error": (_I32, []),
     "coat_bulk_wait_timeouts": (_I32, [ctypes.POINTER(ctypes.c_uint32), _I32]),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
@@ -331,6 +332,35 @@ def coat_unpack_bf16(src, table: PackTable, dsts, *, stream=None):
     _check("coat_unpack_bf16", load().coat_unpack_bf16(
         _ptr(src, torch.float32, "src"), table.numel, table.offset, table.count,
         table.pointers(dsts), src.numel(), _stream(stream)))
+
+
+class CoatStateStats(ctypes.Structure):
+    _fields_ = [("groups", ctypes.c_uint64), ("zero_groups", ctypes.c_uint64),
+                ("k1_groups", ctypes.c_uint64), ("max_codes", ctypes.c_uint64),
+                ("zero_codes", ctypes.c_uint64), ("nonfinite_codes", ctypes.c_uint64),
+                ("k_sum", ctypes.c_double), ("k_min", ctypes.c_float), ("k_max", ctypes.c_float)]
+
+
+def coat_state_stats(code, k, scale, *, group_size: int, fmt: int = COAT_E4M3, out=None,
+                     stream=None) -> dict:
+    """Monitoring counts of one compressed state (see include/coat.h).  With
+    `out` (a CUDA uint8 tensor of sizeof(coat_state_stats_t) bytes) the call
+    stays asynchronous and returns None; otherwise it synchronises and returns
+    the counts as a dict."""
+    import torch
+    size = ctypes.sizeof(CoatStateStats)
+    buf = out if out is not None else torch.empty(size, dtype=torch.uint8, device=code.device)
+    if buf.numel() < size:
+        raise ValueError(f"out needs {size} bytes")
+    _check("coat_state_stats", load().coat_state_stats(
+        _ptr(code, torch.uint8, "code"), _ptr(k, torch.float32, "k"),
+        _ptr(scale, torch.float32, "scale"), code.numel(), group_size, fmt,
+        _ptr(buf, torch.uint8, "out"), _stream(stream)))
+    if out is not None:
+        return None
+    raw = bytes(buf.cpu().numpy().tobytes())
+    st = CoatStateStats.from_buffer_copy(raw)
+    return {name: getattr(st, name) for name, _ in CoatStateStats._fields_}
 
 
 def coat_bulk_wait_timeouts(*, reset: bool = False) -> int:

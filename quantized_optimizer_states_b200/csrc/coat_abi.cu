@@ -14,6 +14,7 @@
 #include "act_kernels.cuh"
 #include "fp8_device.cuh"
 #include "pack_kernels.cuh"
+#include "stats_kernels.cuh"
 #include "step_kernels.cuh"
 
 namespace {
@@ -623,6 +624,34 @@ coat_status_t pack_launch(bool unpack, const void *const *ptrs, const int64_t *n
 }
 
 }  // namespace
+
+extern "C" coat_status_t coat_state_stats(const uint8_t *code, const float *k,
+                                          const float *scale, int64_t n, int32_t group_size,
+                                          int32_t fmt, coat_state_stats_t *stats,
+                                          void *stream) {
+  if (n < 0 || !stats) return COAT_ERR_INVALID_ARG;
+  if (n > 0 && (!code || !k || !scale)) return COAT_ERR_INVALID_ARG;
+  if (group_log2(group_size) < 0 || !valid_fmt(fmt) || n > kMaxElems)
+    return COAT_ERR_UNSUPPORTED;
+  if ((n > 0 && !aligned16(code)) || (reinterpret_cast<uintptr_t>(stats) & 7u) != 0)
+    return COAT_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  coat::state_stats_init_kernel<<<1, 1, 0, s>>>(stats);
+  if (n > 0) {
+    coat::StatsParams p;
+    p.code = code;
+    p.k = k;
+    p.s = scale;
+    p.n = n;
+    p.ngroups = (n + group_size - 1) / group_size;
+    p.max_mag = fmt == COAT_E4M3 ? 0x7Eu : 0x7Bu;
+    p.out = stats;
+    const int64_t want = (n / 16 + coat::kStatsThreads - 1) / coat::kStatsThreads;
+    const unsigned int grid = static_cast<unsigned int>(want < 1184 ? (want > 0 ? want : 1) : 1184);
+    coat::state_stats_kernel<<<grid, coat::kStatsThreads, 0, s>>>(p);
+  }
+  return launch_status();
+}
 
 extern "C" coat_status_t coat_pack_bf16(const void *const *src, const int64_t *numel,
                                         const int64_t *offset, int32_t count, int32_t src_f32,

@@ -245,6 +245,16 @@ class CoatAdamW(torch.optim.Optimizer):
         _lib.coat_dequant(fg.v_code, fg.v_k, fg.v_s, v, group_size=G, fmt=vf)
         return m, v
 
+    def state_stats(self, group_index: int = 0) -> dict:
+        """Monitoring counts of a parameter group's two compressed moments
+        (coat_state_stats): {"m": {...}, "v": {...}}."""
+        fg = self._flat[group_index]
+        G = self.param_groups[group_index]["group_size"]
+        vf = self.param_groups[group_index]["v_fmt"]
+        return {"m": _lib.coat_state_stats(fg.m_code, fg.m_k, fg.m_s, group_size=G,
+                                           fmt=_lib.COAT_E4M3),
+                "v": _lib.coat_state_stats(fg.v_code, fg.v_k, fg.v_s, group_size=G, fmt=vf)}
+
     def flat_master(self, group_index: int = 0) -> torch.Tensor:
         return self._flat[group_index].master
 

@@ -117,6 +117,18 @@ def test_pack_argument_checks(lib):
     assert pk(nulls, tab(0, 8), tab(0, 16), 2, 1, P((1 << 20) + 8), 64, None) == 2
 
 
+def test_state_stats_argument_checks(lib):
+    P = ctypes.c_void_p
+    fake, odd = P(1 << 20), P((1 << 20) + 4)
+    st = lib.coat_state_stats
+    assert st(fake, fake, fake, 64, 128, 0, None, None) == 1      # no output
+    assert st(None, fake, fake, 64, 128, 0, fake, None) == 1      # no codes
+    assert st(fake, fake, fake, 64, 100, 0, fake, None) == 3      # G not a power of 2
+    assert st(fake, fake, fake, 64, 128, 4, fake, None) == 3      # no such format
+    assert st(odd, fake, fake, 64, 128, 0, fake, None) == 2       # codes not 16-byte aligned
+    assert st(fake, fake, fake, 64, 128, 0, odd, None) == 2       # output not 8-byte aligned
+
+
 def test_product_path_fails_loudly_without_library(tmp_path):
     from quantized_optimizer_states_b200 import _lib
     saved = _lib._lib

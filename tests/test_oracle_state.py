@@ -243,3 +243,27 @@ def test_brute_force_tiny_three_steps(orc, G, v_fmt):
     assert rel(th, th64) < 1e-4
     assert np.all(np.isfinite(th))
 
+
+
+def test_state_stats_hand_example(orc):
+    """The monitoring counts on a hand-built state whose answer is worked out
+    by hand: G = 4, a zero group, an expanded group with a signed top code
+    and a -0, a k = 1 group holding a NaN code, and a two-code tail group."""
+    code = np.array([0, 0, 0, 0,
+                     0x7E, 0x01, 0x80, 0xFE,
+                     0x7F, 0x7E, 0x00, 0x33,
+                     0x7E, 0x10], dtype=np.uint8)
+    k = np.array([1.0, 2.0, 1.0, 3.5], dtype=np.float32)
+    s = np.array([0.0, 0.25, 0.5, 1.0], dtype=np.float32)
+    st = orc.state_stats(code, k, s, 4, orc.E4M3)
+    assert st == {"groups": 4, "zero_groups": 1, "k1_groups": 1, "max_codes": 4,
+                  "zero_codes": 6, "nonfinite_codes": 1, "k_sum": 6.5, "k_min": 1.0,
+                  "k_max": 3.5}
+    # E5M2: the top finite magnitude is 0x7B; magnitudes 0x7E / 0x7F are NaN
+    # patterns there (0x7E, 0xFE, 0x7F, 0x7E, 0x7E: five codes)
+    st5 = orc.state_stats(code, k, s, 4, orc.E5M2)
+    assert st5["max_codes"] == 0 and st5["nonfinite_codes"] == 5
+    # no nonzero group at all
+    st0 = orc.state_stats(np.zeros(8, np.uint8), np.ones(2, np.float32),
+                          np.zeros(2, np.float32), 4, orc.E4M3)
+    assert st0["zero_groups"] == 2 and st0["k_min"] == float("inf") and st0["k_sum"] == 0.0

@@ -8,6 +8,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "coat.h"
 
@@ -20,6 +21,14 @@
 namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
+
+// Every compute entry point is one NVTX range named after it, so a profiler's
+// timeline shows which library call issued which launches (header-only
+// NVTX: without a tool attached a range costs a couple of branches).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 coat_status_t launch_status() {
   const cudaError_t e = cudaGetLastError();
@@ -267,6 +276,7 @@ coat_status_t coat_adamw_fp8_step(float *param, const uint16_t *grad, uint8_t *m
                                   float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
                                   float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
                                   void *stream) {
+  NvtxRange nvtx_range("coat_adamw_fp8_step");
   return step_impl(param, grad, false, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
                    nullptr, stream);
 }
@@ -275,6 +285,7 @@ coat_status_t coat_adamw_fp8_step_fp32grad(float *param, const float *grad, uint
                                            float *m_k, float *m_scale, uint8_t *v_code,
                                            float *v_k, float *v_scale, int64_t n,
                                            const coat_adamw_cfg_t *cfg, void *stream) {
+  NvtxRange nvtx_range("coat_adamw_fp8_step_fp32grad");
   return step_impl(param, grad, true, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
                    nullptr, stream);
 }
@@ -284,6 +295,7 @@ coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, ui
                                           float *v_k, float *v_scale, int64_t n,
                                           const coat_adamw_cfg_t *cfg,
                                           const uint32_t *skip_if_nonzero, void *stream) {
+  NvtxRange nvtx_range("coat_adamw_fp8_step_guarded");
   if (!skip_if_nonzero || (reinterpret_cast<uintptr_t>(skip_if_nonzero) & 3u) != 0)
     return skip_if_nonzero ? COAT_ERR_MISALIGNED : COAT_ERR_INVALID_ARG;
   return step_impl(param, grad, false, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
@@ -292,6 +304,7 @@ coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, ui
 
 coat_status_t coat_count_nonfinite_bf16(const uint16_t *x, int64_t n, uint32_t *count,
                                         void *stream) {
+  NvtxRange nvtx_range("coat_count_nonfinite_bf16");
   if (n < 0 || !count) return COAT_ERR_INVALID_ARG;
   if (n > 0 && !x) return COAT_ERR_INVALID_ARG;
   if (n > kMaxElems) return COAT_ERR_UNSUPPORTED;
@@ -309,6 +322,7 @@ coat_status_t coat_count_nonfinite_bf16(const uint16_t *x, int64_t n, uint32_t *
 coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size, int32_t fmt,
                                   int32_t k_range, float k_max, int32_t flags, uint8_t *code,
                                   float *k, float *scale, void *stream) {
+  NvtxRange nvtx_range("coat_quantize_state");
   if (n < 0 || !(k_max >= 0.0f)) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!x || !code || !k || !scale)) return COAT_ERR_INVALID_ARG;
   const int lg = group_log2(group_size);
@@ -339,6 +353,7 @@ coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size,
 coat_status_t coat_dequant(const uint8_t *q, const float *k, const float *scale, int64_t n,
                            int64_t group_size, int32_t fmt, int32_t out_bf16, void *out,
                            void *stream) {
+  NvtxRange nvtx_range("coat_dequant");
   if (n < 0 || group_size < 1) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!q || !scale || !out)) return COAT_ERR_INVALID_ARG;
   if (!valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
@@ -380,6 +395,7 @@ coat_status_t coat_dequant(const uint8_t *q, const float *k, const float *scale,
 coat_status_t coat_group_quant_1xG(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
                                    int32_t group_size, int32_t fmt, uint8_t *q, float *scale,
                                    void *stream) {
+  NvtxRange nvtx_range("coat_group_quant_1xG");
   if (rows < 0 || cols < 0 || ld < cols) return COAT_ERR_INVALID_ARG;
   if (rows > 0 && cols > 0 && (!x || !q || !scale)) return COAT_ERR_INVALID_ARG;
   const int lg = group_log2(group_size);
@@ -433,6 +449,7 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
                                                  int32_t group_size, int32_t fmt,
                                                  float *workspace, int32_t amax_precomputed,
                                                  uint8_t *q, float *scale, void *stream) {
+  NvtxRange nvtx_range("coat_group_scaling_quant_pertensor");
   if (n < 0) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!x || !workspace || !q || !scale)) return COAT_ERR_INVALID_ARG;
   const int lg = group_log2(group_size);
@@ -467,6 +484,7 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
 coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, int64_t n,
                                      int32_t group_size, uint16_t *out, float *group_amax,
                                      void *stream) {
+  NvtxRange nvtx_range("coat_swiglu_group_amax");
   if (n < 0) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!gate || !up || !out || !group_amax)) return COAT_ERR_INVALID_ARG;
   const int lg = group_log2(group_size);
@@ -489,6 +507,7 @@ coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, i
 
 coat_status_t coat_fp8_encode(const float *y, int64_t n, int32_t fmt, uint8_t *q,
                               void *stream) {
+  NvtxRange nvtx_range("coat_fp8_encode");
   if (n < 0) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!y || !q)) return COAT_ERR_INVALID_ARG;
   if (!valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
@@ -629,6 +648,7 @@ extern "C" coat_status_t coat_state_stats(const uint8_t *code, const float *k,
                                           const float *scale, int64_t n, int32_t group_size,
                                           int32_t fmt, coat_state_stats_t *stats,
                                           void *stream) {
+  NvtxRange nvtx_range("coat_state_stats");
   if (n < 0 || !stats) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!code || !k || !scale)) return COAT_ERR_INVALID_ARG;
   if (group_log2(group_size) < 0 || !valid_fmt(fmt) || n > kMaxElems)
@@ -656,12 +676,14 @@ extern "C" coat_status_t coat_state_stats(const uint8_t *code, const float *k,
 extern "C" coat_status_t coat_pack_bf16(const void *const *src, const int64_t *numel,
                                         const int64_t *offset, int32_t count, int32_t src_f32,
                                         uint16_t *dst, int64_t n, void *stream) {
+  NvtxRange nvtx_range("coat_pack_bf16");
   return pack_launch(false, src, numel, offset, count, src_f32, dst, n, stream);
 }
 
 extern "C" coat_status_t coat_unpack_bf16(const float *src, const int64_t *numel,
                                           const int64_t *offset, int32_t count, void *const *dst,
                                           int64_t n, void *stream) {
+  NvtxRange nvtx_range("coat_unpack_bf16");
   return pack_launch(true, const_cast<const void *const *>(dst), numel, offset, count, 1,
                      const_cast<float *>(src), n, stream);
 }
@@ -669,6 +691,7 @@ extern "C" coat_status_t coat_unpack_bf16(const float *src, const int64_t *numel
 extern "C" coat_status_t coat_group_scaling_quant_pertensor_noalloc(
     const uint16_t *x, int64_t n, int32_t group_size, int32_t fmt, uint8_t *q, float *scale,
     void *stream) {
+  NvtxRange nvtx_range("coat_group_scaling_quant_pertensor_noalloc");
   if (n < 0) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!x || !q || !scale)) return COAT_ERR_INVALID_ARG;
   const int lg = group_log2(group_size);

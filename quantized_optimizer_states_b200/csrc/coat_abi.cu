@@ -606,11 +606,16 @@ coat_status_t pack_launch(bool unpack, const void *const *ptrs, const int64_t *n
   if (count == 0) return COAT_OK;
   if (!ptrs || !numel || !offset) return COAT_ERR_INVALID_ARG;
   bool any = false;
+  int64_t chunks_in_launch = 0;
   for (int32_t i = 0; i < count; ++i) {
     if (numel[i] < 0 || offset[i] < 0 || offset[i] > n - numel[i]) return COAT_ERR_INVALID_ARG;
     if (numel[i] > 0 && unpack && !ptrs[i]) return COAT_ERR_INVALID_ARG;
     if (numel[i] > 0 && (offset[i] % 8) != 0) return COAT_ERR_MISALIGNED;
     any = any || numel[i] > 0;
+    // one launch per kPackTensors tensors, its blocks counted in an int32
+    if (i % coat::kPackTensors == 0) chunks_in_launch = 0;
+    chunks_in_launch += (numel[i] + coat::kPackChunk - 1) / coat::kPackChunk;
+    if (chunks_in_launch > 0x7fffffff) return COAT_ERR_UNSUPPORTED;
   }
   if (!any) return COAT_OK;
   if (!flat) return COAT_ERR_INVALID_ARG;
@@ -626,7 +631,6 @@ coat_status_t pack_launch(bool unpack, const void *const *ptrs, const int64_t *n
       p.offset[i] = offset[base + i];
       p.chunk0[i] = static_cast<int32_t>(chunks);
       chunks += (numel[base + i] + coat::kPackChunk - 1) / coat::kPackChunk;
-      if (chunks > 0x7fffffff) return COAT_ERR_UNSUPPORTED;
     }
     p.chunk0[c] = static_cast<int32_t>(chunks);
     p.count = c;

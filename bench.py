@@ -210,8 +210,8 @@ ACT_RING = 8  # distinct activation tensors cycled by the activation bench
 def run_activations(args):
     """The activation-side kernels on the activation workload (BF16 [16384,
     2048], G = 128, E4M3): 1xG quantization, Group Scaling (standalone: steps
-    (i)-(iii)), the SwiGLU producer with fused maxima followed by Group
-    Scaling's steps (ii)-(iii), and dequantization.
+    (i)-(iii)), the SwiGLU and LayerNorm producers with fused maxima, Group
+    Scaling's steps (ii)-(iii) after a producer, and dequantization.
 
     Steady state: each kernel is launched back to back over a ring of
     ACT_RING distinct input (and output) sets -- 8 x 64 MiB of BF16 input
@@ -246,6 +246,7 @@ def run_activations(args):
             "ws_h": torch.empty(wsn, dtype=torch.float32, device=dev),
             "s1": torch.empty(1, dtype=torch.float32, device=dev),
             "h": torch.empty(n, dtype=torch.bfloat16, device=dev),
+            "ln": torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=dev),
             "out": torch.empty(n, dtype=torch.float32, device=dev)})
     for b in ring:  # the producer's outputs that the after-producer case reads
         coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"], group_size=G)
@@ -262,6 +263,9 @@ def run_activations(args):
             lambda b: coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"],
                                                   group_size=G),
             2 + 2 + 2 + 4.0 / G),
+        "layernorm_fused_amax": (
+            lambda b: coat.coat_norm_group_amax(b["x"], b["ln"], b["ws"], group_size=G),
+            2 + 2 + 4.0 / G),
         "group_scaling_after_producer": (
             lambda b: coat.coat_group_scaling_quant_pertensor(b["h"], b["ws_h"], b["q"], b["s1"],
                                                               group_size=G,
@@ -306,7 +310,7 @@ def run_activations(args):
                          "frac": head["frac_of_hbm"], "traffic": recorded_act_traffic(n),
                          "peak_source": f"{peak_kind} copy bandwidth"},
             "kernels": res, "clocks": clocks,
-            "gpu_launches": args.steps * (1 + 2 + 1 + 2 + 1)}
+            "gpu_launches": args.steps * (1 + 2 + 1 + 1 + 2 + 1)}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -396,6 +396,33 @@ coat_status_t coat_state_stats(const uint8_t *code, const float *k, const float 
                                int64_t n, int32_t group_size, int32_t fmt,
                                coat_state_stats_t *stats, void *stream);
 
+/*
+ * coat_norm_group_amax -- a second producer with Group Scaling's step (i)
+ * fused in ([COAT] "混合粒度"; the norm is one of the nonlinear layers of
+ * "激活为什么难压" and produces the input of the QKV and MLP up/gate
+ * projections): row-wise LayerNorm (rms = 0: y = (x - mean) / sqrt(var +
+ * eps), var the mean squared deviation) or RMSNorm (rms = 1: y = x /
+ * sqrt(mean(x^2) + eps)), times weight[c] and plus bias[c] (LayerNorm only)
+ * when given, rounded to BF16; plus the maxima of |out| over every 1xG run
+ * of each row.  Evaluated in binary32, with an error of about
+ * 1e-6 x (|y| + |mean| / std) (x - mean carries the rounding of the mean):
+ * the output is the correctly rounded norm except within that distance of
+ * a BF16 rounding midpoint.
+ *   x           BF16 bits [rows, cols] row-major (16-byte aligned),
+ *               cols a multiple of 16 and of G, cols <= 16384
+ *   weight,bias float32 [cols] or NULL (bias must be NULL when rms = 1)
+ *   out         BF16 bits [rows, cols] (16-byte aligned)
+ *   group_amax  float32 [rows * cols / G]: the slots
+ *               coat_group_scaling_quant_pertensor reads on `out` (flat,
+ *               the same G) with amax_precomputed != 0
+ * Errors: INVALID_ARG (sizes, eps < 0 or not finite, rms not 0/1, bias with
+ * rms), UNSUPPORTED (G, cols > 16384), MISALIGNED, CUDA.
+ */
+coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols, int32_t rms,
+                                   float eps, const float *weight, const float *bias,
+                                   int32_t group_size, uint16_t *out, float *group_amax,
+                                   void *stream);
+
 /* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
  * this thread (0 if none). */
 int32_t coat_last_cuda_error(void);

@@ -296,6 +296,33 @@ def swiglu_bf16(gate_bf16: np.ndarray, up_bf16: np.ndarray) -> np.ndarray:
     return round_to_bf16(h)
 
 
+def norm_f64(x_bf16: np.ndarray, *, rms: bool, eps: float, weight=None,
+             bias=None) -> np.ndarray:
+    """Row-wise LayerNorm (rms=False: (x - mean) / sqrt(var + eps), var the
+    mean squared deviation) or RMSNorm (rms=True: x / sqrt(mean(x^2) + eps))
+    of BF16 rows, times an optional per-column weight plus an optional
+    per-column bias, all in binary64 (eps as the binary32 value the library
+    receives).  The norm is one of the nonlinear layers of the COAT summary
+    page (section "激活为什么难压") and produces a linear layer's input."""
+    x = bf16_bits_to_f64(x_bf16)
+    e = float(np.float32(eps))
+    if rms:
+        y = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + e)
+    else:
+        d = x - np.mean(x, axis=-1, keepdims=True)
+        y = d / np.sqrt(np.mean(d * d, axis=-1, keepdims=True) + e)
+    if weight is not None:
+        y = y * np.asarray(weight, dtype=np.float32).astype(np.float64)
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float32).astype(np.float64)
+    return y
+
+
+def norm_bf16(x_bf16: np.ndarray, **kw) -> np.ndarray:
+    """norm_f64 rounded once to BF16 (bit patterns)."""
+    return round_to_bf16(norm_f64(x_bf16, **kw))
+
+
 def group_amax_of(x_bf16: np.ndarray, G: int) -> np.ndarray:
     """Per-1xG max |x| of a flat BF16 tensor (a shorter last group allowed)."""
     x = np.abs(bf16_bits_to_f64(np.ascontiguousarray(x_bf16).reshape(-1)))

@@ -21,6 +21,7 @@ from ._lib import (  # noqa: F401
     coat_group_scaling_quant_pertensor,
     coat_group_scaling_quant_pertensor_noalloc,
     coat_group_scaling_workspace_bytes,
+    coat_norm_group_amax,
     coat_pack_bf16,
     coat_quantize_state,
     coat_state_stats,

@@ -66,6 +66,7 @@ SIGNATURES = {
     "coat_group_scaling_quant_pertensor_noalloc": (_I32, [_P, _I64, _I32, _I32, _P, _P, _P]),
     "coat_swiglu_group_amax": (_I32, [_P, _P, _I64, _I32, _P, _P, _P]),
     "coat_fp8_encode": (_I32, [_P, _I64, _I32, _P, _P]),
+    "coat_norm_group_amax": (_I32, [_P, _I64, _I64, _I32, _F, _P, _P, _I32, _P, _P, _P]),
     "coat_count_nonfinite_bf16": (_I32, [_P, _I64, _P, _P]),
     "coat_adamw_fp8_step_guarded": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
                                            ctypes.POINTER(CoatAdamwCfg), _P, _P]),
@@ -274,6 +275,26 @@ def coat_swiglu_group_amax(gate, up, out, group_amax, *, group_size: int = 128, 
         _u16(gate, "gate"), _u16(up, "up"), gate.numel(), group_size, _u16(out, "out"),
         _ptr(group_amax, torch.float32, "group_amax"), _stream(stream))
     _check("coat_swiglu_group_amax", st)
+
+
+def coat_norm_group_amax(x, out, group_amax, *, rms: bool = False, eps: float = 1e-5,
+                         weight=None, bias=None, group_size: int = 128, stream=None):
+    """LayerNorm (or RMSNorm) of BF16 rows x [rows, cols] into BF16 `out` with
+    the maxima of every 1xG run of the output in `group_amax` (see
+    include/coat.h)."""
+    import torch
+    if x.dim() != 2 or out.shape != x.shape:
+        raise ValueError("x and out must be [rows, cols] tensors of the same shape")
+    rows, cols = x.shape
+    if group_amax.numel() < rows * (cols // max(group_size, 1)):
+        raise ValueError("group_amax needs rows * cols / G elements")
+    for t, what in ((weight, "weight"), (bias, "bias")):
+        if t is not None and t.numel() != cols:
+            raise ValueError(f"{what} needs cols elements")
+    _check("coat_norm_group_amax", load().coat_norm_group_amax(
+        _u16(x, "x"), rows, cols, int(rms), float(eps), _ptr(weight, torch.float32, "weight"),
+        _ptr(bias, torch.float32, "bias"), group_size, _u16(out, "out"),
+        _ptr(group_amax, torch.float32, "group_amax"), _stream(stream)))
 
 
 def coat_fp8_encode(y, q, *, fmt: int = COAT_E4M3, stream=None):

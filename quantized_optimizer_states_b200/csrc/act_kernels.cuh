@@ -394,6 +394,143 @@ __global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const Swigl
   }
 }
 
+// ---- a second producer with the maxima fused in: LayerNorm / RMSNorm ---------------------
+// The norm of a transformer block (COAT summary page, section "激活为什么难压":
+// LayerNorm/RMSNorm are among the nonlinear layers) produces the input of
+// the linear layers that follow it (QKV, MLP up/gate), so, as for SwiGLU,
+// it emits the per-1xG maxima of its BF16 output for Group Scaling (section
+// "混合粒度").  Per row (token):
+//   LayerNorm  y = (x - mean) / sqrt(var + eps)   (var: mean of squared deviations)
+//   RMSNorm    y = x / sqrt(mean(x^2) + eps)
+// then y * weight[c] (+ bias[c] for LayerNorm) when given, rounded to BF16.
+// One warp per row: the warp stages its row in shared memory (coalesced
+// 16-byte loads), takes the row sums over it in binary32 (per-lane sums,
+// then a fixed xor shuffle tree, so every lane holds the same value), and
+// writes the BF16 output and each 1xG run's maximum.  The binary32
+// statistics (sums of a few thousand terms) and y carry an error of about
+// 1e-6 x (|y| + |mean| / std), so the BF16 output is the correctly rounded
+// norm except within that distance of a rounding midpoint.
+
+struct NormParams {
+  const uint16_t *x;
+  uint16_t *out;
+  float *group_amax;     // [rows * cols / G]
+  const float *weight;   // nullable, [cols]
+  const float *bias;     // nullable, [cols] (LayerNorm)
+  int64_t rows, cols;
+  int log2G;
+  int rms;
+  float eps;
+};
+
+constexpr int kNormMaxCols = 16384;
+
+// Rows of a block: up to kWarps, fewer for long rows so that the staged rows
+// fit 96 KB of shared memory.
+inline int norm_rows_per_block(int64_t cols) {
+  const int64_t fit = (96 * 1024) / (2 * cols);
+  return static_cast<int>(fit < 1 ? 1 : (fit > kWarps ? kWarps : fit));
+}
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormParams p) {
+  extern __shared__ uint4 norm_rows[];
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  if (row >= p.rows) return;   // the whole warp: only warp-level sync below
+  const int nq = static_cast<int>(p.cols >> 3);    // 16-byte chunks of the row
+  uint4 *rs = norm_rows + static_cast<int64_t>(warp) * nq;
+  const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.cols);
+  for (int q = lane; q < nq; q += 32) rs[q] = src[q];
+  __syncwarp();
+
+  const float inv_n = 1.0f / static_cast<float>(p.cols);
+  float acc = 0.0f;
+  for (int q = lane; q < nq; q += 32) {
+    const uint4 c = rs[q];
+    const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = bf16lo_to_float(wv[i]), b = bf16hi_to_float(wv[i]);
+      acc += p.rms ? a * a + b * b : a + b;
+    }
+  }
+  const float s1 = warp_sum_f(acc);
+  float mean = 0.0f, var;
+  if (p.rms) {
+    var = s1 * inv_n;
+  } else {
+    mean = s1 * inv_n;
+    float ss = 0.0f;
+    for (int q = lane; q < nq; q += 32) {
+      const uint4 c = rs[q];
+      const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float a = bf16lo_to_float(wv[i]) - mean, b = bf16hi_to_float(wv[i]) - mean;
+        ss += a * a + b * b;
+      }
+    }
+    var = warp_sum_f(ss) * inv_n;
+  }
+  const float rstd = 1.0f / sqrtf(var + p.eps);
+
+  // output: lane handles 16-element vectors j = lane + 32 v
+  const int nv = static_cast<int>(p.cols >> 4);
+  const int lanes = 1 << (p.log2G - 4);
+  const int64_t groups_per_row = p.cols >> p.log2G;
+  float run = 0.0f;   // running maximum of a group spanning several iterations
+  for (int v = 0; 32 * v < nv; ++v) {
+    const int j = lane + 32 * v;
+    const bool on = j < nv;
+    uint32_t ow[8];
+    float a = 0.0f;
+    if (on) {
+      const uint4 c0 = rs[2 * j], c1 = rs[2 * j + 1];
+      const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = 16 * j + 2 * i;
+        float y0 = (bf16lo_to_float(wv[i]) - mean) * rstd;
+        float y1 = (bf16hi_to_float(wv[i]) - mean) * rstd;
+        if (p.weight) {
+          y0 *= p.weight[c];
+          y1 *= p.weight[c + 1];
+        }
+        if (p.bias) {
+          y0 += p.bias[c];
+          y1 += p.bias[c + 1];
+        }
+        ow[i] = bf16x2_rn(y0, y1);
+        a = fmaxf(a, fmaxf(fabsf(bf16lo_to_float(ow[i])), fabsf(bf16hi_to_float(ow[i]))));
+      }
+      uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.cols + 16 * j);
+      dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      dst[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+    }
+    if (lanes <= 32) {
+      for (int off = 1; off < lanes; off <<= 1)
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      if (on && (lane & (lanes - 1)) == 0)
+        p.group_amax[row * groups_per_row + ((16 * j) >> p.log2G)] = a;
+    } else {
+      a = fmaxf(a, 0.0f);
+      for (int off = 1; off < 32; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      run = fmaxf(run, a);
+      if (((32 * (v + 1)) & (lanes - 1)) == 0) {   // the group's last iteration
+        if (lane == 0) p.group_amax[row * groups_per_row + ((16 * 32 * v) >> p.log2G)] = run;
+        run = 0.0f;
+      }
+    }
+  }
+}
+
 // ---- the FP8 cast alone -------------------------------------------------------------
 // code = RNE_satfinite(y): round to nearest even, finite values beyond the
 // format's largest magnitude (and infinities) saturate to +-max, NaN gives a

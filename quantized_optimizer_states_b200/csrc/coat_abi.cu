@@ -82,11 +82,11 @@ unsigned int blocks_for(int64_t elems) {
 // the kernel may be scheduled while the kernel before it on `s` drains, and
 // it waits for that kernel (pdl_enter) before its first global access.
 template <class... KArgs, class... Args>
-void launch_act(void (*kernel)(KArgs...), unsigned int grid, size_t smem, cudaStream_t s,
-                Args... args) {
+void launch_act_threads(void (*kernel)(KArgs...), unsigned int grid, unsigned int threads,
+                        size_t smem, cudaStream_t s, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(coat::kThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -95,6 +95,12 @@ void launch_act(void (*kernel)(KArgs...), unsigned int grid, size_t smem, cudaSt
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaLaunchKernelEx(&cfg, kernel, args...);  // a failure is reported by launch_status()
+}
+
+template <class... KArgs, class... Args>
+void launch_act(void (*kernel)(KArgs...), unsigned int grid, size_t smem, cudaStream_t s,
+                Args... args) {
+  launch_act_threads(kernel, grid, coat::kThreads, smem, s, args...);
 }
 
 // Streamed launch (tiles through shared memory by bulk copies) over the whole
@@ -502,6 +508,54 @@ coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, i
   p.group_amax = group_amax;
   launch_act(coat::swiglu_group_amax_kernel, coat::act_blocks(n), 0,
              static_cast<cudaStream_t>(stream), p);
+  return launch_status();
+}
+
+coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols, int32_t rms,
+                                   float eps, const float *weight, const float *bias,
+                                   int32_t group_size, uint16_t *out, float *group_amax,
+                                   void *stream) {
+  NvtxRange nvtx_range("coat_norm_group_amax");
+  if (rows < 0 || cols < 1 || (rms != 0 && rms != 1) || !(eps >= 0.0f) || !std::isfinite(eps))
+    return COAT_ERR_INVALID_ARG;
+  if (rms && bias) return COAT_ERR_INVALID_ARG;
+  const int lg = group_log2(group_size);
+  if (lg < 0) return COAT_ERR_UNSUPPORTED;
+  if (cols % group_size != 0 || cols % 16 != 0) return COAT_ERR_INVALID_ARG;
+  if (cols > coat::kNormMaxCols || rows > 0x7fffffff) return COAT_ERR_UNSUPPORTED;
+  if (rows == 0) return COAT_OK;
+  if (!x || !out || !group_amax) return COAT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out) || (reinterpret_cast<uintptr_t>(group_amax) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(weight) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(bias) & 3u) != 0)
+    return COAT_ERR_MISALIGNED;
+  coat::NormParams p;
+  p.x = x;
+  p.out = out;
+  p.group_amax = group_amax;
+  p.weight = weight;
+  p.bias = bias;
+  p.rows = rows;
+  p.cols = cols;
+  p.log2G = lg;
+  p.rms = rms;
+  p.eps = eps;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // one warp per row, rows_pb rows per block, each staging its row in
+  // shared memory
+  const int rows_pb = coat::norm_rows_per_block(cols);
+  const size_t smem = static_cast<size_t>(rows_pb) * static_cast<size_t>(cols) * 2;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(coat::norm_group_amax_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) {
+      g_last_cuda_error = static_cast<int32_t>(e);
+      return COAT_ERR_CUDA;
+    }
+  }
+  const unsigned int grid = static_cast<unsigned int>((rows + rows_pb - 1) / rows_pb);
+  launch_act_threads(coat::norm_group_amax_kernel, grid, 32u * rows_pb, smem, s, p);
   return launch_status();
 }
 

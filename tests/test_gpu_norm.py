@@ -1,0 +1,119 @@
+"""GPU parity of the LayerNorm / RMSNorm producer with fused 1xG maxima
+(coat_norm_group_amax) against the oracle: the BF16 output equals the
+binary64 norm rounded once, except one BF16 step apart where the binary64
+value lies within the binary32 evaluation's error (4e-6 relative) of a
+rounding midpoint, for at most 1e-3 of the elements; the maxima are those
+of the output; Group Scaling with the producer's maxima equals Group
+Scaling on its own."""
+import numpy as np
+import pytest
+
+import parity
+from quantized_optimizer_states_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+E4M3 = 0
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from quantized_optimizer_states_b200 import build
+    build.build()
+    import quantized_optimizer_states_b200 as q
+    q.load()
+    return q
+
+
+WINDOW = 4e-6          # relative error of the binary32 evaluation, with margin
+MAX_FLIPS = 1e-3       # fraction of elements allowed one BF16 step off
+
+
+def _midpoint_ok(orc, y64, got_bits, want_bits, offset):
+    """Every difference is one BF16 step, next to a rounding midpoint: within
+    WINDOW x (|midpoint| + offset), offset = |mean| / std of the element's
+    row scaled like y (x - mean loses the binary32 rounding of the mean)."""
+    bad = np.nonzero(got_bits != want_bits)[0]
+    assert bad.size <= MAX_FLIPS * got_bits.size, bad.size
+    for i in bad:
+        a = orc.bf16_bits_to_f64(np.array([got_bits[i]]))[0]
+        b = orc.bf16_bits_to_f64(np.array([want_bits[i]]))[0]
+        assert abs(int(got_bits[i]) - int(want_bits[i])) == 1, i
+        mid = 0.5 * (a + b)
+        assert abs(y64[i] - mid) <= WINDOW * (abs(mid) + offset[i]), i
+    return bad.size
+
+
+@pytest.mark.parametrize("rows,cols,G", [(64, 2048, 128), (24, 4096, 128), (8, 16384, 4096),
+                                         (40, 768, 256), (16, 5120, 512)])
+@pytest.mark.parametrize("rms", [False, True])
+def test_norm_matches_oracle(lib, orc, rows, cols, G, rms):
+    import torch
+    w = inputs.activations(seed=rows + cols)
+    x = inputs.host_activations(w, rows=rows)
+    x = np.tile(x, (1, -(-cols // x.shape[1])))[:, :cols].copy()
+    x[0, :] = x[0, 0]                          # a constant row
+    rng = np.random.default_rng(cols)
+    weight = (1.0 + 0.1 * rng.standard_normal(cols)).astype(np.float32)
+    bias = None if rms else (0.05 * rng.standard_normal(cols)).astype(np.float32)
+    out = torch.empty(rows, cols, dtype=torch.int16, device="cuda")
+    ga = torch.empty(rows * cols // G, dtype=torch.float32, device="cuda")
+    lib.coat_norm_group_amax(parity.to_dev(x.view(np.int16)), out, ga, rms=rms, eps=1e-5,
+                             weight=parity.to_dev(weight),
+                             bias=None if bias is None else parity.to_dev(bias), group_size=G)
+    torch.cuda.synchronize()
+    got = parity.to_host(out).view(np.uint16).reshape(-1)
+    y64 = orc.norm_f64(x, rms=rms, eps=1e-5, weight=weight, bias=bias).reshape(-1)
+    want = orc.round_to_bf16(y64)
+    xf = orc.bf16_bits_to_f64(x)
+    if rms:
+        offset = np.zeros(x.size)
+    else:
+        mu = xf.mean(axis=1, keepdims=True)
+        sd = np.sqrt(((xf - mu) ** 2).mean(axis=1, keepdims=True) + float(np.float32(1e-5)))
+        offset = np.broadcast_to(np.abs(mu) / sd * np.abs(weight), x.shape).reshape(-1)
+    _midpoint_ok(orc, y64, got, want, offset)
+    assert np.array_equal(parity.to_host(ga), orc.group_amax_of(got, G))
+
+
+def test_norm_feeds_group_scaling(lib, orc):
+    """The producer's maxima make Group Scaling skip its first step with
+    the same codes and scale as the standalone quantizer."""
+    import torch
+    rows, cols, G = 128, 2048, 128
+    x = inputs.host_activations(inputs.activations(seed=3), rows=rows)
+    out = torch.empty(rows, cols, dtype=torch.int16, device="cuda")
+    n = rows * cols
+    ws = torch.empty(lib.coat_group_scaling_workspace_bytes(n, G) // 4, dtype=torch.float32,
+                     device="cuda")
+    lib.coat_norm_group_amax(parity.to_dev(x.view(np.int16)), out, ws[:n // G], group_size=G)
+    q1 = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s1 = torch.empty(1, dtype=torch.float32, device="cuda")
+    lib.coat_group_scaling_quant_pertensor(out.reshape(-1), ws, q1, s1, group_size=G,
+                                           amax_precomputed=True)
+    q2 = torch.empty_like(q1)
+    s2 = torch.empty_like(s1)
+    ws2 = torch.empty_like(ws)
+    lib.coat_group_scaling_quant_pertensor(out.reshape(-1), ws2, q2, s2, group_size=G)
+    torch.cuda.synchronize()
+    assert torch.equal(q1, q2) and torch.equal(s1, s2)
+    q_ref, s_ref, _ = orc.group_scaling_pertensor(parity.to_host(out).view(np.uint16), G, E4M3)
+    assert np.array_equal(parity.to_host(q1), q_ref) and float(s1.item()) == s_ref
+
+
+def test_norm_argument_errors(lib):
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.int16, device="cuda")
+    ga = torch.zeros(4, dtype=torch.float32, device="cuda")
+    b = torch.zeros(128, dtype=torch.float32, device="cuda")
+    with pytest.raises(lib.CoatError) as e:
+        lib.coat_norm_group_amax(x, x.clone(), ga, rms=True, bias=b)   # bias with RMSNorm
+    assert e.value.status == 1
+    with pytest.raises(lib.CoatError) as e:
+        lib.coat_norm_group_amax(x, x.clone(), ga, eps=-1.0)
+    assert e.value.status == 1
+    with pytest.raises(lib.CoatError) as e:
+        lib.coat_norm_group_amax(x, x.clone(), ga, group_size=96)
+    assert e.value.status == 3

@@ -403,10 +403,11 @@ __global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const Swigl
 //   LayerNorm  y = (x - mean) / sqrt(var + eps)   (var: mean of squared deviations)
 //   RMSNorm    y = x / sqrt(mean(x^2) + eps)
 // then y * weight[c] (+ bias[c] for LayerNorm) when given, rounded to BF16.
-// One warp per row: the warp stages its row in shared memory (coalesced
-// 16-byte loads), takes the row sums over it in binary32 (per-lane sums,
-// then a fixed xor shuffle tree, so every lane holds the same value), and
-// writes the BF16 output and each 1xG run's maximum.  The binary32
+// One warp per row: the warp stages its row in shared memory (16-byte
+// asynchronous copies, the next row's issued before the current one is
+// computed), takes the row sums over it in binary32 (per-lane sums, then a
+// fixed xor shuffle tree, so every lane holds the same value), and writes
+// the BF16 output and each 1xG run's maximum.  The binary32
 // statistics (sums of a few thousand terms) and y carry an error of about
 // 1e-6 x (|y| + |mean| / std), so the BF16 output is the correctly rounded
 // norm except within that distance of a rounding midpoint.
@@ -425,10 +426,10 @@ struct NormParams {
 
 constexpr int kNormMaxCols = 16384;
 
-// Rows of a block: up to kWarps, fewer for long rows so that the staged rows
-// fit 96 KB of shared memory.
-inline int norm_rows_per_block(int64_t cols) {
-  const int64_t fit = (96 * 1024) / (2 * cols);
+// Warps (rows in flight) of a block: up to kWarps, fewer for long rows so
+// that the two staged rows of every warp fit 96 KB of shared memory.
+inline int norm_warps_per_block(int64_t cols) {
+  const int64_t fit = (96 * 1024) / (2 * 2 * cols);
   return static_cast<int>(fit < 1 ? 1 : (fit > kWarps ? kWarps : fit));
 }
 
@@ -437,19 +438,22 @@ __device__ __forceinline__ float warp_sum_f(float v) {
   return v;
 }
 
-__global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormParams p) {
-  extern __shared__ uint4 norm_rows[];
-  pdl_enter();
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
-  if (row >= p.rows) return;   // the whole warp: only warp-level sync below
-  const int nq = static_cast<int>(p.cols >> 3);    // 16-byte chunks of the row
-  uint4 *rs = norm_rows + static_cast<int64_t>(warp) * nq;
+// Issue the 16-byte asynchronous copies of one row into shared memory (one
+// commit group per row).
+__device__ __forceinline__ void norm_prefetch_row(const NormParams &p, uint4 *dst, int64_t row,
+                                                  int nq, int lane) {
   const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.cols);
-  for (int q = lane; q < nq; q += 32) rs[q] = src[q];
-  __syncwarp();
+  for (int q = lane; q < nq; q += 32) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst + q));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + q) : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
 
+// One row from its staged copy rs: statistics, output, 1xG maxima.
+__device__ __forceinline__ void norm_one_row(const NormParams &p, const uint4 *rs, int64_t row,
+                                             int lane) {
+  const int nq = static_cast<int>(p.cols >> 3);
   const float inv_n = 1.0f / static_cast<float>(p.cols);
   float acc = 0.0f;
   for (int q = lane; q < nq; q += 32) {
@@ -520,7 +524,6 @@ __global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormPar
       if (on && (lane & (lanes - 1)) == 0)
         p.group_amax[row * groups_per_row + ((16 * j) >> p.log2G)] = a;
     } else {
-      a = fmaxf(a, 0.0f);
       for (int off = 1; off < 32; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
       run = fmaxf(run, a);
       if (((32 * (v + 1)) & (lanes - 1)) == 0) {   // the group's last iteration
@@ -528,6 +531,33 @@ __global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormPar
         run = 0.0f;
       }
     }
+  }
+}
+
+// Persistent warps: warp w of the grid takes rows w, w + W, w + 2W, ... (W
+// the grid's warps), staging each row in one of its two shared-memory
+// buffers while the previous row is computed.
+__global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormParams p) {
+  extern __shared__ uint4 norm_rows[];
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nq = static_cast<int>(p.cols >> 3);    // 16-byte chunks of a row
+  uint4 *buf = norm_rows + static_cast<int64_t>(warp) * 2 * nq;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  if (row >= p.rows) return;   // the whole warp: only warp-level sync below
+  norm_prefetch_row(p, buf, row, nq, lane);
+  for (int it = 0; row < p.rows; ++it, row += step) {
+    const bool more = row + step < p.rows;
+    if (more) norm_prefetch_row(p, buf + ((it + 1) & 1) * nq, row + step, nq, lane);
+    if (more)
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncwarp();   // every lane's copies of this row have landed
+    norm_one_row(p, buf + (it & 1) * nq, row, lane);
+    __syncwarp();   // every lane is done with the buffer the next prefetch reuses
   }
 }
 

@@ -541,10 +541,9 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
   p.rms = rms;
   p.eps = eps;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // one warp per row, rows_pb rows per block, each staging its row in
-  // shared memory
-  const int rows_pb = coat::norm_rows_per_block(cols);
-  const size_t smem = static_cast<size_t>(rows_pb) * static_cast<size_t>(cols) * 2;
+  // persistent warps, each staging two rows in shared memory
+  const int wpb = coat::norm_warps_per_block(cols);
+  const size_t smem = static_cast<size_t>(wpb) * 2 * static_cast<size_t>(cols) * 2;
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(coat::norm_group_amax_kernel,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -554,8 +553,18 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
       return COAT_ERR_CUDA;
     }
   }
-  const unsigned int grid = static_cast<unsigned int>((rows + rows_pb - 1) / rows_pb);
-  launch_act_threads(coat::norm_group_amax_kernel, grid, 32u * rows_pb, smem, s, p);
+  int dev = 0, sms = 1, per_sm = 1;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, coat::norm_group_amax_kernel,
+                                                    32 * wpb, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t blocks_needed = (rows + wpb - 1) / wpb;
+  const int64_t resident = static_cast<int64_t>(sms) * per_sm;
+  const unsigned int grid =
+      static_cast<unsigned int>(blocks_needed < resident ? blocks_needed : resident);
+  launch_act_threads(coat::norm_group_amax_kernel, grid, 32u * wpb, smem, s, p);
   return launch_status();
 }
 

@@ -249,7 +249,8 @@ def run_activations(args):
             "ln": torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=dev),
             "out": torch.empty(n, dtype=torch.float32, device=dev)})
     for b in ring:  # the producer's outputs that the after-producer case reads
-        coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"], group_size=G)
+        coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"], group_size=G,
+                                    tensor_amax=b["ws_h"][ng:])
     cases = {
         # name: (callable on one ring slot, algorithmic bytes per element)
         "group_quant_1xG": (lambda b: coat.coat_group_quant_1xG(b["x"], b["q"], b["sc"],
@@ -261,7 +262,7 @@ def run_activations(args):
             2 + 2 + 1 + 8.0 / G),
         "swiglu_fused_amax": (
             lambda b: coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"],
-                                                  group_size=G),
+                                                  group_size=G, tensor_amax=b["ws_h"][ng:]),
             2 + 2 + 2 + 4.0 / G),
         "layernorm_fused_amax": (
             lambda b: coat.coat_norm_group_amax(b["x"], b["ln"], b["ws"], group_size=G),
@@ -269,8 +270,13 @@ def run_activations(args):
         "group_scaling_after_producer": (
             lambda b: coat.coat_group_scaling_quant_pertensor(b["h"], b["ws_h"], b["q"], b["s1"],
                                                               group_size=G,
-                                                              amax_precomputed=True),
+                                                              amax_precomputed=1),
             2 + 1 + 4.0 / G),
+        "group_scaling_after_producer_with_tensor_max": (
+            lambda b: coat.coat_group_scaling_quant_pertensor(b["h"], b["ws_h"], b["q"], b["s1"],
+                                                              group_size=G,
+                                                              amax_precomputed=2),
+            2 + 1),
         "dequant_pertensor": (
             lambda b: coat.coat_dequant(b["q"], None, b["s1"], b["out"], group_size=n), 1 + 4),
     }
@@ -310,7 +316,7 @@ def run_activations(args):
                          "frac": head["frac_of_hbm"], "traffic": recorded_act_traffic(n),
                          "peak_source": f"{peak_kind} copy bandwidth"},
             "kernels": res, "clocks": clocks,
-            "gpu_launches": args.steps * (1 + 2 + 1 + 1 + 2 + 1)}
+            "gpu_launches": args.steps * (1 + 2 + 1 + 1 + 2 + 1 + 1)}
     print(json.dumps(line), flush=True)
     return 0
 

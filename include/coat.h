@@ -237,8 +237,11 @@ int64_t coat_group_scaling_workspace_bytes(int64_t n, int32_t group_size);
  *   workspace  float32[ceil(n/G) + 1] (4-byte aligned).  Slots
  *              [0, ceil(n/G)) hold the per-group maxima: written by step (i)
  *              when amax_precomputed == 0, or filled beforehand by the
- *              producing kernel when amax_precomputed != 0 (step (i) is then
- *              skipped).  The last slot is scratch for step (ii).
+ *              producing kernel when amax_precomputed == 1 (step (i) is then
+ *              skipped).  The last slot holds the tensor maximum of step
+ *              (ii); amax_precomputed == 2: the producer also wrote that
+ *              slot (its tensor_amax output), and only the cast runs.
+ *              Other amax_precomputed values: INVALID_ARG.
  *   q          uint8[n] codes (16-byte aligned)
  *   scale      float32[1], the per-tensor scale s (amax <= 2^-100 gives 1)
  * Bit-exact: amax is an exact max and s, the reciprocal and the product
@@ -315,11 +318,16 @@ coat_status_t coat_fp8_encode(const float *y, int64_t n, int32_t fmt, uint8_t *q
  *               1xG run of the flat output (the last run may be shorter) --
  *               exactly the slots coat_group_scaling_quant_pertensor reads
  *               when called on `out` with amax_precomputed != 0
+ *   tensor_amax float32[1] or NULL (4-byte aligned): when given, zeroed and
+ *               then set to max |out| over the whole output (step (ii),
+ *               folded into the producer with one atomic max per block):
+ *               pass workspace + ceil(n/G) and call Group Scaling with
+ *               amax_precomputed == 2 to run the cast alone.
  * Errors: INVALID_ARG, UNSUPPORTED (group size), MISALIGNED, CUDA.
  */
 coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, int64_t n,
                                      int32_t group_size, uint16_t *out, float *group_amax,
-                                     void *stream);
+                                     float *tensor_amax, void *stream);
 
 /*
  * coat_pack_bf16 -- gather `count` tensors into one flat BF16 buffer with
@@ -415,13 +423,14 @@ coat_status_t coat_state_stats(const uint8_t *code, const float *k, const float 
  *   group_amax  float32 [rows * cols / G]: the slots
  *               coat_group_scaling_quant_pertensor reads on `out` (flat,
  *               the same G) with amax_precomputed != 0
+ *   tensor_amax float32[1] or NULL: as for coat_swiglu_group_amax
  * Errors: INVALID_ARG (sizes, eps < 0 or not finite, rms not 0/1, bias with
  * rms), UNSUPPORTED (G, cols > 16384), MISALIGNED, CUDA.
  */
 coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols, int32_t rms,
                                    float eps, const float *weight, const float *bias,
                                    int32_t group_size, uint16_t *out, float *group_amax,
-                                   void *stream);
+                                   float *tensor_amax, void *stream);
 
 /* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
  * this thread (0 if none). */

@@ -64,9 +64,9 @@ SIGNATURES = {
     "coat_group_scaling_workspace_bytes": (_I64, [_I64, _I32]),
     "coat_group_scaling_quant_pertensor": (_I32, [_P, _I64, _I32, _I32, _P, _I32, _P, _P, _P]),
     "coat_group_scaling_quant_pertensor_noalloc": (_I32, [_P, _I64, _I32, _I32, _P, _P, _P]),
-    "coat_swiglu_group_amax": (_I32, [_P, _P, _I64, _I32, _P, _P, _P]),
+    "coat_swiglu_group_amax": (_I32, [_P, _P, _I64, _I32, _P, _P, _P, _P]),
     "coat_fp8_encode": (_I32, [_P, _I64, _I32, _P, _P]),
-    "coat_norm_group_amax": (_I32, [_P, _I64, _I64, _I32, _F, _P, _P, _I32, _P, _P, _P]),
+    "coat_norm_group_amax": (_I32, [_P, _I64, _I64, _I32, _F, _P, _P, _I32, _P, _P, _P, _P]),
     "coat_count_nonfinite_bf16": (_I32, [_P, _I64, _P, _P]),
     "coat_adamw_fp8_step_guarded": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
                                            ctypes.POINTER(CoatAdamwCfg), _P, _P]),
@@ -122,6 +122,16 @@ def _ptr(t, dtype=None, what="tensor"):
         raise ValueError(f"{what} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _slot(t):
+    """An optional float32 device slot (e.g. a one-element view of a workspace)."""
+    if t is None:
+        return None
+    import torch
+    if t.dtype != torch.float32 or not t.is_cuda or t.numel() < 1:
+        raise ValueError("tensor_amax must be a float32 CUDA tensor of at least one element")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -234,16 +244,19 @@ def coat_group_scaling_workspace_bytes(n: int, group_size: int) -> int:
 
 
 def coat_group_scaling_quant_pertensor(x, workspace, q, scale, *, group_size: int = 128,
-                                       fmt: int = COAT_E4M3, amax_precomputed: bool = False,
+                                       fmt: int = COAT_E4M3, amax_precomputed: int = 0,
                                        stream=None):
-    """x: BF16 [n]; workspace: float32 [ceil(n/G) + 1]; q: uint8 [n]; scale: float32 [1]."""
+    """x: BF16 [n]; workspace: float32 [ceil(n/G) + 1]; q: uint8 [n]; scale:
+    float32 [1].  amax_precomputed: 0 (steps (i)-(iii)), 1 (the producer
+    wrote the group maxima) or 2 (it also wrote the tensor maximum into the
+    last workspace slot: the cast alone); True counts as 1."""
     import torch
     need = coat_group_scaling_workspace_bytes(x.numel(), group_size)
     if workspace.numel() * workspace.element_size() < need:
         raise ValueError(f"workspace needs {need} bytes")
     st = load().coat_group_scaling_quant_pertensor(
         _u16(x, "x"), x.numel(), group_size, fmt, _ptr(workspace, torch.float32, "workspace"),
-        int(bool(amax_precomputed)), _ptr(q, torch.uint8, "q"),
+        int(amax_precomputed), _ptr(q, torch.uint8, "q"),
         _ptr(scale, torch.float32, "scale"), _stream(stream))
     _check("coat_group_scaling_quant_pertensor", st)
 
@@ -262,9 +275,12 @@ def coat_group_scaling_quant_pertensor_noalloc(x, q, scale, *, group_size: int =
     _check("coat_group_scaling_quant_pertensor_noalloc", st)
 
 
-def coat_swiglu_group_amax(gate, up, out, group_amax, *, group_size: int = 128, stream=None):
+def coat_swiglu_group_amax(gate, up, out, group_amax, *, group_size: int = 128,
+                           tensor_amax=None, stream=None):
     """out = RN_bf16(silu(gate) * up) and the per-1xG maxima of out, ready
-    for coat_group_scaling_quant_pertensor(..., amax_precomputed=True)."""
+    for coat_group_scaling_quant_pertensor(..., amax_precomputed=1); with
+    tensor_amax (a float32 slot, e.g. workspace[ceil(n/G):]) also the maximum
+    of all of out, for amax_precomputed=2."""
     import torch
     if gate.numel() != up.numel() or out.numel() != gate.numel():
         raise ValueError("gate, up and out must have the same number of elements")
@@ -273,12 +289,13 @@ def coat_swiglu_group_amax(gate, up, out, group_amax, *, group_size: int = 128, 
         raise ValueError(f"group_amax needs {ng} float32 slots")
     st = load().coat_swiglu_group_amax(
         _u16(gate, "gate"), _u16(up, "up"), gate.numel(), group_size, _u16(out, "out"),
-        _ptr(group_amax, torch.float32, "group_amax"), _stream(stream))
+        _ptr(group_amax, torch.float32, "group_amax"), _slot(tensor_amax), _stream(stream))
     _check("coat_swiglu_group_amax", st)
 
 
 def coat_norm_group_amax(x, out, group_amax, *, rms: bool = False, eps: float = 1e-5,
-                         weight=None, bias=None, group_size: int = 128, stream=None):
+                         weight=None, bias=None, group_size: int = 128, tensor_amax=None,
+                         stream=None):
     """LayerNorm (or RMSNorm) of BF16 rows x [rows, cols] into BF16 `out` with
     the maxima of every 1xG run of the output in `group_amax` (see
     include/coat.h)."""
@@ -294,7 +311,7 @@ def coat_norm_group_amax(x, out, group_amax, *, rms: bool = False, eps: float = 
     _check("coat_norm_group_amax", load().coat_norm_group_amax(
         _u16(x, "x"), rows, cols, int(rms), float(eps), _ptr(weight, torch.float32, "weight"),
         _ptr(bias, torch.float32, "bias"), group_size, _u16(out, "out"),
-        _ptr(group_amax, torch.float32, "group_amax"), _stream(stream)))
+        _ptr(group_amax, torch.float32, "group_amax"), _slot(tensor_amax), _stream(stream)))
 
 
 def coat_fp8_encode(y, q, *, fmt: int = COAT_E4M3, stream=None):

@@ -78,6 +78,30 @@ __device__ __forceinline__ float group_max(float a, int lanes, float *red) {
   return a;
 }
 
+// Zeroes the tensor-maximum word a producer then accumulates into (a
+// kernel rather than a memset, so that it joins the programmatic
+// dependent launch chain of the kernels around it).
+__global__ void zero_word_kernel(uint32_t *w) {
+  pdl_enter();
+  if (threadIdx.x == 0) *w = 0u;
+}
+
+// Group Scaling's step (ii) folded into a producer: the maximum of the
+// block's group maxima (non-negative, so their bits order as unsigned
+// integers) joins the tensor maximum with one atomic per block.  Every
+// thread of the block calls it.
+__device__ __forceinline__ void block_max_to_tensor(float m, uint32_t *tensor_amax) {
+  __shared__ float bred[kWarps];
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) bred[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = bred[0];
+    for (int i = 1; i < static_cast<int>(blockDim.x >> 5); ++i) t = fmaxf(t, bred[i]);
+    atomicMax(tensor_amax, __float_as_uint(t));
+  }
+}
+
 template <int F>
 __device__ __forceinline__ void cast16(const float *x, float inv, uint32_t *out) {
 #pragma unroll
@@ -343,13 +367,15 @@ struct SwigluParams {
   int64_t n;
   int log2G;
   uint16_t *out;
-  float *group_amax;  // [ceil(n / G)]
+  float *group_amax;     // [ceil(n / G)]
+  uint32_t *tensor_amax; // nullable: also the maximum of all outputs (bits, zeroed first)
 };
 
 __global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const SwigluParams p) {
   __shared__ float red[kActV][kWarps];
   pdl_enter();
   const int lanes = 1 << (p.log2G - 4);
+  float tmax = 0.0f;
   uint32_t gw[kActV][8], uw[kActV][8];
   int64_t e0[kActV];
 #pragma unroll
@@ -381,6 +407,7 @@ __global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const Swigl
       h[2 * i + 1] = bf16hi_to_float(ow[i]);
     }
     const float gmax = group_max(amax16(h), lanes, red[v]);
+    tmax = fmaxf(tmax, gmax);
     if (e0[v] >= p.n) continue;
     if (e0[v] + 16 <= p.n) {
       uint4 *dst = reinterpret_cast<uint4 *>(p.out + e0[v]);
@@ -392,6 +419,7 @@ __global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const Swigl
     }
     if ((threadIdx.x & (lanes - 1)) == 0) p.group_amax[e0[v] >> p.log2G] = gmax;
   }
+  if (p.tensor_amax) block_max_to_tensor(tmax, p.tensor_amax);
 }
 
 // ---- a second producer with the maxima fused in: LayerNorm / RMSNorm ---------------------
@@ -422,6 +450,7 @@ struct NormParams {
   int log2G;
   int rms;
   float eps;
+  uint32_t *tensor_amax; // nullable: also the maximum of all outputs (bits, zeroed first)
 };
 
 constexpr int kNormMaxCols = 16384;
@@ -438,6 +467,11 @@ __device__ __forceinline__ float warp_sum_f(float v) {
   return v;
 }
 
+__device__ __forceinline__ float warp_max_f(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
 // Issue the 16-byte asynchronous copies of one row into shared memory (one
 // commit group per row).
 __device__ __forceinline__ void norm_prefetch_row(const NormParams &p, uint4 *dst, int64_t row,
@@ -450,9 +484,10 @@ __device__ __forceinline__ void norm_prefetch_row(const NormParams &p, uint4 *ds
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// One row from its staged copy rs: statistics, output, 1xG maxima.
-__device__ __forceinline__ void norm_one_row(const NormParams &p, const uint4 *rs, int64_t row,
-                                             int lane) {
+// One row from its staged copy rs: statistics, output, 1xG maxima; returns
+// the row's maximum |output| (in every lane).
+__device__ __forceinline__ float norm_one_row(const NormParams &p, const uint4 *rs, int64_t row,
+                                              int lane) {
   const int nq = static_cast<int>(p.cols >> 3);
   const float inv_n = 1.0f / static_cast<float>(p.cols);
   float acc = 0.0f;
@@ -490,6 +525,7 @@ __device__ __forceinline__ void norm_one_row(const NormParams &p, const uint4 *r
   const int lanes = 1 << (p.log2G - 4);
   const int64_t groups_per_row = p.cols >> p.log2G;
   float run = 0.0f;   // running maximum of a group spanning several iterations
+  float rowmax = 0.0f;
   for (int v = 0; 32 * v < nv; ++v) {
     const int j = lane + 32 * v;
     const bool on = j < nv;
@@ -518,6 +554,7 @@ __device__ __forceinline__ void norm_one_row(const NormParams &p, const uint4 *r
       dst[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
       dst[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
     }
+    rowmax = fmaxf(rowmax, a);
     if (lanes <= 32) {
       for (int off = 1; off < lanes; off <<= 1)
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
@@ -532,6 +569,7 @@ __device__ __forceinline__ void norm_one_row(const NormParams &p, const uint4 *r
       }
     }
   }
+  return warp_max_f(rowmax);
 }
 
 // Persistent warps: warp w of the grid takes rows w, w + W, w + 2W, ... (W
@@ -546,19 +584,22 @@ __global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormPar
   uint4 *buf = norm_rows + static_cast<int64_t>(warp) * 2 * nq;
   const int64_t step = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
-  if (row >= p.rows) return;   // the whole warp: only warp-level sync below
-  norm_prefetch_row(p, buf, row, nq, lane);
-  for (int it = 0; row < p.rows; ++it, row += step) {
-    const bool more = row + step < p.rows;
-    if (more) norm_prefetch_row(p, buf + ((it + 1) & 1) * nq, row + step, nq, lane);
-    if (more)
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    else
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncwarp();   // every lane's copies of this row have landed
-    norm_one_row(p, buf + (it & 1) * nq, row, lane);
-    __syncwarp();   // every lane is done with the buffer the next prefetch reuses
+  float wmax = 0.0f;
+  if (row < p.rows) {   // warp-uniform; a warp without rows only joins the block max
+    norm_prefetch_row(p, buf, row, nq, lane);
+    for (int it = 0; row < p.rows; ++it, row += step) {
+      const bool more = row + step < p.rows;
+      if (more) norm_prefetch_row(p, buf + ((it + 1) & 1) * nq, row + step, nq, lane);
+      if (more)
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncwarp();   // every lane's copies of this row have landed
+      wmax = fmaxf(wmax, norm_one_row(p, buf + (it & 1) * nq, row, lane));
+      __syncwarp();   // every lane is done with the buffer the next prefetch reuses
+    }
   }
+  if (p.tensor_amax) block_max_to_tensor(wmax, p.tensor_amax);
 }
 
 // ---- the FP8 cast alone -------------------------------------------------------------

@@ -456,7 +456,7 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
                                                  float *workspace, int32_t amax_precomputed,
                                                  uint8_t *q, float *scale, void *stream) {
   NvtxRange nvtx_range("coat_group_scaling_quant_pertensor");
-  if (n < 0) return COAT_ERR_INVALID_ARG;
+  if (n < 0 || amax_precomputed < 0 || amax_precomputed > 2) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!x || !workspace || !q || !scale)) return COAT_ERR_INVALID_ARG;
   const int lg = group_log2(group_size);
   if (lg < 0 || !valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
@@ -474,6 +474,11 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
   p.q = q;
   p.scale = scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (amax_precomputed == 2) {
+    // the producer also folded its maxima into workspace[ng]: the cast alone
+    launch_pertensor_cast(p, fmt, s);
+    return launch_status();
+  }
   if (cudaMemsetAsync(p.tensor_amax, 0, sizeof(uint32_t), s) != cudaSuccess) return launch_status();
   if (amax_precomputed) {
     // one pass over the small intermediate: a few blocks per SM suffice
@@ -489,7 +494,7 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
 
 coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, int64_t n,
                                      int32_t group_size, uint16_t *out, float *group_amax,
-                                     void *stream) {
+                                     float *tensor_amax, void *stream) {
   NvtxRange nvtx_range("coat_swiglu_group_amax");
   if (n < 0) return COAT_ERR_INVALID_ARG;
   if (n > 0 && (!gate || !up || !out || !group_amax)) return COAT_ERR_INVALID_ARG;
@@ -497,8 +502,14 @@ coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, i
   if (lg < 0 || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
   if (n == 0) return COAT_OK;
   if (!aligned16(gate) || !aligned16(up) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(group_amax) & 3u) != 0)
+      (reinterpret_cast<uintptr_t>(group_amax) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(tensor_amax) & 3u) != 0)
     return COAT_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the producer's block maxima accumulate with atomicMax from zero
+  if (tensor_amax)
+    launch_act_threads(coat::zero_word_kernel, 1u, 32u, 0, s,
+                       reinterpret_cast<uint32_t *>(tensor_amax));
   coat::SwigluParams p;
   p.gate = gate;
   p.up = up;
@@ -506,15 +517,15 @@ coat_status_t coat_swiglu_group_amax(const uint16_t *gate, const uint16_t *up, i
   p.log2G = lg;
   p.out = out;
   p.group_amax = group_amax;
-  launch_act(coat::swiglu_group_amax_kernel, coat::act_blocks(n), 0,
-             static_cast<cudaStream_t>(stream), p);
+  p.tensor_amax = reinterpret_cast<uint32_t *>(tensor_amax);
+  launch_act(coat::swiglu_group_amax_kernel, coat::act_blocks(n), 0, s, p);
   return launch_status();
 }
 
 coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols, int32_t rms,
                                    float eps, const float *weight, const float *bias,
                                    int32_t group_size, uint16_t *out, float *group_amax,
-                                   void *stream) {
+                                   float *tensor_amax, void *stream) {
   NvtxRange nvtx_range("coat_norm_group_amax");
   if (rows < 0 || cols < 1 || (rms != 0 && rms != 1) || !(eps >= 0.0f) || !std::isfinite(eps))
     return COAT_ERR_INVALID_ARG;
@@ -527,7 +538,8 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
   if (!x || !out || !group_amax) return COAT_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out) || (reinterpret_cast<uintptr_t>(group_amax) & 3u) != 0 ||
       (reinterpret_cast<uintptr_t>(weight) & 3u) != 0 ||
-      (reinterpret_cast<uintptr_t>(bias) & 3u) != 0)
+      (reinterpret_cast<uintptr_t>(bias) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(tensor_amax) & 3u) != 0)
     return COAT_ERR_MISALIGNED;
   coat::NormParams p;
   p.x = x;
@@ -540,7 +552,11 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
   p.log2G = lg;
   p.rms = rms;
   p.eps = eps;
+  p.tensor_amax = reinterpret_cast<uint32_t *>(tensor_amax);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (tensor_amax)
+    launch_act_threads(coat::zero_word_kernel, 1u, 32u, 0, s,
+                       reinterpret_cast<uint32_t *>(tensor_amax));
   // persistent warps, each staging two rows in shared memory
   const int wpb = coat::norm_warps_per_block(cols);
   const size_t smem = static_cast<size_t>(wpb) * 2 * static_cast<size_t>(cols) * 2;

@@ -103,6 +103,36 @@ def test_norm_feeds_group_scaling(lib, orc):
     assert np.array_equal(parity.to_host(q1), q_ref) and float(s1.item()) == s_ref
 
 
+@pytest.mark.parametrize("rms", [False, True])
+def test_norm_tensor_max_feeds_the_cast_alone(lib, orc, rms):
+    """tensor_amax: the producer also writes the tensor maximum; Group
+    Scaling with amax_precomputed=2 then only casts, with the oracle's codes
+    and scale; amax_precomputed outside 0..2 is rejected."""
+    import torch
+    rows, cols, G = 300, 4096, 128
+    x = inputs.host_activations(inputs.activations(seed=8), rows=rows)
+    x = np.tile(x, (1, 2))[:, :cols].copy()
+    n = rows * cols
+    out = torch.empty(rows, cols, dtype=torch.int16, device="cuda")
+    ws = torch.full((lib.coat_group_scaling_workspace_bytes(n, G) // 4,), 3.0,
+                    dtype=torch.float32, device="cuda")
+    lib.coat_norm_group_amax(parity.to_dev(x.view(np.int16)), out, ws[:n // G], rms=rms,
+                             group_size=G, tensor_amax=ws[n // G:])
+    q = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    lib.coat_group_scaling_quant_pertensor(out.reshape(-1), ws, q, s, group_size=G,
+                                           amax_precomputed=2)
+    torch.cuda.synchronize()
+    h = parity.to_host(out).view(np.uint16)
+    q_ref, s_ref, ga_ref = orc.group_scaling_pertensor(h, G, E4M3)
+    assert float(ws[n // G].item()) == float(ga_ref.max())
+    assert np.array_equal(parity.to_host(q), q_ref) and float(s.item()) == s_ref
+    with pytest.raises(lib.CoatError) as e:
+        lib.coat_group_scaling_quant_pertensor(out.reshape(-1), ws, q, s, group_size=G,
+                                               amax_precomputed=3)
+    assert e.value.status == 1
+
+
 def test_norm_argument_errors(lib):
     import torch
     x = torch.zeros(4, 128, dtype=torch.int16, device="cuda")

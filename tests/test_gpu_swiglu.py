@@ -108,6 +108,32 @@ def test_fused_maxima_feed_group_scaling(lib):
     assert float(sc.item()) == s_ref
 
 
+@pytest.mark.parametrize("rows,G", [(32, 128), (17, 512)])
+def test_tensor_max_from_the_producer(lib, rows, G):
+    """With tensor_amax the producer also folds step (ii) in: Group Scaling
+    with amax_precomputed=2 runs the cast alone and gives the oracle's codes
+    and scale (ragged length: 17 rows minus 5 elements)."""
+    w = inputs.activations(seed=rows)
+    gate, up = inputs.host_swiglu_inputs(w, rows=rows)
+    n = gate.size - 5
+    gate, up = gate.reshape(-1)[:n].copy(), up.reshape(-1)[:n].copy()
+    out = torch.empty(n, dtype=torch.int16, device="cuda")
+    ws = torch.full((lib.coat_group_scaling_workspace_bytes(n, G) // 4,), 7.0,
+                    dtype=torch.float32, device="cuda")
+    ng = -(-n // G)
+    lib.coat_swiglu_group_amax(_dev(gate), _dev(up), out, ws, group_size=G,
+                               tensor_amax=ws[ng:])
+    q = torch.empty(n, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(1, dtype=torch.float32, device="cuda")
+    lib.coat_group_scaling_quant_pertensor(out, ws, q, sc, group_size=G, amax_precomputed=2)
+    torch.cuda.synchronize()
+    h = out.cpu().numpy().view(np.uint16)
+    q_ref, s_ref, ga_ref = oracle.group_scaling_pertensor(h, G, 0)
+    assert float(ws[ng].item()) == float(ga_ref.max())
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert float(sc.item()) == s_ref
+
+
 def test_argument_errors(lib):
     from quantized_optimizer_states_b200._lib import CoatError
     x = torch.zeros(256, dtype=torch.int16, device="cuda")

@@ -539,29 +539,31 @@ def main():
     # ---- end to end: gradients from pinned host memory each step ----------------
     e2e = None
     if args.e2e_steps > 0:
-        host_grad = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
-        host_grad.copy_(grad)
-        result = torch.empty(4, dtype=torch.float32, pin_memory=True)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-
         # The step's input (the BF16 gradients) streams in from pinned host
         # memory in group-aligned chunks on a copy stream; the step runs chunk
         # by chunk (the same public call on buffer slices) as soon as its
-        # gradients have arrived, so the transfer overlaps the kernel.
+        # gradients have arrived, so the transfer overlaps the kernel.  Every
+        # chunk crosses PCIe from one pinned staging buffer of chunk size
+        # (2n bytes per step, as with a full host copy, without pinning the
+        # whole gradient on every rank of a multi-GPU run).
         copy_stream = torch.cuda.Stream(device=dev)
         nchunks = 16
         per = -(-n // nchunks)
         per = -(-per // 4096) * 4096
         bounds = [(a, min(n, a + per)) for a in range(0, n, per)]
+        host_grad = torch.empty(per, dtype=torch.bfloat16, pin_memory=True)
+        host_grad.copy_(grad[:per])
+        result = torch.empty(4, dtype=torch.float32, pin_memory=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
 
         def e2e_step():
             t = step_no[0]
             done = []
             for a, b in bounds:
                 with torch.cuda.stream(copy_stream):
-                    grad[a:b].copy_(host_grad[a:b], non_blocking=True)
+                    grad[a:b].copy_(host_grad[:b - a], non_blocking=True)
                     ev = torch.cuda.Event()
                     ev.record(copy_stream)
                 done.append(ev)
@@ -595,9 +597,9 @@ def main():
         e2e = {"value": world * n * args.e2e_steps / (e2e_ms / 1e3), "unit": "params/s",
                "h2d_bytes_per_step": 2 * n, "d2h_bytes_per_step": 16,
                "what": "BF16 gradients copied from pinned host memory every step in 16 chunks "
-                       "on a copy stream, each chunk stepped as soon as it has arrived "
-                       "(coat_adamw_fp8_step on the slices), then a 16-byte read-back of the "
-                       "last group's (k, s) pairs"}
+                       "(from one chunk-sized pinned staging buffer) on a copy stream, each "
+                       "chunk stepped as soon as it has arrived (coat_adamw_fp8_step on the "
+                       "slices), then a 16-byte read-back of the last group's (k, s) pairs"}
         del host_grad
 
     cpu = None

@@ -316,7 +316,10 @@ def run_activations(args):
                          "frac": head["frac_of_hbm"], "traffic": recorded_act_traffic(n),
                          "peak_source": f"{peak_kind} copy bandwidth"},
             "kernels": res, "clocks": clocks,
-            "gpu_launches": args.steps * (1 + 2 + 1 + 1 + 2 + 1 + 1)}
+            # 1xG 1; GS standalone 2; SwiGLU 2 (zeroing the tensor-max slot, the
+            # producer); LayerNorm 1; GS after the producer 2 (step (ii), cast);
+            # the cast alone 1; dequant 1
+            "gpu_launches": args.steps * (1 + 2 + 2 + 1 + 2 + 1 + 1)}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -560,7 +560,9 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
   // persistent warps, each staging two rows in shared memory
   const int wpb = coat::norm_warps_per_block(cols);
   const size_t smem = static_cast<size_t>(wpb) * 2 * static_cast<size_t>(cols) * 2;
-  if (smem > 48 * 1024) {
+  {
+    // always: the kernel's static shared memory comes on top of smem, so
+    // even smem == 48 KB needs the opt-in
     const cudaError_t e = cudaFuncSetAttribute(coat::norm_group_amax_kernel,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));

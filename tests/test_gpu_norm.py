@@ -47,7 +47,7 @@ def _midpoint_ok(orc, y64, got_bits, want_bits, offset):
 
 
 @pytest.mark.parametrize("rows,cols,G", [(64, 2048, 128), (24, 4096, 128), (8, 16384, 4096),
-                                         (40, 768, 256), (16, 5120, 512)])
+                                         (40, 768, 256), (16, 5120, 512), (33, 1536, 128)])
 @pytest.mark.parametrize("rms", [False, True])
 def test_norm_matches_oracle(lib, orc, rows, cols, G, rms):
     import torch

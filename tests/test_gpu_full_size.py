@@ -109,14 +109,18 @@ def _check_every_group(st, G, v_fmt, chunk_groups=1 << 21):
         assert bool(torch.isfinite(st["theta"][off:off + chunk_groups * G]).all())
 
 
-@pytest.mark.parametrize("name,v_fmt", [("olmo-1b", E5M2), ("olmo-7b", E4M3), ("olmo-7b", E5M2)])
-def test_full_size_sampled_groups(lib, orc, name, v_fmt):
+@pytest.mark.parametrize("name,v_fmt,f32_grads", [("olmo-1b", E5M2, False), ("olmo-7b", E4M3, False),
+                                                  ("olmo-7b", E5M2, False),
+                                                  ("olmo-7b", E4M3, True)])
+def test_full_size_sampled_groups(lib, orc, name, v_fmt, f32_grads):
+    """f32_grads: the same BF16 gradients widened to float32 (exactly) and
+    stepped through the float32-gradient form, which rounds them back."""
     import torch
     if name == "olmo-7b":
         w = inputs.olmo_7b(v_fmt="e4m3" if v_fmt == E4M3 else "e5m2")
     else:
         w = inputs.olmo_1b()
-    need = int(w.n * (8 + 32 / w.group_size)) + (4 << 30)  # states + set-up chunks
+    need = int(w.n * (8 + 32 / w.group_size + (4 if f32_grads else 0))) + (4 << 30)
     free, _ = torch.cuda.mem_get_info()
     if free < need:
         pytest.skip(f"needs {need / 2**30:.0f} GiB of free device memory")
@@ -125,9 +129,15 @@ def test_full_size_sampled_groups(lib, orc, name, v_fmt):
     st = _device_state(lib, w, v_fmt, dev)
     groups = _sample_groups(w)
     before = _gather(st, groups, G)
-    lib.coat_adamw_fp8_step(st["theta"], st["grad"], st["mc"], st["mk"], st["ms"], st["vc"],
+    grad = st["grad"]
+    if f32_grads:
+        grad = torch.empty(w.n, dtype=torch.float32, device=dev)
+        for off in range(0, w.n, 1 << 28):
+            grad[off:off + (1 << 28)].copy_(st["grad"][off:off + (1 << 28)])
+    lib.coat_adamw_fp8_step(st["theta"], grad, st["mc"], st["mk"], st["ms"], st["vc"],
                             st["vk"], st["vs"], step=w.step, group_size=G, v_fmt=v_fmt,
                             **w.hyper)
+    del grad
     torch.cuda.synchronize()
     after = _gather(st, groups, G)
     _check_every_group(st, G, v_fmt)
@@ -141,4 +151,4 @@ def test_full_size_sampled_groups(lib, orc, name, v_fmt):
     got = tuple(after[k] for k in ("theta", "mc", "mk", "ms", "vc", "vk", "vs"))
     stats = parity.assert_step_parity(got, ref, w.hyper["lr"], G, v_fmt,
                                       moments=(ref[7], ref[8]))
-    print(f"{name} v_fmt={v_fmt}: {groups.size} groups sampled, {stats}")
+    print(f"{name} v_fmt={v_fmt} f32_grads={f32_grads}: {groups.size} groups sampled, {stats}")

@@ -66,7 +66,7 @@ typedef enum coat_status {
     COAT_ERR_UNSUPPORTED = 3, /* format / group size / flag combination not built */
     COAT_ERR_CUDA = 4,        /* a CUDA launch or query failed */
     COAT_ERR_NONFINITE = 5,   /* reserved */
-    COAT_ERR_TIMEOUT = 6      /* reserved: a bounded device wait ran out */
+    COAT_ERR_TIMEOUT = 6      /* a bounded device wait ran out (coat_selftest_bounded_wait) */
 } coat_status_t;
 
 typedef enum coat_fp8 {
@@ -431,6 +431,20 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
                                    float eps, const float *weight, const float *bias,
                                    int32_t group_size, uint16_t *out, float *group_amax,
                                    float *tensor_amax, void *stream);
+
+/*
+ * coat_selftest_bounded_wait -- exercises, on the device, the bounded wait
+ * the streamed kernels use on their mbarriers: one block waits on a barrier
+ * that needs two arrivals.  leave_open = 0: both arrive, the phase
+ * completes, COAT_OK.  leave_open = 1: one arrives and nothing ever
+ * completes the phase, so every wait runs out after its bounded number of
+ * polls, the block combines the results as the streamed kernels do and
+ * counts the timeout, and the call returns COAT_ERR_TIMEOUT -- with the
+ * CUDA context still usable and the streamed kernels' own counter
+ * (coat_bulk_wait_timeouts) untouched.  No copy is involved.  Synchronises
+ * the stream.  Errors: INVALID_ARG (leave_open not 0/1), CUDA.
+ */
+coat_status_t coat_selftest_bounded_wait(int32_t leave_open, void *stream);
 
 /* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
  * this thread (0 if none). */

@@ -24,6 +24,7 @@ from ._lib import (  # noqa: F401
     coat_norm_group_amax,
     coat_pack_bf16,
     coat_quantize_state,
+    coat_selftest_bounded_wait,
     coat_state_stats,
     coat_status_string,
     coat_swiglu_group_amax,

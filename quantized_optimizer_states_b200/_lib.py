@@ -77,6 +77,7 @@ SIGNATURES = {
     "coat_unpack_bf16": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), _I32,
                                 ctypes.POINTER(_P), _I64, _P]),
     "coat_state_stats": (_I32, [_P, _P, _P, _I64, _I32, _I32, _P, _P]),
+    "coat_selftest_bounded_wait": (_I32, [_I32, _P]),
     "coat_last_cuda_error": (_I32, []),
     "coat_bulk_wait_timeouts": (_I32, [ctypes.POINTER(ctypes.c_uint32), _I32]),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
@@ -408,6 +409,13 @@ def coat_bulk_wait_timeouts(*, reset: bool = False) -> int:
     c = ctypes.c_uint32(0)
     _check("coat_bulk_wait_timeouts", load().coat_bulk_wait_timeouts(ctypes.byref(c), int(reset)))
     return int(c.value)
+
+
+def coat_selftest_bounded_wait(*, leave_open: bool, stream=None):
+    """Run the bounded-wait self-test (see include/coat.h); raises CoatError
+    with status COAT_ERR_TIMEOUT (6) when the wait ran out."""
+    _check("coat_selftest_bounded_wait",
+           load().coat_selftest_bounded_wait(int(bool(leave_open)), _stream(stream)))
 
 
 def coat_version() -> int:

@@ -79,10 +79,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // bounded wait for the phase with the given parity to complete
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kBulkWaitPolls; ++i)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          uint32_t polls = kBulkWaitPolls) {
+  for (uint32_t i = 0; i < polls; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
+}
+
+// a plain arrival (no transaction count)
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // orders this thread's earlier shared-memory reads before later writes by
@@ -140,6 +146,26 @@ struct BulkPipe {
     for (int j = i; j < issued; ++j) wait(j);
   }
 };
+
+// Self-test of the bounded wait: a barrier that needs two arrivals gets
+// `arrivals` of them (2: the phase completes; 1: nothing ever completes
+// it); every thread waits with the same bounded wait the streamed kernels
+// use, the block combines the results as they do, and a wait that ran out
+// is counted in g_wait_selftest_timeouts.  No copy is involved, so nothing
+// is in flight when the block leaves.
+__device__ unsigned int g_wait_selftest_timeouts;
+
+__global__ void bounded_wait_selftest_kernel(uint32_t arrivals, uint32_t polls) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 2);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  if (threadIdx.x < arrivals) mbar_arrive(&bar);
+  const bool ok = mbar_wait(&bar, 0u, polls);
+  if (!__syncthreads_and(ok) && threadIdx.x == 0) atomicAdd(&g_wait_selftest_timeouts, 1u);
+}
 
 // Blocks for a persistent streaming grid of kernel K: every SM filled to
 // the occupancy K allows, never more blocks than tiles.  SMs x resident

@@ -623,6 +623,23 @@ coat_status_t coat_bulk_wait_timeouts(uint32_t *count, int32_t reset) {
   return COAT_OK;
 }
 
+coat_status_t coat_selftest_bounded_wait(int32_t leave_open, void *stream) {
+  if (leave_open != 0 && leave_open != 1) return COAT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned int zero = 0, polls = 1u << 12;
+  if (cudaMemcpyToSymbolAsync(coat::g_wait_selftest_timeouts, &zero, sizeof(zero), 0,
+                              cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return launch_status();
+  coat::bounded_wait_selftest_kernel<<<1, 64, 0, s>>>(leave_open ? 1u : 2u, polls);
+  unsigned int count = 0;
+  if (cudaGetLastError() != cudaSuccess ||
+      cudaMemcpyFromSymbolAsync(&count, coat::g_wait_selftest_timeouts, sizeof(count), 0,
+                                cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return launch_status();
+  return count != 0 ? COAT_ERR_TIMEOUT : COAT_OK;
+}
+
 const char *coat_status_string(coat_status_t status) {
   switch (status) {
     case COAT_OK: return "ok";

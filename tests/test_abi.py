@@ -129,6 +129,10 @@ def test_state_stats_argument_checks(lib):
     assert st(fake, fake, fake, 64, 128, 0, odd, None) == 2       # output not 8-byte aligned
 
 
+def test_selftest_argument_check(lib):
+    assert lib.coat_selftest_bounded_wait(2, None) == 1
+
+
 def test_product_path_fails_loudly_without_library(tmp_path):
     from quantized_optimizer_states_b200 import _lib
     saved = _lib._lib

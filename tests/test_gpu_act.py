@@ -184,6 +184,22 @@ def test_activation_dequant_full_set(lib, orc, out_bf16):
     assert lib.coat_bulk_wait_timeouts(reset=True) == 0
 
 
+def test_bounded_wait_runs_out_and_the_context_survives(lib, orc):
+    """The bounded mbarrier wait of the streamed kernels, made to run out on
+    the device (a barrier phase that nothing completes): the call reports
+    COAT_ERR_TIMEOUT, and afterwards the context still works -- a streamed
+    quantizer run is bit-exact and its own timeout counter is 0."""
+    lib.coat_selftest_bounded_wait(leave_open=False)
+    with pytest.raises(lib.CoatError) as e:
+        lib.coat_selftest_bounded_wait(leave_open=True)
+    assert e.value.status == 6
+    x = inputs.host_activations(inputs.activations(seed=21), rows=12)
+    q, sc = _gpu_1xG(lib, x, 128, E4M3)
+    q_ref, sc_ref = orc.group_quant_1xG(x, 128, E4M3)
+    assert np.array_equal(q, q_ref) and np.array_equal(sc, sc_ref)
+    assert lib.coat_bulk_wait_timeouts(reset=True) == 0
+
+
 def test_hardware_cvt_matches_oracle_encoder(lib, orc):
     """The sm_100a cvt...satfinite path (through the 1xG quantizer with unit
     scale, i.e. a group whose amax is exactly 448) against the oracle's

@@ -15,6 +15,7 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 
 #include "bulk_pipe.cuh"
 #include "fp8_device.cuh"
@@ -599,6 +600,115 @@ __global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormPar
       __syncwarp();   // every lane is done with the buffer the next prefetch reuses
     }
   }
+  if (p.tensor_amax) block_max_to_tensor(wmax, p.tensor_amax);
+}
+
+// Rows of 256 NC columns (NC = 1..8: up to 2048 columns) are held in
+// registers instead: lane l loads the row's 16-byte chunks l, l + 32, ...,
+// l + 32 (NC - 1) with plain 128-bit loads (every load instruction of the
+// warp reads 512 contiguous bytes) and takes the sums, the output and the
+// maxima from them, in the order of the staged kernel above (same sums,
+// same roundings, so the same bits).  Fully unrolled over the row, it
+// executes far fewer instructions than the staged form's three loops over
+// shared memory, which are what limit that form: measured on [16384, 2048],
+// 26.0 us against 32.9 us.  Persistent warps, 8 to a block, 2 blocks per
+// SM (the row and its sums take ~110 registers).
+constexpr int kNormRegWarps = 8;
+constexpr int kNormRegMaxChunks = 8;
+
+template <int NC>
+__device__ __forceinline__ float norm_reg_row(const NormParams &p, int64_t row, int lane) {
+  const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.cols);
+  uint4 c[NC];
+#pragma unroll
+  for (int i = 0; i < NC; ++i) c[i] = src[lane + 32 * i];
+  const float inv_n = 1.0f / static_cast<float>(p.cols);
+  float acc = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = bf16lo_to_float(wv[j]), b = bf16hi_to_float(wv[j]);
+      acc += p.rms ? a * a + b * b : a + b;
+    }
+  }
+  const float s1 = warp_sum_f(acc);
+  float mean = 0.0f, var;
+  if (p.rms) {
+    var = s1 * inv_n;
+  } else {
+    mean = s1 * inv_n;
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float a = bf16lo_to_float(wv[j]) - mean, b = bf16hi_to_float(wv[j]) - mean;
+        ss += a * a + b * b;
+      }
+    }
+    var = warp_sum_f(ss) * inv_n;
+  }
+  const float rstd = 1.0f / sqrtf(var + p.eps);
+
+  // chunk q = lane + 32 i holds columns 8q .. 8q + 7; a 1xG run is G / 8
+  // chunks: consecutive lanes of one i for G <= 256, else all lanes of
+  // G / 256 consecutive i
+  const int clanes = 1 << (p.log2G - 3);
+  const int64_t gbase = (row * p.cols) >> p.log2G;
+  uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.cols);
+  float run = 0.0f, rowmax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+    const int col0 = 8 * (lane + 32 * i);
+    uint32_t ow[4];
+    float a = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int cc = col0 + 2 * j;
+      float y0 = (bf16lo_to_float(wv[j]) - mean) * rstd;
+      float y1 = (bf16hi_to_float(wv[j]) - mean) * rstd;
+      if (p.weight) {
+        y0 *= p.weight[cc];
+        y1 *= p.weight[cc + 1];
+      }
+      if (p.bias) {
+        y0 += p.bias[cc];
+        y1 += p.bias[cc + 1];
+      }
+      ow[j] = bf16x2_rn(y0, y1);
+      a = fmaxf(a, fmaxf(fabsf(bf16lo_to_float(ow[j])), fabsf(bf16hi_to_float(ow[j]))));
+    }
+    dst[lane + 32 * i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    rowmax = fmaxf(rowmax, a);
+    if (clanes <= 32) {
+      for (int off = 1; off < clanes; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      if ((lane & (clanes - 1)) == 0) p.group_amax[gbase + (col0 >> p.log2G)] = a;
+    } else {
+      run = fmaxf(run, warp_max_f(a));
+      if (((i + 1) & ((clanes >> 5) - 1)) == 0) {   // the run's last chunk column
+        if (lane == 0) p.group_amax[gbase + ((256 * i) >> p.log2G)] = run;
+        run = 0.0f;
+      }
+    }
+  }
+  return warp_max_f(rowmax);
+}
+
+// Persistent warps: warp w of the grid takes rows w, w + W, ... (W the
+// grid's warps).
+template <int NC>
+__global__ void __launch_bounds__(32 * kNormRegWarps, 2) norm_reg_group_amax_kernel(const NormParams p) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kNormRegWarps;
+  float wmax = 0.0f;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kNormRegWarps + (threadIdx.x >> 5);
+       row < p.rows; row += step)
+    wmax = fmaxf(wmax, norm_reg_row<NC>(p, row, lane));
   if (p.tensor_amax) block_max_to_tensor(wmax, p.tensor_amax);
 }
 

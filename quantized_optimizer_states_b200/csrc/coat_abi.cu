@@ -274,6 +274,25 @@ coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *
                                  : launch_step_all<coat::kE5M2, false>(lg, n, s, p);
 }
 
+// Register-resident norm rows of 256 NC columns: persistent grid of the
+// blocks that fit the GPU at once (or fewer, for few rows).
+template <int NC>
+void launch_norm_reg(cudaStream_t s, const coat::NormParams &p) {
+  int dev = 0, sms = 1, per_sm = 1;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, coat::norm_reg_group_amax_kernel<NC>,
+                                                    32 * coat::kNormRegWarps, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t blocks_needed = (p.rows + coat::kNormRegWarps - 1) / coat::kNormRegWarps;
+  const int64_t resident = static_cast<int64_t>(sms) * per_sm;
+  const unsigned int grid =
+      static_cast<unsigned int>(blocks_needed < resident ? blocks_needed : resident);
+  launch_act_threads(coat::norm_reg_group_amax_kernel<NC>, grid, 32u * coat::kNormRegWarps, 0, s,
+                     p);
+}
+
 }  // namespace
 
 extern "C" {
@@ -557,7 +576,20 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
   if (tensor_amax)
     launch_act_threads(coat::zero_word_kernel, 1u, 32u, 0, s,
                        reinterpret_cast<uint32_t *>(tensor_amax));
-  // persistent warps, each staging two rows in shared memory
+  if (cols % 256 == 0 && cols / 256 <= coat::kNormRegMaxChunks) {
+    switch (cols / 256) {
+      case 1: launch_norm_reg<1>(s, p); break;
+      case 2: launch_norm_reg<2>(s, p); break;
+      case 3: launch_norm_reg<3>(s, p); break;
+      case 4: launch_norm_reg<4>(s, p); break;
+      case 5: launch_norm_reg<5>(s, p); break;
+      case 6: launch_norm_reg<6>(s, p); break;
+      case 7: launch_norm_reg<7>(s, p); break;
+      default: launch_norm_reg<8>(s, p); break;
+    }
+    return launch_status();
+  }
+  // other widths: persistent warps, each staging two rows in shared memory
   const int wpb = coat::norm_warps_per_block(cols);
   const size_t smem = static_cast<size_t>(wpb) * 2 * static_cast<size_t>(cols) * 2;
   {

@@ -46,8 +46,15 @@ def _midpoint_ok(orc, y64, got_bits, want_bits, offset):
     return bad.size
 
 
+# widths that are multiples of 256 up to 2048 take the register-resident
+# kernel (every chunk count 1..8 below, groups within one load column and
+# across several, more rows than the persistent grid has warps); the others
+# the shared-memory one
 @pytest.mark.parametrize("rows,cols,G", [(64, 2048, 128), (24, 4096, 128), (8, 16384, 4096),
-                                         (40, 768, 256), (16, 5120, 512), (33, 1536, 128)])
+                                         (40, 768, 256), (16, 5120, 512), (33, 1536, 128),
+                                         (3000, 256, 16), (20, 2048, 1024), (12, 2048, 2048),
+                                         (9, 1024, 512), (10, 1280, 256), (16, 1792, 64),
+                                         (7, 512, 32), (24, 1040, 16)])
 @pytest.mark.parametrize("rms", [False, True])
 def test_norm_matches_oracle(lib, orc, rows, cols, G, rms):
     import torch
@@ -103,13 +110,14 @@ def test_norm_feeds_group_scaling(lib, orc):
     assert np.array_equal(parity.to_host(q1), q_ref) and float(s1.item()) == s_ref
 
 
+@pytest.mark.parametrize("cols", [4096, 2048])
 @pytest.mark.parametrize("rms", [False, True])
-def test_norm_tensor_max_feeds_the_cast_alone(lib, orc, rms):
+def test_norm_tensor_max_feeds_the_cast_alone(lib, orc, rms, cols):
     """tensor_amax: the producer also writes the tensor maximum; Group
     Scaling with amax_precomputed=2 then only casts, with the oracle's codes
     and scale; amax_precomputed outside 0..2 is rejected."""
     import torch
-    rows, cols, G = 300, 4096, 128
+    rows, G = 300, 128
     x = inputs.host_activations(inputs.activations(seed=8), rows=rows)
     x = np.tile(x, (1, 2))[:, :cols].copy()
     n = rows * cols

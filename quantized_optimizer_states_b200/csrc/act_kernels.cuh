@@ -435,8 +435,11 @@ __global__ void __launch_bounds__(kThreads) swiglu_group_amax_kernel(const Swigl
 // One warp per row: the warp stages its row in shared memory (16-byte
 // asynchronous copies, the next row's issued before the current one is
 // computed), takes the row sums over it in binary32 (per-lane sums, then a
-// fixed xor shuffle tree, so every lane holds the same value), and writes
-// the BF16 output and each 1xG run's maximum.  The binary32
+// fixed xor shuffle tree, so every lane holds the same value), divides them
+// by the row length with the correctly rounded quotient (a row whose sum is
+// exact, such as a constant row, gets its exact mean: x - mean is then 0,
+// where a product with a rounded 1/n could leave one ulp of x, multiplied by
+// 1/sqrt(eps)), and writes the BF16 output and each 1xG run's maximum.  The binary32
 // statistics (sums of a few thousand terms) and y carry an error of about
 // 1e-6 x (|y| + |mean| / std), so the BF16 output is the correctly rounded
 // norm except within that distance of a rounding midpoint.
@@ -490,7 +493,7 @@ __device__ __forceinline__ void norm_prefetch_row(const NormParams &p, uint4 *ds
 __device__ __forceinline__ float norm_one_row(const NormParams &p, const uint4 *rs, int64_t row,
                                               int lane) {
   const int nq = static_cast<int>(p.cols >> 3);
-  const float inv_n = 1.0f / static_cast<float>(p.cols);
+  const float nf = static_cast<float>(p.cols);   // exact (cols <= 16384)
   float acc = 0.0f;
   for (int q = lane; q < nq; q += 32) {
     const uint4 c = rs[q];
@@ -504,9 +507,9 @@ __device__ __forceinline__ float norm_one_row(const NormParams &p, const uint4 *
   const float s1 = warp_sum_f(acc);
   float mean = 0.0f, var;
   if (p.rms) {
-    var = s1 * inv_n;
+    var = __fdiv_rn(s1, nf);
   } else {
-    mean = s1 * inv_n;
+    mean = __fdiv_rn(s1, nf);
     float ss = 0.0f;
     for (int q = lane; q < nq; q += 32) {
       const uint4 c = rs[q];
@@ -517,7 +520,7 @@ __device__ __forceinline__ float norm_one_row(const NormParams &p, const uint4 *
         ss += a * a + b * b;
       }
     }
-    var = warp_sum_f(ss) * inv_n;
+    var = __fdiv_rn(warp_sum_f(ss), nf);
   }
   const float rstd = 1.0f / sqrtf(var + p.eps);
 
@@ -622,7 +625,7 @@ __device__ __forceinline__ float norm_reg_row(const NormParams &p, int64_t row, 
   uint4 c[NC];
 #pragma unroll
   for (int i = 0; i < NC; ++i) c[i] = src[lane + 32 * i];
-  const float inv_n = 1.0f / static_cast<float>(p.cols);
+  const float nf = static_cast<float>(p.cols);   // exact (cols <= 16384)
   float acc = 0.0f;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
@@ -636,9 +639,9 @@ __device__ __forceinline__ float norm_reg_row(const NormParams &p, int64_t row, 
   const float s1 = warp_sum_f(acc);
   float mean = 0.0f, var;
   if (p.rms) {
-    var = s1 * inv_n;
+    var = __fdiv_rn(s1, nf);
   } else {
-    mean = s1 * inv_n;
+    mean = __fdiv_rn(s1, nf);
     float ss = 0.0f;
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
@@ -649,7 +652,7 @@ __device__ __forceinline__ float norm_reg_row(const NormParams &p, int64_t row, 
         ss += a * a + b * b;
       }
     }
-    var = warp_sum_f(ss) * inv_n;
+    var = __fdiv_rn(warp_sum_f(ss), nf);
   }
   const float rstd = 1.0f / sqrtf(var + p.eps);
 

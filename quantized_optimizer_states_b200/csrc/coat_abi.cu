@@ -275,20 +275,13 @@ coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *
 }
 
 // Register-resident norm rows of 256 NC columns: persistent grid of the
-// blocks that fit the GPU at once (or fewer, for few rows).
+// blocks that fit the GPU at once (or fewer, for few rows), the occupancy
+// looked up once per device.
 template <int NC>
 void launch_norm_reg(cudaStream_t s, const coat::NormParams &p) {
-  int dev = 0, sms = 1, per_sm = 1;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, coat::norm_reg_group_amax_kernel<NC>,
-                                                    32 * coat::kNormRegWarps, 0) != cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
   const int64_t blocks_needed = (p.rows + coat::kNormRegWarps - 1) / coat::kNormRegWarps;
-  const int64_t resident = static_cast<int64_t>(sms) * per_sm;
-  const unsigned int grid =
-      static_cast<unsigned int>(blocks_needed < resident ? blocks_needed : resident);
+  const unsigned int grid = coat::bulk_grid<coat::norm_reg_group_amax_kernel<NC>>(
+      32 * coat::kNormRegWarps, 0, blocks_needed);
   launch_act_threads(coat::norm_reg_group_amax_kernel<NC>, grid, 32u * coat::kNormRegWarps, 0, s,
                      p);
 }

@@ -19,6 +19,7 @@ reduction from the expansion function is "parity unpinned" (direction only).
 from __future__ import annotations
 
 import ctypes
+import os
 
 import numpy as np
 
@@ -48,9 +49,12 @@ class AdamWCfg(ctypes.Structure):
 
 
 def lib():
+    """The compiled C oracle: oracle/liborc.so, built on first use, or the
+    build named by the COAT_ORACLE_LIB environment variable (the mutation
+    tests point it at copies of the oracle with a planted mistake)."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = os.environ.get("COAT_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i64 = ctypes.c_int64
@@ -235,13 +239,16 @@ def adamw_fp64(theta, grad, m, v, *, step, beta1, beta2, lr, eps, weight_decay):
 
 # ---- activations -----------------------------------------------------------
 
-def group_quant_1xG(x_bf16: np.ndarray, G: int, fmt: int = E4M3):
-    """x_bf16: uint16 [rows, cols] -> (q u8 [rows, cols], scale f32 [rows, cols/G])."""
+def group_quant_1xG(x_bf16: np.ndarray, G: int, fmt: int = E4M3, cols: int | None = None):
+    """x_bf16: uint16 [rows, ld] -> (q u8 [rows, cols], scale f32 [rows, cols/G]) for the
+    first `cols` columns of each row (all of them by default): rows of a
+    larger buffer, row stride ld."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
-    rows, cols = x.shape
+    rows, ld = x.shape
+    cols = ld if cols is None else cols
     q = np.empty((rows, cols), dtype=np.uint8)
     sc = np.empty((rows, cols // G), dtype=np.float32)
-    _check(lib().orc_group_quant_1xG(_ptr(x), rows, cols, cols, G, fmt, _ptr(q), _ptr(sc)),
+    _check(lib().orc_group_quant_1xG(_ptr(x), rows, cols, ld, G, fmt, _ptr(q), _ptr(sc)),
            "group_quant_1xG")
     return q, sc
 

@@ -69,6 +69,58 @@ def test_group_scaling_matches_torch_and_single_group(orc, fmt):
 
 
 @pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_group_quant_1xG_row_stride(orc, fmt):
+    """Rows taken from a wider buffer (row stride ld > cols) are quantized as
+    the same rows stored contiguously, and the columns past cols -- here
+    large values that would change every scale -- are never read."""
+    G, rows, cols, ld = 64, 12, 256, 256 + 96
+    x = inputs.host_activations(inputs.activations(seed=3), rows=rows)[:, :cols].copy()
+    wide = np.full((rows, ld), 0x4780, dtype=np.uint16)          # BF16 65536
+    wide[:, :cols] = x
+    q, sc = orc.group_quant_1xG(wide, G, fmt, cols=cols)
+    xf = _bf16_to_f32(x).reshape(rows, -1, G)
+    amax = xf.abs().amax(dim=-1)
+    fmax = torch.tensor(FMAX[fmt], dtype=torch.float32)
+    assert torch.equal(torch.from_numpy(sc), amax / fmax)
+    ref = (xf * (fmax / amax)[..., None]).to(TORCH_DT[fmt]).view(torch.uint8).reshape(rows, -1)
+    assert np.array_equal(q, ref.numpy())
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_group_scaling_max_in_the_last_partial_group(orc, fmt):
+    """The tensor maximum in the shorter last group still sets the scale:
+    s = amax / fmt_max, the largest element encodes to the top code."""
+    n, G = 1000, 128                                 # 7 full groups and one of 104
+    x = np.full(n, 0x3F80, dtype=np.uint16)          # 1.0
+    x[n - 1] = 0x447A                                # BF16 1000.0
+    q, s, ga = orc.group_scaling_pertensor(x, G, fmt)
+    assert ga[-1] == 1000.0 and np.all(ga[:-1] == 1.0)
+    assert s == np.float32(1000.0) / np.float32(FMAX[fmt])
+    top = 0x7E if fmt == E4M3 else 0x7B
+    assert q[n - 1] == top
+    ref = (_bf16_to_f32(x) * (torch.tensor(FMAX[fmt]) / 1000.0)).to(TORCH_DT[fmt])
+    assert np.array_equal(q, ref.view(torch.uint8).numpy())
+
+
+def test_group_scaling_takes_the_producers_maxima(orc):
+    """With maxima supplied (a producer filled the intermediate), step (i) is
+    skipped: the scale comes from the given values even where they differ
+    from the tensor's own maxima (here one entry doubled)."""
+    G = 128
+    x = inputs.host_activations(inputs.activations(seed=4), rows=4).reshape(-1)
+    _, s0, ga = orc.group_scaling_pertensor(x, G, E4M3)
+    given = ga.copy()
+    i = int(np.argmax(given))
+    given[i] = 2.0 * given[i]
+    q, s, ga_out = orc.group_scaling_pertensor(x, G, E4M3, group_amax=given)
+    assert np.array_equal(ga_out, given)
+    amax = torch.tensor(float(given[i]), dtype=torch.float32)
+    assert s == (amax / torch.tensor(448.0)).item() and s == 2.0 * s0
+    ref = (_bf16_to_f32(x) * (torch.tensor(448.0) / amax)).to(torch.float8_e4m3fn)
+    assert np.array_equal(q, ref.view(torch.uint8).numpy())
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
 def test_activation_dequant(orc, fmt):
     w = inputs.activations()
     x = inputs.host_activations(w, rows=8)

@@ -17,6 +17,13 @@ def test_hand_example_closed_forms():
     # mean of squares 30/4: x_i / sqrt(15/2)
     want_rms = np.arange(1, 5) / np.sqrt(7.5)
     assert np.allclose(oracle.norm_f64(x, rms=True, eps=0.0)[0], want_rms, rtol=0, atol=1e-15)
+    # per-column weight and bias act column by column: w = (1, 2, 3, 4),
+    # b = (1/2, 0, 0, -1) give ((2 i - 5) / sqrt 5) i + b_i
+    w = np.array([1.0, 2.0, 3.0, 4.0], np.float32)
+    b = np.array([0.5, 0.0, 0.0, -1.0], np.float32)
+    want_aff = want_ln * np.arange(1, 5) + np.array([0.5, 0.0, 0.0, -1.0])
+    got_aff = oracle.norm_f64(x, rms=False, eps=0.0, weight=w, bias=b)[0]
+    assert np.allclose(got_aff, want_aff, rtol=0, atol=1e-15)
     # with eps the variance term grows by exactly eps (binary32 value of eps)
     e = float(np.float32(1e-3))
     want_eps = (2.0 * np.arange(1, 5) - 5.0) / 2.0 / np.sqrt(1.25 + e)

@@ -36,6 +36,7 @@ bit for bit.
 """
 from __future__ import annotations
 
+import operator
 from dataclasses import dataclass
 
 import torch
@@ -56,6 +57,17 @@ def padded_layout(numels: list[int], group_size: int) -> tuple[list[int], int]:
         offsets.append(off)
         off += -(-n // unit) * unit
     return offsets, off
+
+
+def _check_group_size(G) -> None:
+    """The 1xG group sizes the step kernels are built for: powers of two
+    from 16 to 4096."""
+    try:
+        g = operator.index(G)          # Python or NumPy integers, not floats
+    except TypeError:
+        g = None
+    if g is None or g < 16 or g > 4096 or g & (g - 1):
+        raise ValueError(f"group_size must be a power of two in [16, 4096], got {G!r}")
 
 
 @dataclass
@@ -110,6 +122,11 @@ class CoatAdamW(torch.optim.Optimizer):
             raise ValueError("lr, eps and weight_decay must be non-negative")
         if v_fmt not in _FMT:
             raise ValueError("v_fmt must be 'e4m3' or 'e5m2'")
+        _check_group_size(group_size)
+        if k_range not in (0, 1):
+            raise ValueError("k_range must be 0 (E4M3's range) or 1 (the storage format's)")
+        if not k_max >= 0.0:
+            raise ValueError("k_max must be >= 0 (0: no clamp)")
         defaults = dict(lr=lr, betas=tuple(betas), eps=eps, weight_decay=weight_decay,
                         group_size=group_size, v_fmt=_FMT[v_fmt], k_range=k_range,
                         k_max=k_max)
@@ -132,6 +149,9 @@ class CoatAdamW(torch.optim.Optimizer):
         dev = ps[0].device
         if dev.type != "cuda":
             raise ValueError("CoatAdamW needs CUDA parameters")
+        if any(p.device != dev for p in ps):
+            raise ValueError("the parameters of a group must be on one device")
+        _check_group_size(group["group_size"])
         dtypes = {p.dtype for p in ps}
         if dtypes not in ({torch.float32}, {torch.bfloat16}):
             raise ValueError("a parameter group must be all float32 or all bfloat16")

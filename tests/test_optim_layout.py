@@ -37,3 +37,13 @@ def test_bad_hyperparameters_are_rejected():
         CoatAdamW(p, betas=(1.0, 0.9))
     with pytest.raises(ValueError):
         CoatAdamW(p, v_fmt="e3m4")
+
+
+@pytest.mark.parametrize("kw", [dict(group_size=96), dict(group_size=8), dict(group_size=8192),
+                                dict(group_size=128.0), dict(k_range=2),
+                                dict(k_max=-1.0), dict(k_max=float("nan"))])
+def test_unsupported_group_size_and_expansion_settings_are_rejected(kw):
+    # rejected when the optimizer is made, not at its first step (the check
+    # runs before the parameters' device is looked at, so CPU tensors do)
+    with pytest.raises(ValueError, match="group_size|k_range|k_max"):
+        CoatAdamW([torch.nn.Parameter(torch.zeros(4))], **kw)

@@ -102,7 +102,9 @@ class ClockSampler:
 
     def __init__(self, uuid: str | None):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # the raw samples (the JSON line carries their summary)
+        log_dir = os.environ.get("COAT_BENCH_LOG_DIR") or os.path.join(ROOT, "bench_logs")
+        self.path = os.path.join(log_dir, f"clocks_{os.getpid()}.csv")
         self.uuid = uuid
 
     def start(self):

@@ -1,5 +1,5 @@
 """Guard canaries around the outputs of every activation-side, producer,
-pack and monitoring kernel (compute-sanitizer is closed on this machine): each
+pack and monitoring kernel, a check that needs no memory-checking tool: each
 output is a slice of a larger buffer whose 256 bytes before and after hold
 a sentinel, sizes are ragged (streamed tiles plus a plain remainder, tail
 vectors, tail groups), and after the calls the sentinels must be intact

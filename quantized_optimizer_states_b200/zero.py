@@ -76,6 +76,30 @@ class Zero1Shard:
         self.m_s = torch.zeros(ng, dtype=torch.float32, device=dev)
         self.v_s = torch.zeros(ng, dtype=torch.float32, device=dev)
 
+    _STATE = ("master", "m_code", "m_k", "m_s", "v_code", "v_k", "v_s")
+    _LAYOUT = ("n", "world", "rank", "L", "group_size", "v_fmt", "k_range", "k_max")
+
+    def state_dict(self) -> dict:
+        """This rank's share of the optimizer state (copies) and the layout it
+        belongs to.  Every rank saves its own; loading them back into shards
+        made for the same buffer length, group size, formats and rank count
+        resumes the run bit for bit (the caller keeps the step count t)."""
+        return {**{k: getattr(self, k) for k in self._LAYOUT},
+                **{k: getattr(self, k).detach().clone() for k in self._STATE}}
+
+    def load_state_dict(self, sd: dict) -> None:
+        """Restore a shard saved by state_dict(); the layout must match."""
+        for k in self._LAYOUT:
+            if sd.get(k) != getattr(self, k):
+                raise ValueError(f"checkpoint {k} = {sd.get(k)!r} differs from this shard's "
+                                 f"{getattr(self, k)!r}")
+        with torch.no_grad():
+            for k in self._STATE:
+                dst = getattr(self, k)
+                if tuple(sd[k].shape) != tuple(dst.shape) or sd[k].dtype != dst.dtype:
+                    raise ValueError(f"checkpoint tensor {k} has the wrong shape or type")
+                dst.copy_(sd[k].to(dst.device))
+
     def reduce_gradient_f32(self, grad: torch.Tensor) -> torch.Tensor:
         """Mean over ranks of the full BF16 gradients, this rank's shard, in
         binary32 (sum by the collective, division by the rank count)."""

@@ -109,3 +109,63 @@ def test_two_gloo_ranks_match_the_single_rank_step():
     for rank, full, Lr in res:
         assert Lr == L
         assert np.array_equal(full, th[:n]), f"rank {rank}"
+
+
+def _resume_worker(rank, world, port, n, steps, cut, q):
+    import io
+
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        theta, grads = _inputs(n, world, steps)
+        step_fn = _oracle_step_fn()
+        g = [torch.from_numpy(grads[t, rank]).to(torch.bfloat16) for t in range(steps)]
+        # straight through
+        a = zero.Zero1Shard(torch.from_numpy(theta), group_size=G)
+        for t in range(steps):
+            full_a = a.step(g[t], 10 + t, H, step_fn=step_fn)
+        # stopped after `cut` steps, saved, restored into a fresh shard
+        b = zero.Zero1Shard(torch.from_numpy(theta), group_size=G)
+        for t in range(cut):
+            b.step(g[t], 10 + t, H, step_fn=step_fn)
+        buf = io.BytesIO()
+        torch.save(b.state_dict(), buf)
+        buf.seek(0)
+        c = zero.Zero1Shard(torch.from_numpy(np.zeros(n, np.float32)), group_size=G)
+        c.load_state_dict(torch.load(buf))
+        for t in range(cut, steps):
+            full_c = c.step(g[t], 10 + t, H, step_fn=step_fn)
+        wrong = zero.Zero1Shard(torch.from_numpy(theta), group_size=2 * G)
+        try:
+            wrong.load_state_dict(b.state_dict())
+            rejected = False
+        except ValueError:
+            rejected = True
+        q.put((rank, np.array_equal(full_a.numpy(), full_c.numpy()), rejected))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_resume_from_a_checkpoint_bit_for_bit():
+    """Each rank saves its shard after 2 of 4 steps; fresh shards that load
+    the checkpoints and take steps 3-4 end with the same parameters, bit for
+    bit, as the shards that never stopped; a shard of another group size
+    refuses the checkpoint."""
+    world, n, steps, cut = 2, 5 * 128 + 77, 4, 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_resume_worker, args=(r, world, port, n, steps, cut, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, same, rejected in res:
+        assert same, f"rank {rank}: resumed run differs"
+        assert rejected, f"rank {rank}: mismatched layout accepted"

@@ -40,7 +40,9 @@
  *   - Buffers that the kernels access with 16-byte vector instructions
  *     (parameters, gradients, codes, activations) must start on a 16-byte
  *     boundary, otherwise COAT_ERR_MISALIGNED is returned and nothing runs.
- *     Per-group metadata arrays need only natural (4-byte) alignment.
+ *     Float32 metadata arrays (per-group k and s, scales, maxima) need only
+ *     natural (4-byte) alignment, and every element pointer its element
+ *     size's; a pointer short of that is also COAT_ERR_MISALIGNED.
  *   - Group size G: a power of two, 16 <= G <= 4096
  *     (COAT_ERR_UNSUPPORTED otherwise).
  *   - Sizes are element counts.  n == 0 is valid and launches nothing.
@@ -62,7 +64,7 @@ extern "C" {
 typedef enum coat_status {
     COAT_OK = 0,
     COAT_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad hyper-parameter */
-    COAT_ERR_MISALIGNED = 2,  /* a vector-accessed buffer is not 16-byte aligned */
+    COAT_ERR_MISALIGNED = 2,  /* a buffer short of its required alignment (16-byte for vector-accessed ones) */
     COAT_ERR_UNSUPPORTED = 3, /* format / group size / flag combination not built */
     COAT_ERR_CUDA = 4,        /* a CUDA launch or query failed */
     COAT_ERR_NONFINITE = 5,   /* reserved */

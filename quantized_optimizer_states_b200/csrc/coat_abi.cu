@@ -41,6 +41,9 @@ coat_status_t launch_status() {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// 4-byte alignment of a float array the kernels read or write (null passes)
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
 bool valid_fmt(int32_t f) { return f == COAT_E4M3 || f == COAT_E5M2; }
 
 // log2(G) for a supported group size, else -1.
@@ -210,7 +213,8 @@ coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *
     return COAT_ERR_UNSUPPORTED;
   if (n > kMaxElems) return COAT_ERR_UNSUPPORTED;
   if (n == 0) return COAT_OK;
-  if (!aligned16(param) || !aligned16(grad) || !aligned16(m_code) || !aligned16(v_code))
+  if (!aligned16(param) || !aligned16(grad) || !aligned16(m_code) || !aligned16(v_code) ||
+      !aligned4(m_k) || !aligned4(m_scale) || !aligned4(v_k) || !aligned4(v_scale))
     return COAT_ERR_MISALIGNED;
 
   coat::StepParams p;
@@ -348,7 +352,8 @@ coat_status_t coat_quantize_state(const float *x, int64_t n, int32_t group_size,
       (flags & ~COAT_FORCE_K1) != 0 || n > kMaxElems)
     return COAT_ERR_UNSUPPORTED;
   if (n == 0) return COAT_OK;
-  if (!aligned16(x) || !aligned16(code)) return COAT_ERR_MISALIGNED;
+  if (!aligned16(x) || !aligned16(code) || !aligned4(k) || !aligned4(scale))
+    return COAT_ERR_MISALIGNED;
   coat::QuantParams p;
   p.x = x;
   p.code = code;
@@ -381,7 +386,8 @@ coat_status_t coat_dequant(const uint8_t *q, const float *k, const float *scale,
     if (lg < 0) return COAT_ERR_UNSUPPORTED;
   }
   if (n == 0) return COAT_OK;
-  if (!aligned16(q) || !aligned16(out)) return COAT_ERR_MISALIGNED;
+  if (!aligned16(q) || !aligned16(out) || !aligned4(k) || !aligned4(scale))
+    return COAT_ERR_MISALIGNED;
   coat::DequantParams p;
   p.q = q;
   p.k = k;
@@ -421,7 +427,8 @@ coat_status_t coat_group_quant_1xG(const uint16_t *x, int64_t rows, int64_t cols
   if (cols % group_size != 0) return COAT_ERR_INVALID_ARG;
   if (rows == 0 || cols == 0) return COAT_OK;
   if (rows * cols > kMaxElems) return COAT_ERR_UNSUPPORTED;
-  if (!aligned16(x) || !aligned16(q) || (ld % 8) != 0) return COAT_ERR_MISALIGNED;
+  if (!aligned16(x) || !aligned16(q) || (ld % 8) != 0 || !aligned4(scale))
+    return COAT_ERR_MISALIGNED;
   coat::GroupQuantParams p;
   p.x = x;
   p.rows = rows;
@@ -473,7 +480,7 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
   const int lg = group_log2(group_size);
   if (lg < 0 || !valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
   if (n == 0) return COAT_OK;
-  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+  if (!aligned16(x) || !aligned16(q) || !aligned4(workspace) || !aligned4(scale))
     return COAT_ERR_MISALIGNED;
   const int64_t ng = (n + group_size - 1) / group_size;
   coat::GroupScalingParams p;
@@ -734,6 +741,10 @@ coat_status_t pack_launch(bool unpack, const void *const *ptrs, const int64_t *n
     if (numel[i] < 0 || offset[i] < 0 || offset[i] > n - numel[i]) return COAT_ERR_INVALID_ARG;
     if (numel[i] > 0 && unpack && !ptrs[i]) return COAT_ERR_INVALID_ARG;
     if (numel[i] > 0 && (offset[i] % 8) != 0) return COAT_ERR_MISALIGNED;
+    // element alignment of a source (float32: 4 bytes, BF16: 2) or BF16 target
+    const uintptr_t elem_mask = (!unpack && src_f32) ? 3u : 1u;
+    if (numel[i] > 0 && (reinterpret_cast<uintptr_t>(ptrs[i]) & elem_mask) != 0)
+      return COAT_ERR_MISALIGNED;
     any = any || numel[i] > 0;
     // one launch per kPackTensors tensors, its blocks counted in an int32
     if (i % coat::kPackTensors == 0) chunks_in_launch = 0;
@@ -780,7 +791,8 @@ extern "C" coat_status_t coat_state_stats(const uint8_t *code, const float *k,
   if (n > 0 && (!code || !k || !scale)) return COAT_ERR_INVALID_ARG;
   if (group_log2(group_size) < 0 || !valid_fmt(fmt) || n > kMaxElems)
     return COAT_ERR_UNSUPPORTED;
-  if ((n > 0 && !aligned16(code)) || (reinterpret_cast<uintptr_t>(stats) & 7u) != 0)
+  if ((n > 0 && (!aligned16(code) || !aligned4(k) || !aligned4(scale))) ||
+      (reinterpret_cast<uintptr_t>(stats) & 7u) != 0)
     return COAT_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   coat::state_stats_init_kernel<<<1, 1, 0, s>>>(stats);
@@ -824,7 +836,7 @@ extern "C" coat_status_t coat_group_scaling_quant_pertensor_noalloc(
   const int lg = group_log2(group_size);
   if (lg < 0 || !valid_fmt(fmt) || n > kMaxElems) return COAT_ERR_UNSUPPORTED;
   if (n == 0) return COAT_OK;
-  if (!aligned16(x) || !aligned16(q)) return COAT_ERR_MISALIGNED;
+  if (!aligned16(x) || !aligned16(q) || !aligned4(scale)) return COAT_ERR_MISALIGNED;
   const int64_t ng = (n + group_size - 1) / group_size;
   if (ng > kNoAllocGroups) return COAT_ERR_UNSUPPORTED;
   float *ws = nullptr;

@@ -151,3 +151,90 @@ def test_product_package_never_imports_the_oracle():
             src = open(path).read()
             assert "import oracle" not in src and "from oracle" not in src, path
             assert "coat_oracle" not in src and "liborc" not in src, path
+
+
+def test_more_argument_checks_and_metadata_alignment(lib):
+    """The entry points not covered above, and the 4-byte alignment of float
+    metadata (k, s, scales) and the element alignment of pack pointers: all
+    rejected on the host (these calls never reach the device)."""
+    from quantized_optimizer_states_b200._lib import CoatAdamwCfg
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    fake, odd4, odd2 = P(1 << 20), P((1 << 20) + 2), P((1 << 20) + 1)
+    cfg = CoatAdamwCfg(0.9, 0.999, 1e-4, 1e-8, 0.1, 10, 128, 0, 0, 0, 64.0, 0)
+    a8 = [fake] * 8
+    # metadata of the step (m_k, m_s, v_k, v_s are arguments 3, 4, 6, 7)
+    for i in (3, 4, 6, 7):
+        args = list(a8)
+        args[i] = odd4
+        assert lib.coat_adamw_fp8_step(*args, 16, ctypes.byref(cfg), None) == 2, i
+        assert lib.coat_adamw_fp8_step_fp32grad(*args, 16, ctypes.byref(cfg), None) == 2, i
+    f32 = lib.coat_adamw_fp8_step_fp32grad
+    assert f32(*a8, -1, ctypes.byref(cfg), None) == 1
+    assert f32(P((1 << 20) + 4), *a8[1:], 16, ctypes.byref(cfg), None) == 2
+    gd = lib.coat_adamw_fp8_step_guarded
+    assert gd(*a8, 16, ctypes.byref(cfg), None, None) == 1          # no skip word
+    assert gd(*a8, 16, ctypes.byref(cfg), odd4, None) == 2          # skip word misaligned
+    assert gd(*a8, -1, ctypes.byref(cfg), fake, None) == 1
+    q = lib.coat_quantize_state
+    assert q(fake, 16, 128, 0, 0, 64.0, 0, fake, odd4, fake, None) == 2
+    assert q(fake, 16, 128, 0, 0, 64.0, 0, fake, fake, odd4, None) == 2
+    d = lib.coat_dequant
+    assert d(fake, odd4, fake, 256, 128, 0, 0, fake, None) == 2
+    assert d(fake, None, odd4, 256, 128, 0, 0, fake, None) == 2
+    assert lib.coat_group_quant_1xG(fake, 4, 256, 256, 128, 0, fake, odd4, None) == 2
+    gs = lib.coat_group_scaling_quant_pertensor
+    assert gs(fake, 100, 128, 0, fake, 0, fake, odd4, None) == 2    # scale
+    assert gs(fake, 100, 128, 0, odd4, 0, fake, fake, None) == 2    # workspace
+    assert gs(fake, 100, 128, 0, fake, 3, fake, fake, None) == 1    # amax_precomputed
+    na = lib.coat_group_scaling_quant_pertensor_noalloc
+    assert na(fake, -1, 128, 0, fake, fake, None) == 1
+    assert na(None, 100, 128, 0, fake, fake, None) == 1
+    assert na(fake, 100, 96, 0, fake, fake, None) == 3
+    assert na(fake, 100, 128, 2, fake, fake, None) == 3
+    assert na(odd4, 100, 128, 0, fake, fake, None) == 2
+    assert na(fake, 100, 128, 0, fake, odd4, None) == 2
+    assert na(fake, 0, 128, 0, None, None, None) == 0
+    sw = lib.coat_swiglu_group_amax
+    assert sw(fake, fake, -1, 128, fake, fake, None, None) == 1
+    assert sw(fake, None, 64, 128, fake, fake, None, None) == 1
+    assert sw(fake, fake, 64, 100, fake, fake, None, None) == 3
+    assert sw(fake, odd4, 64, 128, fake, fake, None, None) == 2
+    assert sw(fake, fake, 64, 128, fake, odd4, None, None) == 2
+    assert sw(fake, fake, 64, 128, fake, fake, odd4, None) == 2
+    assert sw(None, None, 0, 128, None, None, None, None) == 0
+    enc = lib.coat_fp8_encode
+    assert enc(fake, -1, 0, fake, None) == 1
+    assert enc(fake, 16, 0, None, None) == 1
+    assert enc(fake, 16, 7, fake, None) == 3
+    assert enc(odd4, 16, 0, fake, None) == 2
+    cnt = lib.coat_count_nonfinite_bf16
+    assert cnt(fake, 16, None, None) == 1
+    assert cnt(None, 16, fake, None) == 1
+    assert cnt(odd4, 16, fake, None) == 2
+    assert cnt(fake, 16, odd2, None) == 2
+    nm = lib.coat_norm_group_amax
+    #      x     rows cols rms eps   weight bias  G    out   ga    tmax
+    assert nm(fake, -1, 256, 0, 1e-5, None, None, 128, fake, fake, None, None) == 1
+    assert nm(fake, 4, 256, 2, 1e-5, None, None, 128, fake, fake, None, None) == 1
+    assert nm(fake, 4, 256, 1, 1e-5, None, fake, 128, fake, fake, None, None) == 1  # RMS + bias
+    assert nm(fake, 4, 256, 0, -1.0, None, None, 128, fake, fake, None, None) == 1
+    assert nm(fake, 4, 200, 0, 1e-5, None, None, 128, fake, fake, None, None) == 1  # G | cols
+    assert nm(fake, 4, 256, 0, 1e-5, None, None, 96, fake, fake, None, None) == 3
+    assert nm(fake, 4, 32768, 0, 1e-5, None, None, 128, fake, fake, None, None) == 3
+    assert nm(odd4, 4, 256, 0, 1e-5, None, None, 128, fake, fake, None, None) == 2
+    assert nm(fake, 4, 256, 0, 1e-5, odd2, None, 128, fake, fake, None, None) == 2
+    assert nm(fake, 4, 256, 0, 1e-5, None, None, 128, fake, fake, odd2, None) == 2
+    assert nm(fake, 0, 256, 0, 1e-5, None, None, 128, None, None, None, None) == 0
+    st = lib.coat_state_stats
+    assert st(fake, odd4, fake, 64, 128, 0, fake, None) == 2       # k
+    assert st(fake, fake, odd4, 64, 128, 0, fake, None) == 2       # s
+
+    def tab(*v):
+        return (I64 * len(v))(*v)
+
+    pk, up = lib.coat_pack_bf16, lib.coat_unpack_bf16
+    f32src = (P * 2)(1 << 20, (1 << 21) + 2)          # second float32 source 2 bytes off
+    assert pk(f32src, tab(8, 8), tab(0, 16), 2, 1, fake, 64, None) == 2
+    bsrc = (P * 2)(1 << 20, (1 << 21) + 1)            # a BF16 source on an odd byte
+    assert pk(bsrc, tab(8, 8), tab(0, 16), 2, 0, fake, 64, None) == 2
+    assert up(fake, tab(8, 8), tab(0, 16), 2, bsrc, 64, None) == 2

@@ -133,12 +133,33 @@ class CoatAdamW(torch.optim.Optimizer):
         super().__init__(params, defaults)
         self.skip_nonfinite = skip_nonfinite
         self.skipped_steps = 0
+        self._flat_grads = flat_grads
         self._flat: list[_FlatGroup] = [self._build(g) for g in self.param_groups]
-        if flat_grads:
-            for fg in self._flat:
-                if not fg.bf16_params:
-                    fg.grad32 = torch.zeros(fg.n, dtype=torch.float32, device=fg.master.device)
-                    self._attach_grad_views(fg)
+
+    def add_param_group(self, param_group):
+        """torch.optim's add_param_group, with the group's COAT settings
+        checked first (v_fmt may be given by name); a group added after
+        construction gets its flat buffers at once -- step() walks one
+        _FlatGroup per parameter group, in the same order -- or, if they
+        cannot be built, is not added."""
+        param_group = dict(param_group)
+        if "v_fmt" in param_group:
+            if param_group["v_fmt"] not in _FMT:
+                raise ValueError("v_fmt must be 'e4m3' or 'e5m2'")
+            param_group["v_fmt"] = _FMT[param_group["v_fmt"]]
+        if "group_size" in param_group:
+            _check_group_size(param_group["group_size"])
+        if param_group.get("k_range", 0) not in (0, 1):
+            raise ValueError("k_range must be 0 (E4M3's range) or 1 (the storage format's)")
+        if not param_group.get("k_max", 0.0) >= 0.0:
+            raise ValueError("k_max must be >= 0 (0: no clamp)")
+        super().add_param_group(param_group)
+        if hasattr(self, "_flat"):
+            try:
+                self._flat.append(self._build(self.param_groups[-1]))
+            except Exception:
+                self.param_groups.pop()
+                raise
 
     # ---- flat buffers --------------------------------------------------------
 
@@ -167,7 +188,7 @@ class CoatAdamW(torch.optim.Optimizer):
                     # the parameter becomes a view of the master buffer
                     p.data = master[off:off + p.numel()].view_as(p)
         z8 = lambda: torch.zeros(n, dtype=torch.uint8, device=dev)  # noqa: E731
-        return _FlatGroup(
+        fg = _FlatGroup(
             params=ps, offsets=offsets, n=n, master=master,
             grad=None,
             m_code=z8(), v_code=z8(),
@@ -176,6 +197,10 @@ class CoatAdamW(torch.optim.Optimizer):
             v_k=torch.ones(ng, dtype=torch.float32, device=dev),
             v_s=torch.zeros(ng, dtype=torch.float32, device=dev),
             bf16_params=bf16, table=_lib.PackTable([p.numel() for p in ps], offsets))
+        if self._flat_grads and not bf16:
+            fg.grad32 = torch.zeros(n, dtype=torch.float32, device=dev)
+            self._attach_grad_views(fg)
+        return fg
 
     def _attach_grad_views(self, fg: _FlatGroup):
         for p, off in zip(fg.params, fg.offsets):

@@ -114,11 +114,22 @@ def _stream(stream):
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
+def _on_current_device(t, what):
+    """The kernels run on the current CUDA device; a tensor of another device
+    would be an illegal address there, so it is refused on the host."""
+    import torch
+    cur = torch.cuda.current_device()
+    if t.get_device() != cur:
+        raise ValueError(f"{what} is on {t.device} but the current device is cuda:{cur} "
+                         f"(call under torch.cuda.device({t.device}))")
+
+
 def _ptr(t, dtype=None, what="tensor"):
     if t is None:
         return None
     if not t.is_cuda:
         raise ValueError(f"{what} must be a CUDA tensor")
+    _on_current_device(t, what)
     if not t.is_contiguous():
         raise ValueError(f"{what} must be contiguous")
     if dtype is not None and t.dtype != dtype:
@@ -133,6 +144,7 @@ def _slot(t):
     import torch
     if t.dtype != torch.float32 or not t.is_cuda or t.numel() < 1:
         raise ValueError("tensor_amax must be a float32 CUDA tensor of at least one element")
+    _on_current_device(t, "tensor_amax")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -232,6 +244,7 @@ def coat_group_quant_1xG(x, q, scale, *, group_size: int = 128, fmt: int = COAT_
     rows, cols = x.shape
     if not x.is_cuda:
         raise ValueError("x must be a CUDA tensor")
+    _on_current_device(x, "x")
     if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
         raise ValueError("x must hold BF16 bit patterns")
     st = load().coat_group_quant_1xG(
@@ -354,6 +367,8 @@ def coat_pack_bf16(srcs, table: PackTable, dst, *, stream=None):
     for t in srcs:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("sources must be contiguous CUDA tensors")
+        if t is not None:
+            _on_current_device(t, "source")
     src_f32 = int(dtypes == {torch.float32})
     _check("coat_pack_bf16", load().coat_pack_bf16(
         table.pointers(srcs), table.numel, table.offset, table.count, src_f32,
@@ -366,7 +381,7 @@ def coat_unpack_bf16(src, table: PackTable, dsts, *, stream=None):
     for t in dsts:
         if t is None or not t.is_cuda or not t.is_contiguous():
             raise ValueError("destinations must be contiguous CUDA tensors")
-        _u16(t, "destination")
+        _u16(t, "destination")     # (checks the device too)
     import torch
     _check("coat_unpack_bf16", load().coat_unpack_bf16(
         _ptr(src, torch.float32, "src"), table.numel, table.offset, table.count,

@@ -238,3 +238,28 @@ def test_more_argument_checks_and_metadata_alignment(lib):
     bsrc = (P * 2)(1 << 20, (1 << 21) + 1)            # a BF16 source on an odd byte
     assert pk(bsrc, tab(8, 8), tab(0, 16), 2, 0, fake, 64, None) == 2
     assert up(fake, tab(8, 8), tab(0, 16), 2, bsrc, 64, None) == 2
+
+
+def test_tensors_of_another_device_are_refused(monkeypatch):
+    """The binding refuses a tensor that is not on the current CUDA device
+    (the kernel would run on the current device and fault on its address).
+    Checked with a stand-in tensor: this machine needs no GPU for it."""
+    import torch
+    from quantized_optimizer_states_b200 import _lib
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+
+    class OnDevice1:
+        device = "cuda:1"
+
+        def get_device(self):
+            return 1
+
+    class OnDevice0(OnDevice1):
+        device = "cuda:0"
+
+        def get_device(self):
+            return 0
+
+    with pytest.raises(ValueError, match="current device is cuda:0"):
+        _lib._on_current_device(OnDevice1(), "x")
+    _lib._on_current_device(OnDevice0(), "x")

@@ -252,28 +252,34 @@ class CoatAdamW(torch.optim.Optimizer):
             with torch.enable_grad():
                 loss = closure()
         for group, fg in zip(self.param_groups, self._flat):
-            direct = (fg.grad32 is not None and not self.skip_nonfinite
-                      and self._grads_are_views(fg))
-            if not direct:
-                self._gather_grads(fg)
-            if self.skip_nonfinite:
-                count = torch.zeros(1, dtype=torch.int32, device=fg.grad.device)
-                _lib.coat_count_nonfinite_bf16(fg.grad, count)
-                if int(count.item()) != 0:
-                    self.skipped_steps += 1
-                    continue
-            fg.step += 1
-            b1, b2 = group["betas"]
-            _lib.coat_adamw_fp8_step(
-                fg.master, fg.grad32 if direct else fg.grad, fg.m_code, fg.m_k, fg.m_s,
-                fg.v_code, fg.v_k, fg.v_s,
-                beta1=b1, beta2=b2, lr=group["lr"], eps=group["eps"],
-                weight_decay=group["weight_decay"], step=fg.step,
-                group_size=group["group_size"], v_fmt=group["v_fmt"],
-                k_range=group["k_range"], k_max=group["k_max"])
-            if fg.bf16_params:
-                self._write_back_bf16(fg)
+            # each group's launches go to its own device (and that device's
+            # current stream), whatever device is current
+            with torch.cuda.device(fg.master.device):
+                self._step_group(group, fg)
         return loss
+
+    def _step_group(self, group, fg: _FlatGroup):
+        direct = (fg.grad32 is not None and not self.skip_nonfinite
+                  and self._grads_are_views(fg))
+        if not direct:
+            self._gather_grads(fg)
+        if self.skip_nonfinite:
+            count = torch.zeros(1, dtype=torch.int32, device=fg.grad.device)
+            _lib.coat_count_nonfinite_bf16(fg.grad, count)
+            if int(count.item()) != 0:
+                self.skipped_steps += 1
+                return
+        fg.step += 1
+        b1, b2 = group["betas"]
+        _lib.coat_adamw_fp8_step(
+            fg.master, fg.grad32 if direct else fg.grad, fg.m_code, fg.m_k, fg.m_s,
+            fg.v_code, fg.v_k, fg.v_s,
+            beta1=b1, beta2=b2, lr=group["lr"], eps=group["eps"],
+            weight_decay=group["weight_decay"], step=fg.step,
+            group_size=group["group_size"], v_fmt=group["v_fmt"],
+            k_range=group["k_range"], k_max=group["k_max"])
+        if fg.bf16_params:
+            self._write_back_bf16(fg)
 
     # ---- inspection ------------------------------------------------------------
 
@@ -286,8 +292,9 @@ class CoatAdamW(torch.optim.Optimizer):
         vf = self.param_groups[group_index]["v_fmt"]
         m = torch.empty(fg.n, dtype=torch.float32, device=fg.master.device)
         v = torch.empty_like(m)
-        _lib.coat_dequant(fg.m_code, fg.m_k, fg.m_s, m, group_size=G, fmt=_lib.COAT_E4M3)
-        _lib.coat_dequant(fg.v_code, fg.v_k, fg.v_s, v, group_size=G, fmt=vf)
+        with torch.cuda.device(fg.master.device):
+            _lib.coat_dequant(fg.m_code, fg.m_k, fg.m_s, m, group_size=G, fmt=_lib.COAT_E4M3)
+            _lib.coat_dequant(fg.v_code, fg.v_k, fg.v_s, v, group_size=G, fmt=vf)
         return m, v
 
     def state_stats(self, group_index: int = 0) -> dict:
@@ -296,9 +303,11 @@ class CoatAdamW(torch.optim.Optimizer):
         fg = self._flat[group_index]
         G = self.param_groups[group_index]["group_size"]
         vf = self.param_groups[group_index]["v_fmt"]
-        return {"m": _lib.coat_state_stats(fg.m_code, fg.m_k, fg.m_s, group_size=G,
-                                           fmt=_lib.COAT_E4M3),
-                "v": _lib.coat_state_stats(fg.v_code, fg.v_k, fg.v_s, group_size=G, fmt=vf)}
+        with torch.cuda.device(fg.master.device):
+            return {"m": _lib.coat_state_stats(fg.m_code, fg.m_k, fg.m_s, group_size=G,
+                                               fmt=_lib.COAT_E4M3),
+                    "v": _lib.coat_state_stats(fg.v_code, fg.v_k, fg.v_s, group_size=G,
+                                               fmt=vf)}
 
     def flat_master(self, group_index: int = 0) -> torch.Tensor:
         return self._flat[group_index].master
@@ -328,4 +337,5 @@ class CoatAdamW(torch.optim.Optimizer):
                     getattr(fg, k).copy_(saved[k].to(getattr(fg, k).device))
                 fg.step = int(saved["step"])
                 if fg.bf16_params:
-                    self._write_back_bf16(fg)
+                    with torch.cuda.device(fg.master.device):
+                        self._write_back_bf16(fg)

@@ -39,10 +39,11 @@ def shard_length(n: int, group_size: int, world: int) -> int:
 
 
 def _coat_step(shard: "Zero1Shard", grad_shard: torch.Tensor, t: int, hyper: dict):
-    _lib.coat_adamw_fp8_step(
-        shard.master, grad_shard, shard.m_code, shard.m_k, shard.m_s, shard.v_code, shard.v_k,
-        shard.v_s, step=t, group_size=shard.group_size, v_fmt=shard.v_fmt,
-        k_range=shard.k_range, k_max=shard.k_max, **hyper)
+    with torch.cuda.device(shard.master.device):      # the shard's own device
+        _lib.coat_adamw_fp8_step(
+            shard.master, grad_shard, shard.m_code, shard.m_k, shard.m_s, shard.v_code,
+            shard.v_k, shard.v_s, step=t, group_size=shard.group_size, v_fmt=shard.v_fmt,
+            k_range=shard.k_range, k_max=shard.k_max, **hyper)
 
 
 class Zero1Shard:

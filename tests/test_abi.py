@@ -263,3 +263,29 @@ def test_tensors_of_another_device_are_refused(monkeypatch):
     with pytest.raises(ValueError, match="current device is cuda:0"):
         _lib._on_current_device(OnDevice1(), "x")
     _lib._on_current_device(OnDevice0(), "x")
+
+
+def test_ctypes_structures_match_the_header(tmp_path):
+    """The binding's ctypes mirrors of coat_adamw_cfg_t and
+    coat_state_stats_t have the C structs' size and field offsets (a C
+    program built against include/coat.h with gcc prints them)."""
+    import subprocess
+    from quantized_optimizer_states_b200._lib import CoatAdamwCfg, CoatStateStats
+    structs = {"coat_adamw_cfg_t": CoatAdamwCfg, "coat_state_stats_t": CoatStateStats}
+    lines = ["#include <stddef.h>", "#include <stdio.h>", '#include "coat.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-I", os.path.join(ROOT, "include"), "-o",
+                    str(exe), str(src)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    got = {tuple(ln.split()[:2]): int(ln.split()[2]) for ln in out.splitlines()}
+    for cname, cls in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for field, _ in cls._fields_:
+            assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)

@@ -289,3 +289,40 @@ def test_ctypes_structures_match_the_header(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(cls), cname
         for field, _ in cls._fields_:
             assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)
+
+
+def _c_kind(decl: str) -> str:
+    decl = decl.strip()
+    if "*" in decl:
+        return "ptr"
+    base = decl.replace("const ", "").split()[0]
+    return {"int64_t": "i64", "int32_t": "i32", "coat_status_t": "i32", "float": "f32",
+            "uint32_t": "u32", "size_t": "u64"}[base]
+
+
+def _ctypes_kind(t) -> str:
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(t, "_type_") and t.__name__.startswith("LP_"):
+        return "ptr"
+    return {ctypes.c_int64: "i64", ctypes.c_int32: "i32", ctypes.c_float: "f32",
+            ctypes.c_uint32: "u32", ctypes.c_uint64: "u64"}[t]
+
+
+def test_binding_signatures_match_the_header():
+    """Every prototype of include/coat.h has a SIGNATURES entry in the binding
+    with the same number of arguments and the same kind of each (pointer,
+    32/64-bit integer, float) and of the result, and the other way round: a
+    stale entry would pass its arguments in the wrong registers."""
+    from quantized_optimizer_states_b200._lib import SIGNATURES
+    with open(os.path.join(ROOT, "include", "coat.h")) as f:
+        text = re.sub(r"/\*.*?\*/", " ", f.read(), flags=re.S)
+    protos = {}
+    for m in re.finditer(r"(coat_status_t|int64_t|int32_t|const\s+char\s*\*)\s*(coat_\w+)\s*"
+                         r"\(([^)]*)\)\s*;", text):
+        res, name, params = m.group(1), m.group(2), m.group(3).strip()
+        args = [] if params in ("", "void") else [p for p in params.split(",")]
+        protos[name] = ("ptr" if "*" in res else _c_kind(res), [_c_kind(a) for a in args])
+    assert set(protos) == set(SIGNATURES), set(protos) ^ set(SIGNATURES)
+    for name, (res, args) in SIGNATURES.items():
+        want_res, want_args = protos[name]
+        assert _ctypes_kind(res) == want_res, name
+        assert [_ctypes_kind(a) for a in args] == want_args, name

@@ -43,3 +43,32 @@ def test_peaks_come_from_the_measured_file():
     peaks, kind = bench.measured_peaks()
     assert kind in ("measured", "fallback")
     assert peaks["hbm_gbs"] > 1000
+
+
+def test_clock_samples_are_summarised(tmp_path, monkeypatch):
+    """The clock record of the timed region: median SM clock, the maximum,
+    and every throttle reason seen active at least once (the lines are
+    nvidia-smi's csv,noheader,nounits output; malformed lines are skipped)."""
+    monkeypatch.setenv("COAT_BENCH_LOG_DIR", str(tmp_path))
+    s = bench.ClockSampler(None)
+
+    class Done:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    rows = ["1965, 1965, 900.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+            "1800, 1965, 1000.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+            "1750, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+            "garbage line",
+            "[N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active"]
+    with open(s.path, "w") as f:
+        f.write("\n".join(rows) + "\n")
+    s.proc, s.out = Done(), open(os.devnull, "w")
+    got = s.stop()
+    assert got == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "samples": 3,
+                   "reasons": ["sw_power_cap"]}
+    s2 = bench.ClockSampler(None)
+    assert s2.stop() is None                    # never started (no nvidia-smi): no record

@@ -72,3 +72,25 @@ def test_clock_samples_are_summarised(tmp_path, monkeypatch):
                    "reasons": ["sw_power_cap"]}
     s2 = bench.ClockSampler(None)
     assert s2.stop() is None                    # never started (no nvidia-smi): no record
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the oracle on the host cores, no GPU)
+    prints one JSON line with the keys the bench contract asks of that arm."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2",
+                        "--warmup", "1", "--ref-sample", "16384"], cwd=bench.ROOT,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "params/s" and line["higher_is_better"] is True
+    assert line["steps"] == 2 and line["warmup"] == 1 and line["value"] > 0
+    assert line["config"]["group_size"] == 128 and line["config"]["v_fmt"] == "e4m3"
+    assert "16384" in line["config"]["workload"]
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "params/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

@@ -119,21 +119,32 @@ class Zero1Shard:
         step uses."""
         return self.reduce_gradient_f32(grad).to(torch.bfloat16)
 
-    def gather_params(self) -> torch.Tensor:
-        """The full updated FP32 parameter buffer (first n elements)."""
-        full = torch.empty(self.world * self.L, dtype=torch.float32, device=self.master.device)
+    def gather_params(self, dtype: torch.dtype = torch.float32) -> torch.Tensor:
+        """The full updated parameter buffer (first n elements): the FP32
+        master weights, or, with dtype=torch.bfloat16, each rank's shard
+        rounded to BF16 (nearest even) before the all-gather, which moves
+        half the bytes -- what a model that holds BF16 weights needs."""
+        if dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError("parameters are gathered as float32 or bfloat16")
+        src = self.master if dtype == torch.float32 else self.master.to(torch.bfloat16)
+        full = torch.empty(self.world * self.L, dtype=dtype, device=self.master.device)
         if self.world > 1:
-            dist.all_gather_into_tensor(full, self.master, group=self.pg)
+            # BF16 moves as pairs of 16-bit patterns in 32-bit words (a shard
+            # is a whole number of 16-element units), which every backend carries
+            view = torch.int32 if dtype == torch.bfloat16 else dtype
+            dist.all_gather_into_tensor(full.view(view), src.view(view), group=self.pg)
         else:
-            full.copy_(self.master)
+            full.copy_(src)
         return full[:self.n]
 
-    def step(self, grad: torch.Tensor, t: int, hyper: dict, step_fn=None) -> torch.Tensor:
+    def step(self, grad: torch.Tensor, t: int, hyper: dict, step_fn=None,
+             gather_dtype: torch.dtype = torch.float32) -> torch.Tensor:
         """One data-parallel step with this rank's full BF16 gradient `grad`;
-        returns the full updated parameters.  `step_fn(shard, grad_shard, t,
-        hyper)` replaces the CUDA step (the CPU tests pass the oracle)."""
+        returns the full updated parameters (FP32, or BF16 with
+        gather_dtype=torch.bfloat16).  `step_fn(shard, grad_shard, t, hyper)`
+        replaces the CUDA step (the CPU tests pass the oracle)."""
         if step_fn is None:
             _coat_step(self, self.reduce_gradient_f32(grad), t, hyper)  # rounded on load
         else:
             step_fn(self, self.reduce_gradient(grad), t, hyper)
-        return self.gather_params()
+        return self.gather_params(gather_dtype)

@@ -414,7 +414,9 @@ coat_status_t coat_state_stats(const uint8_t *code, const float *k, const float 
  * eps), var the mean squared deviation) or RMSNorm (rms = 1: y = x /
  * sqrt(mean(x^2) + eps)), times weight[c] and plus bias[c] (LayerNorm only)
  * when given, rounded to BF16; plus the maxima of |out| over every 1xG run
- * of each row.  Evaluated in binary32, with an error of about
+ * of each row.  Evaluated in binary32 (row sums in a fixed order, divided
+ * by cols with the correctly rounded quotient, so a row whose sum is exact
+ * -- a constant row, say -- gets its exact mean), with an error of about
  * 1e-6 x (|y| + |mean| / std) (x - mean carries the rounding of the mean):
  * the output is the correctly rounded norm except within that distance of
  * a BF16 rounding midpoint.
@@ -427,7 +429,7 @@ coat_status_t coat_state_stats(const uint8_t *code, const float *k, const float 
  *               the same G) with amax_precomputed != 0
  *   tensor_amax float32[1] or NULL: as for coat_swiglu_group_amax
  * Errors: INVALID_ARG (sizes, eps < 0 or not finite, rms not 0/1, bias with
- * rms), UNSUPPORTED (G, cols > 16384), MISALIGNED, CUDA.
+ * rms), UNSUPPORTED (G, cols > 16384, rows > 2^31 - 1), MISALIGNED, CUDA.
  */
 coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols, int32_t rms,
                                    float eps, const float *weight, const float *bias,

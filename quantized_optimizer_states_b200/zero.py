@@ -7,17 +7,30 @@ moments with their per-group k and s (COAT summary page, section
 boundaries, so each rank keeps 1/world of it.  One step:
 
   1. reduce-scatter of the gradients: each rank receives, over its shard,
-     the mean of all ranks' gradients (summed in binary32 by the collective,
-     divided by the rank count, rounded to BF16 nearest-even);
-  2. the COAT step on the shard (one `coat_adamw_fp8_step` call, which takes
-     the binary32 mean and rounds it to BF16 as it loads it, so no separate
-     conversion pass runs);
-  3. all-gather of the updated master weights.
+     the mean of all ranks' gradients.  By default the collective sums the
+     BF16 gradients themselves (2 bytes per parameter on the wire; the
+     collective rounds its partial sums to BF16) and the sum is divided by
+     the rank count in BF16.  With reduce_dtype=torch.float32 the BF16
+     values are widened and summed in binary32 instead (4 bytes per
+     parameter on the wire), one shard-sized chunk at a time so the binary32
+     staging buffer stays bounded, and the mean is rounded to BF16 as the
+     step loads it;
+  2. the COAT step on the shard (one `coat_adamw_fp8_step` call);
+  3. all-gather of the updated master weights (FP32, or each shard rounded
+     to BF16 first: half the bytes).
 
 No 1xG group straddles two shards, so the sharded step computes exactly
 what a single-rank step over the whole buffer computes on the reduced
 gradient.  The collectives go through the default (or given) process group:
 NCCL over NVLink/NVSwitch on B200 nodes, gloo on CPU for the tests.
+
+Costs per parameter of the flat buffer, per rank and step, with W ranks and
+a ring collective: the reduce-scatter moves (W - 1)/W x 2 bytes each way
+(BF16) or (W - 1)/W x 4 bytes (binary32); the all-gather (W - 1)/W x 4
+bytes (FP32 parameters) or x 2 (BF16).  A gradient whose length is not
+W x L (L = shard length) is first copied into a padded buffer (2 bytes read,
+2 written); callers that allocate their flat gradient with
+`padded_numel` elements skip that copy.
 """
 from __future__ import annotations
 
@@ -52,11 +65,16 @@ class Zero1Shard:
 
     `theta` is the full FP32 parameter buffer (the same on every rank); the
     rank keeps a copy of its shard as master weights.  Fresh moments are
-    all-zero groups (codes 0, k = 1, s = 0).
+    all-zero groups (codes 0, k = 1, s = 0).  `reduce_dtype` selects the
+    gradient reduce-scatter: BF16 (default) or binary32.
     """
 
     def __init__(self, theta: torch.Tensor, *, group_size: int = 128, v_fmt: int = 0,
-                 k_range: int = 0, k_max: float = 64.0, group=None):
+                 k_range: int = 0, k_max: float = 64.0, group=None,
+                 reduce_dtype: torch.dtype = torch.bfloat16):
+        if reduce_dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("gradients are reduced as bfloat16 or float32")
+        self.reduce_dtype = reduce_dtype
         self.pg = group
         self.world = dist.get_world_size(group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
@@ -101,22 +119,71 @@ class Zero1Shard:
                     raise ValueError(f"checkpoint tensor {k} has the wrong shape or type")
                 dst.copy_(sd[k].to(dst.device))
 
+    @property
+    def padded_numel(self) -> int:
+        """Length of a flat gradient the reduce-scatter takes without a copy:
+        world x L (the first n elements are the parameters', the rest zero)."""
+        return self.world * self.L
+
+    def _padded(self, grad: torch.Tensor) -> torch.Tensor:
+        g = grad.reshape(-1)
+        if g.numel() == self.padded_numel:
+            return g
+        if g.numel() != self.n:
+            raise ValueError(f"gradient has {g.numel()} elements, expected {self.n} "
+                             f"or {self.padded_numel}")
+        buf = getattr(self, "_gpad", None)
+        if buf is None or buf.dtype != g.dtype or buf.device != g.device:
+            buf = torch.zeros(self.padded_numel, dtype=g.dtype, device=g.device)
+            self._gpad = buf
+        buf[:self.n].copy_(g)
+        return buf
+
+    # binary32 reduce-scatter: elements per chunk of a rank's shard
+    F32_CHUNK = 1 << 24
+
     def reduce_gradient_f32(self, grad: torch.Tensor) -> torch.Tensor:
         """Mean over ranks of the full BF16 gradients, this rank's shard, in
-        binary32 (sum by the collective, division by the rank count)."""
-        full = torch.zeros(self.world * self.L, dtype=torch.float32, device=grad.device)
-        full[:self.n].copy_(grad.reshape(-1))
+        binary32: the values are widened and summed in binary32 by the
+        collective, chunk by chunk (a staging buffer of world x F32_CHUNK
+        floats), and divided by the rank count."""
+        g = self._padded(grad).view(self.world, self.L)
         part = torch.empty(self.L, dtype=torch.float32, device=grad.device)
-        if self.world > 1:
-            dist.reduce_scatter_tensor(part, full, op=dist.ReduceOp.SUM, group=self.pg)
-            part.div_(float(self.world))
-        else:
-            part.copy_(full)
+        if self.world == 1:
+            part.copy_(g[0])
+            return part
+        C = min(self.F32_CHUNK, self.L)
+        stage = torch.empty(self.world * C, dtype=torch.float32, device=grad.device)
+        for off in range(0, self.L, C):
+            c = min(C, self.L - off)
+            st = stage[:self.world * c].view(self.world, c)
+            st.copy_(g[:, off:off + c])
+            dist.reduce_scatter_tensor(part[off:off + c], stage[:self.world * c],
+                                       op=dist.ReduceOp.SUM, group=self.pg)
+        part.div_(float(self.world))
+        return part
+
+    def reduce_gradient_bf16(self, grad: torch.Tensor) -> torch.Tensor:
+        """Mean over ranks of the full BF16 gradients, this rank's shard, with
+        the reduce-scatter on the BF16 values themselves (the collective's
+        partial sums are BF16) and the division by the rank count in BF16."""
+        g = self._padded(grad)
+        if g.dtype != torch.bfloat16:
+            raise ValueError("the BF16 reduce-scatter takes a BF16 gradient")
+        part = torch.empty(self.L, dtype=torch.bfloat16, device=grad.device)
+        if self.world == 1:
+            part.copy_(g)
+            return part
+        dist.reduce_scatter_tensor(part, g, op=dist.ReduceOp.SUM, group=self.pg)
+        part.div_(float(self.world))
         return part
 
     def reduce_gradient(self, grad: torch.Tensor) -> torch.Tensor:
-        """The same mean rounded to BF16 (nearest even): the gradient the
-        step uses."""
+        """The reduced gradient the step uses, as BF16: the BF16 reduce-scatter
+        (reduce_dtype torch.bfloat16) or the binary32 mean rounded to BF16
+        nearest-even (reduce_dtype torch.float32)."""
+        if self.reduce_dtype == torch.bfloat16:
+            return self.reduce_gradient_bf16(grad)
         return self.reduce_gradient_f32(grad).to(torch.bfloat16)
 
     def gather_params(self, dtype: torch.dtype = torch.float32) -> torch.Tensor:
@@ -143,8 +210,10 @@ class Zero1Shard:
         returns the full updated parameters (FP32, or BF16 with
         gather_dtype=torch.bfloat16).  `step_fn(shard, grad_shard, t, hyper)`
         replaces the CUDA step (the CPU tests pass the oracle)."""
-        if step_fn is None:
-            _coat_step(self, self.reduce_gradient_f32(grad), t, hyper)  # rounded on load
-        else:
+        if step_fn is not None:
             step_fn(self, self.reduce_gradient(grad), t, hyper)
+        elif self.reduce_dtype == torch.bfloat16:
+            _coat_step(self, self.reduce_gradient_bf16(grad), t, hyper)
+        else:
+            _coat_step(self, self.reduce_gradient_f32(grad), t, hyper)  # rounded on load
         return self.gather_params(gather_dtype)

@@ -173,3 +173,75 @@ def test_two_gloo_ranks_resume_from_a_checkpoint_bit_for_bit():
     for rank, same, rejected in res:
         assert same, f"rank {rank}: resumed run (or its BF16 gather) differs"
         assert rejected, f"rank {rank}: mismatched layout accepted"
+
+
+def _reduce_worker(rank, world, port, n, q):
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        grads = _exact_grads(n, world)
+        g = torch.from_numpy(grads[rank]).to(torch.bfloat16)
+        f32 = zero.Zero1Shard(torch.zeros(n), group_size=G, reduce_dtype=torch.float32)
+        f32.F32_CHUNK = 100          # several chunks, the last one ragged
+        a = f32.reduce_gradient_f32(g)
+        padded = torch.zeros(f32.padded_numel, dtype=torch.bfloat16)
+        padded[:n] = g
+        b = f32.reduce_gradient_f32(padded)
+        bf = zero.Zero1Shard(torch.zeros(n), group_size=G)
+        c = bf.reduce_gradient(g)
+        q.put((rank, a.numpy().copy(), b.numpy().copy(),
+               c.float().numpy().copy(), c.dtype == torch.bfloat16, f32.L))
+    finally:
+        dist.destroy_process_group()
+
+
+def _exact_grads(n, world):
+    """BF16 gradients whose binary32 sums over ranks are exact (multiples of
+    2^-16 below 1 in magnitude), so the binary32 mean is order-independent."""
+    rng = np.random.default_rng(7)
+    k = rng.integers(-60000, 60000, (world, n))
+    return (k * 2.0 ** -16).astype(np.float32)
+
+
+def test_reduce_scatter_bf16_and_chunked_binary32_three_gloo_ranks():
+    """Three gloo ranks: the binary32 reduce-scatter, done in chunks of 100
+    elements of the shard, gives each rank its shard of the binary32 mean of
+    the BF16 gradients exactly, whether the gradient is passed with n
+    elements or padded to world x L; the BF16 reduce-scatter gives BF16
+    values within 2 BF16 steps of that mean (its partial sums are rounded
+    to BF16)."""
+    import torch
+    world, n = 3, 5 * 128 + 77
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_reduce_worker, args=(r, world, port, n, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    grads = _exact_grads(n, world)
+    gb = torch.from_numpy(grads).to(torch.bfloat16).float().numpy().astype(np.float64)
+    L = res[0][5]
+    mean = np.zeros(world * L)
+    mean[:n] = gb.sum(axis=0) / world
+    mean32 = mean.astype(np.float32)
+    # BF16 keeps 8 significant bits (unit roundoff 2^-8): each rounding of a
+    # partial sum errs by at most 2^-8 of sum |g_i|, the division's by 2^-8 of
+    # the result
+    absum = np.zeros(world * L)
+    absum[:n] = np.abs(gb).sum(axis=0)
+    for rank, a, b, c, is_bf16, Lr in res:
+        assert Lr == L == zero.shard_length(n, G, world)
+        want = mean32[rank * L:(rank + 1) * L]
+        assert np.array_equal(a, want) and np.array_equal(b, want), f"rank {rank}"
+        assert is_bf16
+        bound = (world - 1) * 2.0 ** -8 * absum[rank * L:(rank + 1) * L] / world \
+            + 2.0 ** -8 * np.abs(want)
+        assert np.all(np.abs(c - want) <= bound), f"rank {rank}: BF16 mean too far"

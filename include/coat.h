@@ -78,6 +78,12 @@ typedef enum coat_fp8 {
 
 /* cfg.flags */
 #define COAT_FORCE_K1 0x1 /* ablation: k = 1 for every group (no expansion) */
+/* The step takes no `stats` argument and has no finite-check or statistics
+ * flags: the finite check is coat_count_nonfinite_bf16 followed by
+ * coat_adamw_fp8_step_guarded (a step that becomes a no-op when the count
+ * is nonzero, with no host round trip), and the per-state statistics are
+ * coat_state_stats -- separate calls, so the step kernel carries none of
+ * that counting. */
 
 /* Hyper-parameters and layout of one COAT AdamW step ([COAT] AdamW
  * section; [ATLAS] section 08). */
@@ -277,7 +283,10 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
  * library holds it until the process exits.  The first call on a device
  * resolves that array's address for the current device (a one-time,
  * non-allocating runtime query), so make the first call on each device
- * before any stream capture.  Every call shares the array: calls that
+ * before any stream capture.  The address is kept for the life of the
+ * process: after cudaDeviceReset (which gives the device a new context and
+ * the array a new address) this entry point must not be called again in
+ * that process.  Every call shares the array: calls that
  * overlap on the GPU (on different streams, or from different threads
  * without ordering) race on it and must be serialised by the caller.
  *   x      BF16 bits [n] (16-byte aligned)
@@ -457,13 +466,17 @@ int32_t coat_last_cuda_error(void);
 /* Streamed activation kernels (coat_group_quant_1xG on contiguous rows,
  * the cast of coat_group_scaling_quant_pertensor[_noalloc]) move
  * 4096-element tiles into shared memory with bulk asynchronous copies and
- * wait for each on an mbarrier.  Every such wait is
- * bounded: one that runs out abandons the rest of its block's tiles (their
- * outputs are then not written) and adds 1 to a device counter.
- * coat_bulk_wait_timeouts synchronises the current device, stores the
- * counter in *count (host pointer) and, if reset != 0, sets it to zero.
- * A non-zero count means outputs of the calls since the last reset are
- * incomplete.
+ * wait for each on an mbarrier.  Every such wait is bounded: one that runs
+ * out abandons the rest of its block's tiles (their outputs are then not
+ * written), waits (bounded again) for the block's copies still in flight,
+ * and adds 1 to a device counter.  coat_bulk_wait_timeouts synchronises the current device,
+ * stores the counter in *count (host pointer) and, if reset != 0, sets it
+ * to zero.  A non-zero count means outputs of the calls since the last
+ * reset are incomplete; treat the CUDA context as suspect too (if the
+ * second wait also ran out, a copy may still have been in flight when its
+ * block left).  The launches are asynchronous, so the calls themselves
+ * cannot report this: check the counter where it matters (the tests and
+ * bench.py do after every streamed run).
  * Errors: INVALID_ARG (count NULL), CUDA. */
 coat_status_t coat_bulk_wait_timeouts(uint32_t *count, int32_t reset);
 

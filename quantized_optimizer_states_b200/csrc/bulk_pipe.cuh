@@ -20,8 +20,11 @@
 // Every wait is bounded.  A wait that runs out counts itself in
 // g_bulk_wait_timeouts (read on the host through coat_bulk_wait_timeouts),
 // and the block then waits, again with a bound, for its copies still in
-// flight before it returns, so no copy lands in shared memory that a later
-// block owns.
+// flight before it returns, so that no copy lands in shared memory that a
+// later block owns -- as long as that second wait succeeds.  If it too
+// runs out, a copy may still be in flight when the block leaves: the
+// counter is nonzero either way, and a caller that sees it must treat the
+// outputs as incomplete and the context as suspect.
 #pragma once
 
 #include <atomic>

@@ -498,7 +498,9 @@ coat_status_t coat_group_scaling_quant_pertensor(const uint16_t *x, int64_t n,
     launch_pertensor_cast(p, fmt, s);
     return launch_status();
   }
-  if (cudaMemsetAsync(p.tensor_amax, 0, sizeof(uint32_t), s) != cudaSuccess) return launch_status();
+  // the tensor maximum accumulates with atomicMax from zero (a kernel, not a
+  // memset, so the launches stay one programmatic-dependent-launch chain)
+  launch_act_threads(coat::zero_word_kernel, 1u, 32u, 0, s, p.tensor_amax);
   if (amax_precomputed) {
     // one pass over the small intermediate: a few blocks per SM suffice
     const int64_t want = (ng + coat::kThreads - 1) / coat::kThreads;
@@ -853,7 +855,7 @@ extern "C" coat_status_t coat_group_scaling_quant_pertensor_noalloc(
   p.scale = scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the tensor maximum accumulates with atomicMax and must start at zero
-  if (cudaMemsetAsync(p.tensor_amax, 0, sizeof(uint32_t), s) != cudaSuccess) return launch_status();
+  launch_act_threads(coat::zero_word_kernel, 1u, 32u, 0, s, p.tensor_amax);
   launch_act(coat::group_amax_kernel, coat::act_blocks(n), 0, s, p);
   launch_pertensor_cast(p, fmt, s);
   return launch_status();

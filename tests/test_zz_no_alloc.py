@@ -5,9 +5,10 @@ serving process with a budget fixed at start-up, or a plug-in whose host
 framework owns every allocation.  coat_group_scaling_quant_pertensor_noalloc
 serves them: it uses scratch compiled into the library instead of a
 caller-supplied workspace.  These tests call it through the C ABI and check
-it against the workspace entry point, bit for bit, on consecutive calls
-(the shared scratch keeps the previous call's contents, so the second call
-checks that nothing leaks from the first).  This file is collected last.
+it, bit for bit, against the oracle's Group Scaling and against the
+workspace entry point, on consecutive calls (the shared scratch keeps the
+previous call's contents, so the second call checks that nothing leaks from
+the first).  This file is collected last.
 """
 import ctypes
 
@@ -54,7 +55,8 @@ def _without_workspace(lib, x, G, fmt):
     return q, s
 
 
-def test_noalloc_matches_workspace_variant_on_consecutive_calls(lib):
+def test_noalloc_matches_the_oracle_and_the_workspace_variant_on_consecutive_calls(lib, orc):
+    import numpy as np
     import torch
     # a large tensor first, then a smaller one whose maximum is far below the
     # first call's: stale scratch from call one would change call two
@@ -64,6 +66,10 @@ def test_noalloc_matches_workspace_variant_on_consecutive_calls(lib):
         q_ref, s_ref = _with_workspace(lib, x, G, fmt)
         q, s = _without_workspace(lib, x, G, fmt)
         torch.cuda.synchronize()
+        q_orc, s_orc, _ = orc.group_scaling_pertensor(
+            x.view(torch.int16).cpu().numpy().view(np.uint16), G, fmt)
+        assert s.item() == s_orc
+        assert np.array_equal(q.cpu().numpy(), q_orc)
         assert torch.equal(s, s_ref)
         assert torch.equal(q, q_ref)
 

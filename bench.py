@@ -8,9 +8,14 @@ k and scale, G = 128) resident in HBM.  Prints ONE JSON line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--v-fmt e4m3|e5m2]
   python bench.py --impl reference ...    # the CPU oracle on a bounded sample
 
-Multi-GPU (torchrun): every rank owns its own full parameter set (the step
-has no cross-rank exchange), so per-GPU work is fixed: weak scaling, value =
-parameters stepped by all ranks / max-over-ranks time.
+Multi-GPU (`--gpus N`, N > 1; started through torchrun by this script when
+it is not already running under it): the ZeRO-1 data-parallel step over one
+parameter set split at group boundaries -- BF16 reduce-scatter of every
+rank's full gradient, the fused step on each rank's 1/N shard, BF16
+all-gather of the updated parameters (quantized_optimizer_states_b200.zero).
+Total work is fixed as N grows: strong scaling, value = parameters of the
+set / max-over-ranks time.  `--workload ranks` only checks that all N ranks
+join the process group.
 """
 from __future__ import annotations
 
@@ -149,19 +154,54 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def host_cores() -> int:
+    """Host cores this process may run on (nproc)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def oracle_step_threads(x, st, G: int, v_fmt: int, threads: int, step: int = 10) -> float:
+    """One oracle step over a host sample split into `threads` group-aligned
+    slices, each stepped by its own thread (the oracle is a plain C call
+    through ctypes, which releases the GIL while it runs); returns seconds."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    from quantized_optimizer_states_b200 import inputs
+    n = x["theta"].size
+    ng = -(-n // G)
+    per = -(-ng // threads) * G
+    cuts = [(a, min(n, a + per)) for a in range(0, n, per)]
+
+    def run(ab):
+        a, b = ab
+        g0, g1 = a // G, -(-b // G)
+        oracle.adamw_fp8_step(x["theta"][a:b], x["grad"][a:b], st[0][a:b], st[1][g0:g1],
+                              st[2][g0:g1], st[3][a:b], st[4][g0:g1], st[5][g0:g1], step=step,
+                              group_size=G, v_fmt=v_fmt, **inputs.HYPER)
+
+    with ThreadPoolExecutor(max_workers=len(cuts)) as ex:
+        t0 = time.perf_counter()
+        list(ex.map(run, cuts))
+        return time.perf_counter() - t0
+
+
 def cpu_baseline(workload, G: int, sample: int, v_fmt: int):
-    """The oracle (single-threaded C) on the first `sample` parameters."""
+    """The oracle (plain single-threaded C, run as it stands) on the first
+    `sample` parameters: once on one thread, once split at group boundaries
+    over every host core."""
     import oracle
     from quantized_optimizer_states_b200 import inputs
     x = inputs.host_step_inputs(workload, sample)
     st = oracle.quantize_state(x["m0"], G, 0) + oracle.quantize_state(x["v0"], G, v_fmt)
-    t0 = time.perf_counter()
-    oracle.adamw_fp8_step(x["theta"], x["grad"], *st, step=10, group_size=G, v_fmt=v_fmt,
-                          **inputs.HYPER)
-    dt = time.perf_counter() - t0
-    return {"value": sample / dt, "unit": "params/s", "cores": oracle.threads_used(),
-            "kind": "oracle",
-            "sample": f"first {sample} parameters of the {workload.name} set, one step"}
+    one = oracle_step_threads(x, st, G, v_fmt, 1)
+    cores = host_cores()
+    allc = oracle_step_threads(x, st, G, v_fmt, cores)
+    return {"value": sample / allc, "unit": "params/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {sample} parameters of the {workload.name} set, one step, split "
+                      f"at group boundaries over {cores} threads",
+            "single_thread": {"value": sample / one, "cores": 1}}
 
 
 def run_reference(args):
@@ -177,14 +217,12 @@ def run_reference(args):
     sample = args.ref_sample
     x = inputs.host_step_inputs(w, sample)
     st = oracle.quantize_state(x["m0"], G, 0) + oracle.quantize_state(x["v0"], G, v_fmt)
-    th = x["theta"]
+    cores = host_cores()
     times = []
     for i in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        out = oracle.adamw_fp8_step(th, x["grad"], *st, step=10 + i, group_size=G, v_fmt=v_fmt,
-                                    **inputs.HYPER)
-        dt = time.perf_counter() - t0
-        th, st = out[0], out[1:7]
+        # the oracle on every host core (group-aligned slices, one per thread);
+        # each step starts from the same state, as the steps of one sample
+        dt = oracle_step_threads(x, st, G, v_fmt, cores, step=10 + i)
         if i >= args.warmup:
             times.append(dt)
     total = sum(times)
@@ -196,9 +234,10 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": f"olmo-7b set (bounded sample of {sample} parameters per step)",
                    "group_size": G, "m_fmt": "e4m3", "v_fmt": args.v_fmt},
-        "cpu_baseline": {"value": value, "unit": "params/s", "cores": oracle.threads_used(),
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": cores,
                          "kind": "oracle",
-                         "sample": f"first {sample} parameters of the olmo-7b set per step"},
+                         "sample": f"first {sample} parameters of the olmo-7b set per step, "
+                                   f"split at group boundaries over {cores} threads"},
         "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -209,28 +248,13 @@ def run_reference(args):
 ACT_RING = 8  # distinct activation tensors cycled by the activation bench
 
 
-def run_activations(args):
-    """The activation-side kernels on the activation workload (BF16 [16384,
-    2048], G = 128, E4M3): 1xG quantization, Group Scaling (standalone: steps
-    (i)-(iii)), the SwiGLU and LayerNorm producers with fused maxima, Group
-    Scaling's steps (ii)-(iii) after a producer, and dequantization.
-
-    Steady state: each kernel is launched back to back over a ring of
-    ACT_RING distinct input (and output) sets -- 8 x 64 MiB of BF16 input
-    alone, four times the 126 MB L2 -- so every launch reads its input from
-    HBM, and one pair of CUDA events brackets the K timed launches (the
-    event timer ticks in ~2 us steps on this part, too coarse for a single
-    20 us launch).  One JSON line: elements/s of the 1xG quantizer as the
-    headline; every kernel's time per launch, achieved GB/s and fraction of
-    the measured HBM copy bandwidth in `kernels`."""
+def measure_activations(dev, steps: int, warmup: int):
+    """Time the activation-side kernels on the activation workload (see
+    run_activations); returns (per-kernel results, clock summary, n, G,
+    peak, peak kind)."""
     import torch
     import quantized_optimizer_states_b200 as coat
-    from quantized_optimizer_states_b200 import build as coat_build
     from quantized_optimizer_states_b200 import inputs
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    coat_build.build()
-    coat.load()
     w0 = inputs.activations()
     G = w0.group_size
     n = w0.rows * w0.cols
@@ -289,24 +313,57 @@ def run_activations(args):
     sampler = ClockSampler(None)
     sampler.start()
     time.sleep(0.3)
+    coat.coat_bulk_wait_timeouts(reset=True)
     for name, (fn, bpe) in cases.items():
-        for i in range(max(args.warmup, ACT_RING)):
+        for i in range(max(warmup, ACT_RING)):
             fn(ring[i % ACT_RING])
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             fn(ring[i % ACT_RING])
         e1.record(stream)
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / args.steps
+        ms = e0.elapsed_time(e1) / steps
         gbs = bpe * n / (ms / 1e3) / 1e9
+        # a bounded wait that ran out leaves outputs unwritten: no number then
+        timeouts = coat.coat_bulk_wait_timeouts(reset=True)
         res[name] = {"ms": ms, "elements_per_s": n / (ms / 1e3), "GB/s": gbs,
-                     "frac_of_hbm": gbs / peak, "algorithmic_bytes_per_element": bpe}
+                     "frac_of_hbm": gbs / peak, "algorithmic_bytes_per_element": bpe,
+                     "bulk_wait_timeouts": timeouts}
+        if timeouts:
+            res[name].update(ms=None, elements_per_s=None, frac_of_hbm=None,
+                             error="bounded waits ran out: outputs incomplete")
     clocks = sampler.stop()
+    return res, clocks, n, G, peak, peak_kind
+
+
+def run_activations(args):
+    """The activation-side kernels on the activation workload (BF16 [16384,
+    2048], G = 128, E4M3): 1xG quantization, Group Scaling (standalone: steps
+    (i)-(iii)), the SwiGLU and LayerNorm producers with fused maxima, Group
+    Scaling's steps (ii)-(iii) after a producer, and dequantization.
+
+    Steady state: each kernel is launched back to back over a ring of
+    ACT_RING distinct input (and output) sets -- 8 x 64 MiB of BF16 input
+    alone, four times the 126 MB L2 -- so every launch reads its input from
+    HBM, and one pair of CUDA events brackets the K timed launches (the
+    event timer ticks in ~2 us steps on this part, too coarse for a single
+    20 us launch).  One JSON line: elements/s of the 1xG quantizer as the
+    headline; every kernel's time per launch, achieved GB/s and fraction of
+    the measured HBM copy bandwidth in `kernels`."""
+    import torch
+    import quantized_optimizer_states_b200 as coat
+    from quantized_optimizer_states_b200 import build as coat_build
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    coat_build.build()
+    coat.load()
+    res, clocks, n, G, peak, peak_kind = measure_activations(dev, args.steps, args.warmup)
     head = res["group_quant_1xG"]
     line = {"metric": "elements/s for 1xG FP8 activation quantization (BF16 [16384, 2048], G=128)",
             "value": head["elements_per_s"], "unit": "elements/s", "n_gpus": 1,
+            "valid": all(not r["bulk_wait_timeouts"] for r in res.values()),
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
@@ -318,10 +375,11 @@ def run_activations(args):
                          "frac": head["frac_of_hbm"], "traffic": recorded_act_traffic(n),
                          "peak_source": f"{peak_kind} copy bandwidth"},
             "kernels": res, "clocks": clocks,
-            # 1xG 1; GS standalone 2; SwiGLU 2 (zeroing the tensor-max slot, the
-            # producer); LayerNorm 1; GS after the producer 2 (step (ii), cast);
-            # the cast alone 1; dequant 1
-            "gpu_launches": args.steps * (1 + 2 + 2 + 1 + 2 + 1 + 1)}
+            # 1xG 1; GS standalone 3 (zeroing the tensor maximum, step (i), the
+            # cast); SwiGLU 2 (zeroing its tensor-maximum slot, the producer);
+            # LayerNorm 1; GS after the producer 2 (zeroing, the cast with step
+            # (ii) folded in); the cast alone 1; dequant 1
+            "gpu_launches": args.steps * (1 + 3 + 2 + 1 + 2 + 1 + 1)}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -409,7 +467,7 @@ def run_optimizer(args):
     return 0
 
 
-def main():
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -420,52 +478,330 @@ def main():
                          "workload specifies; e4m3 otherwise)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-sample", type=int, default=1 << 25)
-    ap.add_argument("--ref-sample", type=int, default=1 << 22)
+    ap.add_argument("--ref-sample", type=int, default=1 << 24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the records beside the headline (the other v format, the "
+                         "activation kernels)")
+    ap.add_argument("--variant-steps", type=int, default=10)
     ap.add_argument("--workload", default="olmo-7b",
-                    choices=["olmo-7b", "olmo-1b", "sweep", "activations", "optimizer"])
+                    choices=["olmo-7b", "olmo-1b", "sweep", "activations", "optimizer",
+                             "ranks"])
     ap.add_argument("--group-size", type=int, default=128, help="sweep workload only")
     ap.add_argument("--regime", default="late", choices=["early", "late", "typical"],
                     help="sweep workload only")
-    args = ap.parse_args()
+    ap.add_argument("--zero1", action="store_true",
+                    help="time the ZeRO-1 data-parallel step even on one GPU (a one-rank "
+                         "process group: the collectives reduce to copies)")
+    ap.add_argument("--launch-timeout", type=int, default=3600,
+                    help="seconds before the ranks started by --gpus N are stopped")
+    args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "coat":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.v_fmt is None:
         args.v_fmt = "e5m2" if args.workload == "olmo-1b" else "e4m3"
     if args.impl == "reference":
         return run_reference(args)
+    world = int(os.environ.get("WORLD_SIZE", "0"))
+    if args.gpus > 1 and world == 0:
+        # not started by torchrun: start the N ranks (one process per GPU) here
+        return launch_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv),
+                            args.launch_timeout)
+    if args.workload == "ranks":
+        return run_ranks(args)
     if args.workload == "activations":
         return run_activations(args)
     if args.workload == "optimizer":
         return run_optimizer(args)
+    if world > 1 or args.zero1:
+        return run_zero1(args)
+    return run_step(args)
 
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_command(n: int, argv: list[str], timeout_s: int, port: int) -> list[str]:
+    """torchrun over n local ranks running this script with the same
+    arguments, bounded by `timeout -k 60` (a last resort above the process
+    group's own timeout)."""
+    return ["timeout", "-k", "60", str(timeout_s), sys.executable, "-m",
+            "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port),
+            os.path.abspath(__file__), *argv]
+
+
+def launch_ranks(n: int, argv: list[str], timeout_s: int) -> int:
+    """`bench.py --gpus N` run without torchrun: start N ranks through
+    torchrun (rendezvous on 127.0.0.1) and return their exit status; rank 0
+    prints the JSON line.  NCCL's communicator set-up lines stay on
+    (NCCL_DEBUG=INFO, subsystem INIT) so the ranks can be counted in the log."""
+    env = dict(os.environ)
+    env.setdefault("NCCL_DEBUG", "INFO")
+    env.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+    return subprocess.run(launch_command(n, argv, timeout_s, free_port()), env=env).returncode
+
+
+def init_ranks(timeout_s: int = 300, single: bool = False):
+    """Join the process group torchrun set up: NCCL with one GPU per rank, or
+    gloo where there is no GPU; returns (world, rank, local rank).  With
+    `single`, a process not started by torchrun forms a one-rank group."""
     import torch
     import torch.distributed as dist
+    from datetime import timedelta
+    if single and "WORLD_SIZE" not in os.environ:
+        os.environ.update(WORLD_SIZE="1", RANK="0", LOCAL_RANK="0", MASTER_ADDR="127.0.0.1",
+                          MASTER_PORT=str(free_port()))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if (world > 1 or single) and not dist.is_initialized():
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=timeout_s),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timedelta(seconds=timeout_s))
+    return world, rank, local
+
+
+def run_ranks(args):
+    """--workload ranks: every rank joins the process group and adds one to
+    an all-reduce; rank 0 prints how many ranks took part (no kernels)."""
+    import torch
+    import torch.distributed as dist
+    world, rank, local = init_ranks()
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    joined = world
+    if world > 1:
+        t = torch.ones(1, dtype=torch.float32, device=dev)
+        dist.all_reduce(t)
+        joined = int(t.item())
+    if rank == 0:
+        print(json.dumps({"workload": "ranks", "n_gpus": world, "ranks_joined": joined,
+                          "backend": dist.get_backend() if world > 1 else None}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def step_workload(args, seed_offset: int = 0):
+    from quantized_optimizer_states_b200 import inputs
+    if args.workload == "olmo-7b":
+        return inputs.olmo_7b(seed=1237 + seed_offset, v_fmt=args.v_fmt)
+    if args.workload == "olmo-1b":
+        w = inputs.olmo_1b(seed=1235 + seed_offset)
+        w.v_fmt = args.v_fmt
+        return w
+    return inputs.sweep(args.group_size, args.v_fmt, args.regime, seed=1238 + seed_offset)
+
+
+def run_zero1(args):
+    """N > 1 ranks (one GPU each): the ZeRO-1 data-parallel step over ONE
+    parameter set split at group boundaries (zero.Zero1Shard): BF16
+    reduce-scatter of every rank's full gradient, coat_adamw_fp8_step on the
+    rank's 1/N shard, BF16 all-gather of the updated parameters.  Total work
+    is fixed as N grows (strong scaling); value = parameters of the set per
+    second of the slowest rank.  The three phases are timed with CUDA events
+    on the launching stream (the collectives are ordered on it)."""
+    import torch
+    import torch.distributed as dist
+    import quantized_optimizer_states_b200 as coat
+    from quantized_optimizer_states_b200 import inputs, zero
+    from quantized_optimizer_states_b200 import build as coat_build
+
+    world, rank, local = init_ranks(single=True)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        coat_build.build()
+    dist.barrier()
+    coat.load()
+    v_fmt = coat.COAT_E4M3 if args.v_fmt == "e4m3" else coat.COAT_E5M2
+    # every rank: the same parameters, its own gradient
+    w = step_workload(args)
+    n, G = w.n, w.group_size
+    hyper = dict(w.hyper)
+    theta, grad_unused, chunks = inputs.device_step_inputs(w, dev)
+    del grad_unused
+    shard = zero.Zero1Shard(theta, group_size=G, v_fmt=v_fmt)
+    del theta
+    L, lo = shard.L, rank * shard.L
+    for off, m0, v0 in chunks():          # initial states of this rank's shard
+        a, b = max(off, lo), min(off + m0.numel(), lo + L, n)
+        if a >= b:
+            continue
+        g0, g1 = (a - lo) // G, -(-(b - lo) // G)
+        coat.coat_quantize_state(m0[a - off:b - off], shard.m_code[a - lo:b - lo],
+                                 shard.m_k[g0:g1], shard.m_s[g0:g1], group_size=G,
+                                 fmt=coat.COAT_E4M3)
+        coat.coat_quantize_state(v0[a - off:b - off], shard.v_code[a - lo:b - lo],
+                                 shard.v_k[g0:g1], shard.v_s[g0:g1], group_size=G, fmt=v_fmt)
+    wg = step_workload(args, seed_offset=1000 * (rank + 1))
+    th_unused, g_rank, _ = inputs.device_step_inputs(wg, dev)
+    del th_unused
+    grad = torch.zeros(shard.padded_numel, dtype=torch.bfloat16, device=dev)
+    grad[:n].copy_(g_rank)             # the flat gradient, padded: no copy per step
+    del g_rank
+    torch.cuda.empty_cache()
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream(dev)
+    step_no = [w.step]
+    marks = []
+
+    def step(record=False):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
+        if record:
+            ev[0].record(stream)
+        g = shard.reduce_gradient_bf16(grad)
+        if record:
+            ev[1].record(stream)
+        zero._coat_step(shard, g, step_no[0], hyper)
+        if record:
+            ev[2].record(stream)
+        shard.gather_params(torch.bfloat16)
+        if record:
+            ev[3].record(stream)
+            marks.append(ev)
+        step_no[0] += 1
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(None) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = t0.elapsed_time(t1)
+    rs_ms = sum(e[0].elapsed_time(e[1]) for e in marks) / args.steps
+    st_ms = sum(e[1].elapsed_time(e[2]) for e in marks) / args.steps
+    ag_ms = sum(e[2].elapsed_time(e[3]) for e in marks) / args.steps
+    t = torch.tensor([total_ms, rs_ms, st_ms, ag_ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, rs_ms, st_ms, ag_ms = (float(x) for x in t.tolist())
+
+    # ---- end to end: each rank's gradient from pinned host memory every step ----
+    e2e = None
+    if args.e2e_steps > 0:
+        nchunks = 16
+        per = -(-n // nchunks)
+        host = torch.empty(per, dtype=torch.bfloat16, pin_memory=True)
+        host.copy_(grad[:per])
+        result = torch.empty(4, dtype=torch.float32, pin_memory=True)
+        torch.cuda.synchronize()
+
+        def e2e_step():
+            for a in range(0, n, per):
+                b = min(n, a + per)
+                grad[a:b].copy_(host[:b - a], non_blocking=True)
+            step()
+            result[0:1].copy_(shard.m_k[-1:], non_blocking=True)
+            result[1:2].copy_(shard.m_s[-1:], non_blocking=True)
+            result[2:3].copy_(shard.v_k[-1:], non_blocking=True)
+            result[3:4].copy_(shard.v_s[-1:], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = {"value": n * args.e2e_steps / (float(t.item()) / 1e3), "unit": "params/s",
+               "h2d_bytes_per_step": 2 * n * world, "d2h_bytes_per_step": 16 * world,
+               "what": "every rank's BF16 gradient copied from pinned host memory every step "
+                       "(16 chunks through one chunk-sized pinned staging buffer), then the "
+                       "ZeRO-1 step, then a 16-byte read-back of the last group's (k, s) pairs "
+                       "on every rank"}
+        del host
+
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        peak = float(peaks["hbm_gbs"])
+        achieved = bytes_per_param(G) * L / (st_ms / 1e3) / 1e9
+        # ring collectives: (N - 1)/N of the buffer leaves (and enters) each rank
+        frac = (world - 1) / world
+        rs_bytes, ag_bytes = frac * 2 * shard.padded_numel, frac * 2 * shard.padded_numel
+        line = {
+            "metric": METRIC, "value": n * args.steps / (total_ms / 1e3), "unit": "params/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{w.name} set: {n} FP32 params, BF16 grads, FP8 m (e4m3) / "
+                                   f"v ({args.v_fmt}) + per-group k, scale",
+                       "group_size": G, "m_fmt": "e4m3", "v_fmt": args.v_fmt,
+                       "params_per_gpu": L,
+                       "parallelism": f"zero1 dp{world}: BF16 reduce-scatter of each rank's "
+                                      "full gradient, coat_adamw_fp8_step on the rank's "
+                                      f"1/{world} shard, BF16 all-gather of the parameters",
+                       "l2": "no flush needed: every phase moves far more than the 126 MB L2"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peak_kind} copy bandwidth",
+                         "kernel": "coat_adamw_fp8_step on the shard",
+                         "algorithmic_bytes_per_param": bytes_per_param(G)},
+            "collectives": {"reduce_scatter_ms": rs_ms, "step_ms": st_ms,
+                            "all_gather_ms": ag_ms,
+                            "reduce_scatter_GBps_per_rank": rs_bytes / (rs_ms / 1e3) / 1e9
+                            if rs_bytes else None,
+                            "all_gather_GBps_per_rank": ag_bytes / (ag_ms / 1e3) / 1e9
+                            if ag_bytes else None,
+                            "link_peak_GBps": 770.0,
+                            "link_peak_source": "measured peer copy per direction on this pool",
+                            "bytes_per_rank_per_step": rs_bytes + ag_bytes},
+            "cpu_baseline": None,
+            "e2e": e2e,
+            # the step kernel, plus a tail launch when the shard is not a whole
+            # number of 1024-parameter blocks (the division after the
+            # reduce-scatter and the BF16 rounding before the all-gather are
+            # torch's)
+            "gpu_launches": args.steps * (1 + (L % 1024 != 0)),
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
+def run_step(args):
+    """One GPU: coat_adamw_fp8_step over the whole resident parameter set."""
+    import torch
     import quantized_optimizer_states_b200 as coat
     from quantized_optimizer_states_b200 import inputs
     from quantized_optimizer_states_b200 import build as coat_build
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+    world, rank, local = 1, 0, int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     coat_build.build()
     coat.load()
 
     v_fmt = coat.COAT_E4M3 if args.v_fmt == "e4m3" else coat.COAT_E5M2
-    if args.workload == "olmo-7b":
-        w = inputs.olmo_7b(seed=1237 + rank, v_fmt=args.v_fmt)
-    elif args.workload == "olmo-1b":
-        w = inputs.olmo_1b(seed=1235 + rank)
-        w.v_fmt = args.v_fmt
-    else:
-        w = inputs.sweep(args.group_size, args.v_fmt, args.regime, seed=1238 + rank)
+    w = step_workload(args)
     n, G = w.n, w.group_size
     ng = -(-n // G)
     hyper = dict(w.hyper)
@@ -507,8 +843,6 @@ def main():
     sampler = ClockSampler(uuid)
     sampler.start()
     time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
     torch.cuda.synchronize()
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     # the timed region is an NVTX range, so a profiler can list exactly its launches
@@ -519,16 +853,10 @@ def main():
         evs[i + 1].record(stream)
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_pop()
-    if world > 1:
-        dist.barrier()
     clocks = sampler.stop()
     per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
     total_ms = evs[0].elapsed_time(evs[-1])
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * n * args.steps / (total_ms / 1e3)
+    value = n * args.steps / (total_ms / 1e3)
     kernel_ms = sum(per) / len(per)
 
     peaks, peak_kind = measured_peaks()
@@ -560,8 +888,6 @@ def main():
         host_grad.copy_(grad[:per])
         result = torch.empty(4, dtype=torch.float32, pin_memory=True)
         torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
 
         def e2e_step():
             t = step_no[0]
@@ -595,11 +921,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * n * args.e2e_steps / (e2e_ms / 1e3), "unit": "params/s",
+        e2e = {"value": n * args.e2e_steps / (e2e_ms / 1e3), "unit": "params/s",
                "h2d_bytes_per_step": 2 * n, "d2h_bytes_per_step": 16,
                "what": "BF16 gradients copied from pinned host memory every step in 16 chunks "
                        "(from one chunk-sized pinned staging buffer) on a copy stream, each "
@@ -608,32 +930,73 @@ def main():
         del host_grad
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if not args.no_cpu_baseline:
         cpu = cpu_baseline(w, G, args.cpu_sample, v_fmt)
 
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"{w.name} set: {n} FP32 params, BF16 grads, FP8 m (e4m3) / "
-                                   f"v ({args.v_fmt}) + per-group k, scale",
-                       "group_size": G, "m_fmt": "e4m3", "v_fmt": args.v_fmt,
-                       "params_per_gpu": n, "parallelism": f"{world} independent shards",
-                       "l2": f"no flush needed: {bytes_per_param(G) * n / 1e9:.1f} GB moved "
-                             "per step, far above the 126 MB L2"},
-            "roofline": roofline,
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": args.steps,
-            "clocks": clocks,
-            "kernel_ms": kernel_ms,
-        }
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    # ---- the rest of the path, recorded beside the headline -------------------------
+    variant = acts = None
+    if not args.no_extra:
+        # the other second-moment format of the same set: v re-quantized, timed alone
+        other = coat.COAT_E5M2 if v_fmt == coat.COAT_E4M3 else coat.COAT_E4M3
+        for off, m0, v0 in chunks():
+            c = m0.numel()
+            g0, g1 = off // G, -(-(off + c) // G)
+            coat.coat_quantize_state(v0, v_code[off:off + c], v_k[g0:g1], v_s[g0:g1],
+                                     group_size=G, fmt=other)
+        torch.cuda.synchronize()
+
+        def step_other():
+            coat.coat_adamw_fp8_step(theta, grad, m_code, m_k, m_s, v_code, v_k, v_s,
+                                     step=step_no[0], group_size=G, v_fmt=other, **hyper)
+            step_no[0] += 1
+
+        for _ in range(3):
+            step_other()
+        sampler = ClockSampler(uuid)
+        sampler.start()
+        time.sleep(0.2)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.variant_steps):
+            step_other()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        vclocks = sampler.stop()
+        vms = e0.elapsed_time(e1) / args.variant_steps
+        vgbs = bytes_per_param(G) * n / (vms / 1e3) / 1e9
+        variant = {"v_fmt": "e5m2" if other == coat.COAT_E5M2 else "e4m3", "steps": args.variant_steps,
+                   "ms_per_step": vms, "params_per_s": n / (vms / 1e3), "GB/s": vgbs,
+                   "frac_of_hbm": vgbs / peak, "clocks": vclocks}
+        # the activation-side kernels on the activation workload
+        res, aclocks, an, aG, _, _ = measure_activations(dev, 40, 8)
+        acts = {"workload": "activations [16384, 2048] BF16 with GLU spike channels, G = 128, "
+                            "E4M3; 40 launches over a ring of 8 input sets",
+                "kernels": res, "clocks": aclocks,
+                "roofline_1xG_traffic": recorded_act_traffic(an)}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name} set: {n} FP32 params, BF16 grads, FP8 m (e4m3) / "
+                               f"v ({args.v_fmt}) + per-group k, scale",
+                   "group_size": G, "m_fmt": "e4m3", "v_fmt": args.v_fmt,
+                   "params_per_gpu": n, "parallelism": "one GPU",
+                   "l2": f"no flush needed: {bytes_per_param(G) * n / 1e9:.1f} GB moved "
+                         "per step, far above the 126 MB L2"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "kernel_ms": kernel_ms,
+        # beside the headline, outside its timed region
+        "variant_other_v_fmt": variant,
+        "activation_kernels": acts,
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 

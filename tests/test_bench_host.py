@@ -94,3 +94,30 @@ def test_reference_arm_prints_the_contract_line():
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
     assert line["e2e"] == {"value": line["value"], "unit": "params/s",
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_launch_command_runs_this_script_under_torchrun_on_localhost():
+    cmd = bench.launch_command(8, ["--gpus", "8", "--steps", "3"], 900, 29555)
+    assert cmd[:4] == ["timeout", "-k", "60", "900"]
+    i = cmd.index("torch.distributed.run")
+    assert cmd[i - 1] == "-m"
+    assert "--nproc-per-node=8" in cmd and "--nnodes=1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[cmd.index("--master-port") + 1] == "29555"
+    assert cmd[-4:] == [os.path.abspath(bench.__file__), "--gpus", "8", "--steps", "3"][-4:]
+
+
+def test_gpus_n_starts_n_ranks_that_all_join():
+    """`bench.py --gpus 2` outside torchrun starts two ranks itself; with no
+    GPU here they join over gloo, and rank 0's JSON line reports both."""
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--gpus", "2",
+                          "--workload", "ranks", "--launch-timeout", "240"],
+                         capture_output=True, text=True, timeout=300, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    assert lines[0]["n_gpus"] == 2 and lines[0]["ranks_joined"] == 2

@@ -37,6 +37,24 @@ __device__ __forceinline__ void pdl_enter() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// 16-byte global -> shared copy on the asynchronous copy path (no registers
+// held), and the waits for this thread's own outstanding copy groups.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_one() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
 __device__ __forceinline__ void act_scale(float amax, float fmax, float &s, float &inv) {
   if (amax > 0x1p-100f) {
     s = __fdiv_rn(amax, fmax);
@@ -619,9 +637,11 @@ __global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormPar
 constexpr int kNormRegWarps = 8;
 constexpr int kNormRegMaxChunks = 8;
 
+// One row of 256 NC columns held in registers: src is the row (its 32 NC
+// 16-byte chunks, in global or shared memory), lane l takes chunks l + 32 i.
 template <int NC>
-__device__ __forceinline__ float norm_reg_row(const NormParams &p, int64_t row, int lane) {
-  const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.cols);
+__device__ __forceinline__ float norm_reg_row(const NormParams &p, const uint4 *src, int64_t row,
+                                              int lane) {
   uint4 c[NC];
 #pragma unroll
   for (int i = 0; i < NC; ++i) c[i] = src[lane + 32 * i];
@@ -701,17 +721,53 @@ __device__ __forceinline__ float norm_reg_row(const NormParams &p, int64_t row, 
   return warp_max_f(rowmax);
 }
 
-// Persistent warps: warp w of the grid takes rows w, w + W, ... (W the
-// grid's warps).
+// Shared memory of norm_reg_group_amax_kernel<NC>: two row buffers a warp.
+template <int NC>
+constexpr size_t norm_reg_smem() {
+  return static_cast<size_t>(kNormRegWarps) * 2 * 32 * NC * sizeof(uint4);
+}
+
+// Persistent blocks, one contiguous share of the rows each.  A warp takes
+// the block's next untaken row whenever it starts one (a shared-memory
+// counter), so warps the scheduler favours take more rows and the block's
+// warps finish together, and it copies that next row into the second of its
+// two shared-memory buffers (cp.async, its own chunks only, so no barrier)
+// while it normalises the current one.
 template <int NC>
 __global__ void __launch_bounds__(32 * kNormRegWarps, 2) norm_reg_group_amax_kernel(const NormParams p) {
+  extern __shared__ __align__(16) uint4 nbuf[];
+  __shared__ unsigned int next_row;
   pdl_enter();
   const int lane = threadIdx.x & 31;
-  const int64_t step = static_cast<int64_t>(gridDim.x) * kNormRegWarps;
+  const int warp = threadIdx.x >> 5;
+  const int64_t r0 = p.rows * blockIdx.x / gridDim.x;
+  const int64_t r1 = p.rows * (blockIdx.x + 1) / gridDim.x;
+  if (threadIdx.x == 0) next_row = kNormRegWarps;
+  __syncthreads();
+  uint4 *wb = nbuf + warp * 2 * 32 * NC;
+  const int64_t cv = p.cols / 8;   // 16-byte chunks a row
+  auto fetch = [&](int64_t row, uint4 *dst) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.x) + row * cv;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) cp_async16(dst + lane + 32 * i, src + lane + 32 * i);
+    cp_async_commit();
+  };
   float wmax = 0.0f;
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kNormRegWarps + (threadIdx.x >> 5);
-       row < p.rows; row += step)
-    wmax = fmaxf(wmax, norm_reg_row<NC>(p, row, lane));
+  int64_t row = r0 + warp;
+  if (row < r1) fetch(row, wb);
+  for (int k = 0; row < r1; ++k) {
+    unsigned int g = 0;
+    if (lane == 0) g = atomicAdd(&next_row, 1u);
+    const int64_t nxt = r0 + __shfl_sync(0xffffffffu, g, 0);
+    if (nxt < r1) {
+      fetch(nxt, wb + ((k + 1) & 1) * 32 * NC);
+      cp_async_wait_one();   // the current row's copies (all but the newest group)
+    } else {
+      cp_async_wait_all();
+    }
+    wmax = fmaxf(wmax, norm_reg_row<NC>(p, wb + (k & 1) * 32 * NC, row, lane));
+    row = nxt;
+  }
   if (p.tensor_amax) block_max_to_tensor(wmax, p.tensor_amax);
 }
 

@@ -282,12 +282,20 @@ coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *
 // blocks that fit the GPU at once (or fewer, for few rows), the occupancy
 // looked up once per device.
 template <int NC>
-void launch_norm_reg(cudaStream_t s, const coat::NormParams &p) {
+coat_status_t launch_norm_reg(cudaStream_t s, const coat::NormParams &p) {
+  constexpr auto kernel = coat::norm_reg_group_amax_kernel<NC>;
+  constexpr size_t smem = coat::norm_reg_smem<NC>();
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+  if (e != cudaSuccess) {
+    g_last_cuda_error = static_cast<int32_t>(e);
+    return COAT_ERR_CUDA;
+  }
   const int64_t blocks_needed = (p.rows + coat::kNormRegWarps - 1) / coat::kNormRegWarps;
-  const unsigned int grid = coat::bulk_grid<coat::norm_reg_group_amax_kernel<NC>>(
-      32 * coat::kNormRegWarps, 0, blocks_needed);
-  launch_act_threads(coat::norm_reg_group_amax_kernel<NC>, grid, 32u * coat::kNormRegWarps, 0, s,
-                     p);
+  const unsigned int grid = coat::bulk_grid<kernel>(32 * coat::kNormRegWarps, smem, blocks_needed);
+  launch_act_threads(kernel, grid, 32u * coat::kNormRegWarps, smem, s, p);
+  return launch_status();
 }
 
 }  // namespace
@@ -580,16 +588,15 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
                        reinterpret_cast<uint32_t *>(tensor_amax));
   if (cols % 256 == 0 && cols / 256 <= coat::kNormRegMaxChunks) {
     switch (cols / 256) {
-      case 1: launch_norm_reg<1>(s, p); break;
-      case 2: launch_norm_reg<2>(s, p); break;
-      case 3: launch_norm_reg<3>(s, p); break;
-      case 4: launch_norm_reg<4>(s, p); break;
-      case 5: launch_norm_reg<5>(s, p); break;
-      case 6: launch_norm_reg<6>(s, p); break;
-      case 7: launch_norm_reg<7>(s, p); break;
-      default: launch_norm_reg<8>(s, p); break;
+      case 1: return launch_norm_reg<1>(s, p);
+      case 2: return launch_norm_reg<2>(s, p);
+      case 3: return launch_norm_reg<3>(s, p);
+      case 4: return launch_norm_reg<4>(s, p);
+      case 5: return launch_norm_reg<5>(s, p);
+      case 6: return launch_norm_reg<6>(s, p);
+      case 7: return launch_norm_reg<7>(s, p);
+      default: return launch_norm_reg<8>(s, p);
     }
-    return launch_status();
   }
   // other widths: persistent warps, each staging two rows in shared memory
   const int wpb = coat::norm_warps_per_block(cols);

@@ -482,7 +482,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the records beside the headline (the other v format, the "
-                         "activation kernels)")
+                         "activation kernels, the OLMo-1B set and the 2^28 sweep)")
     ap.add_argument("--variant-steps", type=int, default=10)
     ap.add_argument("--workload", default="olmo-7b",
                     choices=["olmo-7b", "olmo-1b", "sweep", "activations", "optimizer",
@@ -787,6 +787,54 @@ def run_zero1(args):
     return 0
 
 
+def time_step_set(w, v_fmt: int, steps: int, warmup: int, dev) -> dict:
+    """The public step on workload w (inputs built on the device, states
+    quantized with coat_quantize_state), `steps` timed steps after `warmup`,
+    CUDA events on the launching stream; returns its record."""
+    import torch
+    import quantized_optimizer_states_b200 as coat
+    from quantized_optimizer_states_b200 import inputs
+    n, G = w.n, w.group_size
+    ng = -(-n // G)
+    theta, grad, chunks = inputs.device_step_inputs(w, dev)
+    mc = torch.empty(n, dtype=torch.uint8, device=dev)
+    vc = torch.empty(n, dtype=torch.uint8, device=dev)
+    mk, ms, vk, vs = (torch.empty(ng, dtype=torch.float32, device=dev) for _ in range(4))
+    for off, m0, v0 in chunks():
+        c = m0.numel()
+        g0, g1 = off // G, -(-(off + c) // G)
+        coat.coat_quantize_state(m0, mc[off:off + c], mk[g0:g1], ms[g0:g1], group_size=G,
+                                 fmt=coat.COAT_E4M3)
+        coat.coat_quantize_state(v0, vc[off:off + c], vk[g0:g1], vs[g0:g1], group_size=G,
+                                 fmt=v_fmt)
+    t = [w.step]
+
+    def step():
+        coat.coat_adamw_fp8_step(theta, grad, mc, mk, ms, vc, vk, vs, step=t[0], group_size=G,
+                                 v_fmt=v_fmt, **w.hyper)
+        t[0] += 1
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_ = e0.elapsed_time(e1) / steps
+    peak = float(measured_peaks()[0]["hbm_gbs"])
+    gbs = bytes_per_param(G) * n / (ms_ / 1e3) / 1e9
+    del theta, grad, mc, vc, mk, ms, vk, vs
+    torch.cuda.empty_cache()
+    return {"params": n, "group_size": G,
+            "v_fmt": "e4m3" if v_fmt == coat.COAT_E4M3 else "e5m2", "steps": steps,
+            "ms_per_step": ms_, "params_per_s": n / (ms_ / 1e3), "GB/s": gbs,
+            "frac_of_hbm": gbs / peak}
+
+
 def run_step(args):
     """One GPU: coat_adamw_fp8_step over the whole resident parameter set."""
     import torch
@@ -934,7 +982,7 @@ def run_step(args):
         cpu = cpu_baseline(w, G, args.cpu_sample, v_fmt)
 
     # ---- the rest of the path, recorded beside the headline -------------------------
-    variant = acts = None
+    variant = acts = sets = None
     if not args.no_extra:
         # the other second-moment format of the same set: v re-quantized, timed alone
         other = coat.COAT_E5M2 if v_fmt == coat.COAT_E4M3 else coat.COAT_E4M3
@@ -974,6 +1022,23 @@ def run_step(args):
                             "E4M3; 40 launches over a ring of 8 input sets",
                 "kernels": res, "clocks": aclocks,
                 "roofline_1xG_traffic": recorded_act_traffic(an)}
+        # the other parameter sets: OLMo-1B (v E5M2) and the 2^28 group-size /
+        # format sweep (late regime), with the big set's buffers released first
+        del theta, grad, m_code, v_code, m_k, m_s, v_k, v_s
+        torch.cuda.empty_cache()
+        sampler = ClockSampler(uuid)
+        sampler.start()
+        sets = {"olmo_1b_v_e5m2": time_step_set(inputs.olmo_1b(), coat.COAT_E5M2, 10, 3, dev),
+                "sweep_2p28_late": [time_step_set(inputs.sweep(gs, vf, "late"),
+                                                  coat.COAT_E4M3 if vf == "e4m3"
+                                                  else coat.COAT_E5M2, 10, 3, dev)
+                                    for gs in (32, 64, 128, 256, 1024)
+                                    for vf in ("e4m3", "e5m2")],
+                "sweep_2p28_early_G128": [time_step_set(inputs.sweep(128, vf, "early"),
+                                                        coat.COAT_E4M3 if vf == "e4m3"
+                                                        else coat.COAT_E5M2, 10, 3, dev)
+                                          for vf in ("e4m3", "e5m2")]}
+        sets["clocks"] = sampler.stop()
 
     line = {
         "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,
@@ -995,6 +1060,7 @@ def run_step(args):
         # beside the headline, outside its timed region
         "variant_other_v_fmt": variant,
         "activation_kernels": acts,
+        "other_parameter_sets": sets,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -637,8 +637,23 @@ __global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormPar
 constexpr int kNormRegWarps = 8;
 constexpr int kNormRegMaxChunks = 8;
 
+// max of two BF16 pairs, lane by lane (NaN ignored)
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(bf16lo_to_float(w), bf16hi_to_float(w));
+}
+
 // One row of 256 NC columns held in registers: src is the row (its 32 NC
 // 16-byte chunks, in global or shared memory), lane l takes chunks l + 32 i.
+// The arithmetic runs on packed binary32 pairs: the row sums as four partial
+// sums a lane (two packed pairs, alternate pairs of columns), the
+// normalisation two columns an instruction, and each 1xG maximum of |out|
+// on the BF16 outputs themselves (pairs with their sign bits cleared).
 template <int NC>
 __device__ __forceinline__ float norm_reg_row(const NormParams &p, const uint4 *src, int64_t row,
                                               int lane) {
@@ -646,35 +661,39 @@ __device__ __forceinline__ float norm_reg_row(const NormParams &p, const uint4 *
 #pragma unroll
   for (int i = 0; i < NC; ++i) c[i] = src[lane + 32 * i];
   const float nf = static_cast<float>(p.cols);   // exact (cols <= 16384)
-  float acc = 0.0f;
+  float2 s0 = make_float2(0.0f, 0.0f), s1 = s0;
 #pragma unroll
   for (int i = 0; i < NC; ++i) {
     const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float a = bf16lo_to_float(wv[j]), b = bf16hi_to_float(wv[j]);
-      acc += p.rms ? a * a + b * b : a + b;
+      const float2 x2 = bf16x2_to_float2(wv[j]);
+      float2 &acc = (j & 1) ? s1 : s0;
+      acc = p.rms ? fma2_rn(x2, x2, acc) : add2_rn(acc, x2);
     }
   }
-  const float s1 = warp_sum_f(acc);
+  const float sum = warp_sum_f((s0.x + s0.y) + (s1.x + s1.y));
   float mean = 0.0f, var;
   if (p.rms) {
-    var = __fdiv_rn(s1, nf);
+    var = __fdiv_rn(sum, nf);
   } else {
-    mean = __fdiv_rn(s1, nf);
-    float ss = 0.0f;
+    mean = __fdiv_rn(sum, nf);
+    const float2 nm = make_float2(-mean, -mean);
+    float2 q0 = make_float2(0.0f, 0.0f), q1 = q0;
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
       const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float a = bf16lo_to_float(wv[j]) - mean, b = bf16hi_to_float(wv[j]) - mean;
-        ss += a * a + b * b;
+        const float2 d = add2_rn(bf16x2_to_float2(wv[j]), nm);
+        float2 &acc = (j & 1) ? q1 : q0;
+        acc = fma2_rn(d, d, acc);
       }
     }
-    var = __fdiv_rn(warp_sum_f(ss), nf);
+    var = __fdiv_rn(warp_sum_f((q0.x + q0.y) + (q1.x + q1.y)), nf);
   }
   const float rstd = 1.0f / sqrtf(var + p.eps);
+  const float2 NM = make_float2(-mean, -mean), RS = make_float2(rstd, rstd);
 
   // chunk q = lane + 32 i holds columns 8q .. 8q + 7; a 1xG run is G / 8
   // chunks: consecutive lanes of one i for G <= 256, else all lanes of
@@ -688,24 +707,18 @@ __device__ __forceinline__ float norm_reg_row(const NormParams &p, const uint4 *
     const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
     const int col0 = 8 * (lane + 32 * i);
     uint32_t ow[4];
-    float a = 0.0f;
+    uint32_t am = 0u;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int cc = col0 + 2 * j;
-      float y0 = (bf16lo_to_float(wv[j]) - mean) * rstd;
-      float y1 = (bf16hi_to_float(wv[j]) - mean) * rstd;
-      if (p.weight) {
-        y0 *= p.weight[cc];
-        y1 *= p.weight[cc + 1];
-      }
-      if (p.bias) {
-        y0 += p.bias[cc];
-        y1 += p.bias[cc + 1];
-      }
-      ow[j] = bf16x2_rn(y0, y1);
-      a = fmaxf(a, fmaxf(fabsf(bf16lo_to_float(ow[j])), fabsf(bf16hi_to_float(ow[j]))));
+      float2 y = mul2_rn(add2_rn(bf16x2_to_float2(wv[j]), NM), RS);
+      if (p.weight) y = mul2_rn(y, make_float2(p.weight[cc], p.weight[cc + 1]));
+      if (p.bias) y = add2_rn(y, make_float2(p.bias[cc], p.bias[cc + 1]));
+      ow[j] = bf16x2_rn(y.x, y.y);
+      am = bmax2(am, ow[j] & 0x7FFF7FFFu);
     }
     dst[lane + 32 * i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    float a = fmaxf(bf16lo_to_float(am), bf16hi_to_float(am));
     rowmax = fmaxf(rowmax, a);
     if (clanes <= 32) {
       for (int off = 1; off < clanes; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));

@@ -560,6 +560,9 @@ def init_ranks(timeout_s: int = 300, single: bool = False):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if (world > 1 or single) and not dist.is_initialized():
+        # NCCL's communicator set-up lines, so the log shows every rank joining
+        os.environ.setdefault("NCCL_DEBUG", "INFO")
+        os.environ.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
         if torch.cuda.is_available():
             torch.cuda.set_device(local)
             dist.init_process_group("nccl", timeout=timedelta(seconds=timeout_s),

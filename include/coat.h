@@ -68,7 +68,7 @@ typedef enum coat_status {
     COAT_ERR_UNSUPPORTED = 3, /* format / group size / flag combination not built */
     COAT_ERR_CUDA = 4,        /* a CUDA launch or query failed */
     COAT_ERR_NONFINITE = 5,   /* reserved */
-    COAT_ERR_TIMEOUT = 6      /* a bounded device wait ran out (coat_selftest_bounded_wait) */
+    COAT_ERR_TIMEOUT = 6      /* reserved: no kernel of this library waits on the device */
 } coat_status_t;
 
 typedef enum coat_fp8 {
@@ -445,40 +445,9 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
                                    int32_t group_size, uint16_t *out, float *group_amax,
                                    float *tensor_amax, void *stream);
 
-/*
- * coat_selftest_bounded_wait -- exercises, on the device, the bounded wait
- * the streamed kernels use on their mbarriers: one block waits on a barrier
- * that needs two arrivals.  leave_open = 0: both arrive, the phase
- * completes, COAT_OK.  leave_open = 1: one arrives and nothing ever
- * completes the phase, so every wait runs out after its bounded number of
- * polls, the block combines the results as the streamed kernels do and
- * counts the timeout, and the call returns COAT_ERR_TIMEOUT -- with the
- * CUDA context still usable and the streamed kernels' own counter
- * (coat_bulk_wait_timeouts) untouched.  No copy is involved.  Synchronises
- * the stream.  Errors: INVALID_ARG (leave_open not 0/1), CUDA.
- */
-coat_status_t coat_selftest_bounded_wait(int32_t leave_open, void *stream);
-
 /* The last CUDA error code seen by a call that returned COAT_ERR_CUDA in
  * this thread (0 if none). */
 int32_t coat_last_cuda_error(void);
-
-/* Streamed activation kernels (coat_group_quant_1xG on contiguous rows,
- * the cast of coat_group_scaling_quant_pertensor[_noalloc]) move
- * 4096-element tiles into shared memory with bulk asynchronous copies and
- * wait for each on an mbarrier.  Every such wait is bounded: one that runs
- * out abandons the rest of its block's tiles (their outputs are then not
- * written), waits (bounded again) for the block's copies still in flight,
- * and adds 1 to a device counter.  coat_bulk_wait_timeouts synchronises the current device,
- * stores the counter in *count (host pointer) and, if reset != 0, sets it
- * to zero.  A non-zero count means outputs of the calls since the last
- * reset are incomplete; treat the CUDA context as suspect too (if the
- * second wait also ran out, a copy may still have been in flight when its
- * block left).  The launches are asynchronous, so the calls themselves
- * cannot report this: check the counter where it matters (the tests and
- * bench.py do after every streamed run).
- * Errors: INVALID_ARG (count NULL), CUDA. */
-coat_status_t coat_bulk_wait_timeouts(uint32_t *count, int32_t reset);
 
 /* A static, human-readable name for a status code. */
 const char *coat_status_string(coat_status_t status);

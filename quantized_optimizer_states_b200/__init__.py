@@ -13,7 +13,6 @@ from ._lib import (  # noqa: F401
     CoatError,
     PackTable,
     coat_adamw_fp8_step,
-    coat_bulk_wait_timeouts,
     coat_count_nonfinite_bf16,
     coat_dequant,
     coat_fp8_encode,
@@ -24,7 +23,6 @@ from ._lib import (  # noqa: F401
     coat_norm_group_amax,
     coat_pack_bf16,
     coat_quantize_state,
-    coat_selftest_bounded_wait,
     coat_state_stats,
     coat_status_string,
     coat_swiglu_group_amax,

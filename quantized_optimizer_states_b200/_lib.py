@@ -77,9 +77,7 @@ SIGNATURES = {
     "coat_unpack_bf16": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), _I32,
                                 ctypes.POINTER(_P), _I64, _P]),
     "coat_state_stats": (_I32, [_P, _P, _P, _I64, _I32, _I32, _P, _P]),
-    "coat_selftest_bounded_wait": (_I32, [_I32, _P]),
     "coat_last_cuda_error": (_I32, []),
-    "coat_bulk_wait_timeouts": (_I32, [ctypes.POINTER(ctypes.c_uint32), _I32]),
     "coat_status_string": (ctypes.c_char_p, [_I32]),
     "coat_version": (_I32, []),
 }
@@ -107,34 +105,50 @@ def _check(name: str, status: int):
         raise CoatError(name, status, load().coat_last_cuda_error())
 
 
+def _current_device() -> int:
+    """Index of the current CUDA device (torch's own cheap query where it
+    has one: the binding runs on every call of every entry point)."""
+    import torch
+    get = getattr(torch._C, "_cuda_getDevice", None)
+    return int(get()) if get is not None else torch.cuda.current_device()
+
+
 def _stream(stream):
+    """The stream handle: the given one, else torch's current stream on the
+    current device (its raw handle, without building a Stream object)."""
     if stream is not None:
         return ctypes.c_void_p(int(stream))
     import torch
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return raw(_current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _on_current_device(t, what):
     """The kernels run on the current CUDA device; a tensor of another device
     would be an illegal address there, so it is refused on the host."""
-    import torch
-    cur = torch.cuda.current_device()
+    cur = _current_device()
     if t.get_device() != cur:
         raise ValueError(f"{what} is on {t.device} but the current device is cuda:{cur} "
                          f"(call under torch.cuda.device({t.device}))")
 
 
 def _ptr(t, dtype=None, what="tensor"):
+    """The device address of a contiguous CUDA tensor on the current device
+    (an int, which ctypes passes as a pointer)."""
     if t is None:
         return None
-    if not t.is_cuda:
+    dev = t.get_device()
+    if dev < 0:
         raise ValueError(f"{what} must be a CUDA tensor")
-    _on_current_device(t, what)
+    if dev != _current_device():
+        _on_current_device(t, what)
     if not t.is_contiguous():
         raise ValueError(f"{what} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
-    return ctypes.c_void_p(t.data_ptr())
+    return t.data_ptr()
 
 
 def _slot(t):
@@ -242,13 +256,15 @@ def coat_group_quant_1xG(x, q, scale, *, group_size: int = 128, fmt: int = COAT_
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit column stride")
     rows, cols = x.shape
-    if not x.is_cuda:
+    dev = x.get_device()
+    if dev < 0:
         raise ValueError("x must be a CUDA tensor")
-    _on_current_device(x, "x")
+    if dev != _current_device():
+        _on_current_device(x, "x")
     if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
         raise ValueError("x must hold BF16 bit patterns")
     st = load().coat_group_quant_1xG(
-        ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), group_size, fmt,
+        x.data_ptr(), rows, cols, x.stride(0), group_size, fmt,
         _ptr(q, torch.uint8, "q"), _ptr(scale, torch.float32, "scale"), _stream(stream))
     _check("coat_group_quant_1xG", st)
 
@@ -265,11 +281,12 @@ def coat_group_scaling_quant_pertensor(x, workspace, q, scale, *, group_size: in
     wrote the group maxima) or 2 (it also wrote the tensor maximum into the
     last workspace slot: the cast alone); True counts as 1."""
     import torch
-    need = coat_group_scaling_workspace_bytes(x.numel(), group_size)
+    n = x.numel()
+    need = (-(-n // group_size) + 1) * 4 if group_size >= 1 else 0  # as the library sizes it
     if workspace.numel() * workspace.element_size() < need:
         raise ValueError(f"workspace needs {need} bytes")
     st = load().coat_group_scaling_quant_pertensor(
-        _u16(x, "x"), x.numel(), group_size, fmt, _ptr(workspace, torch.float32, "workspace"),
+        _u16(x, "x"), n, group_size, fmt, _ptr(workspace, torch.float32, "workspace"),
         int(amax_precomputed), _ptr(q, torch.uint8, "q"),
         _ptr(scale, torch.float32, "scale"), _stream(stream))
     _check("coat_group_scaling_quant_pertensor", st)
@@ -415,22 +432,6 @@ def coat_state_stats(code, k, scale, *, group_size: int, fmt: int = COAT_E4M3, o
     raw = bytes(buf.cpu().numpy().tobytes())
     st = CoatStateStats.from_buffer_copy(raw)
     return {name: getattr(st, name) for name, _ in CoatStateStats._fields_}
-
-
-def coat_bulk_wait_timeouts(*, reset: bool = False) -> int:
-    """Bounded shared-memory copy waits of the streamed kernels that ran out
-    since the last reset (synchronises the device); 0 when every output is
-    complete."""
-    c = ctypes.c_uint32(0)
-    _check("coat_bulk_wait_timeouts", load().coat_bulk_wait_timeouts(ctypes.byref(c), int(reset)))
-    return int(c.value)
-
-
-def coat_selftest_bounded_wait(*, leave_open: bool, stream=None):
-    """Run the bounded-wait self-test (see include/coat.h); raises CoatError
-    with status COAT_ERR_TIMEOUT (6) when the wait ran out."""
-    _check("coat_selftest_bounded_wait",
-           load().coat_selftest_bounded_wait(int(bool(leave_open)), _stream(stream)))
 
 
 def coat_version() -> int:

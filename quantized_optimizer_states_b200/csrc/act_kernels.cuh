@@ -17,7 +17,6 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
-#include "bulk_pipe.cuh"
 #include "fp8_device.cuh"
 #include "state_codec.cuh"
 #include "step_kernels.cuh"
@@ -193,80 +192,40 @@ __global__ void __launch_bounds__(kThreads) group_quant_1xG_kernel(const GroupQu
   }
 }
 
-// ---- streamed forms: tiles through shared memory by bulk copies -----------------
-// A tile is kElemsPerBlock (4096) consecutive elements of a flat tensor, one
-// 16-element vector per thread; a 1xG group (G <= 4096, a power of two)
-// never straddles two tiles.  These kernels take whole tiles only; the host
-// hands a ragged remainder to the plain kernels above and below.
-constexpr int kTileBf16Bytes = kElemsPerBlock * 2;
-
-// Local tiles of this block: t0, t0 + dt, ... below `tiles`.
-__device__ __forceinline__ int stream_local_tiles(int64_t tiles) {
-  const int64_t t0 = blockIdx.x, dt = gridDim.x;
-  return t0 < tiles ? static_cast<int>((tiles - t0 + dt - 1) / dt) : 0;
-}
-
-__device__ __forceinline__ int64_t stream_tile(int i) {
-  return static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(i) * gridDim.x;
-}
-
-// Thread 0: the first min(n, kBulkStages) tiles of a single-input stream.
-template <int kBytes>
-__device__ __forceinline__ void stream_prologue(const BulkPipe<kBytes> &pipe, const void *src,
-                                                int n) {
-  if (threadIdx.x != 0) return;
-  pipe.init();
-  const int pre = n < kBulkStages ? n : kBulkStages;
-  for (int i = 0; i < pre; ++i) {
-    pipe.expect(i, kBytes);
-    pipe.copy(i, 0, static_cast<const unsigned char *>(src) + stream_tile(i) * kBytes, kBytes);
-  }
-}
-
-// Thread 0, after the block has consumed local tile i: refill its stage.
-template <int kBytes>
-__device__ __forceinline__ void stream_refill(const BulkPipe<kBytes> &pipe, const void *src, int i,
-                                              int n) {
-  const int j = i + kBulkStages;
-  if (threadIdx.x != 0 || j >= n) return;
-  pipe.expect(j, kBytes);
-  pipe.copy(j, 0, static_cast<const unsigned char *>(src) + stream_tile(j) * kBytes, kBytes);
-}
-
-// 1xG quantization of a tensor with contiguous rows (ld == cols), flat.
+// 1xG quantization of a tensor with contiguous rows (ld == cols) as one
+// flat run of n elements: every 1xG group is G consecutive elements, so no
+// row / column split is needed.
 template <int F>
 __global__ void __launch_bounds__(kThreads)
-    group_quant_1xG_stream_kernel(const GroupQuantParams p, int64_t tiles) {
-  extern __shared__ __align__(128) unsigned char stream_buf[];
-  __shared__ __align__(8) uint64_t bars[kBulkStages];
-  __shared__ float red[kWarps];
+    group_quant_1xG_flat_kernel(const GroupQuantParams p, int64_t n) {
+  __shared__ float red[kActV][kWarps];
   pdl_enter();
-  const BulkPipe<kTileBf16Bytes> pipe{stream_buf, bars};
   const int lanes = 1 << (p.log2G - 4);
-  const int n = stream_local_tiles(tiles);
-  stream_prologue(pipe, p.x, n);
-  __syncthreads();
-  for (int i = 0; i < n; ++i) {
-    const bool ok = pipe.wait(i);
-    const uint4 *src = reinterpret_cast<const uint4 *>(pipe.stage(i)) + 2 * threadIdx.x;
-    const uint4 a = src[0], b = src[1];
-    fence_reads_before_async_writes();
-    if (!__syncthreads_and(ok)) {
-      pipe.abandon(i, n < i + kBulkStages ? n : i + kBulkStages);
-      return;
+  uint32_t w[kActV][8];
+  int64_t e0[kActV];
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
+    e0[v] = ((static_cast<int64_t>(blockIdx.x) * kActV + v) * kThreads + threadIdx.x) * kVec;
+    if (e0[v] < n) {
+      load16_bf16<false>(p.x, e0[v], n, w[v]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[v][i] = 0;
     }
-    stream_refill(pipe, p.x, i, n);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  }
+#pragma unroll
+  for (int v = 0; v < kActV; ++v) {
     float x[16];
-    unpack16_bf16(w, x);
-    const float amax = group_max(amax16(x), lanes, red);
+    unpack16_bf16(w[v], x);
+    const float amax = group_max(amax16(x), lanes, red[v]);
     float s, inv;
     act_scale(amax, fmt_max<F>(), s, inv);
     uint32_t o[4];
     cast16<F>(x, inv, o);
-    const int64_t e0 = stream_tile(i) * kElemsPerBlock + threadIdx.x * kVec;
-    *reinterpret_cast<uint4 *>(p.q + e0) = make_uint4(o[0], o[1], o[2], o[3]);
-    if ((threadIdx.x & (lanes - 1)) == 0) p.scale[e0 >> p.log2G] = s;
+    if (e0[v] < n) {
+      store16_u8<false>(p.q, e0[v], n, o);
+      if ((threadIdx.x & (lanes - 1)) == 0) p.scale[e0[v] >> p.log2G] = s;
+    }
   }
 }
 
@@ -979,41 +938,6 @@ __global__ void __launch_bounds__(kThreads) dequant_linear_kernel(const DequantP
         }
       }
     }
-  }
-}
-
-// Step (iii) of Group Scaling, streamed.
-template <int F>
-__global__ void __launch_bounds__(kThreads)
-    pertensor_cast_stream_kernel(const GroupScalingParams p, int64_t tiles) {
-  extern __shared__ __align__(128) unsigned char stream_buf[];
-  __shared__ __align__(8) uint64_t bars[kBulkStages];
-  pdl_enter();
-  const BulkPipe<kTileBf16Bytes> pipe{stream_buf, bars};
-  const int n = stream_local_tiles(tiles);
-  stream_prologue(pipe, p.x, n);
-  const float amax = __uint_as_float(*p.tensor_amax);
-  float s, inv;
-  act_scale(amax, fmt_max<F>(), s, inv);
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.scale = s;
-  __syncthreads();
-  for (int i = 0; i < n; ++i) {
-    const bool ok = pipe.wait(i);
-    const uint4 *src = reinterpret_cast<const uint4 *>(pipe.stage(i)) + 2 * threadIdx.x;
-    const uint4 a = src[0], b = src[1];
-    fence_reads_before_async_writes();
-    if (!__syncthreads_and(ok)) {
-      pipe.abandon(i, n < i + kBulkStages ? n : i + kBulkStages);
-      return;
-    }
-    stream_refill(pipe, p.x, i, n);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float x[16];
-    unpack16_bf16(w, x);
-    uint32_t o[4];
-    cast16<F>(x, inv, o);
-    const int64_t e0 = stream_tile(i) * kElemsPerBlock + threadIdx.x * kVec;
-    *reinterpret_cast<uint4 *>(p.q + e0) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 

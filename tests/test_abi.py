@@ -129,10 +129,6 @@ def test_state_stats_argument_checks(lib):
     assert st(fake, fake, fake, 64, 128, 0, odd, None) == 2       # output not 8-byte aligned
 
 
-def test_selftest_argument_check(lib):
-    assert lib.coat_selftest_bounded_wait(2, None) == 1
-
-
 def test_product_path_fails_loudly_without_library(tmp_path):
     from quantized_optimizer_states_b200 import _lib
     saved = _lib._lib
@@ -246,7 +242,7 @@ def test_tensors_of_another_device_are_refused(monkeypatch):
     Checked with a stand-in tensor: this machine needs no GPU for it."""
     import torch
     from quantized_optimizer_states_b200 import _lib
-    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(_lib, "_current_device", lambda: 0)
 
     class OnDevice1:
         device = "cuda:1"
@@ -263,6 +259,8 @@ def test_tensors_of_another_device_are_refused(monkeypatch):
     with pytest.raises(ValueError, match="current device is cuda:0"):
         _lib._on_current_device(OnDevice1(), "x")
     _lib._on_current_device(OnDevice0(), "x")
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        _lib._ptr(torch.empty(4), torch.float32, "x")
 
 
 def test_ctypes_structures_match_the_header(tmp_path):

@@ -73,18 +73,17 @@ def test_group_quant_strided_rows_and_special_values(lib, orc):
     assert np.array_equal(q, q_ref)
 
 
-def test_group_quant_streamed_group_4096_and_remainders(lib, orc):
-    """Contiguous rows go through the streamed kernel (4096-element tiles by
-    bulk copies) plus the plain kernel for a ragged remainder: G = 4096
-    (a group filling a whole tile), and sizes whose remainder is 0, one group
-    or several groups."""
+def test_group_quant_contiguous_group_4096_and_partial_tiles(lib, orc):
+    """Contiguous rows go through the flat kernel (each block two
+    4096-element tiles): G = 4096 (a group filling a whole tile), and sizes
+    that end on a whole block, in the second tile of a block, or a few
+    groups into a tile."""
     for rows, cols, G in ((5, 8192, 4096), (3, 4096 + 2048, 2048), (7, 1152, 128)):
         x = inputs.host_activations(inputs.activations(seed=rows), rows=rows)
         x = np.tile(x, (1, -(-cols // x.shape[1])))[:, :cols].copy()
         q, sc = _gpu_1xG(lib, x, G, E4M3)
         q_ref, sc_ref = orc.group_quant_1xG(x, G, E4M3)
         assert np.array_equal(sc, sc_ref) and np.array_equal(q, q_ref), (rows, cols, G)
-    assert lib.coat_bulk_wait_timeouts(reset=True) == 0
 
 
 def _gpu_group_scaling(lib, x, G, fmt, group_amax=None):
@@ -156,10 +155,8 @@ def test_activation_dequant_bit_exact(lib, orc, fmt):
 
 @pytest.mark.parametrize("out_bf16", [False, True])
 def test_activation_dequant_full_set(lib, orc, out_bf16):
-    """The activation workload's codes (8192 tiles: every block of the
-    persistent streamed grid cycles its shared-memory stages several times)
-    dequantized per 1xG group, and a per-tensor length that is not a whole
-    number of tiles."""
+    """The activation workload's codes dequantized per 1xG group, and a
+    per-tensor length that is not a whole number of tiles."""
     import torch
     x = inputs.host_activations(inputs.activations())
     q, sc = orc.group_quant_1xG(x, 128, E4M3)
@@ -181,23 +178,6 @@ def test_activation_dequant_full_set(lib, orc, out_bf16):
     else:
         assert np.array_equal(parity.to_host(out), ref)
         assert np.array_equal(parity.to_host(out1), ref1)
-    assert lib.coat_bulk_wait_timeouts(reset=True) == 0
-
-
-def test_bounded_wait_runs_out_and_the_context_survives(lib, orc):
-    """The bounded mbarrier wait of the streamed kernels, made to run out on
-    the device (a barrier phase that nothing completes): the call reports
-    COAT_ERR_TIMEOUT, and afterwards the context still works -- a streamed
-    quantizer run is bit-exact and its own timeout counter is 0."""
-    lib.coat_selftest_bounded_wait(leave_open=False)
-    with pytest.raises(lib.CoatError) as e:
-        lib.coat_selftest_bounded_wait(leave_open=True)
-    assert e.value.status == 6
-    x = inputs.host_activations(inputs.activations(seed=21), rows=12)
-    q, sc = _gpu_1xG(lib, x, 128, E4M3)
-    q_ref, sc_ref = orc.group_quant_1xG(x, 128, E4M3)
-    assert np.array_equal(q, q_ref) and np.array_equal(sc, sc_ref)
-    assert lib.coat_bulk_wait_timeouts(reset=True) == 0
 
 
 def test_hardware_cvt_matches_oracle_encoder(lib, orc):

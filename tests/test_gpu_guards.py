@@ -1,7 +1,7 @@
 """Guard canaries around the outputs of every activation-side, producer,
 pack and monitoring kernel, a check that needs no memory-checking tool: each
 output is a slice of a larger buffer whose 256 bytes before and after hold
-a sentinel, sizes are ragged (streamed tiles plus a plain remainder, tail
+a sentinel, sizes are ragged (partial blocks and tiles, tail
 vectors, tail groups), and after the calls the sentinels must be intact
 (the outputs' values are the parity tests' business)."""
 import numpy as np
@@ -53,13 +53,13 @@ def test_activation_kernels_stay_inside(lib, rows):
     x = inputs.host_activations(inputs.activations(seed=rows), rows=rows)
     n = x.size - 48                                  # ragged flat length
     xf = parity.to_dev(x.reshape(-1)[:n].view(np.int16))
-    # 1xG on contiguous rows (streamed tiles + remainder)
+    # 1xG on contiguous rows (the flat kernel, a partial last block)
     q = Guarded(rows * cols, torch.uint8)
     sc = Guarded(rows * cols // G, torch.float32)
     lib.coat_group_quant_1xG(parity.to_dev(x.view(np.int16)), q.t.view(rows, cols),
                              sc.t.view(rows, cols // G), group_size=G)
     q.check("1xG codes"), sc.check("1xG scales")
-    # Group Scaling on a ragged length (streamed cast + remainder), both workspace modes
+    # Group Scaling on a ragged length (a tail vector), both workspace modes
     ng = -(-n // G)
     ws = Guarded(ng + 1, torch.float32)
     qg = Guarded(n, torch.uint8)

@@ -278,33 +278,40 @@ def measure_activations(dev, steps: int, warmup: int):
         coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"], group_size=G,
                                     tensor_amax=b["ws_h"][ng:])
     cases = {
-        # name: (callable on one ring slot, algorithmic bytes per element)
+        # name: (callable on one ring slot, algorithmic bytes per element,
+        #        kernel launches per call)
         "group_quant_1xG": (lambda b: coat.coat_group_quant_1xG(b["x"], b["q"], b["sc"],
                                                                 group_size=G),
-                            2 + 1 + 4.0 / G),
+                            2 + 1 + 4.0 / G, 1),
+        # zeroing the tensor maximum, step (i), the cast
         "group_scaling_standalone": (
             lambda b: coat.coat_group_scaling_quant_pertensor(b["x"].reshape(-1), b["ws"], b["q"],
                                                               b["s1"], group_size=G),
-            2 + 2 + 1 + 8.0 / G),
+            2 + 2 + 1 + 8.0 / G, 3),
+        # zeroing its tensor-maximum slot, the producer
         "swiglu_fused_amax": (
             lambda b: coat.coat_swiglu_group_amax(b["gate"], b["up"], b["h"], b["ws_h"],
                                                   group_size=G, tensor_amax=b["ws_h"][ng:]),
-            2 + 2 + 2 + 4.0 / G),
+            2 + 2 + 2 + 4.0 / G, 2),
+        # the same two: handed a whole workspace, the producer also writes
+        # the tensor maximum into its last slot
         "layernorm_fused_amax": (
             lambda b: coat.coat_norm_group_amax(b["x"], b["ln"], b["ws"], group_size=G),
-            2 + 2 + 4.0 / G),
+            2 + 2 + 4.0 / G, 2),
+        # zeroing, step (ii), the cast
         "group_scaling_after_producer": (
             lambda b: coat.coat_group_scaling_quant_pertensor(b["h"], b["ws_h"], b["q"], b["s1"],
                                                               group_size=G,
                                                               amax_precomputed=1),
-            2 + 1 + 4.0 / G),
+            2 + 1 + 4.0 / G, 3),
+        # the cast alone
         "group_scaling_after_producer_with_tensor_max": (
             lambda b: coat.coat_group_scaling_quant_pertensor(b["h"], b["ws_h"], b["q"], b["s1"],
                                                               group_size=G,
                                                               amax_precomputed=2),
-            2 + 1),
+            2 + 1, 1),
         "dequant_pertensor": (
-            lambda b: coat.coat_dequant(b["q"], None, b["s1"], b["out"], group_size=n), 1 + 4),
+            lambda b: coat.coat_dequant(b["q"], None, b["s1"], b["out"], group_size=n), 1 + 4, 1),
     }
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
@@ -313,7 +320,7 @@ def measure_activations(dev, steps: int, warmup: int):
     sampler = ClockSampler(None)
     sampler.start()
     time.sleep(0.3)
-    for name, (fn, bpe) in cases.items():
+    for name, (fn, bpe, launches) in cases.items():
         for i in range(max(warmup, ACT_RING)):
             fn(ring[i % ACT_RING])
         torch.cuda.synchronize()
@@ -326,7 +333,8 @@ def measure_activations(dev, steps: int, warmup: int):
         ms = e0.elapsed_time(e1) / steps
         gbs = bpe * n / (ms / 1e3) / 1e9
         res[name] = {"ms": ms, "elements_per_s": n / (ms / 1e3), "GB/s": gbs,
-                     "frac_of_hbm": gbs / peak, "algorithmic_bytes_per_element": bpe}
+                     "frac_of_hbm": gbs / peak, "algorithmic_bytes_per_element": bpe,
+                     "launches_per_call": launches}
     clocks = sampler.stop()
     return res, clocks, n, G, peak, peak_kind
 
@@ -367,11 +375,7 @@ def run_activations(args):
                          "frac": head["frac_of_hbm"], "traffic": recorded_act_traffic(n),
                          "peak_source": f"{peak_kind} copy bandwidth"},
             "kernels": res, "clocks": clocks,
-            # 1xG 1; GS standalone 3 (zeroing the tensor maximum, step (i), the
-            # cast); SwiGLU 2 (zeroing its tensor-maximum slot, the producer);
-            # LayerNorm 1; GS after the producer 2 (zeroing, the cast with step
-            # (ii) folded in); the cast alone 1; dequant 1
-            "gpu_launches": args.steps * (1 + 3 + 2 + 1 + 2 + 1 + 1)}
+            "gpu_launches": args.steps * sum(r["launches_per_call"] for r in res.values())}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -422,13 +422,16 @@ coat_status_t coat_state_stats(const uint8_t *code, const float *k, const float 
  * projections): row-wise LayerNorm (rms = 0: y = (x - mean) / sqrt(var +
  * eps), var the mean squared deviation) or RMSNorm (rms = 1: y = x /
  * sqrt(mean(x^2) + eps)), times weight[c] and plus bias[c] (LayerNorm only)
- * when given, rounded to BF16; plus the maxima of |out| over every 1xG run
- * of each row.  Evaluated in binary32 (row sums in a fixed order, divided
- * by cols with the correctly rounded quotient, so a row whose sum is exact
- * -- a constant row, say -- gets its exact mean), with an error of about
- * 1e-6 x (|y| + |mean| / std) (x - mean carries the rounding of the mean):
- * the output is the correctly rounded norm except within that distance of
- * a BF16 rounding midpoint.
+ * when given (with both, y weight + bias is one fused multiply-add),
+ * rounded to BF16; plus the maxima of |out| over every 1xG run of each row.
+ * Evaluated in binary32 (row sums in a fixed order, divided by cols with
+ * the correctly rounded quotient, so a row whose sum is exact -- a constant
+ * row, say -- gets its exact mean), with an error of about 1e-6 x (|out| +
+ * (|x - mean| + |mean|) / std x |weight|) (x - mean carries the rounding
+ * of the mean; with a bias the error is relative to the product, not to
+ * the sum): the output is the correctly rounded norm except within that
+ * distance of a BF16 rounding midpoint.  weight and bias are read 16 bytes
+ * at a time when both (those given) are 16-byte aligned.
  *   x           BF16 bits [rows, cols] row-major (16-byte aligned),
  *               cols a multiple of 16 and of G, cols <= 16384
  *   weight,bias float32 [cols] or NULL (bias must be NULL when rms = 1)

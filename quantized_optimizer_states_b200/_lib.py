@@ -306,12 +306,25 @@ def coat_group_scaling_quant_pertensor_noalloc(x, q, scale, *, group_size: int =
     _check("coat_group_scaling_quant_pertensor_noalloc", st)
 
 
+def _tensor_amax_slot(tensor_amax, group_amax, ng):
+    """The producers' tensor-maximum slot: "auto" takes the slot after the
+    group maxima when group_amax is a whole Group Scaling workspace
+    (ceil(n/G) + 1 floats), so that Group Scaling can run as the cast alone
+    (amax_precomputed=2); None writes no tensor maximum."""
+    if isinstance(tensor_amax, str):
+        if tensor_amax != "auto":
+            raise ValueError('tensor_amax must be a tensor, None or "auto"')
+        return _slot(group_amax[ng:ng + 1]) if group_amax.numel() > ng else None
+    return _slot(tensor_amax)
+
+
 def coat_swiglu_group_amax(gate, up, out, group_amax, *, group_size: int = 128,
-                           tensor_amax=None, stream=None):
+                           tensor_amax="auto", stream=None):
     """out = RN_bf16(silu(gate) * up) and the per-1xG maxima of out, ready
-    for coat_group_scaling_quant_pertensor(..., amax_precomputed=1); with
-    tensor_amax (a float32 slot, e.g. workspace[ceil(n/G):]) also the maximum
-    of all of out, for amax_precomputed=2."""
+    for coat_group_scaling_quant_pertensor(..., amax_precomputed=1); with a
+    tensor_amax slot (a float32 tensor; by default the slot after the group
+    maxima when group_amax is a whole Group Scaling workspace) also the
+    maximum of all of out, for amax_precomputed=2."""
     import torch
     if gate.numel() != up.numel() or out.numel() != gate.numel():
         raise ValueError("gate, up and out must have the same number of elements")
@@ -320,21 +333,23 @@ def coat_swiglu_group_amax(gate, up, out, group_amax, *, group_size: int = 128,
         raise ValueError(f"group_amax needs {ng} float32 slots")
     st = load().coat_swiglu_group_amax(
         _u16(gate, "gate"), _u16(up, "up"), gate.numel(), group_size, _u16(out, "out"),
-        _ptr(group_amax, torch.float32, "group_amax"), _slot(tensor_amax), _stream(stream))
+        _ptr(group_amax, torch.float32, "group_amax"),
+        _tensor_amax_slot(tensor_amax, group_amax, ng), _stream(stream))
     _check("coat_swiglu_group_amax", st)
 
 
 def coat_norm_group_amax(x, out, group_amax, *, rms: bool = False, eps: float = 1e-5,
-                         weight=None, bias=None, group_size: int = 128, tensor_amax=None,
+                         weight=None, bias=None, group_size: int = 128, tensor_amax="auto",
                          stream=None):
     """LayerNorm (or RMSNorm) of BF16 rows x [rows, cols] into BF16 `out` with
     the maxima of every 1xG run of the output in `group_amax` (see
-    include/coat.h)."""
+    include/coat.h); tensor_amax as for coat_swiglu_group_amax."""
     import torch
     if x.dim() != 2 or out.shape != x.shape:
         raise ValueError("x and out must be [rows, cols] tensors of the same shape")
     rows, cols = x.shape
-    if group_amax.numel() < rows * (cols // max(group_size, 1)):
+    ng = rows * (cols // max(group_size, 1))
+    if group_amax.numel() < ng:
         raise ValueError("group_amax needs rows * cols / G elements")
     for t, what in ((weight, "weight"), (bias, "bias")):
         if t is not None and t.numel() != cols:
@@ -342,7 +357,8 @@ def coat_norm_group_amax(x, out, group_amax, *, rms: bool = False, eps: float = 
     _check("coat_norm_group_amax", load().coat_norm_group_amax(
         _u16(x, "x"), rows, cols, int(rms), float(eps), _ptr(weight, torch.float32, "weight"),
         _ptr(bias, torch.float32, "bias"), group_size, _u16(out, "out"),
-        _ptr(group_amax, torch.float32, "group_amax"), _slot(tensor_amax), _stream(stream)))
+        _ptr(group_amax, torch.float32, "group_amax"),
+        _tensor_amax_slot(tensor_amax, group_amax, ng), _stream(stream)))
 
 
 def coat_fp8_encode(y, q, *, fmt: int = COAT_E4M3, stream=None):

@@ -432,6 +432,7 @@ struct NormParams {
   int rms;
   float eps;
   uint32_t *tensor_amax; // nullable: also the maximum of all outputs (bits, zeroed first)
+  bool affine_vec;       // weight and bias (those given) are 16-byte aligned
 };
 
 constexpr int kNormMaxCols = 16384;
@@ -520,13 +521,15 @@ __device__ __forceinline__ float norm_one_row(const NormParams &p, const uint4 *
         const int c = 16 * j + 2 * i;
         float y0 = (bf16lo_to_float(wv[i]) - mean) * rstd;
         float y1 = (bf16hi_to_float(wv[i]) - mean) * rstd;
-        if (p.weight) {
-          y0 *= p.weight[c];
-          y1 *= p.weight[c + 1];
-        }
-        if (p.bias) {
-          y0 += p.bias[c];
-          y1 += p.bias[c + 1];
+        if (p.weight && p.bias) {   // y w + b, one fused multiply-add
+          y0 = __fmaf_rn(y0, p.weight[c], p.bias[c]);
+          y1 = __fmaf_rn(y1, p.weight[c + 1], p.bias[c + 1]);
+        } else if (p.weight) {
+          y0 = __fmul_rn(y0, p.weight[c]);
+          y1 = __fmul_rn(y1, p.weight[c + 1]);
+        } else if (p.bias) {
+          y0 = __fadd_rn(y0, p.bias[c]);
+          y1 = __fadd_rn(y1, p.bias[c + 1]);
         }
         ow[i] = bf16x2_rn(y0, y1);
         a = fmaxf(a, fmaxf(fabsf(bf16lo_to_float(ow[i])), fabsf(bf16hi_to_float(ow[i]))));
@@ -607,13 +610,30 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
   return make_float2(bf16lo_to_float(w), bf16hi_to_float(w));
 }
 
+// 8 consecutive floats as 4 pairs: two 16-byte loads when `vec` (the
+// vector's base, and so every 8-column chunk of it, is 16-byte aligned),
+// else one load a float.
+__device__ __forceinline__ void load8_f32(const float *a, bool vec, float2 (&o)[4]) {
+  if (vec) {
+    const float4 u = __ldg(reinterpret_cast<const float4 *>(a));
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(a) + 1);
+    o[0] = make_float2(u.x, u.y); o[1] = make_float2(u.z, u.w);
+    o[2] = make_float2(v.x, v.y); o[3] = make_float2(v.z, v.w);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = make_float2(__ldg(a + 2 * j), __ldg(a + 2 * j + 1));
+  }
+}
+
 // One row of 256 NC columns held in registers: src is the row (its 32 NC
 // 16-byte chunks, in global or shared memory), lane l takes chunks l + 32 i.
 // The arithmetic runs on packed binary32 pairs: the row sums as four partial
 // sums a lane (two packed pairs, alternate pairs of columns), the
 // normalisation two columns an instruction, and each 1xG maximum of |out|
 // on the BF16 outputs themselves (pairs with their sign bits cleared).
-template <int NC>
+// kAffine: a weight and/or a bias is given (an instantiation of its own, so
+// the plain norm carries no affine code at all).
+template <int NC, bool kAffine>
 __device__ __forceinline__ float norm_reg_row(const NormParams &p, const uint4 *src, int64_t row,
                                               int lane) {
   uint4 c[NC];
@@ -667,14 +687,29 @@ __device__ __forceinline__ float norm_reg_row(const NormParams &p, const uint4 *
     const int col0 = 8 * (lane + 32 * i);
     uint32_t ow[4];
     uint32_t am = 0u;
+    if constexpr (kAffine) {
+      // the affine terms of the chunk's 8 columns: two 16-byte loads each
+      // where the vectors allow it (one load a column otherwise); with both,
+      // y w + b is one fused multiply-add
+      float2 w2[4], b2[4];
+      if (p.weight) load8_f32(p.weight + col0, p.affine_vec, w2);
+      if (p.bias) load8_f32(p.bias + col0, p.affine_vec, b2);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int cc = col0 + 2 * j;
-      float2 y = mul2_rn(add2_rn(bf16x2_to_float2(wv[j]), NM), RS);
-      if (p.weight) y = mul2_rn(y, make_float2(p.weight[cc], p.weight[cc + 1]));
-      if (p.bias) y = add2_rn(y, make_float2(p.bias[cc], p.bias[cc + 1]));
-      ow[j] = bf16x2_rn(y.x, y.y);
-      am = bmax2(am, ow[j] & 0x7FFF7FFFu);
+      for (int j = 0; j < 4; ++j) {
+        float2 y = mul2_rn(add2_rn(bf16x2_to_float2(wv[j]), NM), RS);
+        if (p.weight && p.bias) y = fma2_rn(y, w2[j], b2[j]);
+        else if (p.weight) y = mul2_rn(y, w2[j]);
+        else y = add2_rn(y, b2[j]);
+        ow[j] = bf16x2_rn(y.x, y.y);
+        am = bmax2(am, ow[j] & 0x7FFF7FFFu);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 y = mul2_rn(add2_rn(bf16x2_to_float2(wv[j]), NM), RS);
+        ow[j] = bf16x2_rn(y.x, y.y);
+        am = bmax2(am, ow[j] & 0x7FFF7FFFu);
+      }
     }
     dst[lane + 32 * i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
     float a = fmaxf(bf16lo_to_float(am), bf16hi_to_float(am));
@@ -705,7 +740,7 @@ constexpr size_t norm_reg_smem() {
 // warps finish together, and it copies that next row into the second of its
 // two shared-memory buffers (cp.async, its own chunks only, so no barrier)
 // while it normalises the current one.
-template <int NC>
+template <int NC, bool kAffine>
 __global__ void __launch_bounds__(32 * kNormRegWarps, 2) norm_reg_group_amax_kernel(const NormParams p) {
   extern __shared__ __align__(16) uint4 nbuf[];
   __shared__ unsigned int next_row;
@@ -737,7 +772,7 @@ __global__ void __launch_bounds__(32 * kNormRegWarps, 2) norm_reg_group_amax_ker
     } else {
       cp_async_wait_all();
     }
-    wmax = fmaxf(wmax, norm_reg_row<NC>(p, wb + (k & 1) * 32 * NC, row, lane));
+    wmax = fmaxf(wmax, norm_reg_row<NC, kAffine>(p, wb + (k & 1) * 32 * NC, row, lane));
     row = nxt;
   }
   if (p.tensor_amax) block_max_to_tensor(wmax, p.tensor_amax);

@@ -258,9 +258,9 @@ coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *
 // Register-resident norm rows of 256 NC columns: persistent grid of the
 // blocks that fit the GPU at once (or fewer, for few rows), the occupancy
 // looked up once per device.
-template <int NC>
-coat_status_t launch_norm_reg(cudaStream_t s, const coat::NormParams &p) {
-  constexpr auto kernel = coat::norm_reg_group_amax_kernel<NC>;
+template <int NC, bool kAffine>
+coat_status_t launch_norm_reg_form(cudaStream_t s, const coat::NormParams &p) {
+  constexpr auto kernel = coat::norm_reg_group_amax_kernel<NC, kAffine>;
   constexpr size_t smem = coat::norm_reg_smem<NC>();
   const cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -273,6 +273,13 @@ coat_status_t launch_norm_reg(cudaStream_t s, const coat::NormParams &p) {
   const unsigned int grid = coat::resident_grid<kernel>(32 * coat::kNormRegWarps, smem, blocks_needed);
   launch_act_threads(kernel, grid, 32u * coat::kNormRegWarps, smem, s, p);
   return launch_status();
+}
+
+// weight or bias given: the instantiation with the affine terms
+template <int NC>
+coat_status_t launch_norm_reg(cudaStream_t s, const coat::NormParams &p) {
+  return (p.weight || p.bias) ? launch_norm_reg_form<NC, true>(s, p)
+                              : launch_norm_reg_form<NC, false>(s, p);
 }
 
 }  // namespace
@@ -553,6 +560,7 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
   p.rms = rms;
   p.eps = eps;
   p.tensor_amax = reinterpret_cast<uint32_t *>(tensor_amax);
+  p.affine_vec = aligned16(weight) && aligned16(bias);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (tensor_amax)
     launch_act_threads(coat::zero_word_kernel, 1u, 32u, 0, s,

@@ -32,18 +32,33 @@ MAX_FLIPS = 1e-3       # fraction of elements allowed one BF16 step off
 
 
 def _midpoint_ok(orc, y64, got_bits, want_bits, offset):
-    """Every difference is one BF16 step, next to a rounding midpoint: within
-    WINDOW x (|midpoint| + offset), offset = |mean| / std of the element's
-    row scaled like y (x - mean loses the binary32 rounding of the mean)."""
+    """Every difference is the correct rounding of a value within the
+    binary32 evaluation's error of the binary64 norm: |got - y| <= half a
+    BF16 step of got + WINDOW x (|y| + offset), offset = (|x - mean| +
+    |mean|) / std x |weight| of the element's row (x - mean carries the
+    rounding of the mean; with a bias the product's rounding is relative
+    to it, not to y).  Without a bias that is one BF16 step next to a
+    rounding midpoint."""
     bad = np.nonzero(got_bits != want_bits)[0]
     assert bad.size <= MAX_FLIPS * got_bits.size, bad.size
     for i in bad:
-        a = orc.bf16_bits_to_f64(np.array([got_bits[i]]))[0]
-        b = orc.bf16_bits_to_f64(np.array([want_bits[i]]))[0]
-        assert abs(int(got_bits[i]) - int(want_bits[i])) == 1, i
-        mid = 0.5 * (a + b)
-        assert abs(y64[i] - mid) <= WINDOW * (abs(mid) + offset[i]), i
+        g = orc.bf16_bits_to_f64(np.array([got_bits[i], got_bits[i] + 1, got_bits[i] - 1],
+                                          dtype=np.uint16))
+        half = 0.5 * max(abs(g[1] - g[0]), abs(g[0] - g[2]))
+        assert abs(g[0] - y64[i]) <= half + WINDOW * (abs(y64[i]) + offset[i]), i
     return bad.size
+
+
+def _offset(orc, x, weight, rms):
+    """(|x - mean| + |mean|) / std x |weight| per element (binary64)."""
+    xf = orc.bf16_bits_to_f64(x)
+    w = np.ones(x.shape[1]) if weight is None else np.abs(weight.astype(np.float64))
+    if rms:
+        sd = np.sqrt((xf ** 2).mean(axis=1, keepdims=True) + float(np.float32(1e-5)))
+        return (np.abs(xf) / sd * w).reshape(-1)
+    mu = xf.mean(axis=1, keepdims=True)
+    sd = np.sqrt(((xf - mu) ** 2).mean(axis=1, keepdims=True) + float(np.float32(1e-5)))
+    return ((np.abs(xf - mu) + np.abs(mu)) / sd * w).reshape(-1)
 
 
 # widths that are multiples of 256 up to 2048 take the register-resident
@@ -74,15 +89,39 @@ def test_norm_matches_oracle(lib, orc, rows, cols, G, rms):
     got = parity.to_host(out).view(np.uint16).reshape(-1)
     y64 = orc.norm_f64(x, rms=rms, eps=1e-5, weight=weight, bias=bias).reshape(-1)
     want = orc.round_to_bf16(y64)
-    xf = orc.bf16_bits_to_f64(x)
-    if rms:
-        offset = np.zeros(x.size)
-    else:
-        mu = xf.mean(axis=1, keepdims=True)
-        sd = np.sqrt(((xf - mu) ** 2).mean(axis=1, keepdims=True) + float(np.float32(1e-5)))
-        offset = np.broadcast_to(np.abs(mu) / sd * np.abs(weight), x.shape).reshape(-1)
-    _midpoint_ok(orc, y64, got, want, offset)
+    _midpoint_ok(orc, y64, got, want, _offset(orc, x, weight, rms))
     assert np.array_equal(parity.to_host(ga), orc.group_amax_of(got, G))
+
+
+@pytest.mark.parametrize("cols", [2048, 768, 1040])
+def test_norm_affine_terms_at_any_4_byte_alignment(lib, orc, cols):
+    """weight and bias 16-byte aligned (the register form loads 8 columns
+    by two 16-byte loads) and at a 4-byte offset (one load a column): the
+    same output and maxima bit for bit, and those of the oracle check."""
+    import torch
+    rows, G = 40, 16
+    x = inputs.host_activations(inputs.activations(seed=cols), rows=rows)
+    x = np.tile(x, (1, -(-cols // x.shape[1])))[:, :cols].copy()
+    rng = np.random.default_rng(cols + 1)
+    weight = (1.0 + 0.1 * rng.standard_normal(cols)).astype(np.float32)
+    bias = (0.05 * rng.standard_normal(cols)).astype(np.float32)
+    runs = []
+    for off in (0, 1):
+        wbuf = torch.zeros(cols + 4, dtype=torch.float32, device="cuda")
+        bbuf = torch.zeros(cols + 4, dtype=torch.float32, device="cuda")
+        wbuf[off:off + cols] = torch.from_numpy(weight)
+        bbuf[off:off + cols] = torch.from_numpy(bias)
+        out = torch.empty(rows, cols, dtype=torch.int16, device="cuda")
+        ga = torch.empty(rows * cols // G, dtype=torch.float32, device="cuda")
+        lib.coat_norm_group_amax(parity.to_dev(x.view(np.int16)), out, ga, eps=1e-5,
+                                 weight=wbuf[off:off + cols], bias=bbuf[off:off + cols],
+                                 group_size=G)
+        torch.cuda.synchronize()
+        runs.append((parity.to_host(out).view(np.uint16).reshape(-1), parity.to_host(ga)))
+    assert np.array_equal(runs[0][0], runs[1][0]) and np.array_equal(runs[0][1], runs[1][1])
+    y64 = orc.norm_f64(x, rms=False, eps=1e-5, weight=weight, bias=bias).reshape(-1)
+    _midpoint_ok(orc, y64, runs[0][0], orc.round_to_bf16(y64), _offset(orc, x, weight, False))
+    assert np.array_equal(runs[0][1], orc.group_amax_of(runs[0][0], G))
 
 
 def test_norm_feeds_group_scaling(lib, orc):

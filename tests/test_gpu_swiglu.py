@@ -142,3 +142,32 @@ def test_argument_errors(lib):
         lib.coat_swiglu_group_amax(x, x, x, ga, group_size=100)
     with pytest.raises(ValueError):
         lib.coat_swiglu_group_amax(x, x[:128], x, ga, group_size=128)
+
+
+def test_producers_write_the_tensor_max_into_a_whole_workspace_by_default(lib):
+    """Handed a whole Group Scaling workspace (ceil(n/G) + 1 floats), both
+    producers write the tensor maximum into its last slot unless told not
+    to (tensor_amax=None leaves the slot as it was); handed exactly the
+    group maxima they write nothing past them."""
+    G, rows, cols = 128, 24, 1024
+    w = inputs.activations(seed=3)
+    gate, up = inputs.host_swiglu_inputs(w, rows=rows)
+    gate, up = gate[:, :cols].copy(), up[:, :cols].copy()
+    n = gate.size
+    ng = n // G
+    for default in (True, False):
+        out = torch.empty(n, dtype=torch.int16, device="cuda")
+        ws = torch.full((ng + 1,), -5.0, dtype=torch.float32, device="cuda")
+        kw = {} if default else {"tensor_amax": None}
+        lib.coat_swiglu_group_amax(_dev(gate), _dev(up), out, ws, group_size=G, **kw)
+        ln = torch.empty(rows, cols, dtype=torch.int16, device="cuda")
+        ws2 = torch.full((ng + 1,), -5.0, dtype=torch.float32, device="cuda")
+        lib.coat_norm_group_amax(out.view(rows, cols), ln, ws2, group_size=G, **kw)
+        torch.cuda.synchronize()
+        for buf in (ws, ws2):
+            want = float(buf[:ng].max().item()) if default else -5.0
+            assert float(buf[ng].item()) == want
+    exact = torch.full((ng + 8,), -5.0, dtype=torch.float32, device="cuda")
+    lib.coat_swiglu_group_amax(_dev(gate), _dev(up), out, exact[:ng], group_size=G)
+    torch.cuda.synchronize()
+    assert torch.all(exact[ng:] == -5.0)

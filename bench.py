@@ -834,6 +834,15 @@ def time_step_set(w, v_fmt: int, steps: int, warmup: int, dev) -> dict:
             "frac_of_hbm": gbs / peak}
 
 
+def clock_normalised(value, clocks):
+    """value x (max SM clock / median SM clock under load), or None when the
+    clocks were not sampled."""
+    med, top = (clocks or {}).get("sm_mhz"), (clocks or {}).get("sm_max_mhz")
+    if not med or not top:
+        return None
+    return {"params_per_s_at_max_clock": value * top / med, "sm_mhz": med, "sm_max_mhz": top}
+
+
 def run_step(args):
     """One GPU: coat_adamw_fp8_step over the whole resident parameter set."""
     import torch
@@ -1055,6 +1064,10 @@ def run_step(args):
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": clocks,
+        # the headline scaled by max / median SM clock of the timed region:
+        # what the same kernel gives where the power cap does not lower the
+        # clock (an estimate beside the measured value, not a measurement)
+        "clock_normalised": clock_normalised(value, clocks),
         "kernel_ms": kernel_ms,
         # beside the headline, outside its timed region
         "variant_other_v_fmt": variant,

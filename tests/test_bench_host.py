@@ -3,6 +3,8 @@ roofline divides by, the source-hash keyed traffic records, the peaks."""
 import json
 import os
 
+import pytest
+
 import bench
 
 
@@ -121,3 +123,11 @@ def test_gpus_n_starts_n_ranks_that_all_join():
     lines = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1, out.stdout
     assert lines[0]["n_gpus"] == 2 and lines[0]["ranks_joined"] == 2
+
+
+def test_clock_normalised_scales_by_max_over_median_clock():
+    import bench
+    got = bench.clock_normalised(3.0e11, {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0})
+    assert got["params_per_s_at_max_clock"] == pytest.approx(3.0e11 * 1965.0 / 1800.0)
+    assert bench.clock_normalised(1.0, None) is None
+    assert bench.clock_normalised(1.0, {"sm_mhz": None, "sm_max_mhz": 1965.0}) is None

@@ -185,6 +185,48 @@ coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, ui
                                           const uint32_t *skip_if_nonzero, void *stream);
 
 /*
+ * coat_adamw_fp8_step_peers -- one ZeRO-1 data-parallel step of this rank's
+ * shard in one kernel ([COAT] "结果和边界": multi-GPU data-parallel
+ * training; the optimizer state is partitioned over the ranks at 1xG group
+ * boundaries): the reduce-scatter of the ranks' gradients, the step of
+ * coat_adamw_fp8_step on the shard, and the all-gather of the updated
+ * parameters, over peer memory (plain loads and stores; NVLink between
+ * GPUs).
+ *   grads      host array of `world` device pointers: rank r's full BF16
+ *              gradient buffer, mapped into this process; the shard's
+ *              gradient element i is the mean of grads[r][grad_offset + i]
+ *              over r, RN_bf16(RN32(sum) / world) with the sum in binary32
+ *              in rank order (world = 1: the gradient itself)
+ *   world      1 .. COAT_MAX_PEERS
+ *   param      float32[n]: this rank's FP32 master weights (its shard),
+ *              updated in place
+ *   params_out host array of `world` device pointers or NULL: rank r's full
+ *              parameter buffer (float32, or BF16 when params_out_bf16 = 1);
+ *              every updated parameter i is also stored at
+ *              params_out[r][params_out_offset + i] (an entry may be NULL:
+ *              that rank gets no copy)
+ *   m_code .. v_scale, n, cfg   this rank's shard, as coat_adamw_fp8_step
+ * Every grads[r] + grad_offset and params_out[r] + params_out_offset must be
+ * 16-byte aligned.  The caller orders the call between two barriers of all
+ * ranks: after every rank's gradient is complete, and before any rank
+ * reads its parameters (the kernel reads other ranks' gradients and writes
+ * their parameter buffers; it waits for nothing on the device).  The
+ * kernel makes its stores to other ranks' memory visible system-wide
+ * before it finishes.
+ * Errors: INVALID_ARG (world, a NULL gradient pointer, offsets < 0,
+ * params_out_bf16 not 0/1, and as coat_adamw_fp8_step), MISALIGNED,
+ * UNSUPPORTED, CUDA.
+ */
+#define COAT_MAX_PEERS 8
+coat_status_t coat_adamw_fp8_step_peers(const uint16_t *const *grads, int32_t world,
+                                        int64_t grad_offset, float *param,
+                                        void *const *params_out, int32_t params_out_bf16,
+                                        int64_t params_out_offset, uint8_t *m_code, float *m_k,
+                                        float *m_scale, uint8_t *v_code, float *v_k,
+                                        float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
+                                        void *stream);
+
+/*
  * coat_quantize_state -- compress an FP32 optimizer state into COAT's FP8
  * form (the re-quantization half of the step, on its own): used to
  * initialize or convert states.  [COAT] "扩展函数".

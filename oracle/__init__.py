@@ -186,6 +186,22 @@ def to_bf16_array(x: np.ndarray) -> np.ndarray:
     return out
 
 
+def grad_mean_bf16(grads) -> np.ndarray:
+    """The data-parallel gradient of one step (COAT summary, section
+    "结果和边界": multi-GPU training, every rank computing a full BF16
+    gradient): the mean of the ranks' BF16 gradients, summed in binary32 in
+    rank order (one rounding per addition), divided by the rank count in
+    binary32 and rounded to BF16 (nearest even).  grads: a sequence of BF16
+    bit arrays of one shape; one rank gives its gradient unchanged."""
+    grads = [np.asarray(g, dtype=np.uint16) for g in grads]
+    acc = bf16_bits_to_f64(grads[0]).astype(np.float32)
+    for g in grads[1:]:
+        acc = np.add(acc, bf16_bits_to_f64(g).astype(np.float32), dtype=np.float32)
+    if len(grads) > 1:
+        acc = np.divide(acc, np.float32(len(grads)), dtype=np.float32)
+    return to_bf16_array(acc)
+
+
 def adamw_fp8_step(theta, grad_bf16, m_code, m_k, m_s, v_code, v_k, v_s, *, beta1, beta2, lr,
                    eps, weight_decay, step, group_size, m_fmt=E4M3, v_fmt=E4M3, k_range=0,
                    k_max=64.0, force_k1=False, return_moments=False):

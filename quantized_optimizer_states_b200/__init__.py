@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     CoatError,
     PackTable,
     coat_adamw_fp8_step,
+    coat_adamw_fp8_step_peers,
     coat_count_nonfinite_bf16,
     coat_dequant,
     coat_fp8_encode,

@@ -68,6 +68,9 @@ SIGNATURES = {
     "coat_fp8_encode": (_I32, [_P, _I64, _I32, _P, _P]),
     "coat_norm_group_amax": (_I32, [_P, _I64, _I64, _I32, _F, _P, _P, _I32, _P, _P, _P, _P]),
     "coat_count_nonfinite_bf16": (_I32, [_P, _I64, _P, _P]),
+    "coat_adamw_fp8_step_peers": (_I32, [ctypes.POINTER(_P), _I32, _I64, _P, ctypes.POINTER(_P),
+                                         _I32, _I64, _P, _P, _P, _P, _P, _P, _I64,
+                                         ctypes.POINTER(CoatAdamwCfg), _P]),
     "coat_adamw_fp8_step_guarded": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
                                            ctypes.POINTER(CoatAdamwCfg), _P, _P]),
     "coat_adamw_fp8_step_fp32grad": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
@@ -213,6 +216,71 @@ def coat_adamw_fp8_step(param, grad, m_code, m_k, m_scale, v_code, v_k, v_scale,
         st = load().coat_adamw_fp8_step_guarded(*args, _ptr(skip_if_nonzero, None, "skip"),
                                                 _stream(stream))
         _check("coat_adamw_fp8_step_guarded", st)
+
+
+COAT_MAX_PEERS = 8  # mirrors include/coat.h
+
+
+def _peer_ptr(t, dtype, what):
+    """Address of a contiguous CUDA tensor that may live on another GPU (a
+    rank's buffer mapped into this process); None stays None."""
+    if t is None:
+        return None
+    if t.get_device() < 0:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous() or t.dtype != dtype:
+        raise ValueError(f"{what} must be a contiguous {dtype} tensor")
+    return t.data_ptr()
+
+
+def coat_adamw_fp8_step_peers(grads, param, m_code, m_k, m_scale, v_code, v_k, v_scale, *,
+                              grad_offset: int, params_out=None, params_out_offset: int = 0,
+                              beta1: float, beta2: float, lr: float, eps: float,
+                              weight_decay: float, step: int, group_size: int = 128,
+                              m_fmt: int = COAT_E4M3, v_fmt: int = COAT_E4M3, k_range: int = 0,
+                              k_max: float = 64.0, flags: int = 0, stream=None):
+    """The ZeRO-1 step of this rank's shard in one kernel (see include/coat.h):
+    grads = every rank's full BF16 gradient buffer (rank order; tensors that
+    may live on other GPUs), the shard starting at grad_offset; params_out =
+    every rank's full parameter buffer (float32 or bfloat16, one dtype for
+    all; None entries or None: no copy), the shard at params_out_offset;
+    param and the states are this rank's shard."""
+    import torch
+    world = len(grads)
+    if not 1 <= world <= COAT_MAX_PEERS:
+        raise ValueError(f"1 to {COAT_MAX_PEERS} ranks")
+    n = param.numel()
+    if m_code.numel() != n or v_code.numel() != n:
+        raise ValueError("m_code and v_code must have as many elements as param")
+    for g in grads:
+        if g.numel() < grad_offset + n:
+            raise ValueError("a gradient buffer ends before the shard does")
+    out_bf16 = 0
+    outs = [None] * world
+    if params_out is not None:
+        if len(params_out) != world:
+            raise ValueError("params_out needs one entry per rank")
+        dts = {t.dtype for t in params_out if t is not None}
+        if len(dts) > 1 or not dts <= {torch.float32, torch.bfloat16}:
+            raise ValueError("params_out tensors must all be float32 or all bfloat16")
+        out_bf16 = int(dts == {torch.bfloat16})
+        for r, t in enumerate(params_out):
+            if t is not None and t.numel() < params_out_offset + n:
+                raise ValueError("a parameter buffer ends before the shard does")
+            outs[r] = _peer_ptr(t, torch.bfloat16 if out_bf16 else torch.float32,
+                                f"params_out[{r}]")
+    gptr = (_P * world)(*[_peer_ptr(g.view(torch.int16) if g.dtype != torch.int16 else g,
+                                    torch.int16, f"grads[{r}]") for r, g in enumerate(grads)])
+    optr = (_P * world)(*outs) if params_out is not None else None
+    cfg = CoatAdamwCfg(beta1, beta2, lr, eps, weight_decay, step, group_size, m_fmt, v_fmt,
+                       k_range, k_max, flags)
+    st = load().coat_adamw_fp8_step_peers(
+        gptr, world, grad_offset, _ptr(param, torch.float32, "param"), optr, out_bf16,
+        params_out_offset, _ptr(m_code, torch.uint8, "m_code"), _ptr(m_k, torch.float32, "m_k"),
+        _ptr(m_scale, torch.float32, "m_scale"), _ptr(v_code, torch.uint8, "v_code"),
+        _ptr(v_k, torch.float32, "v_k"), _ptr(v_scale, torch.float32, "v_scale"), n,
+        ctypes.byref(cfg), _stream(stream))
+    _check("coat_adamw_fp8_step_peers", st)
 
 
 def coat_count_nonfinite_bf16(x, count, *, stream=None):

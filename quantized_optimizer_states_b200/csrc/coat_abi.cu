@@ -134,15 +134,16 @@ coat_status_t launch_step(void (*kernel)(coat::StepParams), unsigned int grid, i
   return launch_status();
 }
 
-// The step kernel is instantiated for each supported group size and for
-// full blocks / the ragged tail block, and for BF16 / float32 gradients.
-template <int VF, bool FULL, bool GF32>
+// The step kernel is instantiated for each supported group size, for full
+// blocks / the ragged tail block, and per gradient source (BF16, float32,
+// or the ranks' BF16 gradients in peer memory).
+template <int VF, bool FULL, int GS>
 coat_status_t launch_step_for(int lg, unsigned int grid, int block, size_t smem, cudaStream_t s,
                               const coat::StepParams &p) {
   switch (lg) {
 #define COAT_LAUNCH(LGV) \
   case LGV:              \
-    return launch_step(coat::adamw_fp8_step_kernel<VF, LGV, FULL, GF32>, grid, block, smem, s, p);
+    return launch_step(coat::adamw_fp8_step_kernel<VF, LGV, FULL, GS>, grid, block, smem, s, p);
     COAT_LAUNCH(4) COAT_LAUNCH(5) COAT_LAUNCH(6) COAT_LAUNCH(7) COAT_LAUNCH(8)
     COAT_LAUNCH(9) COAT_LAUNCH(10) COAT_LAUNCH(11) COAT_LAUNCH(12)
 #undef COAT_LAUNCH
@@ -152,7 +153,7 @@ coat_status_t launch_step_for(int lg, unsigned int grid, int block, size_t smem,
 
 // One launch over the full blocks (no bounds checks), then, if n is not a
 // multiple of the block's parameter count, one block for the ragged tail.
-template <int VF, bool GF32>
+template <int VF, int GS>
 coat_status_t launch_step_all(int lg, int64_t n, cudaStream_t s, coat::StepParams p) {
   size_t smem = 0;
   int block = 0;
@@ -163,22 +164,34 @@ coat_status_t launch_step_all(int lg, int64_t n, cudaStream_t s, coat::StepParam
   if (full > 0) {
     p.block0 = 0;
     const coat_status_t st =
-        launch_step_for<VF, true, GF32>(lg, static_cast<unsigned int>(full), block, smem, s, p);
+        launch_step_for<VF, true, GS>(lg, static_cast<unsigned int>(full), block, smem, s, p);
     if (st != COAT_OK) return st;
   }
   if (n % per != 0) {
     p.block0 = full;
-    return launch_step_for<VF, false, GF32>(lg, 1u, block, smem, s, p);
+    return launch_step_for<VF, false, GS>(lg, 1u, block, smem, s, p);
   }
   return COAT_OK;
 }
 
+static_assert(COAT_MAX_PEERS == coat::kMaxPeers, "peer count of the header and the kernel");
+
+// The ranks' buffers of the peer form (coat_adamw_fp8_step_peers), already
+// offset to this shard.
+struct PeerArgs {
+  const uint16_t *grad[coat::kMaxPeers];
+  void *param[coat::kMaxPeers];
+  int world;
+  int param_bf16;
+};
+
 coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *m_code,
                         float *m_k, float *m_scale, uint8_t *v_code, float *v_k,
                         float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
-                        const uint32_t *skip, void *stream) {
+                        const uint32_t *skip, void *stream, const PeerArgs *peers = nullptr) {
   if (!cfg || n < 0) return COAT_ERR_INVALID_ARG;
-  if (n > 0 && (!param || !grad || !m_code || !m_k || !m_scale || !v_code || !v_k || !v_scale))
+  if (n > 0 && (!param || (!grad && !peers) || !m_code || !m_k || !m_scale || !v_code ||
+                !v_k || !v_scale))
     return COAT_ERR_INVALID_ARG;
   if (cfg->step < 1 || !(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) ||
       !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f) || !(cfg->k_max >= 0.0f) ||
@@ -195,6 +208,20 @@ coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *
     return COAT_ERR_MISALIGNED;
 
   coat::StepParams p;
+  p.world = 1;
+  p.param_peer_bf16 = 0;
+  for (int r = 0; r < coat::kMaxPeers; ++r) {
+    p.grad_peer[r] = nullptr;
+    p.param_peer[r] = nullptr;
+  }
+  if (peers) {
+    p.world = peers->world;
+    p.param_peer_bf16 = peers->param_bf16;
+    for (int r = 0; r < peers->world; ++r) {
+      p.grad_peer[r] = peers->grad[r];
+      p.param_peer[r] = peers->param[r];
+    }
+  }
   p.theta = param;
   p.grad = grad_f32 ? nullptr : static_cast<const uint16_t *>(grad);
   p.grad_f32 = grad_f32 ? static_cast<const float *>(grad) : nullptr;
@@ -248,11 +275,15 @@ coat_status_t step_impl(float *param, const void *grad, bool grad_f32, uint8_t *
   }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool e4 = cfg->v_fmt == COAT_E4M3;
+  if (peers)
+    return e4 ? launch_step_all<coat::kE4M3, coat::kGradPeers>(lg, n, s, p)
+              : launch_step_all<coat::kE5M2, coat::kGradPeers>(lg, n, s, p);
   if (grad_f32)
-    return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3, true>(lg, n, s, p)
-                                   : launch_step_all<coat::kE5M2, true>(lg, n, s, p);
-  return cfg->v_fmt == COAT_E4M3 ? launch_step_all<coat::kE4M3, false>(lg, n, s, p)
-                                 : launch_step_all<coat::kE5M2, false>(lg, n, s, p);
+    return e4 ? launch_step_all<coat::kE4M3, coat::kGradF32>(lg, n, s, p)
+              : launch_step_all<coat::kE5M2, coat::kGradF32>(lg, n, s, p);
+  return e4 ? launch_step_all<coat::kE4M3, coat::kGradBf16>(lg, n, s, p)
+            : launch_step_all<coat::kE5M2, coat::kGradBf16>(lg, n, s, p);
 }
 
 // Register-resident norm rows of 256 NC columns: persistent grid of the
@@ -314,6 +345,39 @@ coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, ui
     return skip_if_nonzero ? COAT_ERR_MISALIGNED : COAT_ERR_INVALID_ARG;
   return step_impl(param, grad, false, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
                    skip_if_nonzero, stream);
+}
+
+coat_status_t coat_adamw_fp8_step_peers(const uint16_t *const *grads, int32_t world,
+                                        int64_t grad_offset, float *param,
+                                        void *const *params_out, int32_t params_out_bf16,
+                                        int64_t params_out_offset, uint8_t *m_code, float *m_k,
+                                        float *m_scale, uint8_t *v_code, float *v_k,
+                                        float *v_scale, int64_t n, const coat_adamw_cfg_t *cfg,
+                                        void *stream) {
+  NvtxRange nvtx_range("coat_adamw_fp8_step_peers");
+  if (world < 1 || world > COAT_MAX_PEERS || !grads || grad_offset < 0 ||
+      params_out_offset < 0 || (params_out_bf16 != 0 && params_out_bf16 != 1))
+    return COAT_ERR_INVALID_ARG;
+  PeerArgs pa;
+  pa.world = world;
+  pa.param_bf16 = params_out_bf16;
+  const size_t pesz = params_out_bf16 ? 2 : 4;
+  for (int r = 0; r < COAT_MAX_PEERS; ++r) {
+    pa.grad[r] = nullptr;
+    pa.param[r] = nullptr;
+  }
+  for (int r = 0; r < world; ++r) {
+    if (!grads[r]) return COAT_ERR_INVALID_ARG;
+    pa.grad[r] = grads[r] + grad_offset;
+    if (!aligned16(pa.grad[r])) return COAT_ERR_MISALIGNED;
+    if (params_out && params_out[r]) {
+      pa.param[r] = static_cast<unsigned char *>(params_out[r]) +
+                    static_cast<size_t>(params_out_offset) * pesz;
+      if (!aligned16(pa.param[r])) return COAT_ERR_MISALIGNED;
+    }
+  }
+  return step_impl(param, nullptr, false, m_code, m_k, m_scale, v_code, v_k, v_scale, n, cfg,
+                   nullptr, stream, &pa);
 }
 
 coat_status_t coat_count_nonfinite_bf16(const uint16_t *x, int64_t n, uint32_t *count,

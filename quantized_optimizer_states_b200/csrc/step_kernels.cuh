@@ -60,10 +60,28 @@ constexpr int kElemsPerBlock = kThreads * kVec;    // 4096
 constexpr int kWarps = kThreads / 32;
 constexpr int kMinTableLog2G = 6;                  // decode tables for G >= 64
 
+// Where the step's gradient comes from (a template parameter of the kernel):
+// BF16 words, float32 values rounded to BF16 as they load, or the mean of
+// the BF16 gradients of `world` data-parallel ranks read from their own
+// buffers (peer memory), with the updated parameters also written into
+// every rank's parameter buffer -- the reduce-scatter, the step and the
+// all-gather of a ZeRO-1 step in one kernel.
+constexpr int kGradBf16 = 0;
+constexpr int kGradF32 = 1;
+constexpr int kGradPeers = 2;
+constexpr int kMaxPeers = 8;
+
 struct StepParams {
   float *theta;
-  const uint16_t *grad;       // BF16 gradients (the kernel's GF32 = false form)
-  const float *grad_f32;      // float32 gradients, rounded to BF16 on load (GF32 = true)
+  const uint16_t *grad;       // BF16 gradients (kGradBf16)
+  const float *grad_f32;      // float32 gradients, rounded to BF16 on load (kGradF32)
+  // kGradPeers: rank r's gradient slice of this shard (element i at
+  // grad_peer[r][i]) and rank r's parameter slice (param_peer[r][i], FP32 or
+  // BF16 by param_peer_bf16; null: not replicated), r < world
+  const uint16_t *grad_peer[kMaxPeers];
+  void *param_peer[kMaxPeers];
+  int world;
+  int param_peer_bf16;
   uint8_t *m_code;
   float *m_k;
   float *m_s;
@@ -468,7 +486,66 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   return r;
 }
 
-template <int VF, int LG, bool FULL, bool GF32>
+// kGradPeers: the 16 gradients of this thread as BF16 words, each the mean
+// over the ranks of their BF16 gradients, RN_bf16(RN32(sum) / world) with
+// the sum taken in binary32 in rank order (one rounding per addition); one
+// rank gives its own gradient unchanged.
+template <bool FULL>
+__device__ __forceinline__ void peer_mean_bf16(const StepParams &p, int64_t e0, uint32_t *gw) {
+  float acc[16];
+#pragma unroll
+  for (int r = 0; r < kMaxPeers; ++r) {
+    if (r >= p.world) break;
+    uint32_t w[8];
+    load16_bf16<FULL>(p.grad_peer[r], e0, p.n, w);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float lo = bf16lo_to_float(w[i]), hi = bf16hi_to_float(w[i]);
+      acc[2 * i] = r == 0 ? lo : __fadd_rn(acc[2 * i], lo);
+      acc[2 * i + 1] = r == 0 ? hi : __fadd_rn(acc[2 * i + 1], hi);
+    }
+  }
+  const float wf = static_cast<float>(p.world);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float lo = p.world == 1 ? acc[2 * i] : __fdiv_rn(acc[2 * i], wf);
+    const float hi = p.world == 1 ? acc[2 * i + 1] : __fdiv_rn(acc[2 * i + 1], wf);
+    gw[i] = bf16x2_rn(lo, hi);
+  }
+}
+
+// kGradPeers: four updated parameters (elements base .. base + 3 of the
+// shard) into every rank's parameter slice, as FP32 or rounded to BF16.
+template <bool FULL>
+__device__ __forceinline__ void store4_to_peers(const StepParams &p, int64_t base,
+                                                const float *o) {
+  const bool whole = FULL || base + 4 <= p.n;
+#pragma unroll
+  for (int r = 0; r < kMaxPeers; ++r) {
+    if (r >= p.world) break;
+    void *dst = p.param_peer[r];
+    if (dst == nullptr) continue;
+    if (p.param_peer_bf16) {
+      uint16_t *d = static_cast<uint16_t *>(dst) + base;
+      if (whole) {
+        *reinterpret_cast<uint2 *>(d) = make_uint2(bf16x2_rn(o[0], o[1]), bf16x2_rn(o[2], o[3]));
+      } else {
+        for (int j = 0; j < 4; ++j)
+          if (base + j < p.n) d[j] = static_cast<uint16_t>(bf16x2_rn(o[j], 0.0f));
+      }
+    } else {
+      float *d = static_cast<float *>(dst) + base;
+      if (whole) {
+        *reinterpret_cast<float4 *>(d) = make_float4(o[0], o[1], o[2], o[3]);
+      } else {
+        for (int j = 0; j < 4; ++j)
+          if (base + j < p.n) d[j] = o[j];
+      }
+    }
+  }
+}
+
+template <int VF, int LG, bool FULL, int GS>
 __global__ void __launch_bounds__(StepLayout<LG>::kBlock, StepLayout<LG>::kMinBlocks)
 adamw_fp8_step_kernel(const StepParams p) {
   using L = StepLayout<LG>;
@@ -520,12 +597,14 @@ adamw_fp8_step_kernel(const StepParams p) {
   float m[16], v[16];
   uint32_t gw[8], mw[4], vw[4];
   if (active) {
-    if constexpr (GF32) {
+    if constexpr (GS == kGradF32) {
       // float32 gradients become the BF16 gradients of the rule right here
       float g16[16];
       load16_f32<FULL>(p.grad_f32, e0, p.n, g16);
 #pragma unroll
       for (int i = 0; i < 8; ++i) gw[i] = bf16x2_rn(g16[2 * i], g16[2 * i + 1]);
+    } else if constexpr (GS == kGradPeers) {
+      peer_mean_bf16<FULL>(p, e0, gw);
     } else {
       load16_bf16<FULL>(p.grad, e0, p.n, gw);
     }
@@ -634,6 +713,10 @@ adamw_fp8_step_kernel(const StepParams p) {
         for (int j = 0; j < 4; ++j)
           if (base + j < p.n) p.theta[base + j] = o[j];
       }
+      if constexpr (GS == kGradPeers) {
+        const float o[4] = {a.x, a.y, b.x, b.y};
+        store4_to_peers<FULL>(p, base, o);
+      }
     }
     if (slow) {
 #pragma unroll
@@ -646,7 +729,14 @@ adamw_fp8_step_kernel(const StepParams p) {
         const int64_t base = e0 + 4 * c;
         for (int j = 0; j < 4; ++j)
           if (FULL || base + j < p.n) p.theta[base + j] = o[j];
+        if constexpr (GS == kGradPeers) store4_to_peers<FULL>(p, base, o);
       }
+    }
+    if constexpr (GS == kGradPeers) {
+      // the replicas written into other ranks' memory are visible to them
+      // (after the host-side barrier that follows the launch) before the
+      // kernel counts as finished
+      if (p.world > 1) __threadfence_system();
     }
   }
 

@@ -217,3 +217,94 @@ class Zero1Shard:
         else:
             _coat_step(self, self.reduce_gradient_f32(grad), t, hyper)  # rounded on load
         return self.gather_params(gather_dtype)
+
+    def step_peers(self, bufs: "PeerBuffers", t: int, hyper: dict) -> torch.Tensor:
+        """One data-parallel step in one kernel per rank: after a barrier (every
+        rank's gradient in `bufs.grad` is complete), this rank's kernel reads the
+        ranks' gradients over its shard from their buffers, averages them
+        (binary32 sum in rank order, divided by the rank count, rounded to
+        BF16), steps its shard and writes the updated parameters into every
+        rank's `bufs.param`; a second barrier follows, so every rank's
+        `bufs.param` holds the whole updated set when this returns (in stream
+        order).  Per parameter of the buffer and per rank: (W - 1)/W x 2 bytes of
+        gradient read from other ranks and (W - 1)/W x 2 (BF16) or x 4 (FP32)
+        bytes of parameters written to them, no staging buffer, one launch.
+        Returns the first n elements of this rank's `bufs.param`."""
+        dev = self.master.device
+        off = self.rank * self.L
+        with torch.cuda.device(dev):
+            _barrier(self, dev)
+            _lib.coat_adamw_fp8_step_peers(
+                bufs.grads, self.master, self.m_code, self.m_k, self.m_s, self.v_code, self.v_k,
+                self.v_s, grad_offset=off, params_out=bufs.params, params_out_offset=off, step=t,
+                group_size=self.group_size, v_fmt=self.v_fmt, k_range=self.k_range,
+                k_max=self.k_max, **hyper)
+            _barrier(self, dev)
+        return bufs.param[:self.n]
+
+
+# ---- the step over peer memory ----------------------------------------------------
+
+def _share(t: torch.Tensor):
+    """A picklable description of a CUDA tensor that another process can map
+    (CUDA IPC, as torch.multiprocessing shares CUDA tensors)."""
+    from torch.multiprocessing.reductions import reduce_tensor
+    return reduce_tensor(t)
+
+
+def _open(shared) -> torch.Tensor:
+    fn, args = shared
+    return fn(*args)
+
+
+class PeerBuffers:
+    """Every rank's flat gradient and parameter buffers, mapped into every
+    rank's process, for `Zero1Shard.step_peers`.
+
+    `grad` (BF16, `shard.padded_numel` elements: the first n are the
+    parameters', the rest stay zero) is where this rank's backward pass
+    leaves its full gradient; `param` (BF16 or FP32, the same length) is where
+    every rank's step writes its updated shard, so after a step it holds the
+    whole updated parameter set.  `grads[r]` and `params[r]` are rank r's
+    buffers as seen from this process (its own are the local tensors).  The
+    buffers are exchanged once, here, through the process group (CUDA IPC
+    handles; on a node with NVLink a peer's buffer is read and written over
+    it).  Every rank keeps its PeerBuffers alive as long as any rank uses
+    them."""
+
+    def __init__(self, shard: "Zero1Shard", param_dtype: torch.dtype = torch.bfloat16):
+        if param_dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("parameters are replicated as bfloat16 or float32")
+        if shard.world > _lib.COAT_MAX_PEERS:
+            raise ValueError(f"at most {_lib.COAT_MAX_PEERS} ranks")
+        dev = shard.master.device
+        total = shard.padded_numel
+        self.grad = torch.zeros(total, dtype=torch.bfloat16, device=dev)
+        self.param = torch.zeros(total, dtype=param_dtype, device=dev)
+        if shard.world == 1:
+            self.grads, self.params = [self.grad], [self.param]
+            return
+        mine = (_share(self.grad), _share(self.param))
+        every = [None] * shard.world
+        dist.all_gather_object(every, mine, group=shard.pg)
+        self.grads = [self.grad if r == shard.rank else _open(every[r][0])
+                      for r in range(shard.world)]
+        self.params = [self.param if r == shard.rank else _open(every[r][1])
+                       for r in range(shard.world)]
+
+
+def _barrier(shard: "Zero1Shard", device: torch.device):
+    """Every rank's work issued so far on its current stream is complete
+    before any rank's later work runs: an all-reduce of one word on the
+    stream (NCCL), or a device synchronisation and a host barrier (other
+    backends)."""
+    if shard.world == 1:
+        return
+    if dist.get_backend(shard.pg) == "nccl":
+        flag = getattr(shard, "_flag", None)
+        if flag is None:
+            flag = shard._flag = torch.zeros(1, dtype=torch.int32, device=device)
+        dist.all_reduce(flag, group=shard.pg)
+    else:
+        torch.cuda.synchronize(device)
+        dist.barrier(group=shard.pg)

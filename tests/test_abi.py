@@ -92,6 +92,30 @@ def test_argument_checks_return_before_any_launch(lib):
     assert gs(fake, 0, 128, 0, fake, 0, fake, fake, None) == 0
 
 
+def test_peer_step_argument_checks(lib):
+    """coat_adamw_fp8_step_peers validates its rank tables on the host (these
+    calls never reach the device)."""
+    from quantized_optimizer_states_b200._lib import CoatAdamwCfg
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    cfg = ctypes.byref(CoatAdamwCfg(0.9, 0.999, 1e-4, 1e-8, 0.1, 10, 128, 0, 0, 0, 64.0, 0))
+    grads = (P * 9)(*([0x10000] * 9))
+    outs = (P * 2)(0x20000, 0x30000)
+    st = [fake] * 6
+    pe = lib.coat_adamw_fp8_step_peers
+    assert pe(grads, 0, 0, fake, None, 0, 0, *st, 16, cfg, None) == 1        # no rank
+    assert pe(grads, 9, 0, fake, None, 0, 0, *st, 16, cfg, None) == 1        # above the maximum
+    assert pe(None, 2, 0, fake, None, 0, 0, *st, 16, cfg, None) == 1         # no gradient table
+    assert pe(grads, 2, -16, fake, None, 0, 0, *st, 16, cfg, None) == 1      # negative offset
+    assert pe(grads, 2, 0, fake, outs, 2, 0, *st, 16, cfg, None) == 1        # bf16 flag not 0/1
+    assert pe((P * 2)(0x10000, None), 2, 0, fake, None, 0, 0, *st, 16, cfg, None) == 1
+    assert pe(grads, 2, 4, fake, None, 0, 0, *st, 16, cfg, None) == 2        # 8-byte offset
+    assert pe(grads, 2, 0, fake, outs, 0, 2, *st, 16, cfg, None) == 2        # FP32 copy at 8 bytes
+    assert pe(grads, 2, 0, fake, outs, 1, 4, *st, 16, cfg, None) == 2        # BF16 copy at 8 bytes
+    assert pe(grads, 2, 0, P(0x10004), outs, 1, 8, *st, 16, cfg, None) == 2  # shard misaligned
+    assert pe(grads, 2, 0, fake, outs, 1, 8, *st, 0, cfg, None) == 0         # empty: no launch
+
+
 def test_pack_argument_checks(lib):
     """coat_pack_bf16 / coat_unpack_bf16 validate their host tables before any
     launch (these calls never reach the device)."""

@@ -486,6 +486,9 @@ def main(argv=None):
     ap.add_argument("--group-size", type=int, default=128, help="sweep workload only")
     ap.add_argument("--regime", default="late", choices=["early", "late", "typical"],
                     help="sweep workload only")
+    ap.add_argument("--zero1-path", default="peers", choices=["peers", "nccl"],
+                    help="ZeRO-1 step: one kernel over peer memory (peers) or NCCL "
+                         "reduce-scatter, step, NCCL all-gather (nccl)")
     ap.add_argument("--zero1", action="store_true",
                     help="time the ZeRO-1 data-parallel step even on one GPU (a one-rank "
                          "process group: the collectives reduce to copies)")
@@ -644,7 +647,13 @@ def run_zero1(args):
     wg = step_workload(args, seed_offset=1000 * (rank + 1))
     th_unused, g_rank, _ = inputs.device_step_inputs(wg, dev)
     del th_unused
-    grad = torch.zeros(shard.padded_numel, dtype=torch.bfloat16, device=dev)
+    peers = args.zero1_path == "peers"
+    if peers:
+        # every rank's gradient and parameter buffers, mapped into every rank
+        bufs = zero.PeerBuffers(shard, torch.bfloat16)
+        grad = bufs.grad
+    else:
+        grad = torch.zeros(shard.padded_numel, dtype=torch.bfloat16, device=dev)
     grad[:n].copy_(g_rank)             # the flat gradient, padded: no copy per step
     del g_rank
     torch.cuda.empty_cache()
@@ -656,6 +665,17 @@ def run_zero1(args):
 
     def step(record=False):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
+        if peers:
+            # phases: barrier + kernel + barrier, the kernel alone in ev[1..2]
+            if record:
+                ev[0].record(stream)
+            shard.step_peers(bufs, step_no[0], hyper,
+                             kernel_events=(ev[1], ev[2]) if record else None)
+            if record:
+                ev[3].record(stream)
+                marks.append(ev)
+            step_no[0] += 1
+            return
         if record:
             ev[0].record(stream)
         g = shard.reduce_gradient_bf16(grad)
@@ -737,7 +757,10 @@ def run_zero1(args):
                        "on every rank"}
         del host
 
-    if rank == 0:
+    if rank == 0 and peers:
+        print(json.dumps(zero1_peers_line(args, w, shard, world, total_ms, rs_ms, st_ms, ag_ms,
+                                          e2e, clocks)), flush=True)
+    elif rank == 0:
         peaks, peak_kind = measured_peaks()
         peak = float(peaks["hbm_gbs"])
         achieved = bytes_per_param(G) * L / (st_ms / 1e3) / 1e9
@@ -781,9 +804,78 @@ def run_zero1(args):
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
+    if peers:
+        del bufs, grad              # unmap the other ranks' buffers before any rank exits
+        torch.cuda.synchronize()
     dist.barrier()
     dist.destroy_process_group()
     return 0
+
+
+LINK_GBPS = 770.0   # measured peer copy per direction on this machine
+
+
+def zero1_peers_bytes(L: int, world: int, G: int) -> dict:
+    """Algorithmic bytes of one rank's one-kernel ZeRO-1 step on a shard of L
+    parameters: HBM of the rank's own GPU (the step's 14 + 32/G B, the
+    BF16 copy of its updated shard into its own buffer, and its gradient
+    read by the other ranks: 2 (W - 1) B per shard parameter) and NVLink
+    per direction (in: the other ranks' gradients of its shard and their
+    updated shards written into its buffer; out: the same amounts in the
+    other direction), 2 (W - 1) + 2 (W - 1) B per shard parameter."""
+    hbm = (bytes_per_param(G) + 2 + 2 * (world - 1) + 2 * (world - 1)) * L
+    link = 4 * (world - 1) * L
+    return {"hbm": hbm, "link_per_direction": link}
+
+
+def zero1_peers_line(args, w, shard, world, total_ms, bar0_ms, kern_ms, bar1_ms, e2e, clocks):
+    """The JSON line of the one-kernel ZeRO-1 path: value = parameters of the
+    set per second of the slowest rank; the kernel's roofline is the slower
+    of its HBM bytes at the measured copy bandwidth and its NVLink bytes at
+    the measured peer-copy bandwidth."""
+    peaks, peak_kind = measured_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    n, G, L = w.n, w.group_size, shard.L
+    b = zero1_peers_bytes(L, world, G)
+    t_hbm = b["hbm"] / (hbm_peak * 1e9)
+    t_link = b["link_per_direction"] / (LINK_GBPS * 1e9)
+    bound = "hbm" if t_hbm >= t_link else "nvlink"
+    target_s = max(t_hbm, t_link)
+    kern_s = kern_ms / 1e3
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": b["hbm"] / kern_s / 1e9, "peak": hbm_peak,
+                "unit": "GB/s", "peak_source": f"{peak_kind} copy bandwidth"}
+    else:
+        roof = {"bound": "nvlink", "achieved": b["link_per_direction"] / kern_s / 1e9,
+                "peak": LINK_GBPS, "unit": "GB/s",
+                "peak_source": "measured peer copy per direction on this pool"}
+    roof.update(frac=target_s / kern_s, traffic=None,
+                kernel="coat_adamw_fp8_step_peers on the shard (gradient mean, step, "
+                       "parameter copies into every rank)",
+                algorithmic_bytes=b)
+    return {
+        "metric": METRIC, "value": n * args.steps / (total_ms / 1e3), "unit": "params/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name} set: {n} FP32 params, BF16 grads, FP8 m (e4m3) / "
+                               f"v ({args.v_fmt}) + per-group k, scale",
+                   "group_size": G, "m_fmt": "e4m3", "v_fmt": args.v_fmt,
+                   "params_per_gpu": L,
+                   "parallelism": f"zero1 dp{world}: one kernel per rank reads every rank's "
+                                  "BF16 gradient of its 1/N shard over peer memory, steps "
+                                  "the shard and writes the BF16 parameters into every "
+                                  "rank's buffer, between two barriers of the ranks",
+                   "l2": "no flush needed: every step moves far more than the 126 MB L2"},
+        "roofline": roof,
+        "phases": {"barrier_ms": bar0_ms + bar1_ms, "kernel_ms": kern_ms},
+        "cpu_baseline": None,
+        "e2e": e2e,
+        # the fused kernel, plus a tail launch when the shard is not a whole
+        # number of 1024-parameter blocks (the barriers are NCCL's)
+        "gpu_launches": args.steps * (1 + (L % 1024 != 0)),
+        "clocks": clocks,
+    }
 
 
 def time_step_set(w, v_fmt: int, steps: int, warmup: int, dev) -> dict:

@@ -19,6 +19,13 @@ boundaries, so each rank keeps 1/world of it.  One step:
   3. all-gather of the updated master weights (FP32, or each shard rounded
      to BF16 first: half the bytes).
 
+`Zero1Shard.step_peers` does all three in one kernel per rank over peer
+memory (`PeerBuffers` maps every rank's gradient and parameter buffers into
+every process): the rank's kernel reads the ranks' gradients over its shard
+from their buffers, averages them in binary32 in rank order, steps the
+shard and writes the updated parameters into every rank's buffer; two
+barriers of the ranks frame it.
+
 No 1xG group straddles two shards, so the sharded step computes exactly
 what a single-rank step over the whole buffer computes on the reduced
 gradient.  The collectives go through the default (or given) process group:
@@ -218,7 +225,8 @@ class Zero1Shard:
             _coat_step(self, self.reduce_gradient_f32(grad), t, hyper)  # rounded on load
         return self.gather_params(gather_dtype)
 
-    def step_peers(self, bufs: "PeerBuffers", t: int, hyper: dict) -> torch.Tensor:
+    def step_peers(self, bufs: "PeerBuffers", t: int, hyper: dict,
+                   kernel_events=None) -> torch.Tensor:
         """One data-parallel step in one kernel per rank: after a barrier (every
         rank's gradient in `bufs.grad` is complete), this rank's kernel reads the
         ranks' gradients over its shard from their buffers, averages them
@@ -229,16 +237,22 @@ class Zero1Shard:
         order).  Per parameter of the buffer and per rank: (W - 1)/W x 2 bytes of
         gradient read from other ranks and (W - 1)/W x 2 (BF16) or x 4 (FP32)
         bytes of parameters written to them, no staging buffer, one launch.
-        Returns the first n elements of this rank's `bufs.param`."""
+        Returns the first n elements of this rank's `bufs.param`.
+        kernel_events: an optional pair of CUDA events recorded on the current
+        stream around the kernel alone (for timing)."""
         dev = self.master.device
         off = self.rank * self.L
         with torch.cuda.device(dev):
             _barrier(self, dev)
+            if kernel_events is not None:
+                kernel_events[0].record()
             _lib.coat_adamw_fp8_step_peers(
                 bufs.grads, self.master, self.m_code, self.m_k, self.m_s, self.v_code, self.v_k,
                 self.v_s, grad_offset=off, params_out=bufs.params, params_out_offset=off, step=t,
                 group_size=self.group_size, v_fmt=self.v_fmt, k_range=self.k_range,
                 k_max=self.k_max, **hyper)
+            if kernel_events is not None:
+                kernel_events[1].record()
             _barrier(self, dev)
         return bufs.param[:self.n]
 

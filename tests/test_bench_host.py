@@ -131,3 +131,17 @@ def test_clock_normalised_scales_by_max_over_median_clock():
     assert got["params_per_s_at_max_clock"] == pytest.approx(3.0e11 * 1965.0 / 1800.0)
     assert bench.clock_normalised(1.0, None) is None
     assert bench.clock_normalised(1.0, {"sm_mhz": None, "sm_max_mhz": 1965.0}) is None
+
+
+def test_zero1_peer_step_bytes():
+    """One rank's one-kernel ZeRO-1 step on L shard parameters: HBM = the
+    step's bytes + the BF16 copy of its shard + its gradient read by and the
+    others' shards written into its memory, 2 (W - 1) B each; NVLink per
+    direction 4 (W - 1) B per shard parameter; one rank moves nothing over
+    links."""
+    L = 1 << 20
+    one = bench.zero1_peers_bytes(L, 1, 128)
+    assert one["hbm"] == (14.25 + 2) * L and one["link_per_direction"] == 0
+    eight = bench.zero1_peers_bytes(L, 8, 128)
+    assert eight["link_per_direction"] == 28 * L
+    assert eight["hbm"] == (14.25 + 2 + 28) * L

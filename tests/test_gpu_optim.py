@@ -220,11 +220,13 @@ def test_flat_fp32_gradients_through_backward(optim):
         assert torch.equal(pa, pb)
 
 
-def test_bench_zero1_path_on_one_rank():
-    """bench.py's ZeRO-1 timing path (BF16 reduce-scatter, the step on the
-    shard, BF16 all-gather) runs end to end as a one-rank process group on
-    the 2^28-parameter sweep set and reports its three phases (a subprocess,
-    so its process group and environment stay out of this one)."""
+@pytest.mark.parametrize("path", ["peers", "nccl"])
+def test_bench_zero1_path_on_one_rank(path):
+    """bench.py's ZeRO-1 timing paths run end to end as a one-rank process
+    group on the 2^28-parameter sweep set (a subprocess, so its process group
+    and environment stay out of this one): the one-kernel step over peer
+    memory with its barrier and kernel phases, and the NCCL path (BF16
+    reduce-scatter, the step on the shard, BF16 all-gather) with its three."""
     import json
     import os
     import subprocess
@@ -233,12 +235,17 @@ def test_bench_zero1_path_on_one_rank():
     env = {k: v for k, v in os.environ.items()
            if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
     out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--zero1",
-                          "--workload", "sweep", "--steps", "2", "--warmup", "1",
-                          "--e2e-steps", "1"], capture_output=True, text=True, timeout=600,
-                         env=env)
+                          "--zero1-path", path, "--workload", "sweep", "--steps", "2",
+                          "--warmup", "1", "--e2e-steps", "1"], capture_output=True, text=True,
+                         timeout=600, env=env)
     assert out.returncode == 0, out.stderr[-3000:]
     line = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
     assert line["n_gpus"] == 1 and line["scaling"] == "strong" and line["value"] > 0
-    c = line["collectives"]
-    assert c["reduce_scatter_ms"] > 0 and c["step_ms"] > 0 and c["all_gather_ms"] > 0
+    if path == "peers":
+        ph = line["phases"]
+        assert ph["kernel_ms"] > 0 and ph["barrier_ms"] >= 0
+        assert line["roofline"]["bound"] == "hbm" and 0 < line["roofline"]["frac"] < 1.5
+    else:
+        c = line["collectives"]
+        assert c["reduce_scatter_ms"] > 0 and c["step_ms"] > 0 and c["all_gather_ms"] > 0
     assert line["e2e"]["value"] > 0 and line["gpu_launches"] == 2

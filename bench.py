@@ -648,9 +648,22 @@ def run_zero1(args):
     th_unused, g_rank, _ = inputs.device_step_inputs(wg, dev)
     del th_unused
     peers = args.zero1_path == "peers"
+    peer_fallback = None
     if peers:
-        # every rank's gradient and parameter buffers, mapped into every rank
-        bufs = zero.PeerBuffers(shard, torch.bfloat16)
+        # every rank's gradient and parameter buffers, mapped into every rank;
+        # if the mapping fails on any rank, every rank takes the NCCL path
+        try:
+            bufs = zero.PeerBuffers(shard, torch.bfloat16)
+            ok = 1
+        except Exception as e:  # noqa: BLE001 -- reported in the JSON line
+            bufs, ok, peer_fallback = None, 0, f"{type(e).__name__}: {e}"[:300]
+        flag = torch.tensor([ok], dtype=torch.int32, device=dev)
+        dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+        if int(flag.item()) == 0:
+            peers = False
+            peer_fallback = peer_fallback or "the peer-buffer mapping failed on another rank"
+            del bufs
+    if peers:
         grad = bufs.grad
     else:
         grad = torch.zeros(shard.padded_numel, dtype=torch.bfloat16, device=dev)
@@ -803,6 +816,8 @@ def run_zero1(args):
             "gpu_launches": args.steps * (1 + (L % 1024 != 0)),
             "clocks": clocks,
         }
+        if peer_fallback:
+            line["peer_path_unavailable"] = peer_fallback
         print(json.dumps(line), flush=True)
     if peers:
         del bufs, grad              # unmap the other ranks' buffers before any rank exits

@@ -293,14 +293,26 @@ class PeerBuffers:
             raise ValueError(f"at most {_lib.COAT_MAX_PEERS} ranks")
         dev = shard.master.device
         total = shard.padded_numel
-        self.grad = torch.zeros(total, dtype=torch.bfloat16, device=dev)
-        self.param = torch.zeros(total, dtype=param_dtype, device=dev)
         if shard.world == 1:
+            self.grad = torch.zeros(total, dtype=torch.bfloat16, device=dev)
+            self.param = torch.zeros(total, dtype=param_dtype, device=dev)
             self.grads, self.params = [self.grad], [self.param]
             return
-        mine = (_share(self.grad), _share(self.param))
+        # every rank reaches the exchange, also when its own part failed, so
+        # that no rank is left waiting in it
+        err = None
+        try:
+            self.grad = torch.zeros(total, dtype=torch.bfloat16, device=dev)
+            self.param = torch.zeros(total, dtype=param_dtype, device=dev)
+            mine = (_share(self.grad), _share(self.param))
+        except Exception as e:  # noqa: BLE001 -- re-raised after the exchange
+            mine, err = None, e
         every = [None] * shard.world
         dist.all_gather_object(every, mine, group=shard.pg)
+        if err is not None:
+            raise err
+        if any(x is None for x in every):
+            raise RuntimeError("another rank could not share its buffers")
         self.grads = [self.grad if r == shard.rank else _open(every[r][0])
                       for r in range(shard.world)]
         self.params = [self.param if r == shard.rank else _open(every[r][1])

@@ -245,3 +245,50 @@ def test_reduce_scatter_bf16_and_chunked_binary32_three_gloo_ranks():
         bound = (world - 1) * 2.0 ** -8 * absum[rank * L:(rank + 1) * L] / world \
             + 2.0 ** -8 * np.abs(want)
         assert np.all(np.abs(c - want) <= bound), f"rank {rank}: BF16 mean too far"
+
+
+def _share_fail_worker(rank, world, port, fail_rank, q):
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        sh = zero.Zero1Shard(torch.zeros(4 * G), group_size=G)
+
+        def share(t):
+            if rank == fail_rank:
+                raise OSError("no shareable memory here")
+            return ("handle", rank)
+
+        zero._share = share
+        zero._open = lambda shared: (_ for _ in ()).throw(AssertionError("not reached"))
+        try:
+            zero.PeerBuffers(sh)
+            q.put((rank, "no error"))
+        except Exception as e:  # noqa: BLE001 -- what the test checks
+            q.put((rank, f"{type(e).__name__}: {e}"))
+        dist.barrier()          # every rank is still in step with the others
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_buffer_exchange_fails_on_every_rank_when_one_rank_cannot_share():
+    """A rank whose buffers cannot be shared (the failure made on the host,
+    in one rank) still takes part in the exchange, so no rank is left
+    waiting: every rank raises, the failing one with its own error, the
+    others naming another rank, and all of them meet at a barrier after."""
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_share_fail_worker, args=(r, world, port, 1, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[1] == "OSError: no shareable memory here"
+    assert res[0].startswith("RuntimeError: another rank") and res[2] == res[0]

@@ -20,7 +20,9 @@
  *             along channels for nonlinear-layer inputs, and Group Scaling
  *             (max per 1xG run, then max of that small intermediate) for the
  *             per-tensor scale of linear-layer inputs;
- *           "结果和边界" -- k follows the target format's range.
+ *           "结果和边界" -- k follows the target format's range; training
+ *             on several GPUs (data-parallel ranks, every rank computing a
+ *             full gradient).
  *   [ATLAS] "LLM Atlas / systems / numerics" (llm-atlas.k1412.top),
  *           section 03 "FP8" (E4M3 max 448, min subnormal 2^-9; E5M2 max
  *           57344, min subnormal 2^-16) and section 08 "Adam -> AdamW"

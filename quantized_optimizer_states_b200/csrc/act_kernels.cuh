@@ -586,16 +586,15 @@ __global__ void __launch_bounds__(kThreads) norm_group_amax_kernel(const NormPar
   if (p.tensor_amax) block_max_to_tensor(wmax, p.tensor_amax);
 }
 
-// Rows of 256 NC columns (NC = 1..8: up to 2048 columns) are held in
-// registers instead: lane l loads the row's 16-byte chunks l, l + 32, ...,
-// l + 32 (NC - 1) with plain 128-bit loads (every load instruction of the
-// warp reads 512 contiguous bytes) and takes the sums, the output and the
-// maxima from them, in the order of the staged kernel above (same sums,
-// same roundings, so the same bits).  Fully unrolled over the row, it
+// Rows of 256 NC columns (NC = 1..8: up to 2048 columns) that the two-warp
+// form further below does not take (an odd chunk count, or 1xG runs wider
+// than half a row) are held in registers by one warp: lane l loads the
+// row's 16-byte chunks l, l + 32, ..., l + 32 (NC - 1) (every load
+// instruction of the warp reads 512 contiguous bytes) and takes the sums,
+// the output and the maxima from them.  Fully unrolled over the row, it
 // executes far fewer instructions than the staged form's three loops over
-// shared memory, which are what limit that form: measured on [16384, 2048],
-// 26.0 us against 32.9 us.  Persistent warps, 8 to a block, 2 blocks per
-// SM (the row and its sums take ~110 registers).
+// shared memory, which are what limit that form.  Persistent warps, 8 to a
+// block, 2 blocks per SM (the row and its sums take ~110 registers).
 constexpr int kNormRegWarps = 8;
 constexpr int kNormRegMaxChunks = 8;
 
@@ -776,6 +775,135 @@ __global__ void __launch_bounds__(32 * kNormRegWarps, 2) norm_reg_group_amax_ker
     row = nxt;
   }
   if (p.tensor_amax) block_max_to_tensor(wmax, p.tensor_amax);
+}
+
+// Rows of 512 NCH columns, two warps a row: warp half h of a pair holds
+// chunk columns NCH h .. NCH h + NCH - 1 (lane l: chunks l + 32 i), so a
+// row's data takes half the registers of the one-warp form and twice the
+// warps fit an SM (latency, not bandwidth, bounds that form: 16 warps per
+// SM).  Each half sums its columns (four partial sums a lane, then the
+// warp), the two halves' sums meet in shared memory (half 0 + half 1), and
+// the mean and the variance follow as in the one-warp form.  The block's
+// four pairs advance in lockstep, two block barriers a round; every warp
+// takes part in every round (a pair without a row in the last round skips
+// only its arithmetic), so every barrier is reached by the whole block.
+// Each warp loads the next round's half row into registers while it works
+// on the current one.  A 1xG run lies within one half (G divides 256 NCH).
+constexpr int kSplitPairs = 4;
+
+template <int NCH, bool kAffine>
+__global__ void __launch_bounds__(256, kAffine ? 3 : 4) norm_split_group_amax_kernel(const NormParams p) {
+  __shared__ float sum_red[kSplitPairs][2], var_red[kSplitPairs][2];
+  pdl_enter();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int pair = warp >> 1, h = warp & 1;
+  const int64_t r0 = p.rows * blockIdx.x / gridDim.x;
+  const int64_t r1 = p.rows * (blockIdx.x + 1) / gridDim.x;
+  const int64_t rounds = (r1 - r0 + kSplitPairs - 1) / kSplitPairs;
+  const float nf = static_cast<float>(p.cols);   // exact (cols <= 16384)
+  const int clanes = 1 << (p.log2G - 3);
+  float rowmax = 0.0f;
+  uint4 nxt[NCH];
+  auto load = [&](int64_t row, uint4 *c) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.cols);
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) c[j] = src[lane + 32 * (NCH * h + j)];
+  };
+  int64_t row = r0 + pair;
+  if (row < r1) load(row, nxt);
+  for (int64_t k = 0; k < rounds; ++k, row += kSplitPairs) {
+    const bool on = row < r1;
+    uint4 c[NCH];
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) c[j] = nxt[j];
+    if (row + kSplitPairs < r1) load(row + kSplitPairs, nxt);
+    float2 s0 = make_float2(0.0f, 0.0f), s1 = s0;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 x2 = bf16x2_to_float2(wv[j]);
+        float2 &acc = (j & 1) ? s1 : s0;
+        acc = p.rms ? fma2_rn(x2, x2, acc) : add2_rn(acc, x2);
+      }
+    }
+    const float ws = warp_sum_f((s0.x + s0.y) + (s1.x + s1.y));
+    if (lane == 0) sum_red[pair][h] = ws;
+    __syncthreads();
+    const float sum = sum_red[pair][0] + sum_red[pair][1];
+    float mean = 0.0f, var;
+    if (p.rms) {
+      var = __fdiv_rn(sum, nf);
+      __syncthreads();   // the same two barriers a round on both forms
+    } else {
+      mean = __fdiv_rn(sum, nf);
+      const float2 nm = make_float2(-mean, -mean);
+      float2 q0 = make_float2(0.0f, 0.0f), q1 = q0;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 d = add2_rn(bf16x2_to_float2(wv[j]), nm);
+          float2 &acc = (j & 1) ? q1 : q0;
+          acc = fma2_rn(d, d, acc);
+        }
+      }
+      const float wq = warp_sum_f((q0.x + q0.y) + (q1.x + q1.y));
+      if (lane == 0) var_red[pair][h] = wq;
+      __syncthreads();
+      var = __fdiv_rn(var_red[pair][0] + var_red[pair][1], nf);
+    }
+    if (!on) continue;   // after both barriers of the round
+    const float rstd = 1.0f / sqrtf(var + p.eps);
+    const float2 NM = make_float2(-mean, -mean), RS = make_float2(rstd, rstd);
+    const int64_t gbase = (row * p.cols) >> p.log2G;
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.cols);
+    float run = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const uint32_t wv[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+      const int ci = NCH * h + i;                     // chunk column in the row
+      const int col0 = 8 * (lane + 32 * ci);
+      uint32_t ow[4], am = 0u;
+      if constexpr (kAffine) {
+        float2 w2[4], b2[4];
+        if (p.weight) load8_f32(p.weight + col0, p.affine_vec, w2);
+        if (p.bias) load8_f32(p.bias + col0, p.affine_vec, b2);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float2 y = mul2_rn(add2_rn(bf16x2_to_float2(wv[j]), NM), RS);
+          if (p.weight && p.bias) y = fma2_rn(y, w2[j], b2[j]);
+          else if (p.weight) y = mul2_rn(y, w2[j]);
+          else y = add2_rn(y, b2[j]);
+          ow[j] = bf16x2_rn(y.x, y.y);
+          am = bmax2(am, ow[j] & 0x7FFF7FFFu);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 y = mul2_rn(add2_rn(bf16x2_to_float2(wv[j]), NM), RS);
+          ow[j] = bf16x2_rn(y.x, y.y);
+          am = bmax2(am, ow[j] & 0x7FFF7FFFu);
+        }
+      }
+      dst[lane + 32 * ci] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      float a = fmaxf(bf16lo_to_float(am), bf16hi_to_float(am));
+      rowmax = fmaxf(rowmax, a);
+      if (clanes <= 32) {
+        for (int off = 1; off < clanes; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+        if ((lane & (clanes - 1)) == 0) p.group_amax[gbase + (col0 >> p.log2G)] = a;
+      } else {
+        run = fmaxf(run, warp_max_f(a));
+        if (((ci + 1) & ((clanes >> 5) - 1)) == 0) {   // the run's last chunk column
+          if (lane == 0) p.group_amax[gbase + ((256 * ci) >> p.log2G)] = run;
+          run = 0.0f;
+        }
+      }
+    }
+  }
+  if (p.tensor_amax) block_max_to_tensor(warp_max_f(rowmax), p.tensor_amax);
 }
 
 // ---- the FP8 cast alone -------------------------------------------------------------

@@ -313,6 +313,23 @@ coat_status_t launch_norm_reg(cudaStream_t s, const coat::NormParams &p) {
                               : launch_norm_reg_form<NC, false>(s, p);
 }
 
+// Rows of 512 NCH columns, two warps a row, persistent blocks of four warp
+// pairs (as many as fit the GPU at once, or fewer, for few rows).
+template <int NCH, bool kAffine>
+coat_status_t launch_norm_split_form(cudaStream_t s, const coat::NormParams &p) {
+  constexpr auto kernel = coat::norm_split_group_amax_kernel<NCH, kAffine>;
+  const int64_t need = (p.rows + coat::kSplitPairs - 1) / coat::kSplitPairs;
+  const unsigned int grid = coat::resident_grid<kernel>(256, 0, need);
+  launch_act_threads(kernel, grid, 256u, 0, s, p);
+  return launch_status();
+}
+
+template <int NCH>
+coat_status_t launch_norm_split(cudaStream_t s, const coat::NormParams &p) {
+  return (p.weight || p.bias) ? launch_norm_split_form<NCH, true>(s, p)
+                              : launch_norm_split_form<NCH, false>(s, p);
+}
+
 }  // namespace
 
 extern "C" {
@@ -629,6 +646,16 @@ coat_status_t coat_norm_group_amax(const uint16_t *x, int64_t rows, int64_t cols
   if (tensor_amax)
     launch_act_threads(coat::zero_word_kernel, 1u, 32u, 0, s,
                        reinterpret_cast<uint32_t *>(tensor_amax));
+  if (cols % 512 == 0 && cols / 512 <= coat::kNormRegMaxChunks / 2 &&
+      (cols / 2) % group_size == 0) {
+    // even chunk counts whose 1xG runs lie within a half row: two warps a row
+    switch (cols / 512) {
+      case 1: return launch_norm_split<1>(s, p);
+      case 2: return launch_norm_split<2>(s, p);
+      case 3: return launch_norm_split<3>(s, p);
+      default: return launch_norm_split<4>(s, p);
+    }
+  }
   if (cols % 256 == 0 && cols / 256 <= coat::kNormRegMaxChunks) {
     switch (cols / 256) {
       case 1: return launch_norm_reg<1>(s, p);

@@ -45,18 +45,32 @@ def bytes_per_param(G: int) -> float:
     return 14.0 + 32.0 / G
 
 
-# sources of the activation quantizers (the traffic record of the 1xG
-# kernel is valid while these are unchanged)
-ACT_KERNEL_SOURCES = ["quantized_optimizer_states_b200/csrc/act_kernels.cuh",
-                      "quantized_optimizer_states_b200/csrc/resident_grid.cuh",
+# sources of the 1xG quantizer (its traffic record is valid while these are
+# unchanged): the activation header up to the end of the 1xG section (the
+# shared helpers and the 1xG kernels; the producers and the other kernels
+# below it do not enter the 1xG launch), and the headers it includes
+ACT_KERNEL_SOURCES = [("quantized_optimizer_states_b200/csrc/act_kernels.cuh",
+                       "// ---- Group Scaling per-tensor quantization"),
+                      "quantized_optimizer_states_b200/csrc/step_kernels.cuh",
+                      "quantized_optimizer_states_b200/csrc/state_codec.cuh",
                       "quantized_optimizer_states_b200/csrc/fp8_device.cuh"]
 
 
 def kernel_source_hash(sources=None) -> str:
+    """Hash of the kernel sources a traffic record was captured from; an
+    entry (path, marker) takes the file up to the line that starts with the
+    marker."""
     h = hashlib.sha256()
-    for rel in (KERNEL_SOURCES if sources is None else sources):
+    for ent in (KERNEL_SOURCES if sources is None else sources):
+        rel, marker = ent if isinstance(ent, tuple) else (ent, None)
         with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+            data = f.read()
+        if marker is not None:
+            cut = data.find(b"\n" + marker.encode())
+            if cut < 0:
+                raise ValueError(f"{rel}: no line starts with {marker!r}")
+            data = data[:cut + 1]
+        h.update(data)
     return h.hexdigest()[:16]
 
 

@@ -802,7 +802,7 @@ __global__ void __launch_bounds__(256, kAffine ? 3 : 4) norm_split_group_amax_ke
   const int64_t rounds = (r1 - r0 + kSplitPairs - 1) / kSplitPairs;
   const float nf = static_cast<float>(p.cols);   // exact (cols <= 16384)
   const int clanes = 1 << (p.log2G - 3);
-  float rowmax = 0.0f;
+  uint32_t rowmax2 = 0u, prev = 0u;   // BF16 pairs of |out| maxima
   uint4 nxt[NCH];
   auto load = [&](int64_t row, uint4 *c) {
     const uint4 *src = reinterpret_cast<const uint4 *>(p.x + row * p.cols);
@@ -889,13 +889,30 @@ __global__ void __launch_bounds__(256, kAffine ? 3 : 4) norm_split_group_amax_ke
         }
       }
       dst[lane + 32 * ci] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-      float a = fmaxf(bf16lo_to_float(am), bf16hi_to_float(am));
-      rowmax = fmaxf(rowmax, a);
+      rowmax2 = bmax2(rowmax2, am);
+      // the chunk's maximum in the low half-word (BF16, exact)
+      const uint32_t m = bmax2(am, am >> 16);
       if (clanes <= 32) {
-        for (int off = 1; off < clanes; off <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-        if ((lane & (clanes - 1)) == 0) p.group_amax[gbase + (col0 >> p.log2G)] = a;
+        // two chunk columns reduced together: chunk i - 1 in the low half,
+        // chunk i in the high half of one word
+        if ((i & 1) == 0 && i + 1 < NCH) {
+          prev = m;
+          continue;
+        }
+        uint32_t w = (i & 1) ? __byte_perm(prev, m, 0x5410) : m;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1)
+          if (off < clanes) w = bmax2(w, __shfl_xor_sync(0xffffffffu, w, off));
+        if ((lane & (clanes - 1)) == 0) {
+          if (i & 1) {
+            p.group_amax[gbase + ((col0 - 256) >> p.log2G)] = bf16lo_to_float(w);
+            p.group_amax[gbase + (col0 >> p.log2G)] = bf16hi_to_float(w);
+          } else {
+            p.group_amax[gbase + (col0 >> p.log2G)] = bf16lo_to_float(w);
+          }
+        }
       } else {
-        run = fmaxf(run, warp_max_f(a));
+        run = fmaxf(run, warp_max_f(bf16lo_to_float(m)));
         if (((ci + 1) & ((clanes >> 5) - 1)) == 0) {   // the run's last chunk column
           if (lane == 0) p.group_amax[gbase + ((256 * ci) >> p.log2G)] = run;
           run = 0.0f;
@@ -903,7 +920,9 @@ __global__ void __launch_bounds__(256, kAffine ? 3 : 4) norm_split_group_amax_ke
       }
     }
   }
-  if (p.tensor_amax) block_max_to_tensor(warp_max_f(rowmax), p.tensor_amax);
+  if (p.tensor_amax)
+    block_max_to_tensor(warp_max_f(fmaxf(bf16lo_to_float(rowmax2), bf16hi_to_float(rowmax2))),
+                        p.tensor_amax);
 }
 
 // ---- the FP8 cast alone -------------------------------------------------------------

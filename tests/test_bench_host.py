@@ -145,3 +145,17 @@ def test_zero1_peer_step_bytes():
     eight = bench.zero1_peers_bytes(L, 8, 128)
     assert eight["link_per_direction"] == 28 * L
     assert eight["hbm"] == (14.25 + 2 + 28) * L
+
+
+def test_source_hash_up_to_a_marker(tmp_path):
+    """A (path, marker) source counts only the text before the marker line:
+    an edit after it keeps the hash, an edit before it changes it."""
+    f = tmp_path / "k.cuh"
+    f.write_text("a\n// ---- B\nb\n")
+    h0 = bench.kernel_source_hash([(str(f), "// ---- B")])
+    f.write_text("a\n// ---- B\nb changed\n")
+    assert bench.kernel_source_hash([(str(f), "// ---- B")]) == h0
+    f.write_text("a changed\n// ---- B\nb\n")
+    assert bench.kernel_source_hash([(str(f), "// ---- B")]) != h0
+    with pytest.raises(ValueError):
+        bench.kernel_source_hash([(str(f), "// ---- missing")])

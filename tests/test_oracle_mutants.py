@@ -26,7 +26,8 @@ from oracle import build as orc_build
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PIN_FILES = ["tests/test_oracle_codec.py", "tests/test_oracle_state.py",
              "tests/test_oracle_act.py"]
-PY_PIN_FILES = PIN_FILES + ["tests/test_oracle_norm.py", "tests/test_oracle_swiglu.py"]
+PY_PIN_FILES = PIN_FILES + ["tests/test_oracle_norm.py", "tests/test_oracle_swiglu.py",
+                            "tests/test_oracle_grad_mean.py"]
 PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
 
 # (name, text in oracle/__init__.py, replacement)
@@ -65,6 +66,14 @@ PY_MUTANTS = [
     ("stats_nonfinite_includes_max", '"nonfinite_codes": int((mag > top).sum())',
      '"nonfinite_codes": int((mag >= top).sum())'),
     ("stats_k_sum_over_all_groups", "kn = k[nz].astype(np.float64)", "kn = k.astype(np.float64)"),
+    ("grad_mean_not_divided", "        acc = np.divide(acc, np.float32(len(grads)), dtype=np.float32)",
+     "        acc = acc"),
+    ("grad_mean_divides_by_world_minus_one",
+     "acc = np.divide(acc, np.float32(len(grads)), dtype=np.float32)",
+     "acc = np.divide(acc, np.float32(len(grads) - 1), dtype=np.float32)"),
+    ("grad_mean_drops_the_last_rank", "    for g in grads[1:]:", "    for g in grads[1:-1]:"),
+    ("grad_mean_first_rank_only", "    for g in grads[1:]:\n        acc = np.add(",
+     "    for g in []:\n        acc = np.add("),
     ("step_wrapper_swaps_k_and_s",
      "_ptr(th), _ptr(g), _ptr(mc), _ptr(mk), _ptr(ms), _ptr(vc),",
      "_ptr(th), _ptr(g), _ptr(mc), _ptr(ms), _ptr(mk), _ptr(vc),"),

@@ -209,7 +209,8 @@ coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, ui
  *              that rank gets no copy)
  *   m_code .. v_scale, n, cfg   this rank's shard, as coat_adamw_fp8_step
  * Every grads[r] + grad_offset and params_out[r] + params_out_offset must be
- * 16-byte aligned.  The caller orders the call between two barriers of all
+ * 16-byte aligned, and the current device must be able to access each of
+ * them (coat_enable_peer_access for another GPU's memory).  The caller orders the call between two barriers of all
  * ranks: after every rank's gradient is complete, and before any rank
  * reads its parameters (the kernel reads other ranks' gradients and writes
  * their parameter buffers; it waits for nothing on the device).  The
@@ -220,6 +221,17 @@ coat_status_t coat_adamw_fp8_step_guarded(float *param, const uint16_t *grad, ui
  * UNSUPPORTED, CUDA.
  */
 #define COAT_MAX_PEERS 8
+
+/*
+ * coat_enable_peer_access -- let kernels launched on the current device read
+ * and write the memory of GPU `peer_device` (a rank's buffers mapped into
+ * this process live there): cudaDeviceEnablePeerAccess from the current
+ * device, where the two can reach each other.  A call for the current
+ * device, or for a peer already enabled, does nothing.
+ * Errors: INVALID_ARG (no such device), UNSUPPORTED (the two devices cannot
+ * reach each other), CUDA.
+ */
+coat_status_t coat_enable_peer_access(int32_t peer_device);
 coat_status_t coat_adamw_fp8_step_peers(const uint16_t *const *grads, int32_t world,
                                         int64_t grad_offset, float *param,
                                         void *const *params_out, int32_t params_out_bf16,

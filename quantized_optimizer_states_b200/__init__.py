@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     coat_adamw_fp8_step_peers,
     coat_count_nonfinite_bf16,
     coat_dequant,
+    coat_enable_peer_access,
     coat_fp8_encode,
     coat_group_quant_1xG,
     coat_group_scaling_quant_pertensor,

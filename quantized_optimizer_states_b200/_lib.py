@@ -71,6 +71,7 @@ SIGNATURES = {
     "coat_adamw_fp8_step_peers": (_I32, [ctypes.POINTER(_P), _I32, _I64, _P, ctypes.POINTER(_P),
                                          _I32, _I64, _P, _P, _P, _P, _P, _P, _I64,
                                          ctypes.POINTER(CoatAdamwCfg), _P]),
+    "coat_enable_peer_access": (_I32, [_I32]),
     "coat_adamw_fp8_step_guarded": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
                                            ctypes.POINTER(CoatAdamwCfg), _P, _P]),
     "coat_adamw_fp8_step_fp32grad": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I64,
@@ -231,6 +232,13 @@ def _peer_ptr(t, dtype, what):
     if not t.is_contiguous() or t.dtype != dtype:
         raise ValueError(f"{what} must be a contiguous {dtype} tensor")
     return t.data_ptr()
+
+
+def coat_enable_peer_access(peer_device: int):
+    """Let the current device's kernels access GPU `peer_device`'s memory
+    (see include/coat.h); raises CoatError where the two cannot reach each
+    other."""
+    _check("coat_enable_peer_access", load().coat_enable_peer_access(int(peer_device)))
 
 
 def coat_adamw_fp8_step_peers(grads, param, m_code, m_k, m_scale, v_code, v_k, v_scale, *,

@@ -397,6 +397,29 @@ coat_status_t coat_adamw_fp8_step_peers(const uint16_t *const *grads, int32_t wo
                    nullptr, stream, &pa);
 }
 
+coat_status_t coat_enable_peer_access(int32_t peer_device) {
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return launch_status();
+  if (peer_device == cur) return COAT_OK;
+  int count = 0;
+  if (cudaGetDeviceCount(&count) != cudaSuccess) return launch_status();
+  if (peer_device < 0 || peer_device >= count) return COAT_ERR_INVALID_ARG;
+  int can = 0;
+  if (cudaDeviceCanAccessPeer(&can, cur, peer_device) != cudaSuccess) return launch_status();
+  if (!can) return COAT_ERR_UNSUPPORTED;
+  const cudaError_t e = cudaDeviceEnablePeerAccess(peer_device, 0);
+  if (e == cudaErrorPeerAccessAlreadyEnabled) {
+    cudaGetLastError();   // not an error here: clear it
+    return COAT_OK;
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_last_cuda_error = static_cast<int32_t>(e);
+    return COAT_ERR_CUDA;
+  }
+  return COAT_OK;
+}
+
 coat_status_t coat_count_nonfinite_bf16(const uint16_t *x, int64_t n, uint32_t *count,
                                         void *stream) {
   NvtxRange nvtx_range("coat_count_nonfinite_bf16");

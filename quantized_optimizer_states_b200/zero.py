@@ -317,6 +317,12 @@ class PeerBuffers:
                       for r in range(shard.world)]
         self.params = [self.param if r == shard.rank else _open(every[r][1])
                        for r in range(shard.world)]
+        # the step kernel runs on this rank's device and reads and writes the
+        # other ranks' buffers where they live: enable access to every other
+        # GPU among them (raises where two GPUs cannot reach each other)
+        with torch.cuda.device(dev):
+            for d in sorted({t.get_device() for t in self.grads + self.params} - {dev.index}):
+                _lib.coat_enable_peer_access(d)
 
 
 def _barrier(shard: "Zero1Shard", device: torch.device):

@@ -107,3 +107,14 @@ def test_peer_step_argument_errors(lib):
     with pytest.raises(lib.CoatError) as e:              # 8-byte gradient offset
         lib.coat_adamw_fp8_step_peers([g, g], th, *st, grad_offset=4, **cfg)
     assert e.value.status == 2
+
+
+def test_enable_peer_access_argument_handling(lib):
+    """The current device needs no enabling; a device index the machine does
+    not have is refused before any CUDA call that could change state."""
+    import torch
+    cur = torch.cuda.current_device()
+    lib.coat_enable_peer_access(cur)                    # a no-op
+    with pytest.raises(lib.CoatError) as e:
+        lib.coat_enable_peer_access(torch.cuda.device_count() + 3)
+    assert e.value.status == 1

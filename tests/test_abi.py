@@ -348,3 +348,27 @@ def test_binding_signatures_match_the_header():
         want_res, want_args = protos[name]
         assert _ctypes_kind(res) == want_res, name
         assert [_ctypes_kind(a) for a in args] == want_args, name
+
+
+def test_peer_step_binding_checks_before_any_call():
+    """The binding of coat_adamw_fp8_step_peers refuses bad rank lists on the
+    host, before it touches a device pointer (CPU tensors stand in)."""
+    import torch
+    from quantized_optimizer_states_b200 import _lib
+    n = 256
+    th = torch.zeros(n)
+    st = [torch.zeros(n, dtype=torch.uint8), torch.ones(2), torch.zeros(2),
+          torch.zeros(n, dtype=torch.uint8), torch.ones(2), torch.zeros(2)]
+    g = torch.zeros(2 * n, dtype=torch.bfloat16)
+    kw = dict(step=1, beta1=0.9, beta2=0.999, lr=1e-4, eps=1e-8, weight_decay=0.0)
+    for grads, extra, what in (
+            ([], {}, "1 to 8 ranks"),
+            ([g] * 9, {}, "1 to 8 ranks"),
+            ([g, g], {"grad_offset": 384}, "ends before the shard"),
+            ([g, g], {"params_out": [g]}, "one entry per rank"),
+            ([g, g], {"params_out": [g, torch.zeros(2 * n)]}, "must all be float32 or all bfloat16"),
+            ([g, g], {"params_out": [g, torch.zeros(n, dtype=torch.bfloat16)],
+                      "params_out_offset": 128}, "ends before the shard")):
+        args = {"grad_offset": 0, **extra}
+        with pytest.raises(ValueError, match=what):
+            _lib.coat_adamw_fp8_step_peers(grads, th, *st, **args, **kw)

@@ -367,7 +367,7 @@ def test_peer_step_binding_checks_before_any_call():
             ([g, g], {"grad_offset": 384}, "ends before the shard"),
             ([g, g], {"params_out": [g]}, "one entry per rank"),
             ([g, g], {"params_out": [g, torch.zeros(2 * n)]}, "must all be float32 or all bfloat16"),
-            ([g, g], {"params_out": [g, torch.zeros(n, dtype=torch.bfloat16)],
+            ([g, g], {"params_out": [torch.zeros(n, dtype=torch.bfloat16), g],
                       "params_out_offset": 128}, "ends before the shard")):
         args = {"grad_offset": 0, **extra}
         with pytest.raises(ValueError, match=what):

@@ -9,7 +9,9 @@ Pages cited (by title and section):
   COAT summary, "COAT: 压缩优化器状态和激活以实现内存高效的 FP8 训练"
   (blog.daoxuan.cc/posts/57954): sections on the AdamW rule and why v is
   sensitive, the expansion function f(x) = sign(x)|x|^k with
-  k = log(R_E4M3)/log(R_X), mixed granularity (1xG groups and Group Scaling).
+  k = log(R_E4M3)/log(R_X), mixed granularity (1xG groups and Group Scaling),
+  and the results section (training on several GPUs: the data-parallel
+  gradient mean of grad_mean_bf16).
   LLM Atlas "systems/numerics" (llm-atlas.k1412.top): section 03 "FP8"
   (format limits) and section 08 "Adam -> AdamW" (the update rule).
 
